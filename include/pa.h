@@ -1,0 +1,254 @@
+/*
+ * pa.h -- C ABI of the B200 paged-attention library (libpagedattn.so).
+ *
+ * The library implements the data-parallel hot path of PagedAttention:
+ * scaled-dot-product attention whose K/V are read through per-sequence block
+ * tables from a fixed pool of non-contiguous physical blocks, the block-table
+ * KV append (reshape_and_cache) and the copy-on-write block copy, plus the
+ * host block manager that decides tables, slot mappings and copies.
+ *
+ * Pages the operations follow (cited by title and section):
+ *   [P1] "abhik.ai examples/pagedattention.py" -- KVPool: physical pool,
+ *        allocation order, append, fork, copy-on-write, release, Eq. 3.
+ *   [P2] "vladkulikov.com modern-llms module 9 notebook" -- PagedKVPool:
+ *        preflighted multi-token append, share_prefix, snapshot, validate.
+ *   [P3] "docs.rs ferrum-kv 0.4.0 src/attention.rs" -- paged_attention:
+ *        query [q_tokens, num_heads, head_dim], GQA (kv_h = h / (H / Hkv)),
+ *        scale = 1/sqrt(head_dim), causal rule max_visible = kv_len -
+ *        q_tokens + qt, softmax, weighted sum of V.
+ *   [P4] "semidirectx cmu11-667 lecture19 infer_world.py", section 3 --
+ *        online softmax (m, l) and the tiled (m, l, acc) recurrence.
+ *
+ * Conventions shared by every entry point
+ *   - Pool layout: k_cache and v_cache are device arrays
+ *     [num_blocks, block_size, num_kv_heads, head_dim], row-major, dtype
+ *     pa_dtype.  Slot s = block * block_size + offset; element
+ *     (blk, off, h, i) sits at ((blk * block_size + off) * num_kv_heads + h)
+ *     * head_dim + i.  This is [P3]'s per-token layout [kv_len, Hkv, d]
+ *     stored block by block.
+ *   - Ownership: every device pointer (pool, key/value, query, output, block
+ *     tables, kv_lens, workspace) belongs to the caller and must stay valid
+ *     until the work queued on the given stream has finished.  The pool
+ *     borrows k_cache/v_cache; pa_free never frees them.  The pool owns its
+ *     manager state (free list, refcounts, tables), a small device staging
+ *     area for append plans and a device error word.
+ *   - Streams: device work is queued asynchronously on the caller's stream
+ *     (cudaStream_t passed as void*; NULL = legacy default stream).  Calls on
+ *     one pool must be issued from one host thread and on one stream, or be
+ *     externally ordered.
+ *   - Errors: status codes only; nothing aborts or traps.  Host-detectable
+ *     errors are checked before any state changes (the preflight of [P1]
+ *     append and [P2] append).  Device-detectable errors (a table entry
+ *     outside [0, num_blocks), a slot outside the pool, kv_len < q_tokens or
+ *     beyond the table, a wait that ran out of iterations) set bits of the
+ *     pool's device error word (PA_DEVERR_*), the affected output rows are
+ *     written as zeros and the kernel finishes; pa_get_error reads them.
+ *   - A pool created with k_cache == v_cache == NULL is host-only: the
+ *     manager calls work (no GPU needed), device calls return
+ *     PA_ERR_NO_DEVICE.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct pa_pool pa_pool; /* opaque */
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,     /* bad size, null pointer, misaligned pointer  */
+  PA_ERR_UNKNOWN_SEQ = 2,     /* sequence id not live ([P1] _existing)       */
+  PA_ERR_DUP_SEQ = 3,         /* sequence id already live ([P1] create)      */
+  PA_ERR_POOL_EXHAUSTED = 4,  /* preflight found too few free blocks         */
+  PA_ERR_CUDA = 5,            /* a CUDA runtime call failed                  */
+  PA_ERR_DEVICE = 6,          /* pa_get_error found device error bits        */
+  PA_ERR_UNSUPPORTED = 7,     /* shape/dtype outside what the kernels take   */
+  PA_ERR_NO_DEVICE = 8,       /* device call on a host-only pool             */
+  PA_ERR_INTERNAL = 9         /* pa_validate found a broken invariant        */
+} pa_status;
+
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits of the device error word. */
+#define PA_DEVERR_BLOCK_ID 1  /* block-table entry outside [0, num_blocks)   */
+#define PA_DEVERR_SLOT 2      /* slot outside [0, num_blocks * block_size)   */
+#define PA_DEVERR_KV_LEN 4    /* kv_len < q_tokens, < 0 or beyond the table  */
+#define PA_DEVERR_TIMEOUT 8   /* a bounded wait gave up                      */
+
+/* [P2] PagedKVPool.snapshot figures (token counts). */
+typedef struct pa_stats {
+  int64_t allocated_blocks;
+  int64_t free_blocks;
+  int64_t physical_capacity_tokens;  /* allocated_blocks * block_size       */
+  int64_t physical_payload_tokens;   /* sum over blocks of max sharer fill  */
+  int64_t logical_tokens;            /* sum of sequence lengths             */
+  int64_t internal_waste_tokens;     /* capacity - payload                  */
+  int64_t sharing_savings_tokens;    /* logical - payload                   */
+  int64_t live_sequences;
+} pa_stats;
+
+/* ---- pool lifetime ----------------------------------------------------- */
+
+/* Create a pool over caller-owned k_cache/v_cache (see layout above).
+ * alloc_order: host array, a permutation of [0, num_blocks); a new block is
+ * the first free id in this order ([P1] KVPool._allocate).  NULL = identity
+ * order.  Copied; the caller may free it after the call.
+ * Errors: PA_ERR_INVALID_ARG (non-positive size, not a permutation, exactly
+ * one of k_cache/v_cache NULL, cache pointer not 16-byte aligned). */
+pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
+                         int32_t num_kv_heads, int32_t head_dim,
+                         pa_dtype kv_dtype, void* k_cache, void* v_cache,
+                         const int32_t* alloc_order, pa_pool** out);
+
+/* Destroy the manager, its staging area and error word (synchronises the
+ * device first).  Never frees k_cache/v_cache.  NULL is a no-op. */
+pa_status pa_free(pa_pool* pool);
+
+/* ---- host block manager ([P1] KVPool, [P2] PagedKVPool) ----------------- */
+
+/* New empty sequence; no block is reserved ([P1] create). */
+pa_status pa_seq_create(pa_pool* pool, int32_t seq);
+
+/* New sequence `child` sharing the blocks that cover the first
+ * prefix_tokens tokens of `parent` (refcount +1 each) ([P2] share_prefix);
+ * prefix_tokens = -1 shares the whole parent ([P1] fork).
+ * Errors: UNKNOWN_SEQ, DUP_SEQ, INVALID_ARG (prefix > parent length). */
+pa_status pa_seq_fork(pa_pool* pool, int32_t parent, int32_t child,
+                      int32_t prefix_tokens);
+
+/* Drop one reference per block of `seq`; blocks reaching zero return to the
+ * free list ([P1] release, [P2] release). */
+pa_status pa_seq_release(pa_pool* pool, int32_t seq);
+
+/* Length and table of `seq`.  blocks_out (host, capacity cap) may be NULL to
+ * query only n_blocks/length.  INVALID_ARG if cap is too small. */
+pa_status pa_seq_table(const pa_pool* pool, int32_t seq, int32_t* blocks_out,
+                       int32_t cap, int32_t* n_blocks, int32_t* length);
+
+/* Batch tables for a decode/prefill call: tables_out host [n, width] int32
+ * (row i = table of seqs[i], padded with 0), kv_lens_out host [n] int32.
+ * INVALID_ARG if a table is wider than `width`. */
+pa_status pa_block_tables(const pa_pool* pool, const int32_t* seqs, int32_t n,
+                          int32_t width, int32_t* tables_out,
+                          int32_t* kv_lens_out);
+
+/* Plan an append on the host only (step a1 of the path): for each i append
+ * n_new[i] tokens to seqs[i] (distinct ids) in order.  The whole batch is
+ * preflighted first ([P2] _blocks_needed_for_append, counting a copy for a
+ * shared partial tail); on PA_ERR_POOL_EXHAUSTED nothing changes.  Then per
+ * sequence a shared partial tail is replaced by a fresh block (a copy pair
+ * (src, dst), [P1] _private_tail) and tokens are placed at
+ * table[pos / block_size] * block_size + pos % block_size, a fresh block
+ * being claimed at each boundary ([P1] append).
+ * Outputs (host, may be NULL): slot_mapping_out [sum n_new] int64 in batch
+ * order; cow_src_out/cow_dst_out [cow_cap] int32; n_cow_out.  INVALID_ARG if
+ * more copies than cow_cap (checked before any change; at most n_seqs). */
+pa_status pa_plan_append(pa_pool* pool, const int32_t* seqs,
+                         const int32_t* n_new, int32_t n_seqs,
+                         int64_t* slot_mapping_out, int32_t* cow_src_out,
+                         int32_t* cow_dst_out, int32_t cow_cap,
+                         int32_t* n_cow_out);
+
+/* [P2] snapshot figures. */
+pa_status pa_pool_stats(const pa_pool* pool, pa_stats* out);
+
+/* Refcount of every block: out host [num_blocks] int32. */
+pa_status pa_refcounts(const pa_pool* pool, int32_t* out);
+
+/* [P2] validate: PA_OK, or PA_ERR_INTERNAL if an invariant is broken. */
+pa_status pa_validate(const pa_pool* pool);
+
+/* ---- device hot path ---------------------------------------------------- */
+
+/* Append tokens to sequences and write their K/V into the pool:
+ * pa_plan_append, then (on `stream`) the copy-on-write block copies, then
+ * reshape_and_cache.  key/value: device [T, num_kv_heads, head_dim] in the
+ * pool dtype, T = sum n_new, rows in batch order (all of seqs[0]'s new tokens
+ * first).  slot_mapping_out: optional host [T] int64 copy of the plan.
+ * Errors: those of pa_plan_append (no change), NO_DEVICE, CUDA. */
+pa_status pa_append_kv(pa_pool* pool, const int32_t* seqs,
+                       const int32_t* n_new, int32_t n_seqs, const void* key,
+                       const void* value, int64_t* slot_mapping_out,
+                       void* stream);
+
+/* reshape_and_cache alone: k_cache[slot] = key[t], v_cache[slot] = value[t]
+ * for t < T, all heads ([P1] append write).  d_slot_mapping: device [T]
+ * int64; a negative slot skips the token; a slot >= num_blocks*block_size
+ * sets PA_DEVERR_SLOT and skips it.  key/value: device [T, Hkv, d]. */
+pa_status pa_reshape_and_cache(pa_pool* pool, const void* key,
+                               const void* value,
+                               const int64_t* d_slot_mapping, int32_t T,
+                               void* stream);
+
+/* Copy-on-write block copies: for i < n, whole block d_dst[i] := block
+ * d_src[i] in both k_cache and v_cache, every slot and head
+ * ([P1] _private_tail).  d_src/d_dst: device [n] int32; an id outside
+ * [0, num_blocks) sets PA_DEVERR_BLOCK_ID and skips the pair.  Pairs must
+ * not chain (no dst of one pair is the src of another). */
+pa_status pa_cow_copy(pa_pool* pool, const int32_t* d_src,
+                      const int32_t* d_dst, int32_t n, void* stream);
+
+/* Scratch bytes pa_decode needs for a batch of B sequences with H query
+ * heads and tables of width max_blocks (max kv_len = max_blocks *
+ * block_size) at the given partition_tokens (0 = automatic choice).  0 when
+ * no split is used. */
+size_t pa_decode_workspace_bytes(const pa_pool* pool, int32_t B, int32_t H,
+                                 int32_t max_blocks, int32_t partition_tokens);
+
+/* Decode attention (q_tokens = 1, every cached token visible; [P3] with
+ * q_tokens = 1, [P1] Eq. 3): out[b, h, :] = sum_j softmax_j(q[b,h].k_j *
+ * scale) v_j over j < kv_lens[b], k_j/v_j of KV head h / (H / Hkv) read
+ * through block_tables[b].
+ *   q: device [B, H, head_dim], pool dtype.  out: device [B, H, head_dim]
+ *   float32.  d_block_tables: device [B, max_blocks] int32.  d_kv_lens:
+ *   device [B] int32 (0 gives a zero row).  scale: usually 1/sqrt(head_dim).
+ *   partition_tokens: 0 = automatic, > 0 = split each sequence into
+ *   partitions of that many tokens (a multiple of block_size) whose softmax
+ *   statistics are merged by a log-sum-exp combine ([P4] recurrence applied
+ *   across partitions).  workspace: device scratch of
+ *   pa_decode_workspace_bytes bytes (16-byte aligned), may be NULL when that
+ *   is 0.
+ * Errors: INVALID_ARG (H not a multiple of Hkv, null/misaligned pointer,
+ * workspace too small, partition not a multiple of block_size), NO_DEVICE,
+ * CUDA. */
+pa_status pa_decode(pa_pool* pool, const void* q, int32_t B, int32_t H,
+                    const int32_t* d_block_tables, int32_t max_blocks,
+                    const int32_t* d_kv_lens, float scale,
+                    int32_t partition_tokens, void* workspace,
+                    size_t workspace_bytes, float* out, void* stream);
+
+/* Chunked prefill attention ([P3] with q_tokens > 1): for each sequence b
+ * the chunk's q_tokens queries are its last q_tokens positions; query qt
+ * sees cached positions j <= kv_lens[b] - q_tokens + qt.  The chunk's own
+ * K/V must already be in the pool (pa_append_kv).
+ *   q: device [B, q_tokens, H, head_dim], pool dtype.  out: device
+ *   [B, q_tokens, H, head_dim] float32.  Tables/kv_lens as pa_decode.
+ * Errors: as pa_decode. */
+pa_status pa_prefill_chunk(pa_pool* pool, const void* q, int32_t B,
+                           int32_t q_tokens, int32_t H,
+                           const int32_t* d_block_tables, int32_t max_blocks,
+                           const int32_t* d_kv_lens, float scale, float* out,
+                           void* stream);
+
+/* Synchronise the device, read and clear the pool's device error word.
+ * *device_code = OR of PA_DEVERR_* bits seen since the last call.  Returns
+ * PA_ERR_DEVICE when it is non-zero. */
+pa_status pa_get_error(pa_pool* pool, int32_t* device_code);
+
+/* Static description of a status code. */
+const char* pa_status_string(pa_status status);
+
+/* Which kernel family pa_decode / pa_prefill_chunk would use for this pool
+ * and batch shape: 0 = generic CUDA-core kernel, 1 = the sm_100a fast path. */
+int32_t pa_decode_path(const pa_pool* pool, int32_t H);
+int32_t pa_prefill_path(const pa_pool* pool, int32_t H);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PA_H_ */

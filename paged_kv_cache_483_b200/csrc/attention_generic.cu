@@ -1,0 +1,148 @@
+// Generic CUDA-core paged attention (any dtype, head_dim <= 512, any block
+// size, any group size, q_tokens >= 1).  One CTA per output row (b, qt, h);
+// keys are visited in chunks of 128 with the one-pass (m, l, acc) update of
+// "semidirectx cmu11-667 lecture19 infer_world.py", section 3
+// (tiled_attention).  The scores follow "docs.rs ferrum-kv 0.4.0
+// src/attention.rs" (paged_attention): kv_h = h / (H / Hkv), query qt sees
+// positions j <= kv_len - q_tokens + qt.  This is the path for fp32 pools and
+// for shapes the tensor-core kernels do not take; it is correct, not fast.
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.hpp"
+
+namespace pa {
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+constexpr int kGenThreads = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int w = 1; w < kGenThreads / 32; ++w) r = fmaxf(r, red[w]);
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = 0.f;
+  for (int w = 0; w < kGenThreads / 32; ++w) r += red[w];
+  __syncthreads();
+  return r;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kGenThreads) attention_generic_kernel(
+    const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
+    const int32_t* __restrict__ tables, int MB, const int32_t* __restrict__ kv_lens,
+    int q_tokens, int H, int Hkv, int d, int bs, int NB, float scale_log2,
+    float* __restrict__ out, int32_t* err) {
+  extern __shared__ float gen_smem[];
+  float* qf = gen_smem;              // [d]
+  float* pr = qf + d;                // [128] scores, then weights
+  int* blk = (int*)(pr + kGenThreads);   // [128] physical block per key
+  float* red = (float*)(blk + kGenThreads);  // [32]
+  __shared__ int bad;
+
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (H / Hkv);
+  const int tid = threadIdx.x;
+  const int kv_len = kv_lens[b];
+  float* orow = out + ((int64_t(b) * q_tokens + qt) * H + h) * d;
+
+  const bool len_bad = kv_len < 0 || kv_len > MB * bs ||
+                       (q_tokens > 1 && kv_len < q_tokens) ||
+                       (q_tokens == 1 && kv_len < 0);
+  if (tid == 0) bad = 0;
+  if (len_bad) {
+    if (tid == 0 && qt == 0 && h == 0) raise_err(err, PA_DEVERR_KV_LEN);
+    for (int i = tid; i < d; i += kGenThreads) orow[i] = 0.f;
+    return;
+  }
+  const int visible = kv_len - q_tokens + qt + 1;  // keys 0 .. visible-1
+  const T* qrow = q + ((int64_t(b) * q_tokens + qt) * H + h) * d;
+  for (int i = tid; i < d; i += kGenThreads) qf[i] = to_f(qrow[i]) * scale_log2;
+  __syncthreads();
+
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // d <= 512 = 4 x 128
+  float m = -INFINITY, l = 0.f;
+  const int64_t tok_stride = int64_t(Hkv) * d;
+  for (int c0 = 0; c0 < visible; c0 += kGenThreads) {
+    const int j = c0 + tid;
+    float s = -INFINITY;
+    int pb = -1;
+    if (j < visible) {
+      pb = tables[int64_t(b) * MB + j / bs];
+      if (pb < 0 || pb >= NB) {
+        bad = 1;
+        pb = -1;
+      } else {
+        const T* krow = kc + (int64_t(pb) * bs + j % bs) * tok_stride + int64_t(kvh) * d;
+        float dot = 0.f;
+        for (int i = 0; i < d; ++i) dot = fmaf(qf[i], to_f(krow[i]), dot);
+        s = dot;
+      }
+    }
+    blk[tid] = pb;
+    const float cmax = block_max(s, red);
+    const float m_new = fmaxf(m, cmax);
+    const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
+    const float p = (s == -INFINITY) ? 0.f : exp2f(s - m_new);
+    pr[tid] = p;
+    const float csum = block_sum(p, red);  // also publishes pr/blk
+    l = l * alpha + csum;
+    m = (cmax == -INFINITY) ? m : m_new;
+    const int n = min(kGenThreads, visible - c0);
+    for (int r = 0; r < 4; ++r) {
+      const int i = tid + r * kGenThreads;
+      if (i >= d) break;
+      float a = acc[r] * alpha;
+      for (int jj = 0; jj < n; ++jj) {
+        const int pbj = blk[jj];
+        if (pbj < 0) continue;
+        const int jt = c0 + jj;
+        a = fmaf(pr[jj], to_f(vc[(int64_t(pbj) * bs + jt % bs) * tok_stride +
+                                 int64_t(kvh) * d + i]),
+                 a);
+      }
+      acc[r] = a;
+    }
+    __syncthreads();
+  }
+  const bool zero = bad || !(l > 0.f);
+  if (bad && tid == 0) raise_err(err, PA_DEVERR_BLOCK_ID);
+  for (int r = 0; r < 4; ++r) {
+    const int i = tid + r * kGenThreads;
+    if (i < d) orow[i] = zero ? 0.f : acc[r] / l;
+  }
+}
+
+cudaError_t launch_attention_generic(const GenericArgs& a, cudaStream_t s) {
+  dim3 grid(a.q_tokens, a.H, a.B);
+  size_t smem = sizeof(float) * (a.d + kGenThreads + 32) + sizeof(int) * kGenThreads;
+  const float sl2 = a.scale * kLog2e;
+  if (a.bf16) {
+    attention_generic_kernel<__nv_bfloat16><<<grid, kGenThreads, smem, s>>>(
+        (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k_cache,
+        (const __nv_bfloat16*)a.v_cache, a.tables, a.MB, a.kv_lens, a.q_tokens,
+        a.H, a.Hkv, a.d, a.bs, a.NB, sl2, a.out, a.err);
+  } else {
+    attention_generic_kernel<float><<<grid, kGenThreads, smem, s>>>(
+        (const float*)a.q, (const float*)a.k_cache, (const float*)a.v_cache,
+        a.tables, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs, a.NB, sl2,
+        a.out, a.err);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace pa

@@ -1,0 +1,207 @@
+// Host block manager (see block_manager.hpp for the pages it follows).
+#include "block_manager.hpp"
+
+#include <algorithm>
+#include <unordered_set>
+
+namespace pa {
+
+BlockManager::BlockManager(int32_t num_blocks, int32_t block_size,
+                           const std::vector<int32_t>& order)
+    : num_blocks_(num_blocks), block_size_(block_size),
+      order_(order), rank_(num_blocks), refs_(num_blocks, 0),
+      is_free_(num_blocks, 1), n_free_(num_blocks) {
+  if (order_.empty()) {
+    order_.resize(num_blocks);
+    for (int32_t i = 0; i < num_blocks; ++i) order_[i] = i;
+  }
+  for (int32_t r = 0; r < num_blocks; ++r) {
+    rank_[order_[r]] = r;
+    free_heap_.push(r);
+  }
+}
+
+bool BlockManager::is_permutation(const int32_t* order, int32_t n) {
+  std::vector<uint8_t> seen(n, 0);
+  for (int32_t i = 0; i < n; ++i) {
+    int32_t b = order[i];
+    if (b < 0 || b >= n || seen[b]) return false;
+    seen[b] = 1;
+  }
+  return true;
+}
+
+int32_t BlockManager::take_block() {
+  int32_t r = free_heap_.top();
+  free_heap_.pop();
+  int32_t b = order_[r];
+  is_free_[b] = 0;
+  --n_free_;
+  refs_[b] = 1;
+  return b;
+}
+
+void BlockManager::give_back(int32_t b) {
+  is_free_[b] = 1;
+  ++n_free_;
+  free_heap_.push(rank_[b]);
+}
+
+MgrStatus BlockManager::create(int32_t seq) {
+  if (seqs_.count(seq)) return MgrStatus::dup_seq;
+  seqs_.emplace(seq, Seq{});
+  return MgrStatus::ok;
+}
+
+MgrStatus BlockManager::share_prefix(int32_t parent, int32_t child,
+                                     int64_t prefix) {
+  auto it = seqs_.find(parent);
+  if (it == seqs_.end()) return MgrStatus::unknown_seq;
+  if (prefix < 0) prefix = it->second.length;  // fork: the whole parent
+  if (prefix > it->second.length) return MgrStatus::invalid;
+  if (seqs_.count(child)) return MgrStatus::dup_seq;
+  Seq s;
+  s.length = prefix;
+  int64_t nb = (prefix + block_size_ - 1) / block_size_;
+  s.blocks.assign(it->second.blocks.begin(), it->second.blocks.begin() + nb);
+  for (int32_t b : s.blocks) ++refs_[b];
+  seqs_.emplace(child, std::move(s));
+  return MgrStatus::ok;
+}
+
+MgrStatus BlockManager::release(int32_t seq) {
+  auto it = seqs_.find(seq);
+  if (it == seqs_.end()) return MgrStatus::unknown_seq;
+  for (int32_t b : it->second.blocks)
+    if (--refs_[b] == 0) give_back(b);
+  seqs_.erase(it);
+  return MgrStatus::ok;
+}
+
+MgrStatus BlockManager::append(const int32_t* seqs, const int32_t* n_new,
+                               int32_t n, std::vector<int64_t>* slots,
+                               std::vector<CowPair>* cow) {
+  // -- preflight: nothing below this block changes state until it passes.
+  std::unordered_set<int32_t> seen;
+  std::unordered_map<int32_t, int32_t> ref_drop;  // copies made earlier in batch
+  int64_t need = 0, total_tokens = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = seqs_.find(seqs[i]);
+    if (it == seqs_.end()) return MgrStatus::unknown_seq;
+    if (n_new[i] < 0 || !seen.insert(seqs[i]).second) return MgrStatus::invalid;
+    const Seq& s = it->second;
+    int64_t cnt = n_new[i];
+    total_tokens += cnt;
+    if (cnt == 0) continue;
+    int64_t used = s.length % block_size_, room = 0;
+    if (!s.blocks.empty() && used) {
+      room = block_size_ - used;
+      int32_t tail = s.blocks.back();
+      auto d = ref_drop.find(tail);
+      int32_t ref = refs_[tail] - (d == ref_drop.end() ? 0 : d->second);
+      if (ref > 1) {
+        need += 1;
+        ++ref_drop[tail];
+      }
+    }
+    int64_t beyond = std::max<int64_t>(0, cnt - room);
+    need += (beyond + block_size_ - 1) / block_size_;
+  }
+  if (need > n_free_) return MgrStatus::exhausted;
+
+  // -- apply: per sequence, copy a shared partial tail, then place tokens.
+  if (slots) slots->reserve(slots->size() + total_tokens);
+  for (int32_t i = 0; i < n; ++i) {
+    Seq& s = seqs_[seqs[i]];
+    int64_t cnt = n_new[i];
+    if (cnt == 0) continue;
+    if (!s.blocks.empty() && (s.length % block_size_) &&
+        refs_[s.blocks.back()] > 1) {
+      int32_t old = s.blocks.back();
+      int32_t fresh = take_block();
+      s.blocks.back() = fresh;
+      --refs_[old];
+      if (cow) cow->push_back({old, fresh});
+    }
+    for (int64_t t = 0; t < cnt; ++t) {
+      int64_t pos = s.length;
+      int64_t logical = pos / block_size_, off = pos % block_size_;
+      if (off == 0) s.blocks.push_back(take_block());
+      if (slots)
+        slots->push_back(int64_t(s.blocks[logical]) * block_size_ + off);
+      s.length = pos + 1;
+    }
+  }
+  return MgrStatus::ok;
+}
+
+const std::vector<int32_t>* BlockManager::table(int32_t seq) const {
+  auto it = seqs_.find(seq);
+  return it == seqs_.end() ? nullptr : &it->second.blocks;
+}
+
+int64_t BlockManager::length(int32_t seq) const {
+  auto it = seqs_.find(seq);
+  return it == seqs_.end() ? -1 : it->second.length;
+}
+
+std::vector<int64_t> BlockManager::fills() const {
+  std::vector<int64_t> fill(num_blocks_, 0);
+  for (const auto& kv : seqs_) {
+    const Seq& s = kv.second;
+    for (size_t j = 0; j < s.blocks.size(); ++j) {
+      int64_t f = std::min<int64_t>(block_size_, s.length - int64_t(j) * block_size_);
+      fill[s.blocks[j]] = std::max(fill[s.blocks[j]], f);
+    }
+  }
+  return fill;
+}
+
+Snapshot BlockManager::snapshot() const {
+  Snapshot r{};
+  std::vector<int64_t> fill = fills();
+  r.free = n_free_;
+  r.allocated = num_blocks_ - n_free_;
+  r.capacity = r.allocated * block_size_;
+  for (int32_t b = 0; b < num_blocks_; ++b)
+    if (refs_[b]) r.payload += fill[b];
+  for (const auto& kv : seqs_) r.logical += kv.second.length;
+  r.waste = r.capacity - r.payload;
+  r.savings = r.logical - r.payload;
+  r.live = int64_t(seqs_.size());
+  return r;
+}
+
+bool BlockManager::validate() const {
+  if (int64_t(free_heap_.size()) != n_free_) return false;
+  std::vector<int32_t> expect(num_blocks_, 0);
+  for (const auto& kv : seqs_) {
+    const Seq& s = kv.second;
+    if (s.length < 0) return false;
+    if (int64_t(s.blocks.size()) != (s.length + block_size_ - 1) / block_size_)
+      return false;
+    std::unordered_set<int32_t> uniq(s.blocks.begin(), s.blocks.end());
+    if (uniq.size() != s.blocks.size()) return false;
+    for (int32_t b : s.blocks) {
+      if (b < 0 || b >= num_blocks_) return false;
+      ++expect[b];
+    }
+  }
+  std::vector<int64_t> fill = fills();
+  int64_t nfree = 0;
+  for (int32_t b = 0; b < num_blocks_; ++b) {
+    if (refs_[b] != expect[b]) return false;
+    if (refs_[b] == 0) {
+      if (!is_free_[b] || fill[b] != 0) return false;
+      ++nfree;
+    } else {
+      if (is_free_[b]) return false;
+      if (fill[b] < 1 || fill[b] > block_size_) return false;
+    }
+  }
+  if (nfree != n_free_) return false;
+  Snapshot s = snapshot();
+  return s.logical >= s.payload;
+}
+
+}  // namespace pa

@@ -1,0 +1,71 @@
+// Host block manager: free list, refcounts, block tables, copy-on-write plans.
+//
+// Semantics follow "abhik.ai examples/pagedattention.py" (KVPool: first free
+// id in a fixed allocation order, copy-on-write of a shared partial tail,
+// release) and "vladkulikov.com modern-llms module 9 notebook" (PagedKVPool:
+// preflighted multi-token append, share_prefix, fill accounting, validate).
+// Pure C++: no CUDA here, so every decision can be tested without a GPU.
+#pragma once
+
+#include <cstdint>
+#include <queue>
+#include <unordered_map>
+#include <vector>
+
+namespace pa {
+
+enum class MgrStatus { ok, unknown_seq, dup_seq, exhausted, invalid };
+
+struct CowPair {
+  int32_t src, dst;
+};
+
+struct Snapshot {
+  int64_t allocated, free, capacity, payload, logical, waste, savings, live;
+};
+
+class BlockManager {
+ public:
+  // order: permutation of [0, num_blocks) or empty (identity).
+  BlockManager(int32_t num_blocks, int32_t block_size,
+               const std::vector<int32_t>& order);
+
+  static bool is_permutation(const int32_t* order, int32_t n);
+
+  MgrStatus create(int32_t seq);
+  MgrStatus share_prefix(int32_t parent, int32_t child, int64_t prefix);
+  MgrStatus release(int32_t seq);
+
+  // Batch append plan; all-or-nothing (preflight over the whole batch with
+  // the refcount changes earlier members of the batch make).
+  MgrStatus append(const int32_t* seqs, const int32_t* n_new, int32_t n,
+                   std::vector<int64_t>* slots, std::vector<CowPair>* cow);
+
+  const std::vector<int32_t>* table(int32_t seq) const;
+  int64_t length(int32_t seq) const;
+  Snapshot snapshot() const;
+  const std::vector<int32_t>& refcounts() const { return refs_; }
+  bool validate() const;
+
+  int32_t num_blocks() const { return num_blocks_; }
+  int32_t block_size() const { return block_size_; }
+
+ private:
+  struct Seq {
+    int64_t length = 0;
+    std::vector<int32_t> blocks;
+  };
+  int32_t take_block();            // first free id in the order
+  void give_back(int32_t block);   // refcount reached zero
+  std::vector<int64_t> fills() const;
+
+  int32_t num_blocks_, block_size_;
+  std::vector<int32_t> order_, rank_, refs_;
+  std::vector<uint8_t> is_free_;
+  int64_t n_free_;
+  // min-heap of the free blocks' positions in the allocation order
+  std::priority_queue<int32_t, std::vector<int32_t>, std::greater<int32_t>> free_heap_;
+  std::unordered_map<int32_t, Seq> seqs_;
+};
+
+}  // namespace pa

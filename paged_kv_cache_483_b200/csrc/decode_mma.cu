@@ -1,0 +1,349 @@
+// Paged decode attention for bf16 K/V, head_dim 128, block_size 16, GQA
+// group G <= 8: one CTA per (partition, KV head, sequence).
+//
+// What it computes ("docs.rs ferrum-kv 0.4.0 src/attention.rs",
+// paged_attention with q_tokens = 1; "abhik.ai examples/pagedattention.py",
+// Eq. 3): for the G query heads of KV head kvh,
+//     o_h = sum_j softmax_j(q_h . k_j * scale) v_j,   j < kv_len,
+// with k_j, v_j read through the block table, and the one-pass (m, l, acc)
+// update of "semidirectx cmu11-667 lecture19 infer_world.py", section 3.
+// With NP > 1 partitions each CTA covers part_blocks blocks and writes
+// (m, l, o = acc / l) for a log-sum-exp combine.
+//
+// B200 design:
+//  * one producer warp streams each 16-token block's K and V tiles
+//    (4 KB each; two 64-column boxes per tile with the 128-byte swizzle)
+//    from the pool into an NSTAGE ring with TMA (cp.async.bulk.tensor),
+//    one full/empty mbarrier pair per stage; loads carry an L2 evict-first
+//    hint because every byte is read exactly once;
+//  * four consumer warps take blocks round-robin.  The G query heads of the
+//    group share each K/V tile: S^T = K Q^T is one m16n8k16 tensor-core tile
+//    per 16 d-columns (M = the block's 16 tokens, N = 8 heads), the softmax
+//    statistics live in the accumulator fragment, P^T is turned into the B
+//    operand of O^T += V^T P^T with movmatrix, and V^T comes from ldmatrix
+//    .trans.  P is split into bf16 hi + lo parts so the product keeps ~16
+//    mantissa bits (the PV error then stays at fp32-accumulation level);
+//  * the four warps' partial (m, l, O) are merged through shared memory.
+// At G <= 8 the whole per-token arithmetic is 2 tensor-core tiles, so the
+// loop stays bound by HBM rather than by the FP32 pipes (a CUDA-core dot
+// product would need ~2 G FMA per byte-pair, near the B200's FP32 ridge at
+// G = 8).
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.hpp"
+
+namespace pa {
+
+constexpr int kDecStages = 12;
+constexpr int kDecThreads = 160;  // 4 consumer warps + 1 producer warp
+constexpr int kStageBytes = 8192;  // K tile 4 KB + V tile 4 KB
+constexpr float kLog2eF = 1.4426950408889634f;
+
+struct DecodeSmemTail {
+  uint64_t full[kDecStages];
+  uint64_t empty[kDecStages];
+  int stage_bad[kDecStages];
+  int any_bad;
+};
+
+__global__ void __launch_bounds__(kDecThreads, 2) decode_mma_kernel(
+    const __grid_constant__ CUtensorMap tmK,
+    const __grid_constant__ CUtensorMap tmV, const DecodeArgs p,
+    float scale_log2) {
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  DecodeSmemTail* tail =
+      reinterpret_cast<DecodeSmemTail*>(smem + kDecStages * kStageBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int part = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int G = p.H / p.Hkv;
+  const int kv_len = p.kv_lens[b];
+  const bool len_bad = kv_len < 0 || kv_len > p.MB * 16;
+  const int nblk_seq = len_bad ? 0 : (kv_len + 15) >> 4;
+  const int blk0 = part * p.part_blocks;
+  const int nblk = max(0, min(blk0 + p.part_blocks, nblk_seq) - blk0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+      tail->stage_bad[s] = 0;
+    }
+    tail->any_bad = len_bad ? 1 : 0;
+    fence_barrier_init();
+    if (len_bad && part == 0 && kvh == 0) raise_err(p.err, PA_DEVERR_KV_LEN);
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nblk > 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      const uint64_t pol = policy_evict_first();
+      const int32_t* trow = p.tables + int64_t(b) * p.MB + blk0;
+      int issued = 0;
+      for (int i = 0; i < nblk; ++i) {
+        const int s = i % kDecStages, round = i / kDecStages;
+        if (round > 0 && !mbar_wait(&tail->empty[s], (round - 1) & 1)) {
+          raise_err(p.err, PA_DEVERR_TIMEOUT);
+          break;
+        }
+        const int blk = trow[i];
+        if (blk < 0 || blk >= p.NB) {
+          tail->stage_bad[s] = 1;
+          tail->any_bad = 1;
+          raise_err(p.err, PA_DEVERR_BLOCK_ID);
+          mbar_arrive(&tail->full[s]);
+        } else {
+          tail->stage_bad[s] = 0;
+          uint8_t* st = smem + s * kStageBytes;
+          mbar_arrive_expect_tx(&tail->full[s], kStageBytes);
+          tma_load_3d(st, &tmK, &tail->full[s], 0, kvh, blk * 16, pol);
+          tma_load_3d(st + 2048, &tmK, &tail->full[s], 64, kvh, blk * 16, pol);
+          tma_load_3d(st + 4096, &tmV, &tail->full[s], 0, kvh, blk * 16, pol);
+          tma_load_3d(st + 6144, &tmV, &tail->full[s], 64, kvh, blk * 16, pol);
+        }
+        issued = i + 1;
+      }
+      // drain: no copy may still be landing in shared memory at exit
+      for (int s = 0; s < kDecStages && s < issued; ++s) {
+        const int count = (issued - 1 - s) / kDecStages + 1;
+        mbar_wait(&tail->full[s], (count - 1) & 1);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------- consumers
+  const int g = lane >> 2, c = lane & 3;
+  uint32_t qb[8][2];
+  {
+    const bool ok = g < G;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        static_cast<const __nv_bfloat16*>(p.q) +
+        (int64_t(b) * p.H + kvh * G + (ok ? g : 0)) * 128);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      qb[kk][0] = ok ? __ldg(qrow + 8 * kk + c) : 0u;
+      qb[kk][1] = ok ? __ldg(qrow + 8 * kk + 4 + c) : 0u;
+    }
+  }
+  float o[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  // per-lane ldmatrix row/chunk pattern
+  const int ld_row = (lane & 7) + ((lane >> 3) & 1) * 8;  // K: token row
+  const int ld_khalf = lane >> 4;                          // K: +0/+1 chunk
+  const int lv_tok = (lane & 7) + ((lane >> 4) << 3);      // V: token row
+  const int lv_dc = (lane >> 3) & 1;                       // V: +0/+1 chunk
+  const int tok_end = kv_len;
+
+  for (int i = warp; i < nblk; i += 4) {
+    const int s = i % kDecStages;
+    const bool landed = __all_sync(0xffffffffu, mbar_wait(&tail->full[s], (i / kDecStages) & 1));
+    if (!landed) {
+      if (lane == 0) {
+        raise_err(p.err, PA_DEVERR_TIMEOUT);
+        tail->any_bad = 1;
+      }
+      break;
+    }
+    if (!tail->stage_bad[s]) {
+      const uint32_t kb = smem_u32(smem + s * kStageBytes);
+      const uint32_t vb = kb + 4096;
+      const int valid = min(16, tok_end - (blk0 + i) * 16);
+      if (valid < 16) {
+        // slots past the sequence end hold stale bytes (possibly NaN
+        // patterns); zero their V rows so p = 0 contributes exactly 0
+        uint4* vt = reinterpret_cast<uint4*>(smem + s * kStageBytes + 4096);
+        for (int idx = lane; idx < (16 - valid) * 16; idx += 32) {
+          const int row = valid + (idx >> 4), ch = idx & 15;
+          vt[(ch >> 3) * 128 + row * 8 + (ch & 7)] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();  // order these writes before later TMA refills
+        __syncwarp();
+      }
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int ch = 2 * kk + ld_khalf;
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(kb + (ch >> 3) * 2048 + swz128(ld_row, ch & 7), a0, a1, a2, a3);
+        mma_bf16_16816(sc, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+      }
+      const int tb = (blk0 + i) * 16;
+      float s0 = sc[0] * scale_log2, s1 = sc[1] * scale_log2;
+      float s2 = sc[2] * scale_log2, s3 = sc[3] * scale_log2;
+      if (tb + g >= tok_end) s0 = s1 = -INFINITY;
+      if (tb + g + 8 >= tok_end) s2 = s3 = -INFINITY;
+      float x0 = fmaxf(s0, s2), x1 = fmaxf(s1, s3);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, off));
+        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, off));
+      }
+      // token tb < tok_end, so x0 and x1 are finite here
+      const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
+      const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
+      const float p0 = exp2f(s0 - n0), p2 = exp2f(s2 - n0);
+      const float p1 = exp2f(s1 - n1), p3 = exp2f(s3 - n1);
+      l0 = l0 * al0 + (p0 + p2);
+      l1 = l1 * al1 + (p1 + p3);
+      m0 = n0;
+      m1 = n1;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        o[j][0] *= al0;
+        o[j][1] *= al1;
+        o[j][2] *= al0;
+        o[j][3] *= al1;
+      }
+      // P^T as B fragments: hi part + lo remainder, both bf16
+      const __nv_bfloat162 h01 = __floats2bfloat162_rn(p0, p1);
+      const __nv_bfloat162 h23 = __floats2bfloat162_rn(p2, p3);
+      const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+      const uint32_t hb0 = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
+      const uint32_t hb1 = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
+      const uint32_t lb0 = movmatrix_trans(pack_bf16x2(p0 - f01.x, p1 - f01.y));
+      const uint32_t lb1 = movmatrix_trans(pack_bf16x2(p2 - f23.x, p3 - f23.y));
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int ch = 2 * j + lv_dc;
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4_trans(vb + (ch >> 3) * 2048 + swz128(lv_tok, ch & 7), a0, a1, a2, a3);
+        mma_bf16_16816(o[j], a0, a1, a2, a3, hb0, hb1);
+        mma_bf16_16816(o[j], a0, a1, a2, a3, lb0, lb1);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tail->empty[s]);
+  }
+
+  // ------------------------------------------- merge the four warps' states
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+  named_bar_sync(1, 128);  // every consumer is done with the ring
+  float* so = reinterpret_cast<float*>(smem);  // [4][8][128]
+  float* sm = so + 4 * 8 * 128;                // [4][8]
+  float* sl = sm + 32;                         // [4][8]
+  {
+    float* w0 = so + (warp * 8 + 2 * c) * 128;
+    float* w1 = w0 + 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      w0[16 * j + g] = o[j][0];
+      w1[16 * j + g] = o[j][1];
+      w0[16 * j + g + 8] = o[j][2];
+      w1[16 * j + g + 8] = o[j][3];
+    }
+    if (g == 0) {
+      sm[warp * 8 + 2 * c] = m0;
+      sm[warp * 8 + 2 * c + 1] = m1;
+      sl[warp * 8 + 2 * c] = l0;
+      sl[warp * 8 + 2 * c + 1] = l1;
+    }
+  }
+  named_bar_sync(1, 128);
+  const int t = threadIdx.x;  // d column
+  const bool zero = tail->any_bad != 0;
+  for (int n = 0; n < G; ++n) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[w * 8 + n]);
+    float num = 0.f, den = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float mw = sm[w * 8 + n];
+        const float sc = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+        num = fmaf(so[(w * 8 + n) * 128 + t], sc, num);
+        den = fmaf(sl[w * 8 + n], sc, den);
+      }
+    }
+    const float val = (den > 0.f && !zero) ? num / den : 0.f;
+    const int64_t bh = int64_t(b) * p.H + kvh * G + n;
+    if (p.NP == 1) {
+      p.out[bh * 128 + t] = val;
+    } else {
+      const int64_t slot = bh * p.NP + part;
+      float* ws_m = p.ws;
+      float* ws_l = ws_m + int64_t(p.B) * p.H * p.NP;
+      float* ws_o = ws_l + int64_t(p.B) * p.H * p.NP;
+      ws_o[slot * 128 + t] = val;
+      if (t == 0) {
+        ws_m[slot] = M;
+        ws_l[slot] = zero ? -1.f : den;  // -1 poisons the whole row
+      }
+    }
+  }
+}
+
+// Log-sum-exp combine of the partitions: M = max_p m_p,
+// w_p = l_p 2^(m_p - M), o = sum_p w_p o_p / sum_p w_p (m in log2 units).
+__global__ void __launch_bounds__(128) decode_combine_kernel(
+    const float* __restrict__ ws, int B, int H, int NP, float* __restrict__ out) {
+  const int64_t bh = blockIdx.x;
+  const float* ws_m = ws + bh * NP;
+  const float* ws_l = ws + int64_t(B) * H * NP + bh * NP;
+  const float* ws_o = ws + 2 * int64_t(B) * H * NP + bh * NP * 128;
+  const int t = threadIdx.x;
+  float M = -INFINITY;
+  bool poison = false;
+  for (int q = 0; q < NP; ++q) {
+    M = fmaxf(M, ws_m[q]);
+    poison |= ws_l[q] < 0.f;
+  }
+  float num = 0.f, den = 0.f;
+  if (M != -INFINITY && !poison) {
+    for (int q = 0; q < NP; ++q) {
+      const float mq = ws_m[q];
+      if (mq == -INFINITY) continue;
+      const float w = ws_l[q] * exp2f(mq - M);
+      num = fmaf(w, ws_o[q * 128 + t], num);
+      den += w;
+    }
+  }
+  out[bh * 128 + t] = den > 0.f ? num / den : 0.f;
+}
+
+bool decode_fast_supported(int dtype_bf16, int d, int bs, int G) {
+  return dtype_bf16 && d == 128 && bs == 16 && G >= 1 && G <= 8;
+}
+
+size_t split_workspace_bytes(int32_t B, int32_t H, int32_t NP, int32_t d) {
+  if (NP <= 1) return 0;
+  return sizeof(float) * size_t(B) * H * NP * (2 + size_t(d));
+}
+
+cudaError_t launch_decode_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
+                               const DecodeArgs& a, int sms,
+                               cudaStream_t stream) {
+  (void)sms;
+  const size_t smem = 1024 + kDecStages * kStageBytes + sizeof(DecodeSmemTail);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(
+        decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid(a.NP, a.Hkv, a.B);
+  decode_mma_kernel<<<grid, kDecThreads, smem, stream>>>(*tmK, *tmV, a,
+                                                          a.scale * kLog2eF);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || a.NP == 1) return e;
+  decode_combine_kernel<<<a.B * a.H, 128, 0, stream>>>(a.ws, a.B, a.H, a.NP,
+                                                       a.out);
+  return cudaGetLastError();
+}
+
+}  // namespace pa

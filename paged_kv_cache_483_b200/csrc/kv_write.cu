@@ -1,0 +1,120 @@
+// K1 reshape_and_cache and K2 copy-on-write block copy.
+//
+// Both are byte copies bounded by HBM bandwidth: 16-byte vector loads and
+// stores, consecutive threads on consecutive 16-byte chunks of a row so every
+// warp moves 512 contiguous bytes, grid sized as a multiple of the SM count.
+//
+// K1 writes token t's K/V rows (all KV heads) into slot slot_mapping[t]
+// ("abhik.ai examples/pagedattention.py", KVPool.append: keys[physical,
+// offset] = key).  K2 copies a whole block, every slot and head, of both
+// caches ("abhik.ai examples/pagedattention.py", KVPool._private_tail).
+#include "common.cuh"
+#include "launch.hpp"
+
+namespace pa {
+
+template <typename V>
+__global__ void __launch_bounds__(256) reshape_and_cache_kernel(
+    const V* __restrict__ key, const V* __restrict__ value,
+    V* __restrict__ k_cache, V* __restrict__ v_cache,
+    const int64_t* __restrict__ slot_mapping, int32_t T, int64_t row_vecs,
+    int64_t num_slots, int32_t* err) {
+  const int64_t total = int64_t(T) * row_vecs;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t t = i / row_vecs, c = i - t * row_vecs;
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot < 0) continue;                    // padding token
+    if (slot >= num_slots) {
+      if (c == 0) raise_err(err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const V kv = key[i];
+    const V vv = value[i];
+    k_cache[slot * row_vecs + c] = kv;
+    v_cache[slot * row_vecs + c] = vv;
+  }
+}
+
+template <typename V>
+__global__ void __launch_bounds__(256) cow_copy_kernel(
+    V* __restrict__ k_cache, V* __restrict__ v_cache,
+    const int32_t* __restrict__ src, const int32_t* __restrict__ dst,
+    int32_t n, int64_t block_vecs, int32_t num_blocks, int32_t* err) {
+  const int64_t total = int64_t(n) * block_vecs;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t p = i / block_vecs, c = i - p * block_vecs;
+    const int32_t s = __ldg(src + p), d = __ldg(dst + p);
+    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) {
+      if (c == 0) raise_err(err, PA_DEVERR_BLOCK_ID);
+      continue;
+    }
+    const V kv = k_cache[int64_t(s) * block_vecs + c];
+    const V vv = v_cache[int64_t(s) * block_vecs + c];
+    k_cache[int64_t(d) * block_vecs + c] = kv;
+    v_cache[int64_t(d) * block_vecs + c] = vv;
+  }
+}
+
+static int grid_for(int64_t work, int sms) {
+  int64_t g = (work + 255) / 256;
+  int64_t cap = int64_t(sms) * 8;
+  if (g > cap) g = cap;
+  return int(g < 1 ? 1 : g);
+}
+
+cudaError_t launch_reshape_and_cache(const void* key, const void* value,
+                                     void* k_cache, void* v_cache,
+                                     const int64_t* slots, int32_t T,
+                                     int64_t row_bytes, int64_t num_slots,
+                                     int32_t* err, int sms,
+                                     cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  auto aligned = [](const void* p, int a) {
+    return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+  };
+  if (row_bytes % 16 == 0 && aligned(key, 16) && aligned(value, 16) &&
+      aligned(k_cache, 16) && aligned(v_cache, 16)) {
+    int64_t rv = row_bytes / 16;
+    reshape_and_cache_kernel<uint4><<<grid_for(T * rv, sms), 256, 0, stream>>>(
+        (const uint4*)key, (const uint4*)value, (uint4*)k_cache,
+        (uint4*)v_cache, slots, T, rv, num_slots, err);
+  } else if (row_bytes % 4 == 0) {
+    int64_t rv = row_bytes / 4;
+    reshape_and_cache_kernel<uint32_t><<<grid_for(T * rv, sms), 256, 0, stream>>>(
+        (const uint32_t*)key, (const uint32_t*)value, (uint32_t*)k_cache,
+        (uint32_t*)v_cache, slots, T, rv, num_slots, err);
+  } else {
+    int64_t rv = row_bytes / 2;
+    reshape_and_cache_kernel<uint16_t><<<grid_for(T * rv, sms), 256, 0, stream>>>(
+        (const uint16_t*)key, (const uint16_t*)value, (uint16_t*)k_cache,
+        (uint16_t*)v_cache, slots, T, rv, num_slots, err);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cow_copy(void* k_cache, void* v_cache, const int32_t* src,
+                            const int32_t* dst, int32_t n, int64_t block_bytes,
+                            int32_t num_blocks, int32_t* err, int sms,
+                            cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  if (block_bytes % 16 == 0) {
+    int64_t bv = block_bytes / 16;
+    cow_copy_kernel<uint4><<<grid_for(n * bv, sms), 256, 0, stream>>>(
+        (uint4*)k_cache, (uint4*)v_cache, src, dst, n, bv, num_blocks, err);
+  } else if (block_bytes % 4 == 0) {
+    int64_t bv = block_bytes / 4;
+    cow_copy_kernel<uint32_t><<<grid_for(n * bv, sms), 256, 0, stream>>>(
+        (uint32_t*)k_cache, (uint32_t*)v_cache, src, dst, n, bv, num_blocks,
+        err);
+  } else {
+    int64_t bv = block_bytes / 2;
+    cow_copy_kernel<uint16_t><<<grid_for(n * bv, sms), 256, 0, stream>>>(
+        (uint16_t*)k_cache, (uint16_t*)v_cache, src, dst, n, bv, num_blocks,
+        err);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace pa

@@ -1,0 +1,75 @@
+// Kernel launchers (host side), one per kernel family.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pa {
+
+cudaError_t launch_reshape_and_cache(const void* key, const void* value,
+                                     void* k_cache, void* v_cache,
+                                     const int64_t* slots, int32_t T,
+                                     int64_t row_bytes, int64_t num_slots,
+                                     int32_t* err, int sms,
+                                     cudaStream_t stream);
+
+cudaError_t launch_cow_copy(void* k_cache, void* v_cache, const int32_t* src,
+                            const int32_t* dst, int32_t n, int64_t block_bytes,
+                            int32_t num_blocks, int32_t* err, int sms,
+                            cudaStream_t stream);
+
+// Generic CUDA-core paged attention: any dtype, head_dim <= 512, any block
+// size and group size, q_tokens >= 1 (causal offset rule).
+struct GenericArgs {
+  const void* q;  // [B, q_tokens, H, d]
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* tables;
+  int32_t MB;
+  const int32_t* kv_lens;
+  int32_t B, q_tokens, H, Hkv, d, bs, NB;
+  float scale;
+  float* out;  // [B, q_tokens, H, d]
+  int32_t* err;
+  bool bf16;
+};
+cudaError_t launch_attention_generic(const GenericArgs& a, cudaStream_t s);
+
+// Tensor-core decode for bf16, head_dim 128, block_size 16, group <= 8.
+struct DecodeArgs {
+  const void* q;  // [B, H, 128] bf16
+  const int32_t* tables;
+  int32_t MB;
+  const int32_t* kv_lens;
+  int32_t B, H, Hkv, NB;
+  float scale;
+  int32_t part_blocks;  // blocks per partition
+  int32_t NP;           // partitions per sequence (1 = no split)
+  float* out;           // [B, H, 128]
+  float* ws;            // split scratch (NP > 1)
+  int32_t* err;
+};
+bool decode_fast_supported(int dtype_bf16, int d, int bs, int G);
+cudaError_t launch_decode_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
+                               const DecodeArgs& a, int sms,
+                               cudaStream_t stream);
+size_t split_workspace_bytes(int32_t B, int32_t H, int32_t NP, int32_t d);
+
+// Chunked prefill on tcgen05 tensor cores (bf16, head_dim 128, block 16).
+struct PrefillArgs {
+  const void* q;  // [B, q_tokens, H, 128] bf16
+  const int32_t* tables;
+  int32_t MB;
+  const int32_t* kv_lens;
+  int32_t B, q_tokens, H, Hkv, NB;
+  float scale;
+  float* out;  // [B, q_tokens, H, 128] fp32
+  int32_t* err;
+};
+bool prefill_fast_supported(int dtype_bf16, int d, int bs, int G);
+cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                const PrefillArgs& a, int sms,
+                                cudaStream_t stream);
+
+}  // namespace pa

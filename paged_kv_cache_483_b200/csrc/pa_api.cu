@@ -1,0 +1,534 @@
+// C ABI of the paged-attention library (declared in include/pa.h).
+//
+// Argument checking, the host block manager, append staging and kernel
+// dispatch.  No compute happens here: every step of the path runs in the
+// kernels of kv_write.cu, attention_generic.cu, decode_mma.cu and
+// prefill_tc.cu.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/pa.h"
+#include "block_manager.hpp"
+#include "launch.hpp"
+
+using pa::BlockManager;
+using pa::MgrStatus;
+
+namespace {
+
+constexpr int kRing = 4;  // append staging slots in flight
+
+struct Staging {
+  int64_t* host = nullptr;   // pinned: [slots (int64) | cow src,dst (int32)]
+  void* dev = nullptr;       // device mirror
+  size_t cap = 0;            // bytes
+  cudaEvent_t done = nullptr;
+  bool pending = false;
+};
+
+}  // namespace
+
+struct pa_pool {
+  BlockManager mgr;
+  int32_t num_blocks, block_size, num_kv_heads, head_dim;
+  pa_dtype dtype;
+  void* k_cache = nullptr;
+  void* v_cache = nullptr;
+  bool device = false;
+  int dev_id = 0;
+  int sms = 148;
+  int32_t* d_err = nullptr;
+  bool tmap_ok = false;
+  CUtensorMap tmK, tmV;
+  Staging ring[kRing];
+  int ring_next = 0;
+  std::vector<int64_t> slots_tmp;
+  std::vector<pa::CowPair> cow_tmp;
+
+  pa_pool(int32_t nb, int32_t bs, const std::vector<int32_t>& order)
+      : mgr(nb, bs, order) {}
+};
+
+namespace {
+
+pa_status from_mgr(MgrStatus s) {
+  switch (s) {
+    case MgrStatus::ok: return PA_OK;
+    case MgrStatus::unknown_seq: return PA_ERR_UNKNOWN_SEQ;
+    case MgrStatus::dup_seq: return PA_ERR_DUP_SEQ;
+    case MgrStatus::exhausted: return PA_ERR_POOL_EXHAUSTED;
+    default: return PA_ERR_INVALID_ARG;
+  }
+}
+
+size_t elem_bytes(pa_dtype t) { return t == PA_BF16 ? 2 : 4; }
+
+bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library needs no link-time dependency on libcuda.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault,
+                                &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// The pool viewed as a 3-D tensor {head_dim, num_kv_heads, num_blocks *
+// block_size}; one box = one block's 16 tokens x 64 columns of one KV head,
+// written to shared memory with the 128-byte swizzle.
+bool make_pool_map(CUtensorMap* map, void* base, const pa_pool* p) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {cuuint64_t(p->head_dim), cuuint64_t(p->num_kv_heads),
+                              cuuint64_t(p->num_blocks) * p->block_size};
+  const cuuint64_t strides[2] = {cuuint64_t(p->head_dim) * 2,
+                                 cuuint64_t(p->head_dim) * p->num_kv_heads * 2};
+  const cuuint32_t box[3] = {64, 1, cuuint32_t(p->block_size)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Blocks per partition for the tensor-core decode.  partition_tokens > 0 is
+// taken as given; 0 picks enough partitions for about two resident CTAs per
+// SM when the batch has fewer (sequence, KV head) groups than that.
+bool decode_partitions(const pa_pool* p, int32_t B, int32_t MB,
+                       int32_t partition_tokens, int32_t* part_blocks,
+                       int32_t* np) {
+  if (partition_tokens > 0) {
+    if (partition_tokens % p->block_size) return false;
+    *part_blocks = partition_tokens / p->block_size;
+  } else {
+    const int64_t groups = int64_t(B) * p->num_kv_heads;
+    const int64_t target = 2 * int64_t(p->sms);
+    int64_t want = 1;
+    if (groups > 0 && groups * 5 < target * 4) want = (target + groups - 1) / groups;
+    const int64_t max_np = std::max<int64_t>(1, (MB + 15) / 16);
+    want = std::min(want, max_np);
+    *part_blocks = int32_t((MB + want - 1) / want);
+  }
+  if (*part_blocks < 1) *part_blocks = 1;
+  *np = (MB + *part_blocks - 1) / *part_blocks;
+  if (*np < 1) *np = 1;
+  return true;
+}
+
+bool use_fast_decode(const pa_pool* p, int32_t H) {
+  return p->tmap_ok && H % p->num_kv_heads == 0 &&
+         pa::decode_fast_supported(p->dtype == PA_BF16, p->head_dim,
+                                   p->block_size, H / p->num_kv_heads);
+}
+
+bool use_fast_prefill(const pa_pool* p, int32_t H) {
+  return p->tmap_ok && H % p->num_kv_heads == 0 &&
+         pa::prefill_fast_supported(p->dtype == PA_BF16, p->head_dim,
+                                    p->block_size, H / p->num_kv_heads);
+}
+
+pa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
+                         int32_t num_kv_heads, int32_t head_dim,
+                         pa_dtype kv_dtype, void* k_cache, void* v_cache,
+                         const int32_t* alloc_order, pa_pool** out) {
+  if (!out) return PA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (kv_dtype != PA_F32 && kv_dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if ((k_cache == nullptr) != (v_cache == nullptr)) return PA_ERR_INVALID_ARG;
+  if (k_cache && (!aligned16(k_cache) || !aligned16(v_cache)))
+    return PA_ERR_INVALID_ARG;
+  if (int64_t(num_blocks) * block_size > (int64_t(1) << 31) - 1)
+    return PA_ERR_INVALID_ARG;
+  std::vector<int32_t> order;
+  if (alloc_order) {
+    if (!BlockManager::is_permutation(alloc_order, num_blocks))
+      return PA_ERR_INVALID_ARG;
+    order.assign(alloc_order, alloc_order + num_blocks);
+  }
+  pa_pool* p = new (std::nothrow) pa_pool(num_blocks, block_size, order);
+  if (!p) return PA_ERR_INVALID_ARG;
+  p->num_blocks = num_blocks;
+  p->block_size = block_size;
+  p->num_kv_heads = num_kv_heads;
+  p->head_dim = head_dim;
+  p->dtype = kv_dtype;
+  p->k_cache = k_cache;
+  p->v_cache = v_cache;
+  if (k_cache) {
+    p->device = true;
+    if (cudaGetDevice(&p->dev_id) != cudaSuccess ||
+        cudaDeviceGetAttribute(&p->sms, cudaDevAttrMultiProcessorCount,
+                               p->dev_id) != cudaSuccess ||
+        cudaMalloc(&p->d_err, sizeof(int32_t)) != cudaSuccess ||
+        cudaMemset(p->d_err, 0, sizeof(int32_t)) != cudaSuccess) {
+      if (p->d_err) cudaFree(p->d_err);
+      delete p;
+      return PA_ERR_CUDA;
+    }
+    if (kv_dtype == PA_BF16 && head_dim == 128 && block_size == 16)
+      p->tmap_ok = make_pool_map(&p->tmK, k_cache, p) &&
+                   make_pool_map(&p->tmV, v_cache, p);
+  }
+  *out = p;
+  return PA_OK;
+}
+
+pa_status pa_free(pa_pool* p) {
+  if (!p) return PA_OK;
+  if (p->device) {
+    cudaDeviceSynchronize();
+    for (auto& r : p->ring) {
+      if (r.host) cudaFreeHost(r.host);
+      if (r.dev) cudaFree(r.dev);
+      if (r.done) cudaEventDestroy(r.done);
+    }
+    if (p->d_err) cudaFree(p->d_err);
+  }
+  delete p;
+  return PA_OK;
+}
+
+pa_status pa_seq_create(pa_pool* p, int32_t seq) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  return from_mgr(p->mgr.create(seq));
+}
+
+pa_status pa_seq_fork(pa_pool* p, int32_t parent, int32_t child,
+                      int32_t prefix_tokens) {
+  if (!p || prefix_tokens < -1) return PA_ERR_INVALID_ARG;
+  return from_mgr(p->mgr.share_prefix(parent, child, prefix_tokens));
+}
+
+pa_status pa_seq_release(pa_pool* p, int32_t seq) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  return from_mgr(p->mgr.release(seq));
+}
+
+pa_status pa_seq_table(const pa_pool* p, int32_t seq, int32_t* blocks_out,
+                       int32_t cap, int32_t* n_blocks, int32_t* length) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  const std::vector<int32_t>* t = p->mgr.table(seq);
+  if (!t) return PA_ERR_UNKNOWN_SEQ;
+  if (n_blocks) *n_blocks = int32_t(t->size());
+  if (length) *length = int32_t(p->mgr.length(seq));
+  if (blocks_out) {
+    if (cap < int32_t(t->size())) return PA_ERR_INVALID_ARG;
+    std::copy(t->begin(), t->end(), blocks_out);
+  }
+  return PA_OK;
+}
+
+pa_status pa_block_tables(const pa_pool* p, const int32_t* seqs, int32_t n,
+                          int32_t width, int32_t* tables_out,
+                          int32_t* kv_lens_out) {
+  if (!p || n < 0 || width <= 0 || (n > 0 && !seqs)) return PA_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n; ++i) {
+    const std::vector<int32_t>* t = p->mgr.table(seqs[i]);
+    if (!t) return PA_ERR_UNKNOWN_SEQ;
+    if (int32_t(t->size()) > width) return PA_ERR_INVALID_ARG;
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    const std::vector<int32_t>* t = p->mgr.table(seqs[i]);
+    if (tables_out) {
+      int32_t* row = tables_out + int64_t(i) * width;
+      std::fill(row, row + width, 0);
+      std::copy(t->begin(), t->end(), row);
+    }
+    if (kv_lens_out) kv_lens_out[i] = int32_t(p->mgr.length(seqs[i]));
+  }
+  return PA_OK;
+}
+
+pa_status pa_plan_append(pa_pool* p, const int32_t* seqs, const int32_t* n_new,
+                         int32_t n_seqs, int64_t* slot_mapping_out,
+                         int32_t* cow_src_out, int32_t* cow_dst_out,
+                         int32_t cow_cap, int32_t* n_cow_out) {
+  if (!p || n_seqs < 0 || (n_seqs > 0 && (!seqs || !n_new)))
+    return PA_ERR_INVALID_ARG;
+  if ((cow_src_out || cow_dst_out) && cow_cap < n_seqs) return PA_ERR_INVALID_ARG;
+  p->slots_tmp.clear();
+  p->cow_tmp.clear();
+  pa_status st = from_mgr(p->mgr.append(seqs, n_new, n_seqs, &p->slots_tmp, &p->cow_tmp));
+  if (st != PA_OK) return st;
+  if (slot_mapping_out)
+    std::copy(p->slots_tmp.begin(), p->slots_tmp.end(), slot_mapping_out);
+  for (size_t i = 0; i < p->cow_tmp.size(); ++i) {
+    if (cow_src_out) cow_src_out[i] = p->cow_tmp[i].src;
+    if (cow_dst_out) cow_dst_out[i] = p->cow_tmp[i].dst;
+  }
+  if (n_cow_out) *n_cow_out = int32_t(p->cow_tmp.size());
+  return PA_OK;
+}
+
+pa_status pa_pool_stats(const pa_pool* p, pa_stats* out) {
+  if (!p || !out) return PA_ERR_INVALID_ARG;
+  pa::Snapshot s = p->mgr.snapshot();
+  out->allocated_blocks = s.allocated;
+  out->free_blocks = s.free;
+  out->physical_capacity_tokens = s.capacity;
+  out->physical_payload_tokens = s.payload;
+  out->logical_tokens = s.logical;
+  out->internal_waste_tokens = s.waste;
+  out->sharing_savings_tokens = s.savings;
+  out->live_sequences = s.live;
+  return PA_OK;
+}
+
+pa_status pa_refcounts(const pa_pool* p, int32_t* out) {
+  if (!p || !out) return PA_ERR_INVALID_ARG;
+  const auto& r = p->mgr.refcounts();
+  std::copy(r.begin(), r.end(), out);
+  return PA_OK;
+}
+
+pa_status pa_validate(const pa_pool* p) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  return p->mgr.validate() ? PA_OK : PA_ERR_INTERNAL;
+}
+
+pa_status pa_append_kv(pa_pool* p, const int32_t* seqs, const int32_t* n_new,
+                       int32_t n_seqs, const void* key, const void* value,
+                       int64_t* slot_mapping_out, void* stream) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  if (!p->device) return PA_ERR_NO_DEVICE;
+  if (n_seqs < 0 || (n_seqs > 0 && (!seqs || !n_new))) return PA_ERR_INVALID_ARG;
+  int64_t T = 0;
+  for (int32_t i = 0; i < n_seqs; ++i) T += std::max<int32_t>(0, n_new[i]);
+  if (T > 0 && (!key || !value)) return PA_ERR_INVALID_ARG;
+  if (T > INT32_MAX) return PA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // staging slot: wait until the kernels of its previous use are done
+  Staging& r = p->ring[p->ring_next];
+  if (r.pending && cudaEventSynchronize(r.done) != cudaSuccess) return PA_ERR_CUDA;
+  r.pending = false;
+  const size_t need = size_t(T) * sizeof(int64_t) + size_t(n_seqs) * 2 * sizeof(int32_t);
+  if (need > r.cap) {
+    size_t cap = std::max<size_t>(need, 4096);
+    cap = std::max(cap, r.cap * 2);
+    if (r.host) cudaFreeHost(r.host);
+    if (r.dev) cudaFree(r.dev);
+    r.host = nullptr;
+    r.dev = nullptr;
+    r.cap = 0;
+    if (cudaMallocHost(reinterpret_cast<void**>(&r.host), cap) != cudaSuccess)
+      return PA_ERR_CUDA;
+    if (cudaMalloc(&r.dev, cap) != cudaSuccess) return PA_ERR_CUDA;
+    r.cap = cap;
+    if (!r.done && cudaEventCreateWithFlags(&r.done, cudaEventDisableTiming) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+
+  // host plan (step a1): all-or-nothing
+  p->slots_tmp.clear();
+  p->cow_tmp.clear();
+  pa_status st = from_mgr(p->mgr.append(seqs, n_new, n_seqs, &p->slots_tmp, &p->cow_tmp));
+  if (st != PA_OK) return st;
+  if (slot_mapping_out)
+    std::copy(p->slots_tmp.begin(), p->slots_tmp.end(), slot_mapping_out);
+  const int32_t n_cow = int32_t(p->cow_tmp.size());
+  int64_t* hs = r.host;
+  std::copy(p->slots_tmp.begin(), p->slots_tmp.end(), hs);
+  int32_t* hc = reinterpret_cast<int32_t*>(hs + T);
+  for (int32_t i = 0; i < n_cow; ++i) {
+    hc[i] = p->cow_tmp[i].src;
+    hc[n_cow + i] = p->cow_tmp[i].dst;
+  }
+  const size_t bytes = size_t(T) * sizeof(int64_t) + size_t(n_cow) * 2 * sizeof(int32_t);
+  if (bytes && cudaMemcpyAsync(r.dev, r.host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  const int64_t* d_slots = static_cast<const int64_t*>(r.dev);
+  const int32_t* d_cow = reinterpret_cast<const int32_t*>(d_slots + T);
+  const size_t eb = elem_bytes(p->dtype);
+  cudaError_t e = pa::launch_cow_copy(
+      p->k_cache, p->v_cache, d_cow, d_cow + n_cow, n_cow,
+      int64_t(p->block_size) * p->num_kv_heads * p->head_dim * eb, p->num_blocks,
+      p->d_err, p->sms, s);
+  if (e == cudaSuccess)
+    e = pa::launch_reshape_and_cache(
+        key, value, p->k_cache, p->v_cache, d_slots, int32_t(T),
+        int64_t(p->num_kv_heads) * p->head_dim * eb,
+        int64_t(p->num_blocks) * p->block_size, p->d_err, p->sms, s);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaEventRecord(r.done, s) != cudaSuccess) return PA_ERR_CUDA;
+  r.pending = true;
+  p->ring_next = (p->ring_next + 1) % kRing;
+  return PA_OK;
+}
+
+pa_status pa_reshape_and_cache(pa_pool* p, const void* key, const void* value,
+                               const int64_t* d_slot_mapping, int32_t T,
+                               void* stream) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  if (!p->device) return PA_ERR_NO_DEVICE;
+  if (T < 0 || (T > 0 && (!key || !value || !d_slot_mapping))) return PA_ERR_INVALID_ARG;
+  const size_t eb = elem_bytes(p->dtype);
+  return cuda_status(pa::launch_reshape_and_cache(
+      key, value, p->k_cache, p->v_cache, d_slot_mapping, T,
+      int64_t(p->num_kv_heads) * p->head_dim * eb,
+      int64_t(p->num_blocks) * p->block_size, p->d_err, p->sms,
+      static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_cow_copy(pa_pool* p, const int32_t* d_src, const int32_t* d_dst,
+                      int32_t n, void* stream) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  if (!p->device) return PA_ERR_NO_DEVICE;
+  if (n < 0 || (n > 0 && (!d_src || !d_dst))) return PA_ERR_INVALID_ARG;
+  const size_t eb = elem_bytes(p->dtype);
+  return cuda_status(pa::launch_cow_copy(
+      p->k_cache, p->v_cache, d_src, d_dst, n,
+      int64_t(p->block_size) * p->num_kv_heads * p->head_dim * eb, p->num_blocks,
+      p->d_err, p->sms, static_cast<cudaStream_t>(stream)));
+}
+
+size_t pa_decode_workspace_bytes(const pa_pool* p, int32_t B, int32_t H,
+                                 int32_t max_blocks, int32_t partition_tokens) {
+  if (!p || B <= 0 || H <= 0 || max_blocks <= 0) return 0;
+  if (!use_fast_decode(p, H)) return 0;
+  int32_t pb = 0, np = 1;
+  if (!decode_partitions(p, B, max_blocks, partition_tokens, &pb, &np)) return 0;
+  return pa::split_workspace_bytes(B, H, np, p->head_dim);
+}
+
+int32_t pa_decode_path(const pa_pool* p, int32_t H) {
+  return (p && use_fast_decode(p, H)) ? 1 : 0;
+}
+
+int32_t pa_prefill_path(const pa_pool* p, int32_t H) {
+  return (p && use_fast_prefill(p, H)) ? 1 : 0;
+}
+
+static pa_status check_attention_args(const pa_pool* p, const void* q, int32_t B,
+                                      int32_t H, const int32_t* tables,
+                                      int32_t MB, const int32_t* kv_lens,
+                                      const float* out) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  if (!p->device) return PA_ERR_NO_DEVICE;
+  if (B < 0 || H <= 0 || MB <= 0 || H % p->num_kv_heads) return PA_ERR_INVALID_ARG;
+  if (B > 0 && (!q || !tables || !kv_lens || !out)) return PA_ERR_INVALID_ARG;
+  if (int64_t(MB) * p->block_size > INT32_MAX) return PA_ERR_INVALID_ARG;
+  if (p->head_dim > 512) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+pa_status pa_decode(pa_pool* p, const void* q, int32_t B, int32_t H,
+                    const int32_t* d_block_tables, int32_t max_blocks,
+                    const int32_t* d_kv_lens, float scale,
+                    int32_t partition_tokens, void* workspace,
+                    size_t workspace_bytes, float* out, void* stream) {
+  pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks,
+                                      d_kv_lens, out);
+  if (st != PA_OK) return st;
+  if (partition_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (B == 0) return PA_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_fast_decode(p, H)) {
+    if (!aligned16(q)) return PA_ERR_INVALID_ARG;
+    pa::DecodeArgs a{};
+    if (!decode_partitions(p, B, max_blocks, partition_tokens, &a.part_blocks, &a.NP))
+      return PA_ERR_INVALID_ARG;
+    const size_t need = pa::split_workspace_bytes(B, H, a.NP, p->head_dim);
+    if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+      return PA_ERR_INVALID_ARG;
+    a.q = q;
+    a.tables = d_block_tables;
+    a.MB = max_blocks;
+    a.kv_lens = d_kv_lens;
+    a.B = B;
+    a.H = H;
+    a.Hkv = p->num_kv_heads;
+    a.NB = p->num_blocks;
+    a.scale = scale;
+    a.out = out;
+    a.ws = static_cast<float*>(workspace);
+    a.err = p->d_err;
+    return cuda_status(pa::launch_decode_fast(&p->tmK, &p->tmV, a, p->sms, s));
+  }
+  if (partition_tokens % p->block_size) return PA_ERR_INVALID_ARG;
+  pa::GenericArgs g{q, p->k_cache, p->v_cache, d_block_tables, max_blocks,
+                    d_kv_lens, B, 1, H, p->num_kv_heads, p->head_dim,
+                    p->block_size, p->num_blocks, scale, out, p->d_err,
+                    p->dtype == PA_BF16};
+  return cuda_status(pa::launch_attention_generic(g, s));
+}
+
+pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,
+                           int32_t q_tokens, int32_t H,
+                           const int32_t* d_block_tables, int32_t max_blocks,
+                           const int32_t* d_kv_lens, float scale, float* out,
+                           void* stream) {
+  pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks,
+                                      d_kv_lens, out);
+  if (st != PA_OK) return st;
+  if (q_tokens <= 0 || q_tokens > 65535) return PA_ERR_INVALID_ARG;
+  if (B == 0) return PA_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_fast_prefill(p, H)) {
+    if (!aligned16(q)) return PA_ERR_INVALID_ARG;
+    pa::PrefillArgs a{q, d_block_tables, max_blocks, d_kv_lens, B, q_tokens, H,
+                      p->num_kv_heads, p->num_blocks, scale, out, p->d_err};
+    return cuda_status(pa::launch_prefill_fast(&p->tmK, &p->tmV, a, p->sms, s));
+  }
+  pa::GenericArgs g{q, p->k_cache, p->v_cache, d_block_tables, max_blocks,
+                    d_kv_lens, B, q_tokens, H, p->num_kv_heads, p->head_dim,
+                    p->block_size, p->num_blocks, scale, out, p->d_err,
+                    p->dtype == PA_BF16};
+  return cuda_status(pa::launch_attention_generic(g, s));
+}
+
+pa_status pa_get_error(pa_pool* p, int32_t* device_code) {
+  if (!p || !device_code) return PA_ERR_INVALID_ARG;
+  *device_code = 0;
+  if (!p->device) return PA_ERR_NO_DEVICE;
+  if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemcpy(device_code, p->d_err, sizeof(int32_t), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaMemset(p->d_err, 0, sizeof(int32_t)) != cudaSuccess) return PA_ERR_CUDA;
+  return *device_code ? PA_ERR_DEVICE : PA_OK;
+}
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNKNOWN_SEQ: return "unknown or released sequence";
+    case PA_ERR_DUP_SEQ: return "duplicate sequence id";
+    case PA_ERR_POOL_EXHAUSTED: return "physical KV pool exhausted";
+    case PA_ERR_CUDA: return "CUDA runtime error";
+    case PA_ERR_DEVICE: return "device error bits set";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PA_ERR_NO_DEVICE: return "host-only pool";
+    case PA_ERR_INTERNAL: return "broken invariant";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

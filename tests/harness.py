@@ -1,0 +1,123 @@
+"""Replays a workload script on the GPU library and on the oracle.
+
+Both sides receive the same seeded arrays from ``workloads``; neither sees the
+other's results.  The oracle side stores data for a chosen subset of KV heads
+(float32 holding bf16-exact values) so full-size configurations fit in host
+memory; its attention then runs on the matching query heads.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import paged_kv_cache_483_b200 as pa
+import workloads
+from oracle import KVPool, paged_attention
+
+
+def torch_dtype(w):
+    return torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+
+class GpuRun:
+    def __init__(self, w, device="cuda", init="zeros"):
+        self.w = w
+        dt = torch_dtype(w)
+        shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
+        alloc = torch.zeros if init == "zeros" else torch.empty
+        self.k_cache = alloc(shape, dtype=dt, device=device)
+        self.v_cache = alloc(shape, dtype=dt, device=device)
+        self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.dtype,
+                            self.k_cache, self.v_cache, alloc_order=w.order)
+        self.slots = {}
+        self.device = device
+
+    def apply(self, ops):
+        for op in ops:
+            if op.kind == "create":
+                self.pool.create(op.args[0])
+            elif op.kind == "share":
+                self.pool.fork(*op.args)
+            elif op.kind == "release":
+                self.pool.release(op.args[0])
+            elif op.kind == "append":
+                k, v = self.w.kv_for(op)
+                self.slots[op.index] = self.pool.append_kv(
+                    [op.args[0]], [op.args[1]], k.to(self.device), v.to(self.device),
+                    return_slots=True)
+            else:
+                raise ValueError(op.kind)
+        return self
+
+    def tables(self, seqs=None):
+        seqs = self.w.decode_seqs if seqs is None else seqs
+        width = max(len(self.pool.table(s)[0]) for s in seqs)
+        t, lens = self.pool.block_tables(seqs, max(width, 1))
+        return (torch.from_numpy(t).to(self.device), torch.from_numpy(lens).to(self.device),
+                t, lens)
+
+    def decode(self, q=None, partition_tokens=0):
+        q = self.w.queries() if q is None else q
+        tables, lens, _, _ = self.tables()
+        out = self.pool.decode(q[:, 0].contiguous().to(self.device), tables, lens,
+                               partition_tokens=partition_tokens)
+        torch.cuda.synchronize()
+        return out.cpu().numpy()
+
+    def prefill(self, q=None):
+        q = self.w.queries() if q is None else q
+        tables, lens, _, _ = self.tables()
+        out = self.pool.prefill_chunk(q.contiguous().to(self.device), tables, lens)
+        torch.cuda.synchronize()
+        return out.cpu().numpy()
+
+
+class OracleRun:
+    def __init__(self, w, heads="all"):
+        self.w = w
+        self.heads = list(range(w.num_kv_heads)) if heads == "all" else list(heads)
+        self.pool = KVPool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim,
+                           w.order, store_heads=self.heads,
+                           dtype=np.float64 if w.dtype == "f32" else np.float32)
+        self.slots, self.cows = {}, {}
+
+    def apply(self, ops):
+        for op in ops:
+            if op.kind == "create":
+                self.pool.create(op.args[0])
+            elif op.kind == "share":
+                self.pool.share_prefix(*op.args)
+            elif op.kind == "release":
+                self.pool.release(op.args[0])
+            elif op.kind == "append":
+                k, v = self.w.kv_for(op)
+                dt = self.pool.keys.dtype
+                s, c = self.pool.append(op.args[0], op.args[1], k.to(torch.float64).numpy().astype(dt),
+                                        v.to(torch.float64).numpy().astype(dt))
+                self.slots[op.index], self.cows[op.index] = s, c
+        return self
+
+    def attention(self, seq_index, q, heads=None):
+        """Output of query rows q [q_tokens, H, d] (float64) for the decode
+        sequence at position seq_index, restricted to query heads whose KV head
+        is stored.  Returns {h: out[q_tokens, d]}."""
+        w = self.w
+        G = w.num_heads // w.num_kv_heads
+        seq = w.decode_seqs[seq_index]
+        k, v = self.pool.gather(seq)
+        res = {}
+        for i, kvh in enumerate(self.heads):
+            hs = list(range(kvh * G, (kvh + 1) * G)) if heads is None else \
+                [h for h in heads if h // G == kvh]
+            if not hs:
+                continue
+            from oracle import attention_two_pass
+            out = attention_two_pass(q[:, hs], k[:, i:i + 1].astype(np.float64),
+                                     v[:, i:i + 1].astype(np.float64))
+            for j, h in enumerate(hs):
+                res[h] = out[:, j]
+        return res
+
+
+def q64(w):
+    return w.queries().to(torch.float64).numpy()

@@ -1,0 +1,249 @@
+"""Parity of the CUDA path with the float64 oracle (needs a B200).
+
+Bars (written in each test): bit-exact for slot mappings, copy-on-write pairs,
+tables, refcounts and KV bytes; attention max-abs error <= 1e-4 for fp32 K/V,
+<= 2e-3 for bf16 decode, <= 5e-3 for bf16 prefill, all against the oracle run
+on the same (bf16-rounded) inputs.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_483_b200 as pa
+import workloads
+from harness import GpuRun, OracleRun, q64
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32, TOL_DECODE, TOL_PREFILL = 1e-4, 2e-3, 5e-3
+
+
+def _max_err(gpu_out, oracle_rows, qt=None):
+    err = 0.0
+    for h, ref in oracle_rows.items():
+        got = gpu_out[:, h] if qt is None else gpu_out[qt, h]
+        err = max(err, float(np.abs(got - (ref[0] if qt is None else ref[0])).max()))
+    return err
+
+
+def _check_decode(g, o, w, tol, partition_tokens=0):
+    out = g.decode(partition_tokens=partition_tokens)
+    q = q64(w)
+    worst = 0.0
+    for i in range(len(w.decode_seqs)):
+        rows = o.attention(i, q[i])
+        for h, ref in rows.items():
+            worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+    assert worst <= tol, worst
+    return out
+
+
+def test_tiny_trace_fp32():
+    w = workloads.tiny()
+    g = GpuRun(w).apply(w.setup)
+    o = OracleRun(w).apply(w.setup)
+    assert g.slots == o.slots                                 # bit-exact plan
+    assert g.pool.refcounts() == o.pool.refs
+    assert len(o.cows[3]) == 1                               # B's shared tail copied
+    torch.cuda.synchronize()
+    # whole pool, bit-exact (both sides start from zeros; no block is reused)
+    assert np.array_equal(g.k_cache.cpu().numpy().astype(np.float64), o.pool.keys)
+    assert np.array_equal(g.v_cache.cpu().numpy().astype(np.float64), o.pool.values)
+    _check_decode(g, o, w, TOL_F32)
+    assert g.pool.get_error() == 0
+
+
+def _small(lens, H, Hkv, d=128, bs=16, dtype="bf16", seed=1, split_last=0):
+    return workloads.custom_decode("small", lens, H, Hkv, d, bs, dtype, seed,
+                                   spare_blocks=4, split_last=split_last)
+
+
+LENS = [1, 15, 16, 17, 33, 100, 255, 256, 513, 1000, 0, 2]
+
+
+@pytest.mark.parametrize("H,Hkv", [(32, 8), (64, 8), (8, 8), (16, 8), (4, 1), (8, 1)])
+@pytest.mark.parametrize("part", [0, 16, 64, 256])
+def test_decode_fast_parity(H, Hkv, part):
+    w = _small(LENS, H, Hkv, seed=H * 7 + Hkv + part)
+    g = GpuRun(w).apply(w.setup)
+    assert g.pool.decode_path(H) == 1
+    o = OracleRun(w).apply(w.setup)
+    _check_decode(g, o, w, TOL_DECODE, part)
+    assert g.pool.get_error() == 0
+
+
+def test_decode_uninitialised_pool_is_safe():
+    # stale slots past a sequence end must not leak into the result
+    w = _small([3, 17, 31], 32, 8, seed=5)
+    g = GpuRun(w, init="empty")
+    g.k_cache.fill_(float("nan"))
+    g.v_cache.fill_(float("inf"))
+    g.apply(w.setup)
+    o = OracleRun(w).apply(w.setup)
+    _check_decode(g, o, w, TOL_DECODE)
+
+
+def test_decode_is_invariant_under_block_permutation():
+    w = _small([700, 1234, 40, 511], 32, 8, seed=11)
+    outs = []
+    for k in range(3):
+        wk = dataclasses.replace(w, order=workloads.permutation(w.num_blocks, 100 + k))
+        outs.append(GpuRun(wk).apply(wk.setup).decode())
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+
+
+def test_generic_path_bf16_head_dim_64():
+    w = _small([5, 70, 129], 8, 2, d=64, seed=3)
+    g = GpuRun(w).apply(w.setup)
+    assert g.pool.decode_path(8) == 0
+    _check_decode(g, OracleRun(w).apply(w.setup), w, TOL_DECODE)
+
+
+def test_generic_path_fp32_gqa():
+    w = _small([9, 40, 64], 8, 2, d=32, bs=8, dtype="f32", seed=4)
+    g = GpuRun(w).apply(w.setup)
+    _check_decode(g, OracleRun(w).apply(w.setup), w, TOL_F32)
+
+
+def test_append_with_sharing_is_bit_exact():
+    # groups sharing prefixes, private tails, a copy-on-write in the step
+    w = workloads.ragged256(groups=3, per_group=4, prefix=40, spare_blocks=8)
+    g = GpuRun(w).apply(w.setup + w.step)
+    o = OracleRun(w).apply(w.setup + w.step)
+    assert g.slots == o.slots
+    assert any(o.cows.values())
+    assert g.pool.refcounts() == o.pool.refs
+    kc = g.k_cache.cpu().float().numpy()
+    vc = g.v_cache.cpu().float().numpy()
+    for s in o.pool.tables:
+        for t in range(o.pool.lengths[s]):
+            blk, off = o.pool.address(s, t)
+            assert np.array_equal(kc[blk, off], o.pool.keys[blk, off])
+            assert np.array_equal(vc[blk, off], o.pool.values[blk, off])
+    _check_decode(g, o, w, TOL_DECODE)
+
+
+def test_reshape_and_cache_and_cow_entry_points():
+    w = workloads.custom_decode("rc", [40], 8, 8, 128, 16, "bf16", 9, spare_blocks=4)
+    g = GpuRun(w)
+    T = 20
+    key = torch.randn(T, 8, 128, device="cuda").to(torch.bfloat16)
+    val = torch.randn(T, 8, 128, device="cuda").to(torch.bfloat16)
+    slots = torch.tensor([5 * 16 + i for i in range(T - 1)] + [-1], device="cuda")
+    g.pool.reshape_and_cache(key, val, slots)
+    src = torch.tensor([5], dtype=torch.int32, device="cuda")
+    dst = torch.tensor([2], dtype=torch.int32, device="cuda")
+    g.pool.cow_copy(src, dst)
+    torch.cuda.synchronize()
+    flat_k = g.k_cache.view(-1, 8, 128)
+    assert torch.equal(flat_k[80:80 + T - 1], key[:T - 1])
+    assert torch.equal(g.k_cache[2], g.k_cache[5]) and torch.equal(g.v_cache[2], g.v_cache[5])
+    assert torch.equal(g.v_cache.view(-1, 8, 128)[80:80 + T - 1], val[:T - 1])
+    assert g.pool.get_error() == 0
+
+
+def test_device_bounds_errors_zero_rows():
+    w = _small([40, 40], 32, 8, seed=21)
+    g = GpuRun(w).apply(w.setup)
+    tables, lens, _, _ = g.tables()
+    q = w.queries()[:, 0].contiguous().cuda()
+    bad = tables.clone()
+    bad[1, 1] = w.num_blocks + 5
+    out = g.pool.decode(q, bad, lens)
+    assert g.pool.get_error() & pa.PA_DEVERR_BLOCK_ID
+    assert torch.all(out[1] == 0) and torch.any(out[0] != 0)
+    long = lens.clone()
+    long[0] = tables.shape[1] * 16 + 1
+    out = g.pool.decode(q, tables, long)
+    assert g.pool.get_error() & pa.PA_DEVERR_KV_LEN
+    assert torch.all(out[0] == 0)
+    key = torch.zeros(1, 8, 128, device="cuda", dtype=torch.bfloat16)
+    g.pool.reshape_and_cache(key, key, torch.tensor([w.num_blocks * 16], device="cuda"))
+    assert g.pool.get_error() & pa.PA_DEVERR_SLOT
+    assert g.pool.get_error() == 0                       # cleared by the read
+
+
+def _prefill_case(batch, cached, chunk, H, Hkv, seed):
+    return workloads.prefill(seed=seed, batch=batch, cached=cached, chunk=chunk)
+
+
+@pytest.mark.parametrize("batch,cached,chunk", [(2, 0, 37), (2, 40, 37), (1, 200, 130), (3, 5, 1)])
+def test_prefill_parity_small(batch, cached, chunk):
+    w = workloads.prefill(seed=batch * 100 + cached + chunk, batch=batch, cached=cached, chunk=chunk)
+    w = dataclasses.replace(w, setup=[op for op in w.setup if not (op.kind == "append" and op.args[1] == 0)])
+    g = GpuRun(w).apply(w.setup + w.step)
+    o = OracleRun(w).apply(w.setup + w.step)
+    out = g.prefill()
+    q = q64(w)
+    worst = 0.0
+    for i in range(batch):
+        rows = o.attention(i, q[i])
+        for h, ref in rows.items():
+            worst = max(worst, float(np.abs(out[i, :, h] - ref).max()))
+    assert worst <= TOL_PREFILL, worst
+    assert g.pool.get_error() == 0
+
+
+# ---------------------------------------------------------------- full sizes
+def _full(w, kv_heads, sample_seqs, decode=True, partition_tokens=0, check_slots=True):
+    g = GpuRun(w).apply(w.setup + w.step)
+    o = OracleRun(w, heads=kv_heads).apply(w.setup + w.step)
+    if check_slots:
+        assert g.slots == o.slots
+    assert g.pool.refcounts() == o.pool.refs
+    _, _, t_gpu, lens = g.tables()
+    assert np.array_equal(t_gpu, o.pool.block_table(w.decode_seqs, t_gpu.shape[1]))
+    q = q64(w)
+    out = g.decode(partition_tokens=partition_tokens) if decode else g.prefill()
+    return g, o, out, q
+
+
+def test_full_decode32_sampled():
+    w = workloads.decode32()
+    g, o, out, q = _full(w, [0, 5], None)
+    worst = 0.0
+    for i in (0, 13, 31):
+        for h, ref in o.attention(i, q[i]).items():
+            worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+    assert worst <= TOL_DECODE, worst
+    assert g.pool.get_error() == 0
+
+
+def test_full_ragged256_sampled():
+    w = workloads.ragged256()
+    g, o, out, q = _full(w, [3], None)
+    assert any(o.cows.values())
+    lens = [o.pool.lengths[s] for s in w.decode_seqs]
+    pick = sorted(set([int(np.argmin(lens)), int(np.argmax(lens))] + list(range(0, 256, 37))))
+    worst = 0.0
+    for i in pick:
+        for h, ref in o.attention(i, q[i]).items():
+            worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+    assert worst <= TOL_DECODE, worst
+    assert g.pool.get_error() == 0
+
+
+def test_full_splitk128k_sampled():
+    w = workloads.splitk128k()
+    g, o, out, q = _full(w, [2], None, partition_tokens=w.partition_tokens)
+    worst = 0.0
+    for i in (0, 3):
+        for h, ref in o.attention(i, q[i]).items():
+            worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+    assert worst <= TOL_DECODE, worst
+    assert g.pool.get_error() == 0
+
+
+def test_full_prefill_sampled():
+    w = workloads.prefill()
+    g, o, out, q = _full(w, [1], None, decode=False)
+    worst = 0.0
+    rows = [0, 1, 127, 128, 255, 511]
+    for i in (0, 7):
+        ref = o.attention(i, q[i])
+        for h, r in ref.items():
+            worst = max(worst, float(np.abs(out[i, rows, h] - r[rows]).max()))
+    assert worst <= TOL_PREFILL, worst
+    assert g.pool.get_error() == 0
