@@ -1,0 +1,557 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-attention hot path on B200.
+
+Default workload (the headline metric): decode batch 32 at 8K context, GQA
+32/8, head_dim 128, block 16, bf16 K/V/Q, a 16384-block pool in a seeded
+permuted order.  One step = append of every sequence's new token (K/V written
+by reshape_and_cache at the slots the host manager planned for position 8191)
+followed by paged decode attention at kv_len 8192.  The host plan itself is
+timed separately (``host_plan_us``) because a repeated step must rewrite the
+same slots.
+
+Metric: effective KV bytes read by decode per second (sum_b kv_len_b * Hkv *
+head_dim * 2 (K and V) * 2 bytes), whole job over all ranks; ``seqs_per_s``
+is the same time expressed as sequences decoded per second.
+
+Other workloads (``--config``): ragged256 (copy-on-write + append + decode),
+splitk128k (split-K decode + log-sum-exp combine), prefill (512-token chunk
+append + causal chunked prefill; metric TFLOP/s of causal pairs).
+
+Multi-GPU: one process per GPU (torchrun); every rank decodes its own replica
+batch (different seeds), no collective on the data path ("scaling": "weak");
+the time is the max over ranks.  ``--impl reference`` times the float64 CPU
+oracle on this host's cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+MIB = 1 << 20
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+# ------------------------------------------------------------------ helpers --
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "paged_kv_cache_483_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_file, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    if d.get("source_hash") != source_hash(kernel_file):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, cuda_index, period=0.02):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:
+                uuid = str(torch.cuda.get_device_properties(cuda_index).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------- distributed --
+class Dist:
+    def __init__(self, want):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.want = want
+        self.pg = None
+
+    def init(self, backend):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x, device=None):
+        if not self.pg:
+            return x
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# --------------------------------------------------------- our CUDA path ----
+class Setup:
+    """A workload brought up on the GPU through the C ABI (untimed)."""
+
+    def __init__(self, w, device):
+        import torch
+        import paged_kv_cache_483_b200 as pa
+        self.w, self.device = w, device
+        dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
+        self.k_cache = torch.empty(shape, dtype=dt, device=device)
+        self.v_cache = torch.empty(shape, dtype=dt, device=device)
+        self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.dtype,
+                            self.k_cache, self.v_cache, alloc_order=w.order)
+        for op in w.setup:
+            if op.kind == "create":
+                self.pool.create(op.args[0])
+            elif op.kind == "share":
+                self.pool.fork(*op.args)
+            elif op.kind == "release":
+                self.pool.release(op.args[0])
+            else:
+                k, v = w.kv_for(op)
+                self.pool.append_kv([op.args[0]], [op.args[1]], k.to(device), v.to(device))
+        torch.cuda.synchronize()
+        # the step's appends: planned once by the host manager (timed alone)
+        self.step_k = self.step_v = None
+        self.slots = None
+        self.cow_src = self.cow_dst = None
+        self.host_plan_us = None
+        if w.step:
+            seqs = [op.args[0] for op in w.step]
+            n_new = [op.args[1] for op in w.step]
+            t0 = time.perf_counter()
+            slots, cow = self.pool.plan_append(seqs, n_new)
+            self.host_plan_us = (time.perf_counter() - t0) * 1e6
+            ks, vs = zip(*[w.kv_for(op) for op in w.step])
+            self.step_k = torch.cat(ks).to(device)
+            self.step_v = torch.cat(vs).to(device)
+            self.slots = torch.tensor(slots, dtype=torch.int64, device=device)
+            if cow:
+                self.cow_src = torch.tensor([c[0] for c in cow], dtype=torch.int32, device=device)
+                self.cow_dst = torch.tensor([c[1] for c in cow], dtype=torch.int32, device=device)
+        t, lens = self.pool.block_tables(w.decode_seqs, max(len(self.pool.table(s)[0])
+                                                            for s in w.decode_seqs))
+        self.tables_h, self.lens_h = t, lens
+        self.tables = torch.from_numpy(t).to(device)
+        self.lens = torch.from_numpy(lens).to(device)
+        q = w.queries()
+        self.q = (q[:, 0] if w.q_tokens == 1 else q).contiguous().to(device)
+        self.out = torch.empty(self.q.shape, dtype=torch.float32, device=device)
+        self.n_cow = 0 if self.cow_src is None else int(self.cow_src.numel())
+
+
+def decode_bytes(w, lens):
+    eb = 2 if w.dtype == "bf16" else 4
+    return int(np.sum(lens.astype(np.int64))) * w.num_kv_heads * w.head_dim * 2 * eb
+
+
+def prefill_flops(w, lens):
+    # 4 * d * H * (q * cached + q (q + 1) / 2) per sequence: causal pairs only
+    q = w.q_tokens
+    return int(sum(4 * w.head_dim * w.num_heads * (q * (int(L) - q) + q * (q + 1) // 2)
+                   for L in lens))
+
+
+def run_ours(args, dist):
+    import torch
+    torch.cuda.set_device(dist.local)
+    device = torch.device("cuda", dist.local)
+    builder = workloads.ALL[args.config]
+    w = builder(seed=workloads.seed_for({"decode32": 2, "ragged256": 3, "splitk128k": 4,
+                                         "prefill": 5}[args.config]) + 1000 * dist.rank)
+    S = Setup(w, device)
+    pool = S.pool
+    is_prefill = w.q_tokens > 1
+    part = w.partition_tokens
+    stream = torch.cuda.current_stream(device)
+
+    split = (not is_prefill) and pool.decode_workspace_bytes(
+        S.q.shape[0], S.q.shape[1], S.tables.shape[1], part) > 0
+    per_step = (1 if S.n_cow else 0) + (1 if S.slots is not None else 0) + (2 if split else 1)
+    launches = {"n": 0}
+
+    def step(ev_pair=None):
+        if S.n_cow:
+            pool.cow_copy(S.cow_src, S.cow_dst, stream)
+        if S.slots is not None:
+            pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        if is_prefill:
+            pool.prefill_chunk(S.q, S.tables, S.lens, out=S.out, stream=stream)
+        else:
+            pool.decode(S.q, S.tables, S.lens, out=S.out, partition_tokens=part, stream=stream)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+        launches["n"] += per_step
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert pool.get_error() == 0, "device error during warm-up"
+
+    # ------------------------------------------------------ timed region --
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches["n"] = 0
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_start.record(stream)
+        for i in range(K):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    dist.barrier()
+    gpu_launches = launches["n"]
+    ms_step = t_start.elapsed_time(t_end) / K
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    ms_step_max = dist.max(ms_step, device)
+    assert pool.get_error() == 0, "device error in the timed region"
+
+    # --------------------------------------------------------------- e2e --
+    e2e = run_e2e(args, S, dist, device, is_prefill, part)
+
+    hbm, bf16, bf16_sus, peak_kind = peaks()
+    lens = S.lens_h
+    if is_prefill:
+        flops = prefill_flops(w, lens)
+        value = dist.world * flops / (ms_step_max * 1e-3) / 1e12
+        metric = "chunked prefill attention TFLOP/s (causal pairs), 8 x 512 over 4608, GQA 32/8"
+        unit = "TFLOP/s"
+        achieved = flops / (kern_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": bf16,
+                "unit": "TFLOP/s", "frac": round(achieved / bf16, 4),
+                "traffic": profiled_traffic("prefill_tc.cu", w.name),
+                "kernel": "prefill", "kernel_ms": round(kern_ms, 5),
+                "peak_source": f"{peak_kind} bf16_tflops (burst)"}
+        extra = {"tflops": round(value, 2)}
+    else:
+        kv = decode_bytes(w, lens)
+        value = dist.world * kv / (ms_step_max * 1e-3) / 1e9
+        metric = "decode KV HBM GB/s (fraction of B200 peak) and seqs/s at 8K ctx, GQA 32/8"
+        unit = "GB/s"
+        achieved = kv / (kern_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4),
+                "traffic": profiled_traffic("decode_mma.cu", w.name),
+                "kernel": "decode_mma_kernel" + (" + decode_combine_kernel" if split else ""),
+                "kernel_ms": round(kern_ms, 5),
+                "algorithmic_bytes_per_launch": kv, "peak_source": f"{peak_kind} hbm_gbs"}
+        extra = {"seqs_per_s": round(dist.world * len(w.decode_seqs) / (ms_step_max * 1e-3), 1),
+                 "frac_of_peak": round(value / hbm, 4)}
+    res = {
+        "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": dist.world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1), bf16-rounded)",
+        "config": config_of(w, args, dist),
+        **extra,
+        "host_plan_us": None if S.host_plan_us is None else round(S.host_plan_us, 1),
+        "gpu_launches": gpu_launches,
+        "roofline": roof,
+        "e2e": e2e,
+        "clocks": clk.summary(),
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, args)
+    pool.close()
+    return res
+
+
+def config_of(w, args, dist):
+    G = w.num_heads // w.num_kv_heads
+    return {"workload": w.name, "batch_per_gpu": len(w.decode_seqs),
+            "global_batch": len(w.decode_seqs) * dist.world,
+            "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads, "group": G,
+            "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
+            "q_tokens": w.q_tokens, "partition_tokens": w.partition_tokens,
+            "parallelism": f"replicas x{dist.world} (no collective)",
+            "l2": "inputs larger than L2 (KV per step > 126 MB)" if w.name != "ragged256"
+            else "KV per step ~0.5 GB > L2 (shared prefixes may hit in L2)"}
+
+
+def run_e2e(args, S, dist, device, is_prefill, part):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs (queries, new K/V, slot mapping, kv_lens) from pinned host memory
+    and reads the output back; copies are inside the timed region."""
+    import torch
+    pool = S.pool
+    stream = torch.cuda.current_stream(device)
+    h_q = S.q.cpu().pin_memory()
+    h_out = torch.empty(S.out.shape, dtype=torch.float32).pin_memory()
+    h_lens = S.lens.cpu().pin_memory()
+    d_q, d_lens = torch.empty_like(S.q), torch.empty_like(S.lens)
+    h_k = h_v = h_slots = None
+    bi = h_q.numel() * h_q.element_size() + h_lens.numel() * 4
+    if S.slots is not None:
+        h_k, h_v = S.step_k.cpu().pin_memory(), S.step_v.cpu().pin_memory()
+        h_slots = S.slots.cpu().pin_memory()
+        d_k, d_v, d_slots = torch.empty_like(S.step_k), torch.empty_like(S.step_v), torch.empty_like(S.slots)
+        bi += 2 * h_k.numel() * h_k.element_size() + h_slots.numel() * 8
+    bo = h_out.numel() * 4
+    K = max(1, min(args.steps, args.e2e_steps))
+
+    def step():
+        d_q.copy_(h_q, non_blocking=True)
+        d_lens.copy_(h_lens, non_blocking=True)
+        if h_k is not None:
+            d_k.copy_(h_k, non_blocking=True)
+            d_v.copy_(h_v, non_blocking=True)
+            d_slots.copy_(h_slots, non_blocking=True)
+            if S.n_cow:
+                pool.cow_copy(S.cow_src, S.cow_dst, stream)
+            pool.reshape_and_cache(d_k, d_v, d_slots, stream)
+        if is_prefill:
+            pool.prefill_chunk(d_q, S.tables, d_lens, out=S.out, stream=stream)
+        else:
+            pool.decode(d_q, S.tables, d_lens, out=S.out, partition_tokens=part, stream=stream)
+        h_out.copy_(S.out, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = dist.max(a.elapsed_time(b) / K, device)
+    w = S.w
+    if is_prefill:
+        v = dist.world * prefill_flops(w, S.lens_h) / (ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+    else:
+        v = dist.world * decode_bytes(w, S.lens_h) / (ms * 1e-3) / 1e9
+        unit = "GB/s"
+    return {"value": round(v, 2), "unit": unit, "h2d_bytes_per_step": int(bi),
+            "d2h_bytes_per_step": int(bo), "ms_per_step": round(ms, 5), "steps": K}
+
+
+# --------------------------------------------------------------- oracle ----
+class OracleSampler:
+    """The float64 oracle (paged gather, then two-pass softmax) run on
+    (sequence, KV head) groups of a workload.  The oracle pool is built once
+    (untimed, data stored as float32 holding the bf16 values exactly); only the
+    attention calls are timed."""
+
+    def __init__(self, w):
+        import torch
+        from oracle import KVPool
+        self.w = w
+        self.G = w.num_heads // w.num_kv_heads
+        self.q = w.queries().to(torch.float64).numpy()
+        p = KVPool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.order,
+                   store_heads="all", dtype=np.float32)
+        for op in w.setup + w.step:
+            if op.kind == "create":
+                p.create(op.args[0])
+            elif op.kind == "share":
+                p.share_prefix(*op.args)
+            elif op.kind == "release":
+                p.release(op.args[0])
+            else:
+                k, v = w.kv_for(op)
+                p.append(op.args[0], op.args[1], k.float().numpy(), v.float().numpy())
+        self.pool = p
+        self.next = 0
+
+    def run(self, budget_s, max_units=None):
+        """Decode (or prefill) whole sequences -- every head -- until the
+        budget is spent; returns (bytes or flops, seconds, sequences)."""
+        from oracle import paged_attention
+        w, p = self.w, self.pool
+        work, spent, done = 0, 0.0, 0
+        while spent < budget_s and (max_units is None or done < max_units):
+            si = self.next % len(w.decode_seqs)
+            self.next += 1
+            seq = w.decode_seqs[si]
+            t0 = time.perf_counter()
+            paged_attention(p, seq, self.q[si])        # gather + two-pass softmax
+            spent += time.perf_counter() - t0
+            L = p.lengths[seq]
+            if w.q_tokens > 1:
+                qn = w.q_tokens
+                work += 4 * w.head_dim * w.num_heads * (qn * (L - qn) + qn * (qn + 1) // 2)
+            else:
+                work += L * w.num_kv_heads * w.head_dim * 2 * (2 if w.dtype == "bf16" else 4)
+            done += 1
+        return work, spent, done
+
+
+def cpu_baseline(w, args):
+    sampler = OracleSampler(w)
+    work, spent, done = sampler.run(args.cpu_budget)
+    desc = (f"{done} of the {len(w.decode_seqs)} sequences of {w.name} (all heads): oracle "
+            f"paged gather + float64 two-pass softmax")
+    if w.q_tokens > 1:
+        val, unit = work / spent / 1e12, "TFLOP/s"
+    else:
+        val, unit = work / spent / 1e9, "GB/s"
+    return {"value": round(val, 6), "unit": unit, "cores": oracle_threads(), "kind": "oracle",
+            "sample": desc, "seconds": round(spent, 2), "host_cpus": os.cpu_count()}
+
+
+def run_reference(args, dist):
+    """The float64 oracle as the reference arm, on this host's cores."""
+    if dist.rank != 0:
+        return None
+    builder = workloads.ALL[args.config]
+    w = builder()
+    sampler = OracleSampler(w)
+    # each step: one bounded sample (whole groups) so the run stays ~2-3 minutes
+    per_step = max(0.005, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        sampler.run(per_step, max_units=1)
+    work, spent, groups, steps = 0, 0.0, 0, 0
+    for _ in range(args.steps):
+        wk, sp, n = sampler.run(per_step)
+        work, spent, groups, steps = work + wk, spent + sp, groups + n, steps + 1
+        if spent > 150:
+            break
+    desc = (f"{groups} sequences (all heads) of {w.name} over {steps} steps: oracle paged "
+            f"gather + float64 two-pass softmax")
+    if w.q_tokens > 1:
+        val, unit, metric = work / spent / 1e12, "TFLOP/s", \
+            "chunked prefill attention TFLOP/s (causal pairs), 8 x 512 over 4608, GQA 32/8"
+    else:
+        val, unit, metric = work / spent / 1e9, "GB/s", \
+            "decode KV HBM GB/s (fraction of B200 peak) and seqs/s at 8K ctx, GQA 32/8"
+    ms = spent / max(1, steps) * 1e3
+    return {"impl": "reference", "metric": metric, "value": round(val, 6), "unit": unit,
+            "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), bf16-rounded)",
+            "config": {"workload": w.name, "sample": desc},
+            "cpu_baseline": {"value": round(val, 6), "unit": unit, "cores": oracle_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(val, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=["decode32", "ragged256", "splitk128k", "prefill"],
+                    default="decode32")
+    ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    dist = Dist(args.gpus)
+    if args.impl == "reference":
+        res = run_reference(args, dist)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    dist.init("nccl")
+    try:
+        res = run_ours(args, dist)
+        if dist.rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()
