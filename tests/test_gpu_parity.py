@@ -165,15 +165,14 @@ def test_device_bounds_errors_zero_rows():
     assert g.pool.get_error() == 0                       # cleared by the read
 
 
-def _prefill_case(batch, cached, chunk, H, Hkv, seed):
-    return workloads.prefill(seed=seed, batch=batch, cached=cached, chunk=chunk)
-
-
-@pytest.mark.parametrize("batch,cached,chunk", [(2, 0, 37), (2, 40, 37), (1, 200, 130), (3, 5, 1)])
-def test_prefill_parity_small(batch, cached, chunk):
-    w = workloads.prefill(seed=batch * 100 + cached + chunk, batch=batch, cached=cached, chunk=chunk)
-    w = dataclasses.replace(w, setup=[op for op in w.setup if not (op.kind == "append" and op.args[1] == 0)])
+@pytest.mark.parametrize("batch,cached,chunk,H,Hkv", [
+    (2, 0, 37, 32, 8), (2, 40, 37, 32, 8), (1, 200, 130, 32, 8), (3, 5, 1, 32, 8),
+    (2, 300, 129, 8, 8), (2, 17, 200, 16, 8), (2, 250, 64, 64, 8), (1, 1000, 300, 32, 8)])
+def test_prefill_parity_small(batch, cached, chunk, H, Hkv):
+    w = workloads.prefill(seed=batch * 100 + cached + chunk + H, batch=batch, cached=cached,
+                          chunk=chunk, num_heads=H, num_kv_heads=Hkv)
     g = GpuRun(w).apply(w.setup + w.step)
+    assert g.pool.prefill_path(H) == 1
     o = OracleRun(w).apply(w.setup + w.step)
     out = g.prefill()
     q = q64(w)

@@ -164,7 +164,7 @@ def ragged256(seed: int = seed_for(3), groups: int = 32, per_group: int = 8,
     for g in range(groups):
         root = 100000 + g
         ops += [("create", root), ("append", root, prefix)]
-        need += prefix // bs
+        need += -(-prefix // bs)
         for m in range(per_group):
             b = g * per_group + m
             L = int(lens[b])
@@ -192,14 +192,15 @@ def splitk128k(seed: int = seed_for(4)) -> Workload:
 
 
 def prefill(seed: int = seed_for(5), batch: int = 8, cached: int = 4096,
-            chunk: int = 512) -> Workload:
+            chunk: int = 512, num_heads: int = 32, num_kv_heads: int = 8) -> Workload:
     """Chunked prefill: cached tokens, then a chunk appended and attended causally."""
     bs = 16
-    ops = [("create", b) for b in range(batch)] + [("append", b, cached) for b in range(batch)]
+    ops = [("create", b) for b in range(batch)]
+    ops += [("append", b, cached) for b in range(batch) if cached > 0]
     setup = _script(ops)
     step = [Op("append", (b, chunk), len(ops) + b) for b in range(batch)]
     nb = batch * (-(-(cached + chunk) // bs)) + 64
-    return Workload("prefill", nb, bs, 32, 8, 128, "bf16", seed,
+    return Workload("prefill", nb, bs, num_heads, num_kv_heads, 128, "bf16", seed,
                     permutation(nb, seed), setup=setup, step=step,
                     decode_seqs=list(range(batch)), q_tokens=chunk)
 
