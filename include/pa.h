@@ -69,7 +69,8 @@ typedef enum pa_status {
   PA_ERR_DEVICE = 6,          /* pa_get_error found device error bits        */
   PA_ERR_UNSUPPORTED = 7,     /* shape/dtype outside what the kernels take   */
   PA_ERR_NO_DEVICE = 8,       /* device call on a host-only pool             */
-  PA_ERR_INTERNAL = 9         /* pa_validate found a broken invariant        */
+  PA_ERR_INTERNAL = 9,        /* pa_validate found a broken invariant        */
+  PA_ERR_SCRATCH_LIMIT = 10   /* request needs more than the fixed scratch   */
 } pa_status;
 
 typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
@@ -234,6 +235,37 @@ pa_status pa_prefill_chunk(pa_pool* pool, const void* q, int32_t B,
                            const int32_t* d_block_tables, int32_t max_blocks,
                            const int32_t* d_kv_lens, float scale, float* out,
                            void* stream);
+
+/* Bytes of the fixed device scratch array used by pa_decode_static_scratch. */
+#define PA_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* pa_decode for callers that cannot allocate device memory.  The pages
+ * describe no counterpart: this is an integration convenience of this
+ * library.  A serving process that gives all device memory to its KV pool and
+ * weights at start-up, or a plugin whose host framework owns the device
+ * allocator, cannot provide pa_decode's workspace; this entry point takes the
+ * partition scratch from a file-scope __device__ array of
+ * PA_STATIC_SCRATCH_BYTES (16 MiB) that every GPU loading the library holds
+ * until the process exits, and calls no cudaMalloc, cudaFree or other
+ * allocating routine.  Arguments and results are those of pa_decode without
+ * the workspace pair; the current device must be the pool's device.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents.  Nothing in it needs to start at zero (each partition
+ *     writes all its entries before they are read), but calls whose kernels
+ *     overlap on the GPU (different streams, no ordering between them) race
+ *     on the array.
+ * Errors: those of pa_decode, plus PA_ERR_SCRATCH_LIMIT (nothing launched)
+ * when pa_decode_workspace_bytes for this shape exceeds
+ * PA_STATIC_SCRATCH_BYTES -- use fewer or larger partitions, or pa_decode. */
+pa_status pa_decode_static_scratch(pa_pool* pool, const void* q, int32_t B,
+                                   int32_t H, const int32_t* d_block_tables,
+                                   int32_t max_blocks,
+                                   const int32_t* d_kv_lens, float scale,
+                                   int32_t partition_tokens, float* out,
+                                   void* stream);
 
 /* Synchronise the device, read and clear the pool's device error word.
  * *device_code = OR of PA_DEVERR_* bits seen since the last call.  Returns

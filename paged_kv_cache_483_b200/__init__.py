@@ -23,14 +23,15 @@ LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
 PA_F32, PA_BF16 = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "unknown sequence", 3: "duplicate sequence",
           4: "pool exhausted", 5: "CUDA error", 6: "device error", 7: "unsupported",
-          8: "host-only pool", 9: "broken invariant"}
+          8: "host-only pool", 9: "broken invariant", 10: "scratch limit"}
 PA_DEVERR_BLOCK_ID, PA_DEVERR_SLOT, PA_DEVERR_KV_LEN, PA_DEVERR_TIMEOUT = 1, 2, 4, 8
 
 EXPORTS = ["pa_pool_create", "pa_free", "pa_seq_create", "pa_seq_fork", "pa_seq_release",
            "pa_seq_table", "pa_block_tables", "pa_plan_append", "pa_pool_stats",
            "pa_refcounts", "pa_validate", "pa_append_kv", "pa_reshape_and_cache",
            "pa_cow_copy", "pa_decode_workspace_bytes", "pa_decode", "pa_prefill_chunk",
-           "pa_get_error", "pa_status_string", "pa_decode_path", "pa_prefill_path"]
+           "pa_get_error", "pa_status_string", "pa_decode_path", "pa_prefill_path",
+           "pa_decode_static_scratch"]
 
 
 class PAError(RuntimeError):
@@ -81,6 +82,7 @@ def lib():
         "pa_status_string": ([C.c_int], C.c_char_p),
         "pa_decode_path": ([_P, _I32], _I32),
         "pa_prefill_path": ([_P, _I32], _I32),
+        "pa_decode_static_scratch": ([_P, _P, _I32, _I32, _P, _I32, _P, _F, _I32, _P, _P], C.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)

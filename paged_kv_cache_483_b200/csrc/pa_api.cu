@@ -527,6 +527,7 @@ const char* pa_status_string(pa_status s) {
     case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
     case PA_ERR_NO_DEVICE: return "host-only pool";
     case PA_ERR_INTERNAL: return "broken invariant";
+    case PA_ERR_SCRATCH_LIMIT: return "request exceeds the fixed device scratch";
   }
   return "unknown status";
 }

@@ -1,0 +1,69 @@
+"""pa_decode_static_scratch: decode for callers that cannot allocate.
+
+A serving process that gives all device memory to its KV pool and weights at
+start-up, or a plugin whose host framework owns the device allocator, cannot
+hand pa_decode a workspace for its split-K partitions.  The static-scratch
+entry point takes that scratch from a fixed device array inside the library
+instead.  These checks call it through the C ABI and compare it with
+pa_decode given a caller workspace, on two calls in a row (the array keeps the
+first call's contents), and check that a request larger than the array is
+refused with PA_ERR_SCRATCH_LIMIT.
+"""
+import ctypes as C
+import math
+
+import pytest
+import torch
+
+import paged_kv_cache_483_b200 as pa
+import workloads
+from harness import GpuRun
+
+pytestmark = pytest.mark.gpu
+
+TOL_DECODE = 2e-3          # the bf16 decode tolerance of the parity tests
+PA_ERR_SCRATCH_LIMIT = 10
+
+
+def _call(L, g, q, tables, lens, part, out):
+    return L.pa_decode_static_scratch(
+        g.pool.handle, C.c_void_p(q.data_ptr()), q.shape[0], q.shape[1],
+        C.c_void_p(tables.data_ptr()), tables.shape[1], C.c_void_p(lens.data_ptr()),
+        C.c_float(1.0 / math.sqrt(128)), part, C.c_void_p(out.data_ptr()),
+        C.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+def test_static_scratch_matches_workspace_decode_twice():
+    w = workloads.custom_decode("noalloc", [700, 1234, 40, 4097, 1, 0, 333], 64, 8, 128, 16,
+                                "bf16", seed=99, spare_blocks=4)
+    g = GpuRun(w).apply(w.setup)
+    tables, lens, _, _ = g.tables()
+    q = w.queries()[:, 0].contiguous().cuda()
+    part = 256     # several partitions per sequence, so the scratch is used
+    assert g.pool.decode_workspace_bytes(q.shape[0], q.shape[1], tables.shape[1], part) > 0
+    ref = g.pool.decode(q, tables, lens, partition_tokens=part)
+    torch.cuda.synchronize()
+    L = pa.lib()
+    for _ in range(2):
+        out = torch.full_like(ref, float("nan"))
+        assert _call(L, g, q, tables, lens, part, out) == 0
+        torch.cuda.synchronize()
+        assert torch.isfinite(out).all()
+        assert (out - ref).abs().max().item() <= TOL_DECODE
+    assert g.pool.get_error() == 0
+
+
+def test_static_scratch_refuses_oversized_requests():
+    w = workloads.custom_decode("noalloc_big", [64] * 8, 64, 8, 128, 16, "bf16", seed=5,
+                                spare_blocks=4)
+    g = GpuRun(w).apply(w.setup)
+    q = w.queries()[:, 0].contiguous().cuda()
+    wide = torch.zeros((8, 4096), dtype=torch.int32, device="cuda")
+    lens = torch.full((8,), 64, dtype=torch.int32, device="cuda")
+    need = g.pool.decode_workspace_bytes(8, 64, 4096, 16)
+    assert need > (16 << 20)
+    out = torch.zeros((8, 64, 128), dtype=torch.float32, device="cuda")
+    assert _call(pa.lib(), g, q, wide, lens, 16, out) == PA_ERR_SCRATCH_LIMIT
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out).item() == 0          # nothing was launched
+    assert g.pool.get_error() == 0
