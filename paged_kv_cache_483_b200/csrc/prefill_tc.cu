@@ -8,22 +8,27 @@
 // softmax(q.k * scale) weighted sum of V, with the one-pass (m, l, acc)
 // update of "semidirectx cmu11-667 lecture19 infer_world.py", section 3.
 //
-// One CTA = one 128-row query tile of one (sequence, KV head): rows are
-// (token, head) pairs, 128/G tokens x G heads, so the G query heads that share
-// a KV head share every K/V tile.  Keys are visited in tiles of 128 (eight
+// One CTA = two 128-row query tiles (A and B) of one (sequence, KV head).
+// Rows are (token, head) pairs, 128/G tokens x G heads, so the G query heads
+// that share a KV head share every K/V tile, and both tiles share each K/V
+// tile fetched into shared memory.  Keys are visited in tiles of 128 (eight
 // paged blocks, each fetched by TMA as two 64-column boxes with the 128-byte
-// swizzle, landing exactly in the UMMA K-major layout).
-//   warp 0      TMA producer (Q once; K and V tiles into a 2-stage ring)
-//   warp 1      one thread issues tcgen05.mma: S = Q K^T into TMEM (double
-//               buffered, 2 x 128 columns), then O += P V (O: 128 columns)
-//   warps 2-5   softmax, one thread per row = TMEM lane: load the S row,
-//               causal mask, running max, exp2, row sum, P as bf16 into shared
-//               memory (K-major, swizzled) for the PV MMA; O is rescaled in
-//               TMEM only when a row's max grows by more than 2^8 (a stale max
-//               below that keeps every exponent <= 2^8, exact in fp32)
-//   epilogue    O / l from TMEM to global fp32.
-// The QK^T of tile j+1 runs on the tensor core while the softmax of tile j
-// runs on the CUDA cores.  P is rounded to bf16 for the PV product.
+// swizzle, landing in the UMMA K-major layout).
+//   warp 0      TMA producer: Q_A, Q_B once; K and V tiles into 2-stage rings
+//               (K(j+1) is issued before V(j): a K stage frees after its two
+//               QK^T, well before the V stage of the same tile).
+//   warp 1      one thread issues tcgen05.mma in the order
+//                 ... PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1) ...
+//               S_X = Q_X K^T lands in TMEM; O_X += P_X V reads P_X from TMEM
+//               (the softmax writes it over S_X) and V from shared memory.
+//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B; one thread per
+//               row = TMEM lane.  While one tile's softmax runs on the CUDA
+//               cores the tensor core works on the other tile.
+// TMEM (512 columns): S_A/P_A [0,128), S_B/P_B [128,256), O_A, O_B.
+// The tensor core executes one CTA's MMAs in issue order, so when QK_X(j) has
+// completed, PV_X(j-1) has too: the softmax may then rescale O_X in TMEM.  O
+// is rescaled only when a row's max grows by more than 2^8 (a stale max below
+// that keeps every exponent <= 2^8, exact in fp32).  P is rounded to bf16.
 #include <math.h>
 
 #include "common.cuh"
@@ -34,15 +39,14 @@ namespace pa {
 
 namespace {
 
-constexpr int kPfThreads = 192;
+constexpr int kPfThreads = 320;
 constexpr int kPfStages = 2;
 constexpr uint32_t kTile = 32768;  // 128 x 128 bf16
 constexpr uint32_t kHalf = 16384;  // 128 x 64 bf16 (one 128-byte-swizzled half)
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kTile;
-constexpr uint32_t kOffV = kTile * (1 + kPfStages);
-constexpr uint32_t kOffP = kTile * (1 + 2 * kPfStages);
-constexpr uint32_t kDataBytes = kTile * (2 + 2 * kPfStages);
+constexpr uint32_t kOffQ = 0;      // Q_A, then Q_B
+constexpr uint32_t kOffK = 2 * kTile;
+constexpr uint32_t kOffV = (2 + kPfStages) * kTile;
+constexpr uint32_t kDataBytes = (2 + 2 * kPfStages) * kTile;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr float kRescaleTau = 8.0f;
@@ -53,8 +57,8 @@ struct PfBars {
   uint64_t q_full;
   uint64_t k_full[kPfStages], k_empty[kPfStages];
   uint64_t v_full[kPfStages], v_empty[kPfStages];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full, o_done;
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_final;
   uint32_t tmem_base;
   int abort;
   int bad;
@@ -74,6 +78,17 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
   return false;
 }
 
+// Warp-uniform wait used by the softmax warps (tcgen05.ld/st are collective).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, PfBars* bars,
+                                          int32_t* err, int lane) {
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity));
+  if (!ok && lane == 0) {
+    raise_err(err, PA_DEVERR_TIMEOUT);
+    atomicExch(&bars->abort, 1);
+  }
+  return ok;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
@@ -86,13 +101,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.H / p.Hkv, TQ = 128 / G;
-  const int mt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int t0 = mt * TQ;
+  const int kvh = blockIdx.y, b = blockIdx.z;
+  const int t0 = blockIdx.x * 2 * TQ;                 // first token of tile A
   const int q_tokens = p.q_tokens;
   const int kv_len = p.kv_lens[b];
-  const int valid_tokens = min(TQ, q_tokens - t0);
+  const int valid_tokens = min(2 * TQ, q_tokens - t0);  // of both tiles
   const bool len_bad = kv_len < q_tokens || kv_len > p.MB * 16;
-  const int qpos0 = kv_len - q_tokens + t0;        // key limit of the first token
+  const int qpos0 = kv_len - q_tokens + t0;           // key limit of token t0
   const int key_end = len_bad ? 0 : qpos0 + valid_tokens;
   const int n_tiles = (key_end + 127) >> 7;
   const int n_blk = (key_end + 15) >> 4;
@@ -103,7 +118,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
     bars->bad = len_bad ? 1 : 0;
   }
   __syncthreads();
-  // every block id the tile will touch must be inside the pool
+  // every block id the CTA will touch must be inside the pool
   for (int i = threadIdx.x; i < n_blk; i += blockDim.x) {
     const int blk = trow[i];
     if (blk < 0 || blk >= p.NB) bars->bad = 2;
@@ -128,12 +143,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->s_free[s], 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_full[x], 128);
     }
-    mbar_init(&bars->p_full, 128);
-    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->o_final, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -153,129 +167,143 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
       prefetch_tensormap(&tmV);
       const uint64_t pol_q = policy_evict_first();
       const uint64_t pol_kv = policy_evict_last();
-      mbar_arrive_expect_tx(&bars->q_full, kTile);
-      tma_load_3d(smem + kOffQ, &tmQ, &bars->q_full, 0, kvh * G, b * q_tokens + t0, pol_q);
-      tma_load_3d(smem + kOffQ + kHalf, &tmQ, &bars->q_full, 64, kvh * G, b * q_tokens + t0,
-                  pol_q);
-      int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kPfStages, round = j / kPfStages;
-        if (round > 0) {
-          if (!wait_or_abort(&bars->k_empty[s], (round - 1) & 1, bars, p.err)) break;
-          if (!wait_or_abort(&bars->v_empty[s], (round - 1) & 1, bars, p.err)) break;
-        }
-        if (bars->abort) break;
+      mbar_arrive_expect_tx(&bars->q_full, 2 * kTile);
+      for (int x = 0; x < 2; ++x) {
+        const int z = b * q_tokens + t0 + x * TQ;
+        tma_load_3d(smem + kOffQ + x * kTile, &tmQ, &bars->q_full, 0, kvh * G, z, pol_q);
+        tma_load_3d(smem + kOffQ + x * kTile + kHalf, &tmQ, &bars->q_full, 64, kvh * G, z,
+                    pol_q);
+      }
+      int k_issued = 0, v_issued = 0;
+      auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* full, int j) {
         const int nb = min(8, n_blk - j * 8);
-        uint8_t* kst = smem + kOffK + s * kTile;
-        uint8_t* vst = smem + kOffV + s * kTile;
-        mbar_arrive_expect_tx(&bars->k_full[s], nb * 4096);
+        mbar_arrive_expect_tx(full, nb * 4096);
         for (int i = 0; i < nb; ++i) {
           const int z = trow[j * 8 + i] * 16;
-          tma_load_3d(kst + i * 2048, &tmK, &bars->k_full[s], 0, kvh, z, pol_kv);
-          tma_load_3d(kst + kHalf + i * 2048, &tmK, &bars->k_full[s], 64, kvh, z, pol_kv);
+          tma_load_3d(dst + i * 2048, map, full, 0, kvh, z, pol_kv);
+          tma_load_3d(dst + kHalf + i * 2048, map, full, 64, kvh, z, pol_kv);
         }
-        mbar_arrive_expect_tx(&bars->v_full[s], nb * 4096);
-        for (int i = 0; i < nb; ++i) {
-          const int z = trow[j * 8 + i] * 16;
-          tma_load_3d(vst + i * 2048, &tmV, &bars->v_full[s], 0, kvh, z, pol_kv);
-          tma_load_3d(vst + kHalf + i * 2048, &tmV, &bars->v_full[s], 64, kvh, z, pol_kv);
+      };
+      bool ok = true;
+      for (int j = -1; ok && j < n_tiles; ++j) {
+        const int jk = j + 1;                          // K tile to issue
+        if (jk < n_tiles) {
+          const int s = jk % kPfStages, round = jk / kPfStages;
+          if (round > 0) ok = wait_or_abort(&bars->k_empty[s], (round - 1) & 1, bars, p.err);
+          if (!ok || bars->abort) break;
+          load_tile(smem + kOffK + s * kTile, &tmK, &bars->k_full[s], jk);
+          k_issued = jk + 1;
         }
-        issued = j + 1;
+        if (j >= 0) {                                  // V tile j
+          const int s = j % kPfStages, round = j / kPfStages;
+          if (round > 0) ok = wait_or_abort(&bars->v_empty[s], (round - 1) & 1, bars, p.err);
+          if (!ok || bars->abort) break;
+          load_tile(smem + kOffV + s * kTile, &tmV, &bars->v_full[s], j);
+          v_issued = j + 1;
+        }
       }
       // drain: every issued copy has landed before the CTA may exit
       mbar_wait(&bars->q_full, 0);
-      for (int s = 0; s < kPfStages && s < issued; ++s) {
-        const int count = (issued - 1 - s) / kPfStages + 1;
-        mbar_wait(&bars->k_full[s], (count - 1) & 1);
-        mbar_wait(&bars->v_full[s], (count - 1) & 1);
+      for (int s = 0; s < kPfStages; ++s) {
+        if (s < k_issued) mbar_wait(&bars->k_full[s], ((k_issued - 1 - s) / kPfStages) & 1);
+        if (s < v_issued) mbar_wait(&bars->v_full[s], ((v_issued - 1 - s) / kPfStages) & 1);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      bool ok = wait_or_abort(&bars->q_full, 0, bars, p.err);
-      tc_fence_after();
       const uint32_t qa = smem_u32(smem + kOffQ);
-      const uint32_t pa_ = smem_u32(smem + kOffP);
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          const int s = j % kPfStages;
-          ok = wait_or_abort(&bars->k_full[s], (j / kPfStages) & 1, bars, p.err);
-          if (ok && j >= 2)
-            ok = wait_or_abort(&bars->s_free[j & 1], ((j - 2) >> 1) & 1, bars, p.err);
-          if (!ok || bars->abort) break;
-          tc_fence_after();
-          const uint32_t kb = smem_u32(smem + kOffK + s * kTile);
-          const uint32_t d = tbase + kColS + (j & 1) * 128;
+      auto qk = [&](int x, int j) {                    // S_x = Q_x K(j)^T
+        const uint32_t kb = smem_u32(smem + kOffK + (j % kPfStages) * kTile);
+        const uint32_t q = qa + x * kTile;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            umma_bf16(d, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(kb + off), kIdescQK,
-                      kk > 0);
-          }
-          umma_commit(&bars->s_full[j & 1]);
-          umma_commit(&bars->k_empty[s]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          umma_bf16(tbase + kColS + x * 128, desc_kmajor_sw128(q + off),
+                    desc_kmajor_sw128(kb + off), kIdescQK, kk > 0);
         }
-        if (j >= 1) {
-          const int jj = j - 1, s = jj % kPfStages;
-          ok = wait_or_abort(&bars->p_full, jj & 1, bars, p.err);
-          if (ok) ok = wait_or_abort(&bars->v_full[s], (jj / kPfStages) & 1, bars, p.err);
-          if (!ok || bars->abort) break;
-          tc_fence_after();
-          const uint32_t vb = smem_u32(smem + kOffV + s * kTile);
+        umma_commit(&bars->s_full[x]);
+      };
+      auto pv = [&](int x, int j) {                    // O_x += P_x V(j)
+        const uint32_t vb = smem_u32(smem + kOffV + (j % kPfStages) * kTile);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            umma_bf16(tbase + kColO, desc_kmajor_sw128(pa_ + off),
-                      desc_mnmajor_sw128(vb + kk * 2048, kHalf, 1024), kIdescPV,
-                      (jj > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&bars->o_done);
-          umma_commit(&bars->v_empty[s]);
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_tmem_a(tbase + kColO + x * 128, tbase + kColS + x * 128 + kk * 8,
+                           desc_mnmajor_sw128(vb + kk * 2048, kHalf, 1024), kIdescPV,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait_or_abort(&bars->q_full, 0, bars, p.err) &&
+                wait_or_abort(&bars->k_full[0], 0, bars, p.err);
+      if (ok) {
+        tc_fence_after();
+        qk(0, 0);
+        qk(1, 0);
+        umma_commit(&bars->k_empty[0]);
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kPfStages;
+        const bool more = j + 1 < n_tiles;
+        ok = wait_or_abort(&bars->v_full[s], (j / kPfStages) & 1, bars, p.err) &&
+             wait_or_abort(&bars->p_full[0], j & 1, bars, p.err);
+        if (!ok || bars->abort) break;
+        tc_fence_after();
+        pv(0, j);
+        if (more) {
+          const int s1 = (j + 1) % kPfStages;
+          ok = wait_or_abort(&bars->k_full[s1], ((j + 1) / kPfStages) & 1, bars, p.err);
+          if (!ok) break;
+          tc_fence_after();
+          qk(0, j + 1);
+        }
+        ok = wait_or_abort(&bars->p_full[1], j & 1, bars, p.err);
+        if (!ok || bars->abort) break;
+        tc_fence_after();
+        pv(1, j);
+        umma_commit(&bars->v_empty[s]);
+        if (more) {
+          qk(1, j + 1);
+          umma_commit(&bars->k_empty[(j + 1) % kPfStages]);
         }
       }
+      umma_commit(&bars->o_final);
     }
   } else {
     // ------------------------------------------------ softmax / epilogue
+    const int x = (warp - 2) >> 2;                     // query tile A (0) or B (1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                 // row = TMEM lane
     const int t_local = r / G, g = r % G;
-    const bool row_valid = t_local < valid_tokens;
-    const int qpos = qpos0 + t_local;
+    const int tok = t0 + x * TQ + t_local;             // query token of this row
+    const bool row_valid = tok < q_tokens;
+    const int qpos = kv_len - q_tokens + tok;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    uint8_t* prow = smem + kOffP + r * 128;
+    const uint32_t s_addr = tbase + lane_off + kColS + x * 128;
+    const uint32_t o_addr = tbase + lane_off + kColO + x * 128;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1));
-      if (!ok) {
-        if (lane == 0) {
-          raise_err(p.err, PA_DEVERR_TIMEOUT);
-          atomicExch(&bars->abort, 1);
-        }
-        break;
-      }
+      ok = warp_wait(&bars->s_full[x], j & 1, bars, p.err, lane);
+      if (!ok) break;
       tc_fence_after();
       float s[128];
       {
-        const uint32_t sb = tbase + lane_off + kColS + (j & 1) * 128;
+        uint32_t v[128];
+        tmem_ld128(s_addr, v);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(sb + c * 32, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[i]);
-        }
+        for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(v[i]);
       }
-      tc_fence_before();
-      mbar_arrive(&bars->s_free[j & 1]);
       const int lim = qpos - j * 128;                  // columns c <= lim are visible
-      float mx = -INFINITY;
+      if (lim < 127) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        s[c] = (c <= lim) ? s[c] : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 128; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
       }
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float mt = mx * scale_log2;
       float alpha = 1.f;
       bool rescale = false;
@@ -284,78 +312,62 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
         rescale = (j > 0);
         m_ref = mt;
       }
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (j - 1) & 1));
-        if (!ok) {
-          if (lane == 0) {
-            raise_err(p.err, PA_DEVERR_TIMEOUT);
-            atomicExch(&bars->abort, 1);
-          }
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
-          const uint32_t ob = tbase + lane_off + kColO;
+      // PV_x(j-1) has completed (it precedes QK_x(j) on the tensor core)
+      if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[32];
-            tmem_ld32(ob + c * 32, v);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(o_addr + c * 32, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-            tmem_st32(ob + c * 32, v);
-          }
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+          tmem_st32(o_addr + c * 32, v);
         }
       }
       l *= alpha;
-      if (j == n_tiles - 1) {
+      if (x == 0 && j == n_tiles - 1) {
         // V rows at or past key_end hold stale bytes: zero them (p = 0 there,
-        // and 0 x NaN would poison the product)
-        const int s = j % kPfStages;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->v_full[s], (j / kPfStages) & 1));
-        if (ok && j * 128 + r >= key_end) {
-          uint4* v0 = reinterpret_cast<uint4*>(smem + kOffV + s * kTile + r * 128);
-          uint4* v1 = reinterpret_cast<uint4*>(smem + kOffV + s * kTile + kHalf + r * 128);
+        // and 0 x NaN would poison the product); PV_B is issued after PV_A
+        const int st = j % kPfStages;
+        const bool landed = warp_wait(&bars->v_full[st], (j / kPfStages) & 1, bars, p.err, lane);
+        if (landed && j * 128 + r >= key_end) {
+          uint4* v0 = reinterpret_cast<uint4*>(smem + kOffV + st * kTile + r * 128);
+          uint4* v1 = reinterpret_cast<uint4*>(smem + kOffV + st * kTile + kHalf + r * 128);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             v0[c] = make_uint4(0u, 0u, 0u, 0u);
             v1[c] = make_uint4(0u, 0u, 0u, 0u);
           }
         }
+        fence_proxy_async_smem();
       }
-      float sum = 0.f;
+      // P = 2^(s*scale - m_ref) as bf16 pairs, written over S_x in TMEM
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
       const float nm = -m_ref;
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        uint32_t w[4];
+      for (int hcol = 0; hcol < 2; ++hcol) {
+        uint32_t w[32];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2(fmaf(s[ch * 8 + 2 * e], scale_log2, nm));
-          const float p1 = ex2(fmaf(s[ch * 8 + 2 * e + 1], scale_log2, nm));
-          sum += p0 + p1;
-          w[e] = pack_bf16x2(p0, p1);
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2(fmaf(s[hcol * 64 + 2 * i], scale_log2, nm));
+          const float p1 = ex2(fmaf(s[hcol * 64 + 2 * i + 1], scale_log2, nm));
+          sum4[i & 3] += p0 + p1;
+          w[i] = pack_bf16x2(p0, p1);
         }
-        *reinterpret_cast<uint4*>(prow + (ch >> 3) * kHalf + (((ch & 7) ^ (r & 7)) << 4)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        tmem_st32(s_addr + hcol * 32, w);
       }
-      l += sum;
-      fence_proxy_async_smem();
+      l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       tc_fence_before();
-      mbar_arrive(&bars->p_full);
+      mbar_arrive(&bars->p_full[x]);
     }
     // epilogue: O / l
-    bool done = ok && __all_sync(0xffffffffu,
-                                 mbar_wait(&bars->o_done, (n_tiles - 1) & 1));
-    if (!done && lane == 0) {
-      raise_err(p.err, PA_DEVERR_TIMEOUT);
-      atomicExch(&bars->abort, 1);
-    }
+    const bool done = ok && warp_wait(&bars->o_final, 0, bars, p.err, lane);
     tc_fence_after();
     const float inv = (done && l > 0.f) ? 1.f / l : 0.f;
-    float* orow = p.out + ((int64_t(b) * q_tokens + t0 + t_local) * p.H + kvh * G + g) * 128;
+    float* orow = p.out + ((int64_t(b) * q_tokens + tok) * p.H + kvh * G + g) * 128;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t v[32];
-      tmem_ld32(tbase + lane_off + kColO + c * 32, v);
+      tmem_ld32(o_addr + c * 32, v);
       if (row_valid) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
@@ -414,7 +426,7 @@ cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((a.q_tokens + TQ - 1) / TQ, a.Hkv, a.B);
+  dim3 grid((a.q_tokens + 2 * TQ - 1) / (2 * TQ), a.Hkv, a.B);
   prefill_tc_kernel<<<grid, kPfThreads, smem, stream>>>(tmQ, *tmK, *tmV, a,
                                                          a.scale * 1.4426950408889634f);
   return cudaGetLastError();
