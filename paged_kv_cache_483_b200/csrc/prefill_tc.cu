@@ -70,6 +70,12 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               PfBars* bars, int32_t* err) {
   if (mbar_wait(bar, parity)) return true;
@@ -299,11 +305,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
       }
       float mx8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+      for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(s[i], s[i + 8]);
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      for (int c = 16; c < 128; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = max3(mx8[i], s[c + i], s[c + 8 + i]);
+      const float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]),
+                            fmaxf(mx8[6], mx8[7]));
       const float mt = mx * scale_log2;
       float alpha = 1.f;
       bool rescale = false;
@@ -341,21 +349,23 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
         fence_proxy_async_smem();
       }
       // P = 2^(s*scale - m_ref) as bf16 pairs, written over S_x in TMEM
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-      const float nm = -m_ref;
+      float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      const float2 sl2 = make_float2(scale_log2, scale_log2);
+      const float2 nm2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
       for (int hcol = 0; hcol < 2; ++hcol) {
         uint32_t w[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(fmaf(s[hcol * 64 + 2 * i], scale_log2, nm));
-          const float p1 = ex2(fmaf(s[hcol * 64 + 2 * i + 1], scale_log2, nm));
-          sum4[i & 3] += p0 + p1;
-          w[i] = pack_bf16x2(p0, p1);
+          const float2 e = __ffma2_rn(make_float2(s[hcol * 64 + 2 * i], s[hcol * 64 + 2 * i + 1]),
+                                      sl2, nm2);
+          const float2 pp = make_float2(ex2(e.x), ex2(e.y));
+          sum2[i & 1] = __fadd2_rn(sum2[i & 1], pp);
+          w[i] = pack_bf16x2(pp.x, pp.y);
         }
         tmem_st32(s_addr + hcol * 32, w);
       }
-      l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      l += (sum2[0].x + sum2[1].x) + (sum2[0].y + sum2[1].y);
       tc_fence_before();
       mbar_arrive(&bars->p_full[x]);
     }
