@@ -23,7 +23,10 @@
 //    operand of O^T += V^T P^T with movmatrix, and V^T comes from ldmatrix
 //    .trans.  P is split into bf16 hi + lo parts so the product keeps ~16
 //    mantissa bits (the PV error then stays at fp32-accumulation level);
-//  * the four warps' partial (m, l, O) are merged through shared memory.
+//  * the four warps' partial (m, l, O) are merged through shared memory;
+//  * when an unsplit grid spans several waves (many sequences of mixed
+//    lengths), a one-CTA prepass orders the sequences longest-first so the
+//    long ones do not form the tail.
 // At G <= 8 the whole per-token arithmetic is 2 tensor-core tiles, so the
 // loop stays bound by HBM rather than by the FP32 pipes (a CUDA-core dot
 // product would need ~2 G FMA per byte-pair, near the B200's FP32 ridge at
@@ -35,18 +38,26 @@
 
 namespace pa {
 
-constexpr int kDecStages = 12;
 constexpr int kDecThreads = 160;  // 4 consumer warps + 1 producer warp
+// Ring depth.  Block i of a CTA goes to consumer warp i % 4 and stage
+// i % stages; with a multiple of 4 stages every stage belongs to one warp, so
+// its rounds are waited on in order (a parity wait can only tell the current
+// round from the previous one).  12 stages x 8 KB keep 96 KB in flight per
+// CTA at 2 CTAs per SM (measured best of 4, 6 and 12 on the decode workloads).
+constexpr int kRingStages = 12;
 constexpr int kStageBytes = 8192;  // K tile 4 KB + V tile 4 KB
 constexpr float kLog2eF = 1.4426950408889634f;
 
+template <int kDecStages>
 struct DecodeSmemTail {
+  static_assert(kDecStages % 4 == 0, "stages must be a multiple of the 4 consumer warps");
   uint64_t full[kDecStages];
   uint64_t empty[kDecStages];
   int stage_bad[kDecStages];
   int any_bad;
 };
 
+template <int kDecStages>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_mma_kernel(
     const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const DecodeArgs p,
@@ -54,11 +65,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_mma_kernel(
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-  DecodeSmemTail* tail =
-      reinterpret_cast<DecodeSmemTail*>(smem + kDecStages * kStageBytes);
+  DecodeSmemTail<kDecStages>* tail =
+      reinterpret_cast<DecodeSmemTail<kDecStages>*>(smem + kDecStages * kStageBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int part = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int part = blockIdx.x, kvh = blockIdx.y;
+  const int b = p.order ? p.order[blockIdx.z] : int(blockIdx.z);
   const int G = p.H / p.Hkv;
   const int kv_len = p.kv_lens[b];
   const bool len_bad = kv_len < 0 || kv_len > p.MB * 16;
@@ -315,6 +327,43 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
   out[bh * 128 + t] = den > 0.f ? num / den : 0.f;
 }
 
+// Longest-first order of the sequences (counting sort on the block count,
+// descending; one CTA).  Launching long sequences first keeps them from
+// forming the tail of a ragged batch; the result of each sequence does not
+// depend on when its CTAs run.
+constexpr int kOrderBuckets = 4096;
+__global__ void __launch_bounds__(1024) decode_order_kernel(const int32_t* __restrict__ kv_lens,
+                                                            int B, int32_t* __restrict__ order) {
+  __shared__ int count[kOrderBuckets];
+  for (int i = threadIdx.x; i < kOrderBuckets; i += blockDim.x) count[i] = 0;
+  __syncthreads();
+  auto bucket = [&](int b) {
+    const int L = kv_lens[b];
+    const int nb = L > 0 ? (L + 15) >> 4 : 0;
+    return kOrderBuckets - 1 - min(nb, kOrderBuckets - 1);   // descending
+  };
+  for (int b = threadIdx.x; b < B; b += blockDim.x) atomicAdd(&count[bucket(b)], 1);
+  __syncthreads();
+  if (threadIdx.x == 0) {                       // exclusive prefix sum
+    int run = 0;
+    for (int i = 0; i < kOrderBuckets; ++i) {
+      const int c = count[i];
+      count[i] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < B; b += blockDim.x) order[atomicAdd(&count[bucket(b)], 1)] = b;
+}
+
+// Only unsplit grids of several waves are reordered: split grids already cut
+// long sequences into partitions, one wave runs everything at once anyway.
+bool decode_wants_order(int32_t B, int32_t Hkv, int32_t NP, int sms) {
+  return NP == 1 && int64_t(B) * Hkv > 2 * int64_t(sms);
+}
+
+size_t order_workspace_bytes(int32_t B) { return sizeof(int32_t) * size_t(B); }
+
 bool decode_fast_supported(int dtype_bf16, int d, int bs, int G) {
   return dtype_bf16 && d == 128 && bs == 16 && G >= 1 && G <= 8;
 }
@@ -324,22 +373,33 @@ size_t split_workspace_bytes(int32_t B, int32_t H, int32_t NP, int32_t d) {
   return sizeof(float) * size_t(B) * H * NP * (2 + size_t(d));
 }
 
-cudaError_t launch_decode_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
-                               const DecodeArgs& a, int sms,
-                               cudaStream_t stream) {
-  (void)sms;
-  const size_t smem = 1024 + kDecStages * kStageBytes + sizeof(DecodeSmemTail);
+template <int NST>
+static cudaError_t launch_ring(const CUtensorMap* tmK, const CUtensorMap* tmV,
+                               const DecodeArgs& a, cudaStream_t stream) {
+  const size_t smem = 1024 + NST * kStageBytes + sizeof(DecodeSmemTail<NST>);
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(
-        decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NST>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   dim3 grid(a.NP, a.Hkv, a.B);
-  decode_mma_kernel<<<grid, kDecThreads, smem, stream>>>(*tmK, *tmV, a,
-                                                          a.scale * kLog2eF);
-  cudaError_t e = cudaGetLastError();
+  decode_mma_kernel<NST><<<grid, kDecThreads, smem, stream>>>(*tmK, *tmV, a,
+                                                              a.scale * kLog2eF);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
+                               const DecodeArgs& a, int sms,
+                               cudaStream_t stream) {
+  (void)sms;
+  if (a.order) {
+    decode_order_kernel<<<1, 1024, 0, stream>>>(a.kv_lens, a.B, a.order);
+    cudaError_t eo = cudaGetLastError();
+    if (eo != cudaSuccess) return eo;
+  }
+  cudaError_t e = launch_ring<kRingStages>(tmK, tmV, a, stream);
   if (e != cudaSuccess || a.NP == 1) return e;
   decode_combine_kernel<<<a.B * a.H, 128, 0, stream>>>(a.ws, a.B, a.H, a.NP,
                                                        a.out);

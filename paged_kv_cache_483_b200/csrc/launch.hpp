@@ -49,12 +49,16 @@ struct DecodeArgs {
   float* out;           // [B, H, 128]
   float* ws;            // split scratch (NP > 1)
   int32_t* err;
+  int32_t* order;       // longest-first sequence order (device, [B]) or null
 };
 bool decode_fast_supported(int dtype_bf16, int d, int bs, int G);
 cudaError_t launch_decode_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
                                const DecodeArgs& a, int sms,
                                cudaStream_t stream);
 size_t split_workspace_bytes(int32_t B, int32_t H, int32_t NP, int32_t d);
+// Scratch for the longest-first order when the grid spans several waves.
+bool decode_wants_order(int32_t B, int32_t Hkv, int32_t NP, int sms);
+size_t order_workspace_bytes(int32_t B);
 
 // Chunked prefill on tcgen05 tensor cores (bf16, head_dim 128, block 16).
 struct PrefillArgs {

@@ -414,7 +414,10 @@ size_t pa_decode_workspace_bytes(const pa_pool* p, int32_t B, int32_t H,
   if (!use_fast_decode(p, H)) return 0;
   int32_t pb = 0, np = 1;
   if (!decode_partitions(p, B, max_blocks, partition_tokens, &pb, &np)) return 0;
-  return pa::split_workspace_bytes(B, H, np, p->head_dim);
+  size_t bytes = pa::split_workspace_bytes(B, H, np, p->head_dim);
+  if (pa::decode_wants_order(B, p->num_kv_heads, np, p->sms))
+    bytes += pa::order_workspace_bytes(B);
+  return bytes;
 }
 
 int32_t pa_decode_path(const pa_pool* p, int32_t H) {
@@ -454,9 +457,13 @@ pa_status pa_decode(pa_pool* p, const void* q, int32_t B, int32_t H,
     pa::DecodeArgs a{};
     if (!decode_partitions(p, B, max_blocks, partition_tokens, &a.part_blocks, &a.NP))
       return PA_ERR_INVALID_ARG;
-    const size_t need = pa::split_workspace_bytes(B, H, a.NP, p->head_dim);
+    const size_t split_bytes = pa::split_workspace_bytes(B, H, a.NP, p->head_dim);
+    const bool order = pa::decode_wants_order(B, p->num_kv_heads, a.NP, p->sms);
+    const size_t need = split_bytes + (order ? pa::order_workspace_bytes(B) : 0);
     if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
       return PA_ERR_INVALID_ARG;
+    a.order = order ? reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + split_bytes)
+                    : nullptr;
     a.q = q;
     a.tables = d_block_tables;
     a.MB = max_blocks;
