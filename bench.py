@@ -256,8 +256,10 @@ def run_ours(args, dist):
     part = w.partition_tokens
     stream = torch.cuda.current_stream(device)
 
-    split = (not is_prefill) and pool.decode_workspace_bytes(
-        S.q.shape[0], S.q.shape[1], S.tables.shape[1], part) > 0
+    ws_bytes = 0 if is_prefill else pool.decode_workspace_bytes(
+        S.q.shape[0], S.q.shape[1], S.tables.shape[1], part)
+    split = ws_bytes > 0                    # a second launch: order prepass or combine
+    order_only = ws_bytes == 4 * S.q.shape[0]
     per_step = (1 if S.n_cow else 0) + (1 if S.slots is not None else 0) + (2 if split else 1)
     launches = {"n": 0}
 
@@ -328,7 +330,9 @@ def run_ours(args, dist):
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4),
                 "traffic": profiled_traffic("decode_mma.cu", w.name),
-                "kernel": "decode_mma_kernel" + (" + decode_combine_kernel" if split else ""),
+                "kernel": ("decode_order_kernel + decode_mma_kernel" if order_only else
+                           "decode_mma_kernel + decode_combine_kernel" if split else
+                           "decode_mma_kernel"),
                 "kernel_ms": round(kern_ms, 5),
                 "algorithmic_bytes_per_launch": kv, "peak_source": f"{peak_kind} hbm_gbs"}
         extra = {"seqs_per_s": round(dist.world * len(w.decode_seqs) / (ms_step_max * 1e-3), 1),

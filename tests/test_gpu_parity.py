@@ -246,3 +246,40 @@ def test_full_prefill_sampled():
             worst = max(worst, float(np.abs(out[i, rows, h] - r[rows]).max()))
     assert worst <= TOL_PREFILL, worst
     assert g.pool.get_error() == 0
+
+
+def test_prefill_device_errors_zero_rows():
+    w = workloads.prefill(seed=41, batch=2, cached=100, chunk=70)
+    g = GpuRun(w).apply(w.setup + w.step)
+    tables, lens, _, _ = g.tables()
+    q = w.queries().contiguous().cuda()
+    assert g.pool.prefill_path(32) == 1
+    bad = tables.clone()
+    bad[1, 2] = w.num_blocks + 3
+    out = g.pool.prefill_chunk(q, bad, lens)
+    assert g.pool.get_error() & pa.PA_DEVERR_BLOCK_ID
+    assert torch.all(out[1] == 0) and torch.any(out[0] != 0)
+    short = lens.clone()
+    short[0] = 50                                        # fewer keys than the chunk
+    out = g.pool.prefill_chunk(q, tables, short)
+    assert g.pool.get_error() & pa.PA_DEVERR_KV_LEN
+    assert torch.all(out[0] == 0) and torch.any(out[1] != 0)
+    assert g.pool.get_error() == 0
+
+
+def test_prefill_uninitialised_pool_is_safe():
+    # stale slots past the sequence end (NaN / Inf bit patterns) must not leak
+    w = workloads.prefill(seed=43, batch=2, cached=37, chunk=60)
+    g = GpuRun(w, init="empty")
+    g.k_cache.fill_(float("nan"))
+    g.v_cache.fill_(float("inf"))
+    g.apply(w.setup + w.step)
+    o = OracleRun(w).apply(w.setup + w.step)
+    out = g.prefill()
+    q = q64(w)
+    worst = 0.0
+    for i in range(2):
+        for h, ref in o.attention(i, q[i]).items():
+            worst = max(worst, float(np.abs(out[i, :, h] - ref).max()))
+    assert np.isfinite(out).all()
+    assert worst <= TOL_PREFILL, worst
