@@ -39,7 +39,9 @@ namespace pa {
 
 namespace {
 
-constexpr int kPfThreads = 320;
+constexpr int kPfThreads = 384;      // 3 warpgroups: control, softmax A, softmax B
+constexpr int kCtrlRegs = 64;        // 128 x 64 + 256 x 216 <= 384 x 168 at launch
+constexpr int kSoftmaxRegs = 216;
 constexpr int kPfStages = 2;
 constexpr uint32_t kTile = 32768;  // 128 x 128 bf16
 constexpr uint32_t kHalf = 16384;  // 128 x 64 bf16 (one 128-byte-swizzled half)
@@ -165,6 +167,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
   tc_fence_after();
   const uint32_t tbase = bars->tmem_base;
 
+  if (warp < 4) {
+  regs_dealloc<kCtrlRegs>();
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
     if (lane == 0) {
@@ -273,9 +277,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
       }
       umma_commit(&bars->o_final);
     }
+  }
   } else {
     // ------------------------------------------------ softmax / epilogue
-    const int x = (warp - 2) >> 2;                     // query tile A (0) or B (1)
+    regs_alloc<kSoftmaxRegs>();
+    const int x = (warp - 4) >> 2;                     // query tile A (0) or B (1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                 // row = TMEM lane
     const int t_local = r / G, g = r % G;
