@@ -309,25 +309,39 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
       }
-      float mx8[8];
+      const float2 sl2 = make_float2(scale_log2, scale_log2);
+      // P = 2^(s*scale - m_ref) as bf16 pairs over the first 64 columns of S;
+      // returns the row sum of this tile's P
+      auto write_p = [&](float mref) -> float {
+        float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float2 nm2 = make_float2(-mref, -mref);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(s[i], s[i + 8]);
+        for (int hcol = 0; hcol < 2; ++hcol) {
+          uint32_t w[32];
 #pragma unroll
-      for (int c = 16; c < 128; c += 16)
+          for (int i = 0; i < 32; ++i) {
+            const float2 e = __ffma2_rn(
+                make_float2(s[hcol * 64 + 2 * i], s[hcol * 64 + 2 * i + 1]), sl2, nm2);
+            const float2 pp = make_float2(ex2(e.x), ex2(e.y));
+            sum2[i & 1] = __fadd2_rn(sum2[i & 1], pp);
+            w[i] = pack_bf16x2(pp.x, pp.y);
+          }
+          tmem_st32(s_addr + hcol * 32, w);
+        }
+        return (sum2[0].x + sum2[1].x) + (sum2[0].y + sum2[1].y);
+      };
+      auto row_max = [&]() -> float {
+        float mx8[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = max3(mx8[i], s[c + i], s[c + 8 + i]);
-      const float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]),
-                            fmaxf(mx8[6], mx8[7]));
-      const float mt = mx * scale_log2;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (mt != -INFINITY && (m_ref == -INFINITY || mt > m_ref + kRescaleTau)) {
-        alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mt);
-        rescale = (j > 0);
-        m_ref = mt;
-      }
-      // PV_x(j-1) has completed (it precedes QK_x(j) on the tensor core)
-      if (__any_sync(0xffffffffu, rescale)) {
+        for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(s[i], s[i + 8]);
+#pragma unroll
+        for (int c = 16; c < 128; c += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx8[i] = max3(mx8[i], s[c + i], s[c + 8 + i]);
+        return max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]),
+                    fmaxf(mx8[6], mx8[7])) * scale_log2;
+      };
+      auto rescale_o = [&](float alpha) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
@@ -336,11 +350,46 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
           for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
           tmem_st32(o_addr + c * 32, v);
         }
+      };
+      // PV_x(j-1) has completed (it precedes QK_x(j) on the tensor core), so
+      // O_x may be rescaled here.
+      float tile_sum;
+      if (!__any_sync(0xffffffffu, m_ref == -INFINITY)) {
+        // Speculative: exponentiate against the current reference max while
+        // the row max is formed in the same pass; only a row whose max grew
+        // by more than 2^8 makes the warp rescale O and redo P.
+        tile_sum = write_p(m_ref);
+        const float mt = row_max();
+        const bool grow = mt > m_ref + kRescaleTau;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float alpha = grow ? ex2(m_ref - mt) : 1.f;
+          if (grow) m_ref = mt;
+          rescale_o(alpha);
+          l *= alpha;
+          tile_sum = write_p(m_ref);
+        }
+      } else {
+        // a row without a visible key so far: its reference max comes first
+        const float mt = row_max();
+        float alpha = 1.f;
+        bool grow = false;
+        if (mt != -INFINITY) {
+          if (m_ref == -INFINITY) {
+            alpha = 0.f;
+            m_ref = mt;
+          } else if (mt > m_ref + kRescaleTau) {
+            alpha = ex2(m_ref - mt);
+            m_ref = mt;
+            grow = true;
+          }
+        }
+        if (__any_sync(0xffffffffu, grow)) rescale_o(alpha);
+        l *= alpha;
+        tile_sum = write_p(m_ref == -INFINITY ? 0.f : m_ref);
       }
-      l *= alpha;
       if (x == 0 && j == n_tiles - 1) {
         // V rows at or past key_end hold stale bytes: zero them (p = 0 there,
-        // and 0 x NaN would poison the product); PV_B is issued after PV_A
+        // and 0 x NaN would poison the product); PV_B follows PV_A
         const int st = j % kPfStages;
         const bool landed = warp_wait(&bars->v_full[st], (j / kPfStages) & 1, bars, p.err, lane);
         if (landed && j * 128 + r >= key_end) {
@@ -354,24 +403,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
         }
         fence_proxy_async_smem();
       }
-      // P = 2^(s*scale - m_ref) as bf16 pairs, written over S_x in TMEM
-      float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      const float2 sl2 = make_float2(scale_log2, scale_log2);
-      const float2 nm2 = make_float2(-m_ref, -m_ref);
-#pragma unroll
-      for (int hcol = 0; hcol < 2; ++hcol) {
-        uint32_t w[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 e = __ffma2_rn(make_float2(s[hcol * 64 + 2 * i], s[hcol * 64 + 2 * i + 1]),
-                                      sl2, nm2);
-          const float2 pp = make_float2(ex2(e.x), ex2(e.y));
-          sum2[i & 1] = __fadd2_rn(sum2[i & 1], pp);
-          w[i] = pack_bf16x2(pp.x, pp.y);
-        }
-        tmem_st32(s_addr + hcol * 32, w);
-      }
-      l += (sum2[0].x + sum2[1].x) + (sum2[0].y + sum2[1].y);
+      l += tile_sum;
       tc_fence_before();
       mbar_arrive(&bars->p_full[x]);
     }
