@@ -42,9 +42,11 @@ constexpr int kDecThreads = 160;  // 4 consumer warps + 1 producer warp
 // Ring depth.  Block i of a CTA goes to consumer warp i % 4 and stage
 // i % stages; with a multiple of 4 stages every stage belongs to one warp, so
 // its rounds are waited on in order (a parity wait can only tell the current
-// round from the previous one).  12 stages x 8 KB keep 96 KB in flight per
-// CTA at 2 CTAs per SM (measured best of 4, 6 and 12 on the decode workloads).
-constexpr int kRingStages = 12;
+// round from the previous one).  8 stages x 8 KB (64 KB) with 125 registers
+// fit 3 CTAs per SM: 192 KB in flight per SM, and more resident CTAs to hide
+// the per-CTA latency of short sequences (measured against 4 and 12 stages at
+// 2 CTAs per SM: equal at 8K context, +5 % on the ragged batch, +2 % split-K).
+constexpr int kRingStages = 8;
 constexpr int kStageBytes = 8192;  // K tile 4 KB + V tile 4 KB
 constexpr float kLog2eF = 1.4426950408889634f;
 
@@ -58,7 +60,7 @@ struct DecodeSmemTail {
 };
 
 template <int kDecStages>
-__global__ void __launch_bounds__(kDecThreads, 2) decode_mma_kernel(
+__global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_mma_kernel(
     const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const DecodeArgs p,
     float scale_log2) {
