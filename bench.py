@@ -4,8 +4,8 @@
 Default workload (the headline metric): decode batch 32 at 8K context, GQA
 32/8, head_dim 128, block 16, bf16 K/V/Q, a 16384-block pool in a seeded
 permuted order.  One step = append of every sequence's new token (K/V written
-by reshape_and_cache at the slots the host manager planned for position 8191)
-followed by paged decode attention at kv_len 8192.  The host plan itself is
+at the slots the host manager planned for position 8191) and paged decode
+attention at kv_len 8192, fused in one kernel (pa_decode_append).  The host plan itself is
 timed separately (``host_plan_us``) because a repeated step must rewrite the
 same slots.
 
@@ -260,18 +260,24 @@ def run_ours(args, dist):
         S.q.shape[0], S.q.shape[1], S.tables.shape[1], part)
     split = ws_bytes > 0                    # a second launch: order prepass or combine
     order_only = ws_bytes == 4 * S.q.shape[0]
-    per_step = (1 if S.n_cow else 0) + (1 if S.slots is not None else 0) + (2 if split else 1)
+    # decode steps fuse the new token's append into the decode kernel
+    fused = (not is_prefill) and S.slots is not None
+    per_step = ((1 if S.n_cow else 0) + (1 if (S.slots is not None and not fused) else 0)
+                + (2 if split else 1))
     launches = {"n": 0}
 
     def step(ev_pair=None):
         if S.n_cow:
             pool.cow_copy(S.cow_src, S.cow_dst, stream)
-        if S.slots is not None:
+        if S.slots is not None and not fused:
             pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
         if ev_pair is not None:
             ev_pair[0].record(stream)
         if is_prefill:
             pool.prefill_chunk(S.q, S.tables, S.lens, out=S.out, stream=stream)
+        elif fused:
+            pool.decode_append(S.q, S.step_k, S.step_v, S.slots, S.tables, S.lens, out=S.out,
+                               partition_tokens=part, stream=stream)
         else:
             pool.decode(S.q, S.tables, S.lens, out=S.out, partition_tokens=part, stream=stream)
         if ev_pair is not None:
@@ -398,9 +404,13 @@ def run_e2e(args, S, dist, device, is_prefill, part):
             d_slots.copy_(h_slots, non_blocking=True)
             if S.n_cow:
                 pool.cow_copy(S.cow_src, S.cow_dst, stream)
-            pool.reshape_and_cache(d_k, d_v, d_slots, stream)
+            if is_prefill:
+                pool.reshape_and_cache(d_k, d_v, d_slots, stream)
         if is_prefill:
             pool.prefill_chunk(d_q, S.tables, d_lens, out=S.out, stream=stream)
+        elif h_k is not None:
+            pool.decode_append(d_q, d_k, d_v, d_slots, S.tables, d_lens, out=S.out,
+                               partition_tokens=part, stream=stream)
         else:
             pool.decode(d_q, S.tables, d_lens, out=S.out, partition_tokens=part, stream=stream)
         h_out.copy_(S.out, non_blocking=True)

@@ -223,6 +223,24 @@ pa_status pa_decode(pa_pool* pool, const void* q, int32_t B, int32_t H,
                     int32_t partition_tokens, void* workspace,
                     size_t workspace_bytes, float* out, void* stream);
 
+/* Decode step with the new token's append fused in: for each sequence b,
+ * token kv_lens[b] - 1 is the one being decoded; its K/V rows
+ * key[b]/value[b] (device [B, Hkv, head_dim], pool dtype) are written to pool
+ * slot d_slot_mapping[b] (device [B] int64, from pa_plan_append; negative =
+ * no write) and attended in the same pass -- the result equals
+ * pa_reshape_and_cache followed by pa_decode ([P1] append, then Eq. 3).
+ * Tables and kv_lens already include the new token; a copy-on-write the plan
+ * asked for must have been issued (pa_cow_copy) on the same stream before.
+ * On the tensor-core path it is one kernel; elsewhere the two calls.
+ * Other arguments, workspace and errors as pa_decode. */
+pa_status pa_decode_append(pa_pool* pool, const void* q, const void* key,
+                           const void* value, const int64_t* d_slot_mapping,
+                           int32_t B, int32_t H, const int32_t* d_block_tables,
+                           int32_t max_blocks, const int32_t* d_kv_lens,
+                           float scale, int32_t partition_tokens,
+                           void* workspace, size_t workspace_bytes, float* out,
+                           void* stream);
+
 /* Chunked prefill attention ([P3] with q_tokens > 1): for each sequence b
  * the chunk's q_tokens queries are its last q_tokens positions; query qt
  * sees cached positions j <= kv_lens[b] - q_tokens + qt.  The chunk's own

@@ -31,7 +31,7 @@ EXPORTS = ["pa_pool_create", "pa_free", "pa_seq_create", "pa_seq_fork", "pa_seq_
            "pa_refcounts", "pa_validate", "pa_append_kv", "pa_reshape_and_cache",
            "pa_cow_copy", "pa_decode_workspace_bytes", "pa_decode", "pa_prefill_chunk",
            "pa_get_error", "pa_status_string", "pa_decode_path", "pa_prefill_path",
-           "pa_decode_static_scratch"]
+           "pa_decode_static_scratch", "pa_decode_append"]
 
 
 class PAError(RuntimeError):
@@ -83,6 +83,8 @@ def lib():
         "pa_decode_path": ([_P, _I32], _I32),
         "pa_prefill_path": ([_P, _I32], _I32),
         "pa_decode_static_scratch": ([_P, _P, _I32, _I32, _P, _I32, _P, _F, _I32, _P, _P], C.c_int),
+        "pa_decode_append": ([_P, _P, _P, _P, _P, _I32, _I32, _P, _I32, _P, _F, _I32, _P, _SZ, _P,
+                              _P], C.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -286,6 +288,34 @@ class Pool:
                                workspace.numel() if need else 0,
                                _dev_ptr(out, torch.float32, "out"), _stream(stream)),
                "pa_decode")
+        return out
+
+    def decode_append(self, q, key, value, slot_mapping, block_tables, kv_lens, out=None,
+                      scale=None, partition_tokens=0, workspace=None, stream=None):
+        """Fused step: write each sequence's new token (key/value [B, Hkv, d]
+        at slot_mapping [B] int64) and decode q [B, H, d] over kv_lens."""
+        import torch
+        B, H, d = q.shape
+        MB = block_tables.shape[1]
+        if out is None:
+            out = torch.empty((B, H, d), dtype=torch.float32, device=q.device)
+        scale = 1.0 / math.sqrt(self.head_dim) if scale is None else scale
+        need = self.decode_workspace_bytes(B, H, MB, partition_tokens)
+        if need and workspace is None:
+            if self._ws is None or self._ws.numel() < need:
+                self._ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+            workspace = self._ws
+        wp = _dev_ptr(workspace, None, "workspace") if need else None
+        dt = self._torch_dtype()
+        _check(lib().pa_decode_append(self._h, _dev_ptr(q, dt, "q"), _dev_ptr(key, dt, "key"),
+                                      _dev_ptr(value, dt, "value"),
+                                      _dev_ptr(slot_mapping, torch.int64, "slot_mapping"), B, H,
+                                      _dev_ptr(block_tables, torch.int32, "block_tables"), MB,
+                                      _dev_ptr(kv_lens, torch.int32, "kv_lens"), float(scale),
+                                      int(partition_tokens), wp,
+                                      workspace.numel() if need else 0,
+                                      _dev_ptr(out, torch.float32, "out"), _stream(stream)),
+               "pa_decode_append")
         return out
 
     def prefill_chunk(self, q, block_tables, kv_lens, out=None, scale=None, stream=None):

@@ -133,6 +133,25 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
   }
 
   // ------------------------------------------------------------- consumers
+  // Fused append: the CTA whose partition holds token kv_len-1 writes that
+  // token's K/V row of its KV head into the pool (and patches it into the
+  // staged tile below, so the TMA copy of the stale slot is never used).
+  const bool appends = p.new_k != nullptr && nblk > 0 && blk0 + nblk == nblk_seq;
+  const int64_t new_slot = appends ? p.new_slots[b] : -1;
+  if (appends && warp == 0) {
+    if (new_slot >= int64_t(p.NB) * 16) {
+      if (lane == 0) raise_err(p.err, PA_DEVERR_SLOT);
+    } else if (new_slot >= 0) {
+      const int64_t src = (int64_t(b) * p.Hkv + kvh) * 16;        // uint4 units
+      const int64_t dst = (new_slot * p.Hkv + kvh) * 16;
+      if (lane < 16)
+        reinterpret_cast<uint4*>(p.k_cache)[dst + lane] =
+            reinterpret_cast<const uint4*>(p.new_k)[src + lane];
+      else
+        reinterpret_cast<uint4*>(p.v_cache)[dst + lane - 16] =
+            reinterpret_cast<const uint4*>(p.new_v)[src + lane - 16];
+    }
+  }
   const int g = lane >> 2, c = lane & 3;
   uint32_t qb[8][2];
   {
@@ -172,6 +191,16 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
       const uint32_t kb = smem_u32(smem + s * kStageBytes);
       const uint32_t vb = kb + 4096;
       const int valid = min(16, tok_end - (blk0 + i) * 16);
+      if (appends && new_slot >= 0 && new_slot < int64_t(p.NB) * 16 && blk0 + i == nblk_seq - 1) {
+        // the new token's row: 2 x 128 bytes in each of the K and V tiles
+        const int row = valid - 1, ch = lane & 15;
+        const uint4* src = reinterpret_cast<const uint4*>(lane < 16 ? p.new_k : p.new_v) +
+                           (int64_t(b) * p.Hkv + kvh) * 16;
+        uint8_t* tile = smem + s * kStageBytes + (lane < 16 ? 0 : 4096);
+        *reinterpret_cast<uint4*>(tile + (ch >> 3) * 2048 + swz128(row, ch & 7)) = src[ch];
+        fence_proxy_async_smem();  // a later TMA refill of this stage comes after it
+        __syncwarp();
+      }
       if (valid < 16) {
         // slots past the sequence end hold stale bytes (possibly NaN
         // patterns); zero their V rows so p = 0 contributes exactly 0

@@ -50,6 +50,13 @@ struct DecodeArgs {
   float* ws;            // split scratch (NP > 1)
   int32_t* err;
   int32_t* order;       // longest-first sequence order (device, [B]) or null
+  // fused append (all null/0 when off): token kv_len-1 of sequence b is new;
+  // its K/V rows new_k/new_v [B, Hkv, 128] go to pool slot new_slots[b]
+  const void* new_k;
+  const void* new_v;
+  const int64_t* new_slots;
+  void* k_cache;
+  void* v_cache;
 };
 bool decode_fast_supported(int dtype_bf16, int d, int bs, int G);
 cudaError_t launch_decode_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,

@@ -428,6 +428,44 @@ int32_t pa_prefill_path(const pa_pool* p, int32_t H) {
   return (p && use_fast_prefill(p, H)) ? 1 : 0;
 }
 
+static pa_status decode_fast(pa_pool* p, const void* q, int32_t B, int32_t H,
+                             const int32_t* d_block_tables, int32_t max_blocks,
+                             const int32_t* d_kv_lens, float scale, int32_t partition_tokens,
+                             void* workspace, size_t workspace_bytes, float* out,
+                             void* stream, const void* new_k, const void* new_v,
+                             const int64_t* new_slots) {
+  if (!aligned16(q)) return PA_ERR_INVALID_ARG;
+  pa::DecodeArgs a{};
+  if (!decode_partitions(p, B, max_blocks, partition_tokens, &a.part_blocks, &a.NP))
+    return PA_ERR_INVALID_ARG;
+  const size_t split_bytes = pa::split_workspace_bytes(B, H, a.NP, p->head_dim);
+  const bool order = pa::decode_wants_order(B, p->num_kv_heads, a.NP, p->sms);
+  const size_t need = split_bytes + (order ? pa::order_workspace_bytes(B) : 0);
+  if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return PA_ERR_INVALID_ARG;
+  a.order = order ? reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + split_bytes)
+                  : nullptr;
+  a.q = q;
+  a.tables = d_block_tables;
+  a.MB = max_blocks;
+  a.kv_lens = d_kv_lens;
+  a.B = B;
+  a.H = H;
+  a.Hkv = p->num_kv_heads;
+  a.NB = p->num_blocks;
+  a.scale = scale;
+  a.out = out;
+  a.ws = static_cast<float*>(workspace);
+  a.err = p->d_err;
+  a.new_k = new_k;
+  a.new_v = new_v;
+  a.new_slots = new_slots;
+  a.k_cache = p->k_cache;
+  a.v_cache = p->v_cache;
+  return cuda_status(pa::launch_decode_fast(&p->tmK, &p->tmV, a, p->sms,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 static pa_status check_attention_args(const pa_pool* p, const void* q, int32_t B,
                                       int32_t H, const int32_t* tables,
                                       int32_t MB, const int32_t* kv_lens,
@@ -452,38 +490,39 @@ pa_status pa_decode(pa_pool* p, const void* q, int32_t B, int32_t H,
   if (partition_tokens < 0) return PA_ERR_INVALID_ARG;
   if (B == 0) return PA_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (use_fast_decode(p, H)) {
-    if (!aligned16(q)) return PA_ERR_INVALID_ARG;
-    pa::DecodeArgs a{};
-    if (!decode_partitions(p, B, max_blocks, partition_tokens, &a.part_blocks, &a.NP))
-      return PA_ERR_INVALID_ARG;
-    const size_t split_bytes = pa::split_workspace_bytes(B, H, a.NP, p->head_dim);
-    const bool order = pa::decode_wants_order(B, p->num_kv_heads, a.NP, p->sms);
-    const size_t need = split_bytes + (order ? pa::order_workspace_bytes(B) : 0);
-    if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
-      return PA_ERR_INVALID_ARG;
-    a.order = order ? reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + split_bytes)
-                    : nullptr;
-    a.q = q;
-    a.tables = d_block_tables;
-    a.MB = max_blocks;
-    a.kv_lens = d_kv_lens;
-    a.B = B;
-    a.H = H;
-    a.Hkv = p->num_kv_heads;
-    a.NB = p->num_blocks;
-    a.scale = scale;
-    a.out = out;
-    a.ws = static_cast<float*>(workspace);
-    a.err = p->d_err;
-    return cuda_status(pa::launch_decode_fast(&p->tmK, &p->tmV, a, p->sms, s));
-  }
+  if (use_fast_decode(p, H))
+    return decode_fast(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale,
+                       partition_tokens, workspace, workspace_bytes, out, stream, nullptr,
+                       nullptr, nullptr);
   if (partition_tokens % p->block_size) return PA_ERR_INVALID_ARG;
   pa::GenericArgs g{q, p->k_cache, p->v_cache, d_block_tables, max_blocks,
                     d_kv_lens, B, 1, H, p->num_kv_heads, p->head_dim,
                     p->block_size, p->num_blocks, scale, out, p->d_err,
                     p->dtype == PA_BF16};
   return cuda_status(pa::launch_attention_generic(g, s));
+}
+
+pa_status pa_decode_append(pa_pool* p, const void* q, const void* key, const void* value,
+                           const int64_t* d_slot_mapping, int32_t B, int32_t H,
+                           const int32_t* d_block_tables, int32_t max_blocks,
+                           const int32_t* d_kv_lens, float scale, int32_t partition_tokens,
+                           void* workspace, size_t workspace_bytes, float* out, void* stream) {
+  pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, out);
+  if (st != PA_OK) return st;
+  if (B > 0 && (!key || !value || !d_slot_mapping)) return PA_ERR_INVALID_ARG;
+  if (partition_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (B == 0) return PA_OK;
+  if (!use_fast_decode(p, H)) {
+    // same result in two launches on the other paths
+    st = pa_reshape_and_cache(p, key, value, d_slot_mapping, B, stream);
+    if (st != PA_OK) return st;
+    return pa_decode(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale,
+                     partition_tokens, workspace, workspace_bytes, out, stream);
+  }
+  if (!aligned16(key) || !aligned16(value)) return PA_ERR_INVALID_ARG;
+  return decode_fast(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale,
+                     partition_tokens, workspace, workspace_bytes, out, stream, key, value,
+                     d_slot_mapping);
 }
 
 pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,

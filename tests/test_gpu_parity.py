@@ -283,3 +283,80 @@ def test_prefill_uninitialised_pool_is_safe():
             worst = max(worst, float(np.abs(out[i, :, h] - ref).max()))
     assert np.isfinite(out).all()
     assert worst <= TOL_PREFILL, worst
+
+
+def _fused_step(w, fused=True, init="zeros"):
+    """Setup through the library, then the step's one-token appends either
+    fused into the decode or as reshape_and_cache + decode."""
+    g = GpuRun(w, init=init).apply(w.setup)
+    seqs = [op.args[0] for op in w.step]
+    slots, cow = g.pool.plan_append(seqs, [1] * len(seqs))
+    if cow:
+        src = torch.tensor([c[0] for c in cow], dtype=torch.int32, device="cuda")
+        dst = torch.tensor([c[1] for c in cow], dtype=torch.int32, device="cuda")
+        g.pool.cow_copy(src, dst)
+    ks, vs = zip(*[w.kv_for(op) for op in w.step])
+    key = torch.cat(ks).cuda()
+    val = torch.cat(vs).cuda()
+    d_slots = torch.tensor(slots, dtype=torch.int64, device="cuda")
+    tables, lens, _, _ = g.tables()
+    q = w.queries()[:, 0].contiguous().cuda()
+    if fused:
+        out = g.pool.decode_append(q, key, val, d_slots, tables, lens)
+    else:
+        g.pool.reshape_and_cache(key, val, d_slots)
+        out = g.pool.decode(q, tables, lens)
+    torch.cuda.synchronize()
+    return g, out.cpu().numpy(), slots, key, val
+
+
+@pytest.mark.parametrize("H,Hkv", [(32, 8), (64, 8), (8, 8)])
+def test_decode_append_matches_oracle_and_two_calls(H, Hkv):
+    # new tokens land mid-block, at block starts (a fresh block) and at ends
+    lens = [1, 2, 16, 17, 32, 33, 300, 513, 1024, 1025]
+    w = workloads.custom_decode("fused", lens, H, Hkv, 128, 16, "bf16", seed=H + 3,
+                                spare_blocks=8, split_last=1)
+    g, out, slots, key, val = _fused_step(w, fused=True)
+    assert g.pool.decode_path(H) == 1
+    _, out2, _, _, _ = _fused_step(w, fused=False)
+    assert np.array_equal(out, out2)                       # same arithmetic, same order
+    o = OracleRun(w).apply(w.setup + w.step)
+    assert slots == o.slots[w.step[0].index] + sum((o.slots[op.index] for op in w.step[1:]), [])
+    q = q64(w)
+    worst = 0.0
+    for i in range(len(lens)):
+        for h, ref in o.attention(i, q[i]).items():
+            worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+    assert worst <= TOL_DECODE, worst
+    flat_k = g.k_cache.view(-1, Hkv, 128)
+    flat_v = g.v_cache.view(-1, Hkv, 128)
+    assert torch.equal(flat_k[torch.tensor(slots)], key) and torch.equal(flat_v[torch.tensor(slots)], val)
+    assert g.pool.get_error() == 0
+
+
+def test_decode_append_with_copy_on_write_and_stale_pool():
+    w = workloads.ragged256(groups=2, per_group=4, prefix=40, spare_blocks=8)
+    g, out, _, _, _ = _fused_step(w, fused=True, init="empty")
+    o = OracleRun(w).apply(w.setup + w.step)
+    assert any(o.cows.values())
+    q = q64(w)
+    worst = 0.0
+    for i in range(len(w.decode_seqs)):
+        for h, ref in o.attention(i, q[i]).items():
+            worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+    assert np.isfinite(out).all() and worst <= TOL_DECODE, worst
+    assert g.pool.get_error() == 0
+
+
+def test_decode_append_generic_path_fp32():
+    w = workloads.custom_decode("fused32", [5, 16, 40], 8, 2, 32, 8, "f32", seed=8,
+                                spare_blocks=4, split_last=1)
+    g, out, _, _, _ = _fused_step(w, fused=True)
+    assert g.pool.decode_path(8) == 0
+    o = OracleRun(w).apply(w.setup + w.step)
+    q = q64(w)
+    worst = 0.0
+    for i in range(3):
+        for h, ref in o.attention(i, q[i]).items():
+            worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+    assert worst <= TOL_F32, worst
