@@ -366,25 +366,48 @@ constexpr int kOrderBuckets = 4096;
 __global__ void __launch_bounds__(1024) decode_order_kernel(const int32_t* __restrict__ kv_lens,
                                                             int B, int32_t* __restrict__ order) {
   __shared__ int count[kOrderBuckets];
-  for (int i = threadIdx.x; i < kOrderBuckets; i += blockDim.x) count[i] = 0;
+  __shared__ int warp_tot[32];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  for (int i = tid; i < kOrderBuckets; i += blockDim.x) count[i] = 0;
   __syncthreads();
   auto bucket = [&](int b) {
     const int L = kv_lens[b];
     const int nb = L > 0 ? (L + 15) >> 4 : 0;
     return kOrderBuckets - 1 - min(nb, kOrderBuckets - 1);   // descending
   };
-  for (int b = threadIdx.x; b < B; b += blockDim.x) atomicAdd(&count[bucket(b)], 1);
+  for (int b = tid; b < B; b += blockDim.x) atomicAdd(&count[bucket(b)], 1);
   __syncthreads();
-  if (threadIdx.x == 0) {                       // exclusive prefix sum
-    int run = 0;
-    for (int i = 0; i < kOrderBuckets; ++i) {
-      const int c = count[i];
-      count[i] = run;
-      run += c;
+  // exclusive prefix sum: each thread owns 4 consecutive buckets
+  constexpr int kPer = kOrderBuckets / 1024;
+  int local[kPer], run = 0;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    local[k] = run;
+    run += count[tid * kPer + k];
+  }
+  int incl = run;                                  // inclusive scan across the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_tot[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    int t = warp_tot[lane], it = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, it, o);
+      if (lane >= o) it += v;
     }
+    warp_tot[lane] = it - t;                       // exclusive warp offsets
   }
   __syncthreads();
-  for (int b = threadIdx.x; b < B; b += blockDim.x) order[atomicAdd(&count[bucket(b)], 1)] = b;
+  const int base = warp_tot[wid] + incl - run;     // exclusive start of this thread
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) count[tid * kPer + k] = base + local[k];
+  __syncthreads();
+  for (int b = tid; b < B; b += blockDim.x) order[atomicAdd(&count[bucket(b)], 1)] = b;
 }
 
 // Only unsplit grids of several waves are reordered: split grids already cut

@@ -101,7 +101,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, PfBars
 
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-    const __grid_constant__ CUtensorMap tmV, const PrefillArgs p, float scale_log2) {
+    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+    const PrefillArgs p, float scale_log2, int use_tma_store) {
   extern __shared__ uint8_t pf_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(pf_raw) + 1023) & ~uintptr_t(1023));
@@ -411,17 +412,44 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
     const bool done = ok && warp_wait(&bars->o_final, 0, bars, p.err, lane);
     tc_fence_after();
     const float inv = (done && l > 0.f) ? 1.f / l : 0.f;
-    float* orow = p.out + ((int64_t(b) * q_tokens + tok) * p.H + kvh * G + g) * 128;
+    if (use_tma_store && valid_tokens == 2 * TQ) {
+      // Both tiles are full: every MMA is done, so the whole shared memory is
+      // free.  Each row goes into four 32-column boxes with the 128-byte
+      // swizzle (conflict-free), then one thread per tile stores them with TMA.
+      uint8_t* stage = smem + x * 65536;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t v[32];
-      tmem_ld32(o_addr + c * 32, v);
-      if (row_valid) {
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(o_addr + c * 32, v);
+        uint8_t* box = stage + c * 16384;
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(orow + c * 32 + i) =
-              make_float4(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv,
-                          __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<float4*>(box + swz128(r, q4)) =
+              make_float4(__uint_as_float(v[4 * q4]) * inv, __uint_as_float(v[4 * q4 + 1]) * inv,
+                          __uint_as_float(v[4 * q4 + 2]) * inv,
+                          __uint_as_float(v[4 * q4 + 3]) * inv);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + x, 128);
+      if (r == 0) {
+        const int z = b * q_tokens + t0 + x * TQ;
+        for (int c = 0; c < 4; ++c) tma_store_3d(&tmO, stage + c * 16384, c * 32, kvh * G, z);
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+    } else {
+      float* orow = p.out + ((int64_t(b) * q_tokens + tok) * p.H + kvh * G + g) * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(o_addr + c * 32, v);
+        if (row_valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(orow + c * 32 + i) =
+                make_float4(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv,
+                            __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
+        }
       }
     }
   }
@@ -466,6 +494,22 @@ cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  // O viewed as {head_dim, H, B * q_tokens} fp32; one box = 32 columns of
+  // the tile's rows, 128-byte swizzle
+  CUtensorMap tmO;
+  int use_tma_store = 0;
+  {
+    const cuuint64_t odims[3] = {128, cuuint64_t(a.H), cuuint64_t(a.B) * a.q_tokens};
+    const cuuint64_t ostr[2] = {128 * 4, cuuint64_t(a.H) * 128 * 4};
+    const cuuint32_t obox[3] = {32, cuuint32_t(G), cuuint32_t(TQ)};
+    if ((reinterpret_cast<uintptr_t>(a.out) & 15) == 0 &&
+        fn(&tmO, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.out, odims, ostr, obox, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+      use_tma_store = 1;
+    else
+      tmO = tmQ;   // never used
+  }
   const size_t smem = 1024 + kDataBytes + sizeof(PfBars);
   static bool attr_set = false;
   if (!attr_set) {
@@ -475,8 +519,9 @@ cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
     attr_set = true;
   }
   dim3 grid((a.q_tokens + 2 * TQ - 1) / (2 * TQ), a.Hkv, a.B);
-  prefill_tc_kernel<<<grid, kPfThreads, smem, stream>>>(tmQ, *tmK, *tmV, a,
-                                                         a.scale * 1.4426950408889634f);
+  prefill_tc_kernel<<<grid, kPfThreads, smem, stream>>>(tmQ, *tmK, *tmV, tmO, a,
+                                                         a.scale * 1.4426950408889634f,
+                                                         use_tma_store);
   return cudaGetLastError();
 }
 
