@@ -247,12 +247,19 @@ pa_status pa_decode_append(pa_pool* pool, const void* q, const void* key,
  * K/V must already be in the pool (pa_append_kv).
  *   q: device [B, q_tokens, H, head_dim], pool dtype.  out: device
  *   [B, q_tokens, H, head_dim] float32.  Tables/kv_lens as pa_decode.
- * Errors: as pa_decode. */
+ *   max_kv_splits: on the tensor-core path, the query tiles of the last,
+ *   partial wave of CTAs may be split over their keys (at most this many
+ *   parts; 0 = automatic, up to 4; 1 = never) and merged with the [P4]
+ *   log-sum-exp rule, so that the wave fills the GPU.  The split uses
+ *   scratch owned by the pool (about 20 MB, allocated with it): calls on one
+ *   pool that overlap on the GPU (unordered streams) race on it unless they
+ *   pass 1.
+ * Errors: as pa_decode (INVALID_ARG also for max_kv_splits < 0). */
 pa_status pa_prefill_chunk(pa_pool* pool, const void* q, int32_t B,
                            int32_t q_tokens, int32_t H,
                            const int32_t* d_block_tables, int32_t max_blocks,
-                           const int32_t* d_kv_lens, float scale, float* out,
-                           void* stream);
+                           const int32_t* d_kv_lens, float scale,
+                           int32_t max_kv_splits, float* out, void* stream);
 
 /* Bytes of the fixed device scratch array used by pa_decode_static_scratch. */
 #define PA_STATIC_SCRATCH_BYTES (16u << 20)

@@ -77,7 +77,8 @@ def lib():
         "pa_cow_copy": ([_P, _P, _P, _I32, _P], C.c_int),
         "pa_decode_workspace_bytes": ([_P, _I32, _I32, _I32, _I32], _SZ),
         "pa_decode": ([_P, _P, _I32, _I32, _P, _I32, _P, _F, _I32, _P, _SZ, _P, _P], C.c_int),
-        "pa_prefill_chunk": ([_P, _P, _I32, _I32, _I32, _P, _I32, _P, _F, _P, _P], C.c_int),
+        "pa_prefill_chunk": ([_P, _P, _I32, _I32, _I32, _P, _I32, _P, _F, _I32, _P, _P],
+                             C.c_int),
         "pa_get_error": ([_P, _PI32], C.c_int),
         "pa_status_string": ([C.c_int], C.c_char_p),
         "pa_decode_path": ([_P, _I32], _I32),
@@ -318,8 +319,12 @@ class Pool:
                "pa_decode_append")
         return out
 
-    def prefill_chunk(self, q, block_tables, kv_lens, out=None, scale=None, stream=None):
-        """q [B, q_tokens, H, d] CUDA (pool dtype) -> out float32, same shape."""
+    def prefill_chunk(self, q, block_tables, kv_lens, out=None, scale=None, stream=None,
+                      max_kv_splits=0):
+        """q [B, q_tokens, H, d] CUDA (pool dtype) -> out float32, same shape.
+
+        max_kv_splits: 0 = split the last wave's query tiles over their keys
+        as the library chooses, 1 = never split, n = at most n parts."""
         import torch
         B, T, H, d = q.shape
         MB = block_tables.shape[1]
@@ -329,7 +334,8 @@ class Pool:
         _check(lib().pa_prefill_chunk(self._h, _dev_ptr(q, self._torch_dtype(), "q"), B, T, H,
                                       _dev_ptr(block_tables, torch.int32, "block_tables"), MB,
                                       _dev_ptr(kv_lens, torch.int32, "kv_lens"), float(scale),
-                                      _dev_ptr(out, torch.float32, "out"), _stream(stream)),
+                                      int(max_kv_splits), _dev_ptr(out, torch.float32, "out"),
+                                      _stream(stream)),
                "pa_prefill_chunk")
         return out
 

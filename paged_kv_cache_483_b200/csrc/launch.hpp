@@ -77,6 +77,14 @@ struct PrefillArgs {
   float scale;
   float* out;  // [B, q_tokens, H, 128] fp32
   int32_t* err;
+  // key-split scratch of the last wave (null = no split): split_slots slots
+  // of 2 x 128 x 128 fp32 (split_o) and 2 x 128 (m, l) pairs (split_ml), and
+  // 2 tickets per split unit (tickets, zero between calls)
+  int32_t max_splits;  // 0 = automatic, 1 = never split, n = at most n parts
+  float* split_o;
+  float* split_ml;
+  int32_t* tickets;
+  int32_t split_slots;
 };
 bool prefill_fast_supported(int dtype_bf16, int d, int bs, int G);
 cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,

@@ -46,6 +46,10 @@ struct pa_pool {
   int32_t* d_err = nullptr;
   bool tmap_ok = false;
   CUtensorMap tmK, tmV;
+  // tensor-core prefill: key-split scratch for one wave (one slot per SM)
+  float* split_o = nullptr;
+  float* split_ml = nullptr;
+  int32_t* tickets = nullptr;
   Staging ring[kRing];
   int ring_next = 0;
   std::vector<int64_t> slots_tmp;
@@ -147,6 +151,14 @@ bool use_fast_prefill(const pa_pool* p, int32_t H) {
 
 pa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
 
+void free_split(pa_pool* p) {
+  if (p->split_o) cudaFree(p->split_o);
+  if (p->split_ml) cudaFree(p->split_ml);
+  if (p->tickets) cudaFree(p->tickets);
+  p->split_o = p->split_ml = nullptr;
+  p->tickets = nullptr;
+}
+
 }  // namespace
 
 extern "C" {
@@ -194,6 +206,17 @@ pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
     if (kv_dtype == PA_BF16 && head_dim == 128 && block_size == 16)
       p->tmap_ok = make_pool_map(&p->tmK, k_cache, p) &&
                    make_pool_map(&p->tmV, v_cache, p);
+    if (p->tmap_ok) {
+      // without it the prefill runs unsplit
+      const size_t slots = size_t(p->sms);
+      if (cudaMalloc(&p->split_o, slots * 2 * 128 * 128 * sizeof(float)) != cudaSuccess ||
+          cudaMalloc(&p->split_ml, slots * 2 * 128 * 2 * sizeof(float)) != cudaSuccess ||
+          cudaMalloc(&p->tickets, slots * 2 * sizeof(int32_t)) != cudaSuccess ||
+          cudaMemset(p->tickets, 0, slots * 2 * sizeof(int32_t)) != cudaSuccess) {
+        free_split(p);
+        cudaGetLastError();
+      }
+    }
   }
   *out = p;
   return PA_OK;
@@ -209,6 +232,7 @@ pa_status pa_free(pa_pool* p) {
       if (r.done) cudaEventDestroy(r.done);
     }
     if (p->d_err) cudaFree(p->d_err);
+    free_split(p);
   }
   delete p;
   return PA_OK;
@@ -528,18 +552,20 @@ pa_status pa_decode_append(pa_pool* p, const void* q, const void* key, const voi
 pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,
                            int32_t q_tokens, int32_t H,
                            const int32_t* d_block_tables, int32_t max_blocks,
-                           const int32_t* d_kv_lens, float scale, float* out,
-                           void* stream) {
+                           const int32_t* d_kv_lens, float scale,
+                           int32_t max_kv_splits, float* out, void* stream) {
   pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks,
                                       d_kv_lens, out);
   if (st != PA_OK) return st;
-  if (q_tokens <= 0 || q_tokens > 65535) return PA_ERR_INVALID_ARG;
+  if (q_tokens <= 0 || q_tokens > 65535 || max_kv_splits < 0) return PA_ERR_INVALID_ARG;
   if (B == 0) return PA_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_fast_prefill(p, H)) {
     if (!aligned16(q)) return PA_ERR_INVALID_ARG;
     pa::PrefillArgs a{q, d_block_tables, max_blocks, d_kv_lens, B, q_tokens, H,
-                      p->num_kv_heads, p->num_blocks, scale, out, p->d_err};
+                      p->num_kv_heads, p->num_blocks, scale, out, p->d_err,
+                      max_kv_splits, p->split_o, p->split_ml, p->tickets,
+                      p->split_o ? p->sms : 0};
     return cuda_status(pa::launch_prefill_fast(&p->tmK, &p->tmV, a, p->sms, s));
   }
   pa::GenericArgs g{q, p->k_cache, p->v_cache, d_block_tables, max_blocks,

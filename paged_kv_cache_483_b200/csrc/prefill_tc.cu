@@ -31,6 +31,8 @@
 // that keeps every exponent <= 2^8, exact in fp32).  P is rounded to bf16.
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.hpp"
 #include "tcgen05.cuh"
@@ -52,6 +54,7 @@ constexpr uint32_t kDataBytes = (2 + 2 * kPfStages) * kTile;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr float kRescaleTau = 8.0f;
+constexpr int kMaxSplit = 4;         // parts per split unit at most
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
 
@@ -63,7 +66,19 @@ struct PfBars {
   uint64_t o_final;
   uint32_t tmem_base;
   int abort;
-  int bad;
+  int bad_vote[2][4];
+  int ticket[2];
+};
+
+// Work decomposition.  A unit is one CTA's query tile pair of one (sequence,
+// KV head); units are numbered with the query tile fastest.  Units below
+// first_split run whole; each unit from first_split on is split into k parts
+// over its key tiles (one CTA per part) whose partial results are merged by
+// the part that finishes last.
+struct PfPlan {
+  int nq;           // query tile pairs per (sequence, KV head)
+  int first_split;  // first unit that is split
+  int k;            // parts per split unit (1 = none)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -102,7 +117,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, PfBars
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-    const PrefillArgs p, float scale_log2, int use_tma_store) {
+    const PrefillArgs p, const PfPlan pl, float scale_log2, int use_tma_store) {
   extern __shared__ uint8_t pf_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(pf_raw) + 1023) & ~uintptr_t(1023));
@@ -110,40 +125,29 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.H / p.Hkv, TQ = 128 / G;
-  const int kvh = blockIdx.y, b = blockIdx.z;
-  const int t0 = blockIdx.x * 2 * TQ;                 // first token of tile A
+  int u = blockIdx.x, part = 0;
+  if (u >= pl.first_split) {
+    const int t = u - pl.first_split;
+    u = pl.first_split + t / pl.k;
+    part = t % pl.k;
+  }
+  const int split_k = u >= pl.first_split ? pl.k : 1;
+  const int xq = u % pl.nq, kvh = (u / pl.nq) % p.Hkv, b = u / (pl.nq * p.Hkv);
+  const int t0 = xq * 2 * TQ;                         // first token of tile A
   const int q_tokens = p.q_tokens;
   const int kv_len = p.kv_lens[b];
   const int valid_tokens = min(2 * TQ, q_tokens - t0);  // of both tiles
   const bool len_bad = kv_len < q_tokens || kv_len > p.MB * 16;
   const int qpos0 = kv_len - q_tokens + t0;           // key limit of token t0
   const int key_end = len_bad ? 0 : qpos0 + valid_tokens;
-  const int n_tiles = (key_end + 127) >> 7;
+  const int n_all = (key_end + 127) >> 7;             // key tiles of the unit
+  const int j0 = part * n_all / split_k;              // this part: [j0, j0 + n_tiles)
+  const int n_tiles = (part + 1) * n_all / split_k - j0;
   const int n_blk = (key_end + 15) >> 4;
   const int32_t* trow = p.tables + int64_t(b) * p.MB;
 
-  if (threadIdx.x == 0) {
-    bars->abort = 0;
-    bars->bad = len_bad ? 1 : 0;
-  }
-  __syncthreads();
-  // every block id the CTA will touch must be inside the pool
-  for (int i = threadIdx.x; i < n_blk; i += blockDim.x) {
-    const int blk = trow[i];
-    if (blk < 0 || blk >= p.NB) bars->bad = 2;
-  }
-  __syncthreads();
-  if (bars->bad) {
-    if (threadIdx.x == 0)
-      raise_err(p.err, bars->bad == 1 ? PA_DEVERR_KV_LEN : PA_DEVERR_BLOCK_ID);
-    for (int idx = threadIdx.x; idx < valid_tokens * G * 32; idx += blockDim.x) {
-      const int row = idx >> 5, c4 = idx & 31;
-      const int64_t o = ((int64_t(b) * q_tokens + t0 + row / G) * p.H + kvh * G + row % G) * 128;
-      reinterpret_cast<float4*>(p.out + o)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    return;
-  }
-
+  if (threadIdx.x == 0 && len_bad && xq == 0 && kvh == 0 && part == 0)
+    raise_err(p.err, PA_DEVERR_KV_LEN);
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     for (int s = 0; s < kPfStages; ++s) {
@@ -157,6 +161,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
       mbar_init(&bars->p_full[x], 128);
     }
     mbar_init(&bars->o_final, 1);
+    bars->abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -172,7 +177,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
   regs_dealloc<kCtrlRegs>();
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
-    if (lane == 0) {
+    if (lane == 0 && n_tiles > 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
@@ -190,9 +195,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
         const int nb = min(8, n_blk - j * 8);
         mbar_arrive_expect_tx(full, nb * 4096);
         for (int i = 0; i < nb; ++i) {
-          const int z = trow[j * 8 + i] * 16;
-          tma_load_3d(dst + i * 2048, map, full, 0, kvh, z, pol_kv);
-          tma_load_3d(dst + kHalf + i * 2048, map, full, 64, kvh, z, pol_kv);
+          int blk = trow[j * 8 + i];
+          if (blk < 0 || blk >= p.NB) blk = 0;     // reported and zeroed by the softmax
+          tma_load_3d(dst + i * 2048, map, full, 0, kvh, blk * 16, pol_kv);
+          tma_load_3d(dst + kHalf + i * 2048, map, full, 64, kvh, blk * 16, pol_kv);
         }
       };
       bool ok = true;
@@ -202,14 +208,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
           const int s = jk % kPfStages, round = jk / kPfStages;
           if (round > 0) ok = wait_or_abort(&bars->k_empty[s], (round - 1) & 1, bars, p.err);
           if (!ok || bars->abort) break;
-          load_tile(smem + kOffK + s * kTile, &tmK, &bars->k_full[s], jk);
+          load_tile(smem + kOffK + s * kTile, &tmK, &bars->k_full[s], j0 + jk);
           k_issued = jk + 1;
         }
         if (j >= 0) {                                  // V tile j
           const int s = j % kPfStages, round = j / kPfStages;
           if (round > 0) ok = wait_or_abort(&bars->v_empty[s], (round - 1) & 1, bars, p.err);
           if (!ok || bars->abort) break;
-          load_tile(smem + kOffV + s * kTile, &tmV, &bars->v_full[s], j);
+          load_tile(smem + kOffV + s * kTile, &tmV, &bars->v_full[s], j0 + j);
           v_issued = j + 1;
         }
       }
@@ -243,7 +249,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
                            desc_mnmajor_sw128(vb + kk * 2048, kHalf, 1024), kIdescPV,
                            (j > 0 || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_or_abort(&bars->q_full, 0, bars, p.err) &&
+      bool ok = n_tiles > 0 && wait_or_abort(&bars->q_full, 0, bars, p.err) &&
                 wait_or_abort(&bars->k_full[0], 0, bars, p.err);
       if (ok) {
         tc_fence_after();
@@ -276,7 +282,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
           umma_commit(&bars->k_empty[(j + 1) % kPfStages]);
         }
       }
-      umma_commit(&bars->o_final);
+      if (n_tiles > 0) umma_commit(&bars->o_final);
     }
   }
   } else {
@@ -292,6 +298,20 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t s_addr = tbase + lane_off + kColS + x * 128;
     const uint32_t o_addr = tbase + lane_off + kColO + x * 128;
+    // every block id the CTA touches must be inside the pool (checked here,
+    // while the first QK^T is still running)
+    bool bad_blk = false;
+    const int blk_end = min(n_blk, (j0 + n_tiles) * 8);
+    for (int i = j0 * 8 + r; i < blk_end; i += 128) {
+      const int blk = trow[i];
+      bad_blk |= (blk < 0 || blk >= p.NB);
+    }
+    bad_blk = __any_sync(0xffffffffu, bad_blk);
+    if (lane == 0) bars->bad_vote[x][quarter] = bad_blk ? 1 : 0;
+    named_bar_sync(1 + x, 128);
+    bad_blk = (bars->bad_vote[x][0] | bars->bad_vote[x][1] | bars->bad_vote[x][2] |
+               bars->bad_vote[x][3]) != 0;
+    if (bad_blk && r == 0 && x == 0) raise_err(p.err, PA_DEVERR_BLOCK_ID);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
@@ -305,7 +325,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(v[i]);
       }
-      const int lim = qpos - j * 128;                  // columns c <= lim are visible
+      const int lim = qpos - (j0 + j) * 128;           // columns c <= lim are visible
       if (lim < 127) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
@@ -388,12 +408,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
         l *= alpha;
         tile_sum = write_p(m_ref == -INFINITY ? 0.f : m_ref);
       }
-      if (x == 0 && j == n_tiles - 1) {
+      if (x == 0 && j0 + j == n_all - 1) {
         // V rows at or past key_end hold stale bytes: zero them (p = 0 there,
         // and 0 x NaN would poison the product); PV_B follows PV_A
         const int st = j % kPfStages;
         const bool landed = warp_wait(&bars->v_full[st], (j / kPfStages) & 1, bars, p.err, lane);
-        if (landed && j * 128 + r >= key_end) {
+        if (landed && (j0 + j) * 128 + r >= key_end) {
           uint4* v0 = reinterpret_cast<uint4*>(smem + kOffV + st * kTile + r * 128);
           uint4* v1 = reinterpret_cast<uint4*>(smem + kOffV + st * kTile + kHalf + r * 128);
 #pragma unroll
@@ -408,48 +428,147 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
       tc_fence_before();
       mbar_arrive(&bars->p_full[x]);
     }
-    // epilogue: O / l
-    const bool done = ok && warp_wait(&bars->o_final, 0, bars, p.err, lane);
+    // ------------------------------------------------------------ epilogue
+    // o_final: every MMA of the CTA has completed, so TMEM and the whole
+    // shared memory may be reused.  Rows of a part that found an error are
+    // zeros (not O * 0: O may hold non-finite values or was never written).
+    const bool fin_ok = ok && (n_tiles == 0 || warp_wait(&bars->o_final, 0, bars, p.err, lane));
     tc_fence_after();
-    const float inv = (done && l > 0.f) ? 1.f / l : 0.f;
-    if (use_tma_store && valid_tokens == 2 * TQ) {
-      // Both tiles are full: every MMA is done, so the whole shared memory is
-      // free.  Each row goes into four 32-column boxes with the 128-byte
-      // swizzle (conflict-free), then one thread per tile stores them with TMA.
-      uint8_t* stage = smem + x * 65536;
+    const bool part_err = !fin_ok || bad_blk;
+    const bool have = !part_err && n_tiles > 0 && l > 0.f;
+    const float inv = have ? 1.f / l : 0.f;
+    // this part's O / l, columns [32c, 32c + 32)
+    auto own_chunk = [&](int c, float (&o)[32]) {
+      uint32_t v[32];
+      tmem_ld32(o_addr + c * 32, v);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(o_addr + c * 32, v);
-        uint8_t* box = stage + c * 16384;
+      for (int i = 0; i < 32; ++i) o[i] = have ? __uint_as_float(v[i]) * inv : 0.f;
+    };
+    // write the tile's final rows
+    auto emit = [&](auto&& chunk) {
+      if (use_tma_store && valid_tokens == 2 * TQ) {
+        // Both tiles are full: each row goes into four 32-column boxes with
+        // the 128-byte swizzle (conflict-free), then one thread per tile
+        // stores them with TMA.
+        uint8_t* stage = smem + x * 65536;
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          *reinterpret_cast<float4*>(box + swz128(r, q4)) =
-              make_float4(__uint_as_float(v[4 * q4]) * inv, __uint_as_float(v[4 * q4 + 1]) * inv,
-                          __uint_as_float(v[4 * q4 + 2]) * inv,
-                          __uint_as_float(v[4 * q4 + 3]) * inv);
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          chunk(c, o);
+          uint8_t* box = stage + c * 16384;
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            *reinterpret_cast<float4*>(box + swz128(r, q4)) =
+                make_float4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1 + x, 128);
+        if (r == 0) {
+          const int z = b * q_tokens + t0 + x * TQ;
+          for (int c = 0; c < 4; ++c) tma_store_3d(&tmO, stage + c * 16384, c * 32, kvh * G, z);
+          bulk_commit();
+          bulk_wait_read_all();
+        }
+      } else {
+        float* orow = p.out + ((int64_t(b) * q_tokens + tok) * p.H + kvh * G + g) * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          chunk(c, o);
+          if (row_valid) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(orow + c * 32 + i) =
+                  make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+          }
+        }
       }
-      fence_proxy_async_smem();
+    };
+    if (split_k == 1) {
+      emit(own_chunk);
+    } else {
+      // A part of a split unit publishes its normalised O rows and (m, l) --
+      // l < 0 marks a part that failed -- then takes a ticket; the part that
+      // takes the last ticket merges all parts with the log-sum-exp rule:
+      // out = sum_q w_q O_q / l_q, w_q = l_q 2^(m_q - M) / sum_q' l_q' 2^(m_q' - M).
+      const int us = u - pl.first_split;
+      const int64_t slot0 = int64_t(us) * split_k;
+      // a part's O tile is stored as [32 column quads][128 rows][4]: a warp
+      // moves 512 contiguous bytes per access
+      auto part_o = [&](int q) {
+        return reinterpret_cast<float4*>(p.split_o + ((slot0 + q) * 2 + x) * (128 * 128)) + r;
+      };
+      auto part_ml = [&](int q) {
+        return reinterpret_cast<float2*>(p.split_ml) + ((slot0 + q) * 2 + x) * 128 + r;
+      };
+      {
+        float4* dst = part_o(part);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          own_chunk(c, o);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[(c * 8 + i) * 128] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        }
+        *part_ml(part) = make_float2(m_ref, part_err ? -1.f : (have ? l : 0.f));
+      }
+      __threadfence();
       named_bar_sync(1 + x, 128);
       if (r == 0) {
-        const int z = b * q_tokens + t0 + x * TQ;
-        for (int c = 0; c < 4; ++c) tma_store_3d(&tmO, stage + c * 16384, c * 32, kvh * G, z);
-        bulk_commit();
-        bulk_wait_read_all();
+        int32_t* tk = p.tickets + us * 2 + x;
+        const int t = atomicAdd(tk, 1);
+        if (t == split_k - 1) *tk = 0;                 // every part is in: reset
+        bars->ticket[x] = t;
+        __threadfence();
       }
-    } else {
-      float* orow = p.out + ((int64_t(b) * q_tokens + tok) * p.H + kvh * G + g) * 128;
+      named_bar_sync(1 + x, 128);
+      if (bars->ticket[x] == split_k - 1) {
+        float w[kMaxSplit], mq[kMaxSplit];
+        float M = -INFINITY, L = 0.f;
+        bool failed = false;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(o_addr + c * 32, v);
-        if (row_valid) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(orow + c * 32 + i) =
-                make_float4(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv,
-                            __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
+        for (int q = 0; q < kMaxSplit; ++q) {
+          const float2 ml = q < split_k ? __ldcg(part_ml(q)) : make_float2(0.f, 0.f);
+          failed |= ml.y < 0.f;
+          w[q] = fmaxf(ml.y, 0.f);                     // l_q; 2^(m_q - M) below
+          mq[q] = ml.x;
+          if (ml.y > 0.f) M = fmaxf(M, ml.x);
         }
+#pragma unroll
+        for (int q = 0; q < kMaxSplit; ++q) {
+          w[q] = w[q] > 0.f ? w[q] * ex2(mq[q] - M) : 0.f;
+          L += w[q];
+        }
+        const float invL = (!failed && L > 0.f) ? 1.f / L : 0.f;
+#pragma unroll
+        for (int q = 0; q < kMaxSplit; ++q) w[q] *= invL;
+        emit([&](int c, float (&o)[32]) {
+          // every part's loads first (one round trip to L2 per chunk)
+          float4 v[kMaxSplit][8];
+#pragma unroll
+          for (int q = 0; q < kMaxSplit; ++q) {
+            if (q < split_k) {
+              const float4* src = part_o(q);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[q][i] = __ldcg(src + (c * 8 + i) * 128);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+#pragma unroll
+          for (int q = 0; q < kMaxSplit; ++q) {
+            if (q < split_k && w[q] != 0.f) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                o[4 * i] = fmaf(w[q], v[q][i].x, o[4 * i]);
+                o[4 * i + 1] = fmaf(w[q], v[q][i].y, o[4 * i + 1]);
+                o[4 * i + 2] = fmaf(w[q], v[q][i].z, o[4 * i + 2]);
+                o[4 * i + 3] = fmaf(w[q], v[q][i].w, o[4 * i + 3]);
+              }
+            }
+          }
+        });
       }
     }
   }
@@ -480,7 +599,6 @@ static PFN_cuTensorMapEncodeTiled_v12000 q_encode_fn() {
 
 cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
                                 const PrefillArgs& a, int sms, cudaStream_t stream) {
-  (void)sms;
   const int G = a.H / a.Hkv, TQ = 128 / G;
   // Q viewed as {head_dim, H, B * q_tokens}; one box = TQ tokens x G heads x 64
   CUtensorMap tmQ;
@@ -518,10 +636,28 @@ cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((a.q_tokens + 2 * TQ - 1) / (2 * TQ), a.Hkv, a.B);
-  prefill_tc_kernel<<<grid, kPfThreads, smem, stream>>>(tmQ, *tmK, *tmV, tmO, a,
-                                                         a.scale * 1.4426950408889634f,
-                                                         use_tma_store);
+  PfPlan pl;
+  pl.nq = (a.q_tokens + 2 * TQ - 1) / (2 * TQ);
+  const int64_t units = int64_t(pl.nq) * a.Hkv * a.B;
+  if (units > (int64_t(1) << 30)) return cudaErrorInvalidValue;
+  pl.first_split = int(units);
+  pl.k = 1;
+  // The units of the last, partial wave (one CTA per SM) are split over
+  // their keys so that the wave fills the GPU: k parts each, k * tail <= SMs.
+  if (a.split_o && a.split_ml && a.tickets && a.max_splits != 1 && sms > 0) {
+    const int64_t tail = units % sms;
+    if (tail > 0) {
+      int64_t k = sms / tail;
+      k = std::min<int64_t>(k, a.max_splits > 1 ? std::min(a.max_splits, kMaxSplit) : kMaxSplit);
+      if (k >= 2 && tail * k <= a.split_slots) {
+        pl.first_split = int(units - tail);
+        pl.k = int(k);
+      }
+    }
+  }
+  const int64_t ctas = pl.first_split + (units - pl.first_split) * pl.k;
+  prefill_tc_kernel<<<unsigned(ctas), kPfThreads, smem, stream>>>(
+      tmQ, *tmK, *tmV, tmO, a, pl, a.scale * 1.4426950408889634f, use_tma_store);
   return cudaGetLastError();
 }
 

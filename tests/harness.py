@@ -64,10 +64,11 @@ class GpuRun:
         torch.cuda.synchronize()
         return out.cpu().numpy()
 
-    def prefill(self, q=None):
+    def prefill(self, q=None, max_kv_splits=0):
         q = self.w.queries() if q is None else q
         tables, lens, _, _ = self.tables()
-        out = self.pool.prefill_chunk(q.contiguous().to(self.device), tables, lens)
+        out = self.pool.prefill_chunk(q.contiguous().to(self.device), tables, lens,
+                                      max_kv_splits=max_kv_splits)
         torch.cuda.synchronize()
         return out.cpu().numpy()
 

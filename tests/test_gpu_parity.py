@@ -168,13 +168,16 @@ def test_device_bounds_errors_zero_rows():
 @pytest.mark.parametrize("batch,cached,chunk,H,Hkv", [
     (2, 0, 37, 32, 8), (2, 40, 37, 32, 8), (1, 200, 130, 32, 8), (3, 5, 1, 32, 8),
     (2, 300, 129, 8, 8), (2, 17, 200, 16, 8), (2, 250, 64, 64, 8), (1, 1000, 300, 32, 8)])
-def test_prefill_parity_small(batch, cached, chunk, H, Hkv):
+@pytest.mark.parametrize("splits", [0, 1])
+def test_prefill_parity_small(batch, cached, chunk, H, Hkv, splits):
+    # these grids are smaller than one wave: splits=0 cuts every query tile
+    # over its keys (up to 4 parts, some of them empty), splits=1 never does
     w = workloads.prefill(seed=batch * 100 + cached + chunk + H, batch=batch, cached=cached,
                           chunk=chunk, num_heads=H, num_kv_heads=Hkv)
     g = GpuRun(w).apply(w.setup + w.step)
     assert g.pool.prefill_path(H) == 1
     o = OracleRun(w).apply(w.setup + w.step)
-    out = g.prefill()
+    out = g.prefill(max_kv_splits=splits)
     q = q64(w)
     worst = 0.0
     for i in range(batch):
@@ -248,7 +251,8 @@ def test_full_prefill_sampled():
     assert g.pool.get_error() == 0
 
 
-def test_prefill_device_errors_zero_rows():
+@pytest.mark.parametrize("splits", [0, 1])
+def test_prefill_device_errors_zero_rows(splits):
     w = workloads.prefill(seed=41, batch=2, cached=100, chunk=70)
     g = GpuRun(w).apply(w.setup + w.step)
     tables, lens, _, _ = g.tables()
@@ -256,15 +260,46 @@ def test_prefill_device_errors_zero_rows():
     assert g.pool.prefill_path(32) == 1
     bad = tables.clone()
     bad[1, 2] = w.num_blocks + 3
-    out = g.pool.prefill_chunk(q, bad, lens)
+    out = g.pool.prefill_chunk(q, bad, lens, max_kv_splits=splits)
     assert g.pool.get_error() & pa.PA_DEVERR_BLOCK_ID
     assert torch.all(out[1] == 0) and torch.any(out[0] != 0)
     short = lens.clone()
     short[0] = 50                                        # fewer keys than the chunk
-    out = g.pool.prefill_chunk(q, tables, short)
+    out = g.pool.prefill_chunk(q, tables, short, max_kv_splits=splits)
     assert g.pool.get_error() & pa.PA_DEVERR_KV_LEN
     assert torch.all(out[0] == 0) and torch.any(out[1] != 0)
+    out = g.pool.prefill_chunk(q, tables, lens, max_kv_splits=splits)   # recovers
+    assert g.pool.get_error() == 0 and torch.all(torch.isfinite(out))
     assert g.pool.get_error() == 0
+
+
+@pytest.mark.parametrize("splits", [0, 2, 3, 4])
+def test_prefill_tail_split(splits):
+    # 10 sequences x 8 KV heads x 4 query tile pairs = 320 CTAs of work: two
+    # full waves on 148 SMs and a tail of 24 that is split over its keys; a
+    # second call must give the same bits (the merge tickets reset themselves)
+    w = workloads.prefill(seed=47, batch=10, cached=500, chunk=256)
+    g = GpuRun(w).apply(w.setup + w.step)
+    o = OracleRun(w).apply(w.setup + w.step)
+    out = g.prefill(max_kv_splits=splits)
+    again = g.prefill(max_kv_splits=splits)
+    assert np.array_equal(out, again)
+    q = q64(w)
+    worst = 0.0
+    for i in range(10):
+        for h, ref in o.attention(i, q[i]).items():
+            worst = max(worst, float(np.abs(out[i, :, h] - ref).max()))
+    assert worst <= TOL_PREFILL, worst
+    unsplit = g.prefill(max_kv_splits=1)
+    assert float(np.abs(out - unsplit).max()) <= TOL_PREFILL
+    assert g.pool.get_error() == 0
+
+
+def test_prefill_split_arg_checked():
+    w = workloads.prefill(seed=48, batch=1, cached=20, chunk=30)
+    g = GpuRun(w).apply(w.setup + w.step)
+    with pytest.raises(pa.PAError):
+        g.prefill(max_kv_splits=-1)
 
 
 def test_prefill_uninitialised_pool_is_safe():
