@@ -97,17 +97,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map,
       : "memory");
 }
 
-__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map,
-                                            uint64_t* bar, int32_t x,
-                                            int32_t y, int32_t z, int32_t w,
-                                            uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-
 // Shared -> global tile store (no multicast); completion tracked per thread
 // with bulk async-groups.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src,

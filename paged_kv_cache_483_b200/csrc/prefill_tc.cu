@@ -44,13 +44,14 @@ namespace {
 constexpr int kPfThreads = 384;      // 3 warpgroups: control, softmax A, softmax B
 constexpr int kCtrlRegs = 64;        // 128 x 64 + 256 x 216 <= 384 x 168 at launch
 constexpr int kSoftmaxRegs = 216;
-constexpr int kPfStages = 2;
+constexpr int kKStages = 2;         // K ring (tiles)
+constexpr int kVStages = 2;         // V ring (tiles)
 constexpr uint32_t kTile = 32768;  // 128 x 128 bf16
 constexpr uint32_t kHalf = 16384;  // 128 x 64 bf16 (one 128-byte-swizzled half)
 constexpr uint32_t kOffQ = 0;      // Q_A, then Q_B
 constexpr uint32_t kOffK = 2 * kTile;
-constexpr uint32_t kOffV = (2 + kPfStages) * kTile;
-constexpr uint32_t kDataBytes = (2 + 2 * kPfStages) * kTile;
+constexpr uint32_t kOffV = (2 + kKStages) * kTile;
+constexpr uint32_t kDataBytes = (2 + kKStages + kVStages) * kTile;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr float kRescaleTau = 8.0f;
@@ -60,8 +61,8 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
 
 struct PfBars {
   uint64_t q_full;
-  uint64_t k_full[kPfStages], k_empty[kPfStages];
-  uint64_t v_full[kPfStages], v_empty[kPfStages];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];
   uint64_t o_final;
   uint32_t tmem_base;
@@ -150,9 +151,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
     raise_err(p.err, PA_DEVERR_KV_LEN);
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kPfStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
@@ -175,63 +178,72 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
 
   if (warp < 4) {
   regs_dealloc<kCtrlRegs>();
-  if (warp == 0) {
-    // ------------------------------------------------------- TMA producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------- TMA producers: Q and K (warp 0), V (warp 2)
+    // Two threads issue the copies: one thread's TMA issue rate does not
+    // keep up with the K and V tiles of both query tiles.
+    const bool is_k = warp == 0;
     if (lane == 0 && n_tiles > 0) {
-      prefetch_tensormap(&tmQ);
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      const uint64_t pol_q = policy_evict_first();
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      prefetch_tensormap(map);
       const uint64_t pol_kv = policy_evict_last();
-      mbar_arrive_expect_tx(&bars->q_full, 2 * kTile);
-      for (int x = 0; x < 2; ++x) {
-        const int z = b * q_tokens + t0 + x * TQ;
-        tma_load_3d(smem + kOffQ + x * kTile, &tmQ, &bars->q_full, 0, kvh * G, z, pol_q);
-        tma_load_3d(smem + kOffQ + x * kTile + kHalf, &tmQ, &bars->q_full, 64, kvh * G, z,
-                    pol_q);
+      if (is_k) {
+        prefetch_tensormap(&tmQ);
+        const uint64_t pol_q = policy_evict_first();
+        mbar_arrive_expect_tx(&bars->q_full, 2 * kTile);
+        for (int x = 0; x < 2; ++x) {
+          const int z = b * q_tokens + t0 + x * TQ;
+          tma_load_3d(smem + kOffQ + x * kTile, &tmQ, &bars->q_full, 0, kvh * G, z, pol_q);
+          tma_load_3d(smem + kOffQ + x * kTile + kHalf, &tmQ, &bars->q_full, 64, kvh * G, z,
+                      pol_q);
+        }
       }
-      int k_issued = 0, v_issued = 0;
-      auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* full, int j) {
-        const int nb = min(8, n_blk - j * 8);
-        mbar_arrive_expect_tx(full, nb * 4096);
-        for (int i = 0; i < nb; ++i) {
-          int blk = trow[j * 8 + i];
-          if (blk < 0 || blk >= p.NB) blk = 0;     // reported and zeroed by the softmax
-          tma_load_3d(dst + i * 2048, map, full, 0, kvh, blk * 16, pol_kv);
-          tma_load_3d(dst + kHalf + i * 2048, map, full, 64, kvh, blk * 16, pol_kv);
+      // Block ids of a tile, read one tile ahead of their use: the TMA
+      // issues are ordered with every memory access, so an id read next to
+      // its copy would cost one global-memory round trip per block.
+      auto tile_ids = [&](int j, int (&ids)[8]) {
+        const int nb = min(8, n_blk - (j0 + j) * 8);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          int blk = i < nb ? trow[(j0 + j) * 8 + i] : 0;
+          ids[i] = (blk < 0 || blk >= p.NB) ? 0 : blk;   // reported and zeroed by the softmax
         }
       };
-      bool ok = true;
-      for (int j = -1; ok && j < n_tiles; ++j) {
-        const int jk = j + 1;                          // K tile to issue
-        if (jk < n_tiles) {
-          const int s = jk % kPfStages, round = jk / kPfStages;
-          if (round > 0) ok = wait_or_abort(&bars->k_empty[s], (round - 1) & 1, bars, p.err);
-          if (!ok || bars->abort) break;
-          load_tile(smem + kOffK + s * kTile, &tmK, &bars->k_full[s], j0 + jk);
-          k_issued = jk + 1;
+      uint64_t* full = is_k ? bars->k_full : bars->v_full;
+      uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
+      uint8_t* ring = smem + (is_k ? kOffK : kOffV);
+      const int stages = is_k ? kKStages : kVStages;
+      int ids[8];
+      tile_ids(0, ids);
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % stages, round = j / stages;
+        if (round > 0 && !wait_or_abort(&empty[s], (round - 1) & 1, bars, p.err)) break;
+        if (bars->abort) break;
+        uint8_t* dst = ring + s * kTile;
+        const int nb = min(8, n_blk - (j0 + j) * 8);
+        mbar_arrive_expect_tx(&full[s], nb * 4096);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (i < nb) {
+            tma_load_3d(dst + i * 2048, map, &full[s], 0, kvh, ids[i] * 16, pol_kv);
+            tma_load_3d(dst + kHalf + i * 2048, map, &full[s], 64, kvh, ids[i] * 16, pol_kv);
+          }
         }
-        if (j >= 0) {                                  // V tile j
-          const int s = j % kPfStages, round = j / kPfStages;
-          if (round > 0) ok = wait_or_abort(&bars->v_empty[s], (round - 1) & 1, bars, p.err);
-          if (!ok || bars->abort) break;
-          load_tile(smem + kOffV + s * kTile, &tmV, &bars->v_full[s], j0 + j);
-          v_issued = j + 1;
-        }
+        issued = j + 1;
+        if (j + 1 < n_tiles) tile_ids(j + 1, ids);
       }
       // drain: every issued copy has landed before the CTA may exit
-      mbar_wait(&bars->q_full, 0);
-      for (int s = 0; s < kPfStages; ++s) {
-        if (s < k_issued) mbar_wait(&bars->k_full[s], ((k_issued - 1 - s) / kPfStages) & 1);
-        if (s < v_issued) mbar_wait(&bars->v_full[s], ((v_issued - 1 - s) / kPfStages) & 1);
-      }
+      if (is_k) mbar_wait(&bars->q_full, 0);
+      for (int s = 0; s < stages; ++s)
+        if (s < issued) mbar_wait(&full[s], ((issued - 1 - s) / stages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t qa = smem_u32(smem + kOffQ);
       auto qk = [&](int x, int j) {                    // S_x = Q_x K(j)^T
-        const uint32_t kb = smem_u32(smem + kOffK + (j % kPfStages) * kTile);
+        const uint32_t kb = smem_u32(smem + kOffK + (j % kKStages) * kTile);
         const uint32_t q = qa + x * kTile;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -242,7 +254,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
         umma_commit(&bars->s_full[x]);
       };
       auto pv = [&](int x, int j) {                    // O_x += P_x V(j)
-        const uint32_t vb = smem_u32(smem + kOffV + (j % kPfStages) * kTile);
+        const uint32_t vb = smem_u32(smem + kOffV + (j % kVStages) * kTile);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_bf16_tmem_a(tbase + kColO + x * 128, tbase + kColS + x * 128 + kk * 8,
@@ -258,16 +270,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
         umma_commit(&bars->k_empty[0]);
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kPfStages;
+        const int s = j % kVStages;
         const bool more = j + 1 < n_tiles;
-        ok = wait_or_abort(&bars->v_full[s], (j / kPfStages) & 1, bars, p.err) &&
+        ok = wait_or_abort(&bars->v_full[s], (j / kVStages) & 1, bars, p.err) &&
              wait_or_abort(&bars->p_full[0], j & 1, bars, p.err);
         if (!ok || bars->abort) break;
         tc_fence_after();
         pv(0, j);
         if (more) {
-          const int s1 = (j + 1) % kPfStages;
-          ok = wait_or_abort(&bars->k_full[s1], ((j + 1) / kPfStages) & 1, bars, p.err);
+          const int s1 = (j + 1) % kKStages;
+          ok = wait_or_abort(&bars->k_full[s1], ((j + 1) / kKStages) & 1, bars, p.err);
           if (!ok) break;
           tc_fence_after();
           qk(0, j + 1);
@@ -279,7 +291,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
         umma_commit(&bars->v_empty[s]);
         if (more) {
           qk(1, j + 1);
-          umma_commit(&bars->k_empty[(j + 1) % kPfStages]);
+          umma_commit(&bars->k_empty[(j + 1) % kKStages]);
         }
       }
       if (n_tiles > 0) umma_commit(&bars->o_final);
@@ -411,8 +423,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
       if (x == 0 && j0 + j == n_all - 1) {
         // V rows at or past key_end hold stale bytes: zero them (p = 0 there,
         // and 0 x NaN would poison the product); PV_B follows PV_A
-        const int st = j % kPfStages;
-        const bool landed = warp_wait(&bars->v_full[st], (j / kPfStages) & 1, bars, p.err, lane);
+        const int st = j % kVStages;
+        const bool landed = warp_wait(&bars->v_full[st], (j / kVStages) & 1, bars, p.err, lane);
         if (landed && (j0 + j) * 128 + r >= key_end) {
           uint4* v0 = reinterpret_cast<uint4*>(smem + kOffV + st * kTile + r * 128);
           uint4* v1 = reinterpret_cast<uint4*>(smem + kOffV + st * kTile + kHalf + r * 128);
