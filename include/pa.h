@@ -126,6 +126,39 @@ pa_status pa_seq_fork(pa_pool* pool, int32_t parent, int32_t child,
  * free list ([P1] release, [P2] release). */
 pa_status pa_seq_release(pa_pool* pool, int32_t seq);
 
+/* Prefix cache ([P2] prefix-hash trace, "complete block boundaries"): the
+ * block that ends at token `end` is identified by (scope, revision, every
+ * token id before `end`), and only full blocks are keyed.  The cache maps a
+ * key to the physical block that first held it and keeps one reference of
+ * its own on that block, so cached blocks outlive their writers until
+ * pa_prefix_clear.  scope and revision are caller-chosen 64-bit ids (a hash
+ * of a tenant name, of a model revision, ...); token ids are compared
+ * exactly, not by hash.
+ *
+ * pa_seq_create_cached: new sequence `seq` that starts with the longest run
+ * of leading full blocks of tokens[0, n_tokens) (host) whose keys are cached,
+ * shared with their current holders (refcount + 1 each).  *hit_tokens =
+ * the tokens covered (a multiple of block_size); append the rest with
+ * pa_append_kv.  Errors: DUP_SEQ, INVALID_ARG (n_tokens < 0, tokens NULL). */
+pa_status pa_seq_create_cached(pa_pool* pool, int32_t seq, uint64_t scope,
+                               uint64_t revision, const int32_t* tokens,
+                               int32_t n_tokens, int32_t* hit_tokens);
+
+/* Key the full blocks of `seq` among its first n_tokens tokens, whose ids
+ * are tokens[0, n_tokens) (host; n_tokens <= the sequence length).  A key
+ * already cached keeps its block.  *added_blocks = new keys.  Errors:
+ * UNKNOWN_SEQ, INVALID_ARG. */
+pa_status pa_prefix_publish(pa_pool* pool, int32_t seq, uint64_t scope,
+                            uint64_t revision, const int32_t* tokens,
+                            int32_t n_tokens, int32_t* added_blocks);
+
+/* Drop every reference the prefix cache holds; *freed_blocks = blocks that
+ * returned to the free list (may be NULL). */
+pa_status pa_prefix_clear(pa_pool* pool, int32_t* freed_blocks);
+
+/* Number of keys the prefix cache holds. */
+int64_t pa_prefix_entries(const pa_pool* pool);
+
 /* Length and table of `seq`.  blocks_out (host, capacity cap) may be NULL to
  * query only n_blocks/length.  INVALID_ARG if cap is too small. */
 pa_status pa_seq_table(const pa_pool* pool, int32_t seq, int32_t* blocks_out,

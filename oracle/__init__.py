@@ -16,6 +16,8 @@ Pages this oracle follows (cited by title and section):
     grouping, the causal rule max_visible = kv_len - q_tokens + qt, softmax.
   * "semidirectx cmu11-667 lecture19 infer_world.py", section 3 (online
     softmax and tiled attention) -- the (m, l, acc) recurrence.
+  * "vladkulikov.com modern-llms module 9 notebook", prefix-hash trace --
+    ``PrefixCache``: content-keyed identity of full blocks.
 
 Parity status: every function is pinned by a ``-m "not gpu"`` test in
 ``tests/test_oracle_pins.py`` (page-printed traces, closed forms, brute force
@@ -23,6 +25,7 @@ in 40-digit decimal arithmetic, invariants).  No function is unpinned.
 """
 
 from .kv_pool import KVPool, PoolError, PoolExhausted  # noqa: F401
+from .prefix_cache import PrefixCache, prefix_key, run_prefix_trace, trace_tokens  # noqa: F401
 from .attention import (  # noqa: F401
     attention_two_pass, paged_attention, attention_tiled, partition_stats,
     combine_partitions, attention_split_kv, online_softmax_stats,

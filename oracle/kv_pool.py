@@ -56,6 +56,8 @@ class KVPool:
         self._free_heap = list(range(self.num_blocks))
         self._free = set(range(self.num_blocks))
         self.refs = [0] * self.num_blocks
+        # references held outside the sequence tables (a prefix cache), per block
+        self.external: dict = {}
         self.tables: dict = {}
         self.lengths: dict = {}
         if store_heads is None:
@@ -228,6 +230,8 @@ class KVPool:
     # -- accounting ("vladkulikov.com ... _refresh_fills, snapshot") -----------
     def fills(self):
         fill = [0] * self.num_blocks
+        for blk in self.external:              # blocks a prefix cache maps are full
+            fill[blk] = self.block_size
         for seq, table in self.tables.items():
             length = self.lengths[seq]
             for j, blk in enumerate(table):
@@ -289,6 +293,8 @@ class KVPool:
                 if not 0 <= blk < self.num_blocks:
                     raise AssertionError("invalid block id in a table")
                 expect[blk] += 1
+        for blk, cnt in self.external.items():
+            expect[blk] += cnt
         fill = self.fills()
         for blk in range(self.num_blocks):
             if self.refs[blk] != expect[blk]:
@@ -302,5 +308,8 @@ class KVPool:
                 if not 1 <= fill[blk] <= self.block_size:
                     raise AssertionError("referenced block has an invalid fill")
         snap = self.snapshot()
-        if snap["logical_tokens"] < snap["physical_payload_tokens"]:
+        # a block only a prefix cache holds is payload no live sequence counts
+        held = set(b for table in self.tables.values() for b in table)
+        cache_only = sum(self.block_size for b in self.external if b not in held)
+        if snap["logical_tokens"] + cache_only < snap["physical_payload_tokens"]:
             raise AssertionError("physical payload exceeds logical payload")

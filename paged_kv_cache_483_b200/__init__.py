@@ -31,7 +31,8 @@ EXPORTS = ["pa_pool_create", "pa_free", "pa_seq_create", "pa_seq_fork", "pa_seq_
            "pa_refcounts", "pa_validate", "pa_append_kv", "pa_reshape_and_cache",
            "pa_cow_copy", "pa_decode_workspace_bytes", "pa_decode", "pa_prefill_chunk",
            "pa_get_error", "pa_status_string", "pa_decode_path", "pa_prefill_path",
-           "pa_decode_static_scratch", "pa_decode_append"]
+           "pa_decode_static_scratch", "pa_decode_append", "pa_seq_create_cached",
+           "pa_prefix_publish", "pa_prefix_clear", "pa_prefix_entries"]
 
 
 class PAError(RuntimeError):
@@ -67,6 +68,10 @@ def lib():
         "pa_seq_fork": ([_P, _I32, _I32, _I32], C.c_int),
         "pa_seq_release": ([_P, _I32], C.c_int),
         "pa_seq_table": ([_P, _I32, _PI32, _I32, _PI32, _PI32], C.c_int),
+        "pa_seq_create_cached": ([_P, _I32, C.c_uint64, C.c_uint64, _PI32, _I32, _PI32], C.c_int),
+        "pa_prefix_publish": ([_P, _I32, C.c_uint64, C.c_uint64, _PI32, _I32, _PI32], C.c_int),
+        "pa_prefix_clear": ([_P, _PI32], C.c_int),
+        "pa_prefix_entries": ([_P], _I64),
         "pa_block_tables": ([_P, _PI32, _I32, _I32, _PI32, _PI32], C.c_int),
         "pa_plan_append": ([_P, _PI32, _PI32, _I32, _PI64, _PI32, _PI32, _I32, _PI32], C.c_int),
         "pa_pool_stats": ([_P, C.POINTER(Stats)], C.c_int),
@@ -183,6 +188,32 @@ class Pool:
 
     def release(self, seq):
         _check(lib().pa_seq_release(self._h, int(seq)), "pa_seq_release")
+
+    # -- prefix cache (content-keyed full blocks) ----------------------------
+    def create_cached(self, seq, tokens, scope=0, revision=0):
+        """New sequence starting with the cached blocks of ``tokens``'s
+        longest cached full-block prefix; returns the tokens it covers."""
+        toks, tp = _i32(tokens)
+        hit = C.c_int32()
+        _check(lib().pa_seq_create_cached(self._h, int(seq), int(scope), int(revision), tp,
+                                          len(toks), C.byref(hit)), "pa_seq_create_cached")
+        return hit.value
+
+    def publish(self, seq, tokens, scope=0, revision=0):
+        """Key ``seq``'s full blocks (token ids ``tokens``); returns new keys."""
+        toks, tp = _i32(tokens)
+        added = C.c_int32()
+        _check(lib().pa_prefix_publish(self._h, int(seq), int(scope), int(revision), tp,
+                                       len(toks), C.byref(added)), "pa_prefix_publish")
+        return added.value
+
+    def prefix_clear(self):
+        freed = C.c_int32()
+        _check(lib().pa_prefix_clear(self._h, C.byref(freed)), "pa_prefix_clear")
+        return freed.value
+
+    def prefix_entries(self):
+        return int(lib().pa_prefix_entries(self._h))
 
     def table(self, seq):
         n, length = C.c_int32(), C.c_int32()

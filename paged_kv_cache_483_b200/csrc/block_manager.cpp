@@ -10,7 +10,7 @@ BlockManager::BlockManager(int32_t num_blocks, int32_t block_size,
                            const std::vector<int32_t>& order)
     : num_blocks_(num_blocks), block_size_(block_size),
       order_(order), rank_(num_blocks), refs_(num_blocks, 0),
-      is_free_(num_blocks, 1), n_free_(num_blocks) {
+      is_free_(num_blocks, 1), n_free_(num_blocks), cache_refs_(num_blocks, 0) {
   if (order_.empty()) {
     order_.resize(num_blocks);
     for (int32_t i = 0; i < num_blocks; ++i) order_[i] = i;
@@ -147,6 +147,8 @@ int64_t BlockManager::length(int32_t seq) const {
 
 std::vector<int64_t> BlockManager::fills() const {
   std::vector<int64_t> fill(num_blocks_, 0);
+  for (int32_t b = 0; b < num_blocks_; ++b)
+    if (cache_refs_[b]) fill[b] = block_size_;   // cached blocks are full
   for (const auto& kv : seqs_) {
     const Seq& s = kv.second;
     for (size_t j = 0; j < s.blocks.size(); ++j) {
@@ -187,6 +189,14 @@ bool BlockManager::validate() const {
       ++expect[b];
     }
   }
+  std::vector<uint8_t> in_seq(num_blocks_, 0);
+  for (const auto& kv : seqs_)
+    for (int32_t b : kv.second.blocks) in_seq[b] = 1;
+  int64_t cache_only = 0;
+  for (int32_t b = 0; b < num_blocks_; ++b) {
+    expect[b] += cache_refs_[b];
+    if (cache_refs_[b] && !in_seq[b]) cache_only += block_size_;
+  }
   std::vector<int64_t> fill = fills();
   int64_t nfree = 0;
   for (int32_t b = 0; b < num_blocks_; ++b) {
@@ -201,7 +211,101 @@ bool BlockManager::validate() const {
   }
   if (nfree != n_free_) return false;
   Snapshot s = snapshot();
-  return s.logical >= s.payload;
+  return s.logical + cache_only >= s.payload;
+}
+
+uint64_t BlockManager::phash(int32_t parent, uint64_t scope, uint64_t revision,
+                             const int32_t* tokens) const {
+  // FNV-1a over the entry's identity (parent entry, scope, revision, ids)
+  uint64_t h = 1469598103934665603ull;
+  auto mix = [&h](uint64_t v) {
+    for (int i = 0; i < 8; ++i) {
+      h ^= (v >> (8 * i)) & 0xFF;
+      h *= 1099511628211ull;
+    }
+  };
+  mix(uint64_t(int64_t(parent)));
+  mix(scope);
+  mix(revision);
+  for (int32_t i = 0; i < block_size_; ++i) mix(uint64_t(uint32_t(tokens[i])));
+  return h;
+}
+
+int32_t BlockManager::pfind(int32_t parent, uint64_t scope, uint64_t revision,
+                            const int32_t* tokens, uint64_t* hash_out) const {
+  const uint64_t h = phash(parent, scope, revision, tokens);
+  if (hash_out) *hash_out = h;
+  auto range = pidx_.equal_range(h);
+  for (auto it = range.first; it != range.second; ++it) {
+    const PEntry& e = pent_[it->second];
+    if (e.parent == parent && e.scope == scope && e.revision == revision &&
+        std::equal(e.tokens.begin(), e.tokens.end(), tokens))
+      return it->second;
+  }
+  return -1;
+}
+
+MgrStatus BlockManager::create_cached(int32_t seq, uint64_t scope, uint64_t revision,
+                                      const int32_t* tokens, int64_t n,
+                                      int64_t* hit_tokens) {
+  if (n < 0 || (n > 0 && !tokens)) return MgrStatus::invalid;
+  if (seqs_.count(seq)) return MgrStatus::dup_seq;
+  Seq s;
+  int32_t parent = -1;
+  for (int64_t end = block_size_; end <= n; end += block_size_) {
+    const int32_t e = pfind(parent, scope, revision, tokens + end - block_size_, nullptr);
+    if (e < 0) break;
+    s.blocks.push_back(pent_[e].block);
+    parent = e;
+  }
+  s.length = int64_t(s.blocks.size()) * block_size_;
+  for (int32_t b : s.blocks) ++refs_[b];
+  if (hit_tokens) *hit_tokens = s.length;
+  seqs_.emplace(seq, std::move(s));
+  return MgrStatus::ok;
+}
+
+MgrStatus BlockManager::publish(int32_t seq, uint64_t scope, uint64_t revision,
+                                const int32_t* tokens, int64_t n, int64_t* added) {
+  auto it = seqs_.find(seq);
+  if (it == seqs_.end()) return MgrStatus::unknown_seq;
+  if (n < 0 || (n > 0 && !tokens) || n > it->second.length) return MgrStatus::invalid;
+  const Seq& s = it->second;
+  int64_t count = 0;
+  int32_t parent = -1;
+  for (int64_t end = block_size_; end <= n; end += block_size_) {
+    const int32_t* blk_tokens = tokens + end - block_size_;
+    uint64_t h = 0;
+    int32_t e = pfind(parent, scope, revision, blk_tokens, &h);
+    if (e < 0) {
+      PEntry pe{parent, scope, revision,
+                std::vector<int32_t>(blk_tokens, blk_tokens + block_size_),
+                s.blocks[size_t(end / block_size_ - 1)], h};
+      e = int32_t(pent_.size());
+      pent_.push_back(std::move(pe));
+      pidx_.emplace(h, e);
+      ++refs_[pent_[e].block];
+      ++cache_refs_[pent_[e].block];
+      ++count;
+    }
+    parent = e;
+  }
+  if (added) *added = count;
+  return MgrStatus::ok;
+}
+
+int64_t BlockManager::prefix_clear() {
+  int64_t freed = 0;
+  for (const PEntry& e : pent_) {
+    --cache_refs_[e.block];
+    if (--refs_[e.block] == 0) {
+      give_back(e.block);
+      ++freed;
+    }
+  }
+  pent_.clear();
+  pidx_.clear();
+  return freed;
 }
 
 }  // namespace pa

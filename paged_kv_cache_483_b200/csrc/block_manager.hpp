@@ -8,6 +8,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cstddef>
 #include <queue>
 #include <unordered_map>
 #include <vector>
@@ -50,6 +51,22 @@ class BlockManager {
   int32_t num_blocks() const { return num_blocks_; }
   int32_t block_size() const { return block_size_; }
 
+  // Prefix cache ("vladkulikov.com modern-llms module 9 notebook", the
+  // prefix-hash trace): the block that ends at token `end` is identified by
+  // (scope, revision, every token id before `end`), at full block boundaries.
+  // create_cached: a new sequence starting with the longest run of leading
+  // full blocks whose keys are cached (shared, refcount + 1 each).
+  MgrStatus create_cached(int32_t seq, uint64_t scope, uint64_t revision,
+                          const int32_t* tokens, int64_t n, int64_t* hit_tokens);
+  // publish: key the sequence's full blocks among tokens[0, n) (n <= its
+  // length); a key already cached keeps its block.  The cache holds one
+  // reference per block it maps.
+  MgrStatus publish(int32_t seq, uint64_t scope, uint64_t revision,
+                    const int32_t* tokens, int64_t n, int64_t* added);
+  // Drop every cache reference; returns the blocks that became free.
+  int64_t prefix_clear();
+  int64_t prefix_entries() const { return int64_t(pent_.size()); }
+
  private:
   struct Seq {
     int64_t length = 0;
@@ -66,6 +83,24 @@ class BlockManager {
   // min-heap of the free blocks' positions in the allocation order
   std::priority_queue<int32_t, std::vector<int32_t>, std::greater<int32_t>> free_heap_;
   std::unordered_map<int32_t, Seq> seqs_;
+
+  // A key is stored as (its parent's entry, the block's own tokens): two
+  // keys are equal exactly when their parents are and their last
+  // block_size tokens are, so a chain of entries spells the whole prefix.
+  struct PEntry {
+    int32_t parent;        // entry of the previous block, -1 at the first
+    uint64_t scope, revision;
+    std::vector<int32_t> tokens;  // block_size ids
+    int32_t block;
+    uint64_t hash;
+  };
+  int32_t pfind(int32_t parent, uint64_t scope, uint64_t revision,
+                const int32_t* tokens, uint64_t* hash_out) const;
+  uint64_t phash(int32_t parent, uint64_t scope, uint64_t revision,
+                 const int32_t* tokens) const;
+  std::vector<PEntry> pent_;
+  std::unordered_multimap<uint64_t, int32_t> pidx_;
+  std::vector<int32_t> cache_refs_;  // per block: references the cache holds
 };
 
 }  // namespace pa

@@ -254,6 +254,35 @@ pa_status pa_seq_release(pa_pool* p, int32_t seq) {
   return from_mgr(p->mgr.release(seq));
 }
 
+pa_status pa_seq_create_cached(pa_pool* p, int32_t seq, uint64_t scope,
+                               uint64_t revision, const int32_t* tokens,
+                               int32_t n_tokens, int32_t* hit_tokens) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  int64_t hit = 0;
+  pa_status st = from_mgr(p->mgr.create_cached(seq, scope, revision, tokens, n_tokens, &hit));
+  if (st == PA_OK && hit_tokens) *hit_tokens = int32_t(hit);
+  return st;
+}
+
+pa_status pa_prefix_publish(pa_pool* p, int32_t seq, uint64_t scope,
+                            uint64_t revision, const int32_t* tokens,
+                            int32_t n_tokens, int32_t* added_blocks) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  int64_t added = 0;
+  pa_status st = from_mgr(p->mgr.publish(seq, scope, revision, tokens, n_tokens, &added));
+  if (st == PA_OK && added_blocks) *added_blocks = int32_t(added);
+  return st;
+}
+
+pa_status pa_prefix_clear(pa_pool* p, int32_t* freed_blocks) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  const int64_t freed = p->mgr.prefix_clear();
+  if (freed_blocks) *freed_blocks = int32_t(freed);
+  return PA_OK;
+}
+
+int64_t pa_prefix_entries(const pa_pool* p) { return p ? p->mgr.prefix_entries() : 0; }
+
 pa_status pa_seq_table(const pa_pool* p, int32_t seq, int32_t* blocks_out,
                        int32_t cap, int32_t* n_blocks, int32_t* length) {
   if (!p) return PA_ERR_INVALID_ARG;
