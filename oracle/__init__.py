@@ -18,6 +18,8 @@ Pages this oracle follows (cited by title and section):
     softmax and tiled attention) -- the (m, l, acc) recurrence.
   * "vladkulikov.com modern-llms module 9 notebook", prefix-hash trace --
     ``PrefixCache``: content-keyed identity of full blocks.
+  * "vladkulikov.com modern-llms module 9 notebook", KV quantisation --
+    ``quantize_rows``: per-row absmax integer codes.
 
 Parity status: every function is pinned by a ``-m "not gpu"`` test in
 ``tests/test_oracle_pins.py`` (page-printed traces, closed forms, brute force
@@ -26,6 +28,7 @@ in 40-digit decimal arithmetic, invariants).  No function is unpinned.
 
 from .kv_pool import KVPool, PoolError, PoolExhausted  # noqa: F401
 from .prefix_cache import PrefixCache, prefix_key, run_prefix_trace, trace_tokens  # noqa: F401
+from .quant import quantize_rows, dequantize_rows, fake_quantize_rows, stored_rows  # noqa: F401
 from .attention import (  # noqa: F401
     attention_two_pass, paged_attention, attention_tiled, partition_stats,
     combine_partitions, attention_split_kv, online_softmax_stats,
