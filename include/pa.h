@@ -73,7 +73,9 @@ typedef enum pa_status {
   PA_ERR_SCRATCH_LIMIT = 10   /* request needs more than the fixed scratch   */
 } pa_status;
 
-typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+/* PA_INT8: int8 codes with one float32 scale per (token, head) row; only
+ * through pa_pool_create_int8. */
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_INT8 = 2 } pa_dtype;
 
 /* Bits of the device error word. */
 #define PA_DEVERR_BLOCK_ID 1  /* block-table entry outside [0, num_blocks)   */
@@ -100,11 +102,39 @@ typedef struct pa_stats {
  * the first free id in this order ([P1] KVPool._allocate).  NULL = identity
  * order.  Copied; the caller may free it after the call.
  * Errors: PA_ERR_INVALID_ARG (non-positive size, not a permutation, exactly
- * one of k_cache/v_cache NULL, cache pointer not 16-byte aligned). */
+ * one of k_cache/v_cache NULL, cache pointer not 16-byte aligned, kv_dtype
+ * PA_INT8: use pa_pool_create_int8). */
 pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
                          int32_t num_kv_heads, int32_t head_dim,
                          pa_dtype kv_dtype, void* k_cache, void* v_cache,
                          const int32_t* alloc_order, pa_pool** out);
+
+/* Pool of int8 KV rows ([P2] KV quantisation experiment, 8 bits: per
+ * (token, head) row, scale = max|x| / 127 (1 for a zero row), code =
+ * round-half-even(x / scale) clipped to +-127, decided in float64; the
+ * scale is stored as float32 and a row reads back as code * scale).
+ *   kv_records: device bytes [num_blocks, num_kv_heads, PA_INT8_RECORD_BYTES],
+ *   16-byte aligned, caller-owned.  One record per (block, head):
+ *     [0, 2048)     K codes, 16 tokens x 128; token t's 16-byte chunk k is
+ *                   stored at t * 128 + (k ^ (t & 7)) * 16 (pre-swizzled)
+ *     [2048, 4096)  V codes, 128 rows d of 16 bytes (token t at d * 16 + t)
+ *     [4096, 4160)  16 float32 K scales, token order
+ *     [4160, 4224)  16 float32 V scales
+ *   A block's record moves with one bulk copy.  Only block_size 16 and
+ *   head_dim 128.
+ * On such a pool pa_append_kv / pa_reshape_and_cache take bf16 key/value
+ * [T, Hkv, 128] and quantise them into their slots; pa_cow_copy copies whole
+ * records; pa_decode (and pa_decode_append, as two launches) dequantise in
+ * the kernel for H / Hkv <= 8.  pa_prefill_chunk and groups above 8 return
+ * PA_ERR_UNSUPPORTED.
+ * Errors: PA_ERR_UNSUPPORTED (block_size != 16 or head_dim != 128),
+ * PA_ERR_INVALID_ARG (NULL or misaligned kv_records, bad size or order),
+ * PA_ERR_CUDA. */
+#define PA_INT8_RECORD_BYTES 4224
+pa_status pa_pool_create_int8(int32_t num_blocks, int32_t block_size,
+                              int32_t num_kv_heads, int32_t head_dim,
+                              void* kv_records, const int32_t* alloc_order,
+                              pa_pool** out);
 
 /* Destroy the manager, its staging area and error word (synchronises the
  * device first).  Never frees k_cache/v_cache.  NULL is a no-op. */

@@ -99,29 +99,48 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
       prefetch_tensormap(&tmV);
       const uint64_t pol = policy_evict_first();
       const int32_t* trow = p.tables + int64_t(b) * p.MB + blk0;
+      // Block ids in groups of 8, read one group ahead: an id read right
+      // before its copies puts a table round trip on every block.
+      auto load8 = [&](int base, int (&ids)[8]) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ids[u] = base + u < nblk ? trow[base + u] : 0;
+      };
+      int cur[8], nxt[8];
+      load8(0, cur);
+      load8(8, nxt);
       int issued = 0;
-      for (int i = 0; i < nblk; ++i) {
-        const int s = i % kDecStages, round = i / kDecStages;
-        if (round > 0 && !mbar_wait(&tail->empty[s], (round - 1) & 1)) {
-          raise_err(p.err, PA_DEVERR_TIMEOUT);
-          break;
+      bool stop = false;
+      for (int base = 0; base < nblk && !stop; base += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = base + u;
+          if (i >= nblk) break;
+          const int s = i % kDecStages, round = i / kDecStages;
+          if (round > 0 && !mbar_wait(&tail->empty[s], (round - 1) & 1)) {
+            raise_err(p.err, PA_DEVERR_TIMEOUT);
+            stop = true;
+            break;
+          }
+          const int blk = cur[u];
+          if (blk < 0 || blk >= p.NB) {
+            tail->stage_bad[s] = 1;
+            tail->any_bad = 1;
+            raise_err(p.err, PA_DEVERR_BLOCK_ID);
+            mbar_arrive(&tail->full[s]);
+          } else {
+            tail->stage_bad[s] = 0;
+            uint8_t* st = smem + s * kStageBytes;
+            mbar_arrive_expect_tx(&tail->full[s], kStageBytes);
+            tma_load_3d(st, &tmK, &tail->full[s], 0, kvh, blk * 16, pol);
+            tma_load_3d(st + 2048, &tmK, &tail->full[s], 64, kvh, blk * 16, pol);
+            tma_load_3d(st + 4096, &tmV, &tail->full[s], 0, kvh, blk * 16, pol);
+            tma_load_3d(st + 6144, &tmV, &tail->full[s], 64, kvh, blk * 16, pol);
+          }
+          issued = i + 1;
         }
-        const int blk = trow[i];
-        if (blk < 0 || blk >= p.NB) {
-          tail->stage_bad[s] = 1;
-          tail->any_bad = 1;
-          raise_err(p.err, PA_DEVERR_BLOCK_ID);
-          mbar_arrive(&tail->full[s]);
-        } else {
-          tail->stage_bad[s] = 0;
-          uint8_t* st = smem + s * kStageBytes;
-          mbar_arrive_expect_tx(&tail->full[s], kStageBytes);
-          tma_load_3d(st, &tmK, &tail->full[s], 0, kvh, blk * 16, pol);
-          tma_load_3d(st + 2048, &tmK, &tail->full[s], 64, kvh, blk * 16, pol);
-          tma_load_3d(st + 4096, &tmV, &tail->full[s], 0, kvh, blk * 16, pol);
-          tma_load_3d(st + 6144, &tmV, &tail->full[s], 64, kvh, blk * 16, pol);
-        }
-        issued = i + 1;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) cur[u] = nxt[u];
+        load8(base + 16, nxt);
       }
       // drain: no copy may still be landing in shared memory at exit
       for (int s = 0; s < kDecStages && s < issued; ++s) {
@@ -444,20 +463,29 @@ static cudaError_t launch_ring(const CUtensorMap* tmK, const CUtensorMap* tmV,
   return cudaGetLastError();
 }
 
+cudaError_t launch_decode_order(const int32_t* kv_lens, int32_t B, int32_t* order,
+                                cudaStream_t stream) {
+  decode_order_kernel<<<1, 1024, 0, stream>>>(kv_lens, B, order);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_combine(const float* ws, int32_t B, int32_t H, int32_t NP,
+                                  float* out, cudaStream_t stream) {
+  decode_combine_kernel<<<B * H, 128, 0, stream>>>(ws, B, H, NP, out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
                                const DecodeArgs& a, int sms,
                                cudaStream_t stream) {
   (void)sms;
   if (a.order) {
-    decode_order_kernel<<<1, 1024, 0, stream>>>(a.kv_lens, a.B, a.order);
-    cudaError_t eo = cudaGetLastError();
+    cudaError_t eo = launch_decode_order(a.kv_lens, a.B, a.order, stream);
     if (eo != cudaSuccess) return eo;
   }
   cudaError_t e = launch_ring<kRingStages>(tmK, tmV, a, stream);
   if (e != cudaSuccess || a.NP == 1) return e;
-  decode_combine_kernel<<<a.B * a.H, 128, 0, stream>>>(a.ws, a.B, a.H, a.NP,
-                                                       a.out);
-  return cudaGetLastError();
+  return launch_decode_combine(a.ws, a.B, a.H, a.NP, a.out, stream);
 }
 
 }  // namespace pa

@@ -1,0 +1,469 @@
+// Paged decode attention over an int8 KV pool: per-(token, head) rows of 128
+// int8 codes with one float32 scale each, head_dim 128, block_size 16, GQA
+// group G <= 8.  One CTA per (partition, KV head, sequence).
+//
+// What it computes: the decode of "docs.rs ferrum-kv 0.4.0 src/attention.rs"
+// (paged_attention, q_tokens = 1) on the K/V rows the pool holds, i.e.
+// k_j = code_k[j] * scale_k[j], v_j = code_v[j] * scale_v[j], the per-row
+// absmax quantisation of "vladkulikov.com modern-llms module 9 notebook"
+// (KV quantisation experiment, 8 bits), with the one-pass (m, l, acc) update
+// of "semidirectx cmu11-667 lecture19 infer_world.py", section 3.
+//
+// Same machinery as the bf16 decode (producer warp + TMA ring, four consumer
+// warps on tensor-core tiles, (m, l, O) merge, split partitions), with half
+// the bytes per token:
+//  * the pool keeps each (block, head) as one packed 4224-byte record
+//    [K codes 2 KB | V codes 2 KB | 16 K scales | 16 V scales], staged with a
+//    single bulk copy (one copy instruction per block: the producer thread's
+//    issue rate, not HBM, limited a design with one copy per array).  K rows
+//    are token-major with their 16-byte chunks stored pre-swizzled (chunk k of
+//    token t at k ^ (t & 7)); V is d-major (row d = the 16 tokens' codes);
+//  * S^T = K Q^T runs on the int8 tensor-core MMA (m16n8k32, s32
+//    accumulators) straight from the codes: Q is split per head into
+//    int8 hi and lo parts, q = sq (hi + lo / 254) (error <= max|q| / 64516
+//    per element), two MMAs per 32 columns, and
+//    q.k_j = sq scale_k[j] (acc_hi + acc_lo / 254);
+//  * O^T += V^T P^T runs on the fp16 MMA: two adjacent V codes become one
+//    half2 with a byte permute and one subtraction (fp16 holds 1024 + u
+//    exactly), and sum_j p_j v_j = 2^E sum_j (p_j scale_v[j] 2^-E) code_v[j]
+//    with 2^E the block's largest V scale (a power of two, so the fp16 P
+//    keeps its precision; O is rescaled by the ratio of successive 2^E
+//    together with the online-softmax factor).  P goes in as fp16 hi + lo
+//    parts; l sums the unscaled p_j.
+// Token order: row r of a block's S^T tile holds token kPerm[r].  With it a
+// thread's P^T fragment covers tokens 4c .. 4c + 3 (two per register), the
+// four bytes of one 32-bit word of a V d-row, and the K rows a warp reads at
+// once have distinct swizzle phases (no bank conflicts).
+#include <math.h>
+
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "launch.hpp"
+
+namespace pa {
+
+namespace {
+
+constexpr int kQ8Threads = 160;     // 4 consumer warps + 1 producer warp
+constexpr int kQ8Stages = 16;       // multiple of the 4 consumer warps
+constexpr int kQ8StageBytes = kQ8RecordBytes;  // one packed (block, head) record
+constexpr float kLog2e = 1.4426950408889634f;
+// S^T row r of a block holds token kPerm[r] (see the file comment)
+__constant__ int kPerm[16] = {0, 1, 4, 5, 10, 11, 14, 15, 2, 3, 6, 7, 8, 9, 12, 13};
+
+struct Q8Tail {
+  uint64_t full[kQ8Stages];
+  uint64_t empty[kQ8Stages];
+  int stage_bad[kQ8Stages];
+  int any_bad;
+};
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// D (s32) += A (16 x 32 s8, row) * B (32 x 8 s8, col)
+__device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t a1,
+                                             uint32_t a2, uint32_t a3, uint32_t b0,
+                                             uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D (f32) += A (16 x 16 f16, row) * B (16 x 8 f16, col)
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                              uint32_t a2, uint32_t a3, uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two codes of the biased word u = w ^ 0x80808080 (bytes picked by sel,
+// low then high) as an exact half2: the permute builds 0x64uu halves, i.e.
+// 1024 + u, and 1152 = 1024 + 128 taken away leaves the signed code.
+__device__ __forceinline__ uint32_t codes_half2(uint32_t u, uint32_t sel) {
+  const uint32_t x = __byte_perm(u, 0x64646464u, sel);
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&x),
+                            __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
+    const DecodeArgs p, float scale_log2) {
+  extern __shared__ uint8_t q8_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(q8_raw) + 127) & ~uintptr_t(127));
+  Q8Tail* tail = reinterpret_cast<Q8Tail*>(smem + kQ8Stages * kQ8StageBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int part = blockIdx.x, kvh = blockIdx.y;
+  const int b = p.order ? p.order[blockIdx.z] : int(blockIdx.z);
+  const int G = p.H / p.Hkv;
+  const int kv_len = p.kv_lens[b];
+  const bool len_bad = kv_len < 0 || kv_len > p.MB * 16;
+  const int nblk_seq = len_bad ? 0 : (kv_len + 15) >> 4;
+  const int blk0 = part * p.part_blocks;
+  const int nblk = max(0, min(blk0 + p.part_blocks, nblk_seq) - blk0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQ8Stages; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+      tail->stage_bad[s] = 0;
+    }
+    tail->any_bad = len_bad ? 1 : 0;
+    fence_barrier_init();
+    if (len_bad && part == 0 && kvh == 0) raise_err(p.err, PA_DEVERR_KV_LEN);
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nblk > 0) {
+      const uint64_t pol = policy_evict_first();
+      const int32_t* trow = p.tables + int64_t(b) * p.MB + blk0;
+      // Block ids in groups of 8, read one group ahead: an id read right
+      // before its copy puts a table round trip on every block.
+      auto load8 = [&](int base, int (&ids)[8]) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ids[u] = base + u < nblk ? trow[base + u] : 0;
+      };
+      int cur[8], nxt[8];
+      load8(0, cur);
+      load8(8, nxt);
+      int issued = 0;
+      bool stop = false;
+      for (int base = 0; base < nblk && !stop; base += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = base + u;
+          if (i >= nblk) break;
+          const int s = i % kQ8Stages, round = i / kQ8Stages;
+          if (round > 0 && !mbar_wait(&tail->empty[s], (round - 1) & 1)) {
+            raise_err(p.err, PA_DEVERR_TIMEOUT);
+            stop = true;
+            break;
+          }
+          const int blk = cur[u];
+          if (blk < 0 || blk >= p.NB) {
+            tail->stage_bad[s] = 1;
+            tail->any_bad = 1;
+            raise_err(p.err, PA_DEVERR_BLOCK_ID);
+            mbar_arrive(&tail->full[s]);
+          } else {
+            tail->stage_bad[s] = 0;
+            uint8_t* st = smem + s * kQ8StageBytes;
+            mbar_arrive_expect_tx(&tail->full[s], kQ8StageBytes);
+            bulk_load(st,
+                      static_cast<const uint8_t*>(p.k_cache) +
+                          (int64_t(blk) * p.Hkv + kvh) * kQ8StageBytes,
+                      kQ8StageBytes, &tail->full[s], pol);
+          }
+          issued = i + 1;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) cur[u] = nxt[u];
+        load8(base + 16, nxt);
+      }
+      // drain: no copy may still be landing in shared memory at exit
+      for (int s = 0; s < kQ8Stages && s < issued; ++s) {
+        const int count = (issued - 1 - s) / kQ8Stages + 1;
+        mbar_wait(&tail->full[s], (count - 1) & 1);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------- consumers
+  const int g = lane >> 2, c = lane & 3;
+  // Q of head g as int8 hi + lo parts in the B-fragment order of m16n8k32:
+  // word kk*2 + h covers d = 32 kk + 16 h + 4c .. + 3
+  uint32_t qh[4][2], ql[4][2];
+  float qs0, qs1;   // sq * scale_log2 of heads 2c and 2c + 1 (S^T columns)
+  {
+    const bool ok = g < G;
+    const uint2* qrow = reinterpret_cast<const uint2*>(
+        static_cast<const __nv_bfloat16*>(p.q) + (int64_t(b) * p.H + kvh * G + (ok ? g : 0)) * 128);
+    float x[4][2][4];
+    float amax = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint2 w = ok ? __ldg(qrow + 8 * kk + 4 * h + c) : make_uint2(0u, 0u);
+        x[kk][h][0] = __uint_as_float(w.x << 16);
+        x[kk][h][1] = __uint_as_float(w.x & 0xFFFF0000u);
+        x[kk][h][2] = __uint_as_float(w.y << 16);
+        x[kk][h][3] = __uint_as_float(w.y & 0xFFFF0000u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(x[kk][h][e]));
+      }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const float sq = amax > 0.f ? amax / 127.f : 1.f;
+    const float inv = amax > 0.f ? 127.f / amax : 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t hw = 0, lw = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float t = fminf(fmaxf(x[kk][h][e] * inv, -127.f), 127.f);
+          const float hi = rintf(t);
+          const float lo = rintf((t - hi) * 254.f);
+          hw |= (uint32_t(int32_t(hi)) & 0xFFu) << (8 * e);
+          lw |= (uint32_t(int32_t(lo)) & 0xFFu) << (8 * e);
+        }
+        qh[kk][h] = hw;
+        ql[kk][h] = lw;
+      }
+    qs0 = __shfl_sync(0xffffffffu, sq, 8 * c) * scale_log2;
+    qs1 = __shfl_sync(0xffffffffu, sq, 8 * c + 4) * scale_log2;
+  }
+  const int tokA = kPerm[g], tokB = kPerm[g + 8];       // tokens of S^T rows g, g + 8
+  const uint32_t rowA = tokA * 128, rowB = tokB * 128;
+  const uint32_t keyA = tokA & 7, keyB = tokB & 7;      // their swizzle phases
+  // V^T A fragments: tokens kPerm[2c], kPerm[2c+1] are bytes (0,1) of word c
+  // for c < 2 and bytes (2,3) otherwise; kPerm[2c+8], kPerm[2c+9] the others
+  const uint32_t sel_a = c < 2 ? 0x4140u : 0x4342u;
+  const uint32_t sel_b = c < 2 ? 0x4342u : 0x4140u;
+  float o[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float unit = 0.f;    // 2^-E of the warp's O (0 before its first block)
+  const int tok_end = kv_len;
+
+  // S^T of one staged block (rows g, g + 8 = tokens tokA, tokB), already in
+  // log2 units, -inf where the slot is past the sequence end; also returns
+  // the two rows' V scales (0 past the end).
+  auto block_scores = [&](uint32_t kb, int tb, float (&sc)[4], float& vA, float& vB) {
+    int ih[4] = {0, 0, 0, 0}, il[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint32_t c0 = 2 * kk, c1 = 2 * kk + 1;
+      const uint32_t a0 = lds32(kb + rowA + ((c0 ^ keyA) << 4) + 4 * c);
+      const uint32_t a2 = lds32(kb + rowA + ((c1 ^ keyA) << 4) + 4 * c);
+      const uint32_t a1 = lds32(kb + rowB + ((c0 ^ keyB) << 4) + 4 * c);
+      const uint32_t a3 = lds32(kb + rowB + ((c1 ^ keyB) << 4) + 4 * c);
+      mma_s8_16832(ih, a0, a1, a2, a3, qh[kk][0], qh[kk][1]);
+      mma_s8_16832(il, a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
+    }
+    const float* scl = reinterpret_cast<const float*>(smem + (kb - smem_u32(smem)) + 4096);
+    const bool live0 = tb + tokA < tok_end, live1 = tb + tokB < tok_end;
+    const float kA = scl[tokA], kB = scl[tokB];
+    sc[0] = live0 ? fmaf(float(il[0]), 1.f / 254.f, float(ih[0])) * (kA * qs0) : -INFINITY;
+    sc[1] = live0 ? fmaf(float(il[1]), 1.f / 254.f, float(ih[1])) * (kA * qs1) : -INFINITY;
+    sc[2] = live1 ? fmaf(float(il[2]), 1.f / 254.f, float(ih[2])) * (kB * qs0) : -INFINITY;
+    sc[3] = live1 ? fmaf(float(il[3]), 1.f / 254.f, float(ih[3])) * (kB * qs1) : -INFINITY;
+    // past the end: the V scale is zeroed so the (finite) codes add exactly 0
+    vA = live0 ? scl[16 + tokA] : 0.f;
+    vB = live1 ? scl[16 + tokB] : 0.f;
+  };
+  // O^T += V^T P^T for one staged block (P^T as fp16 hi + lo fragments)
+  auto block_pv = [&](uint32_t vb, uint32_t hb0, uint32_t hb1, uint32_t lb0, uint32_t lb1) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t w0 = lds32(vb + (16 * j + g) * 16 + 4 * c) ^ 0x80808080u;
+      const uint32_t w1 = lds32(vb + (16 * j + g + 8) * 16 + 4 * c) ^ 0x80808080u;
+      const uint32_t a0 = codes_half2(w0, sel_a), a2 = codes_half2(w0, sel_b);
+      const uint32_t a1 = codes_half2(w1, sel_a), a3 = codes_half2(w1, sel_b);
+      mma_f16_16816(o[j], a0, a1, a2, a3, hb0, hb1);
+      mma_f16_16816(o[j], a0, a1, a2, a3, lb0, lb1);
+    }
+  };
+
+  // Each warp takes its blocks two at a time (i and i + 4): one online-softmax
+  // step over 32 tokens, and two independent MMA chains to overlap.
+  for (int i = warp; i < nblk; i += 8) {
+    const int i2 = i + 4;
+    const int sa = i % kQ8Stages, sb = i2 % kQ8Stages;
+    const bool has2 = i2 < nblk;
+    bool landed = mbar_wait(&tail->full[sa], (i / kQ8Stages) & 1);
+    if (has2) landed = landed && mbar_wait(&tail->full[sb], (i2 / kQ8Stages) & 1);
+    if (!__all_sync(0xffffffffu, landed)) {
+      if (lane == 0) {
+        raise_err(p.err, PA_DEVERR_TIMEOUT);
+        tail->any_bad = 1;
+      }
+      break;
+    }
+    const bool use1 = !tail->stage_bad[sa], use2 = has2 && !tail->stage_bad[sb];
+    if (use1 || use2) {
+      const uint32_t k1 = smem_u32(smem + sa * kQ8StageBytes);
+      const uint32_t k2 = smem_u32(smem + sb * kQ8StageBytes);
+      float s1[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float s2[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float v1A = 0.f, v1B = 0.f, v2A = 0.f, v2B = 0.f;
+      if (use1) block_scores(k1, (blk0 + i) * 16, s1, v1A, v1B);
+      if (use2) block_scores(k2, (blk0 + i2) * 16, s2, v2A, v2B);
+      float x0 = fmaxf(fmaxf(s1[0], s1[2]), fmaxf(s2[0], s2[2]));
+      float x1 = fmaxf(fmaxf(s1[1], s1[3]), fmaxf(s2[1], s2[3]));
+      float vmax = fmaxf(fmaxf(v1A, v1B), fmaxf(v2A, v2B));
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, off));
+        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, off));
+        vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+      }
+      // a used block's first token is live, so x0 and x1 are finite here
+      const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
+      const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
+      float p1[4], p2[4];
+      p1[0] = exp2f(s1[0] - n0), p1[1] = exp2f(s1[1] - n1);
+      p1[2] = exp2f(s1[2] - n0), p1[3] = exp2f(s1[3] - n1);
+      p2[0] = exp2f(s2[0] - n0), p2[1] = exp2f(s2[1] - n1);
+      p2[2] = exp2f(s2[2] - n0), p2[3] = exp2f(s2[3] - n1);
+      l0 = l0 * al0 + ((p1[0] + p1[2]) + (p2[0] + p2[2]));
+      l1 = l1 * al1 + ((p1[1] + p1[3]) + (p2[1] + p2[3]));
+      m0 = n0;
+      m1 = n1;
+      // power-of-two V unit 2^(E+1) > the largest live V scale of the pair
+      const uint32_t e = min(max((__float_as_uint(vmax) >> 23) & 0xFFu, 1u), 252u);
+      const float bunit = __uint_as_float((253u - e) << 23);   // 2^-(E + 1)
+      const float ratio = unit == 0.f ? 1.f : bunit / unit;     // O in the new unit
+      unit = bunit;
+      const float r0 = al0 * ratio, r1 = al1 * ratio;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        o[j][0] *= r0;
+        o[j][1] *= r1;
+        o[j][2] *= r0;
+        o[j][3] *= r1;
+      }
+      auto frag = [&](const float (&pp)[4], float vA, float vB, uint32_t (&hb)[4]) {
+        const float q0 = pp[0] * (vA * bunit), q1 = pp[1] * (vA * bunit);
+        const float q2 = pp[2] * (vB * bunit), q3 = pp[3] * (vB * bunit);
+        const __half2 h01 = __floats2half2_rn(q0, q1), h23 = __floats2half2_rn(q2, q3);
+        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+        hb[0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
+        hb[1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
+        hb[2] = movmatrix_trans(pack_half2(q0 - f01.x, q1 - f01.y));
+        hb[3] = movmatrix_trans(pack_half2(q2 - f23.x, q3 - f23.y));
+      };
+      if (use1) {
+        uint32_t f[4];
+        frag(p1, v1A, v1B, f);
+        block_pv(k1 + 2048, f[0], f[1], f[2], f[3]);
+      }
+      if (use2) {
+        uint32_t f[4];
+        frag(p2, v2A, v2B, f);
+        block_pv(k2 + 2048, f[0], f[1], f[2], f[3]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&tail->empty[sa]);
+      if (has2) mbar_arrive(&tail->empty[sb]);
+    }
+  }
+  // O back to absolute units
+  if (unit > 0.f) {
+    const float back = 1.f / unit;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[j][k] *= back;
+  }
+
+  // ------------------------------------------- merge the four warps' states
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+  named_bar_sync(1, 128);  // every consumer is done with the ring
+  float* so = reinterpret_cast<float*>(smem);  // [4][8][128]
+  float* sm = so + 4 * 8 * 128;                // [4][8]
+  float* sl = sm + 32;                         // [4][8]
+  {
+    float* w0 = so + (warp * 8 + 2 * c) * 128;
+    float* w1 = w0 + 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      w0[16 * j + g] = o[j][0];
+      w1[16 * j + g] = o[j][1];
+      w0[16 * j + g + 8] = o[j][2];
+      w1[16 * j + g + 8] = o[j][3];
+    }
+    if (g == 0) {
+      sm[warp * 8 + 2 * c] = m0;
+      sm[warp * 8 + 2 * c + 1] = m1;
+      sl[warp * 8 + 2 * c] = l0;
+      sl[warp * 8 + 2 * c + 1] = l1;
+    }
+  }
+  named_bar_sync(1, 128);
+  const int t = threadIdx.x;  // d column
+  const bool zero = tail->any_bad != 0;
+  for (int n = 0; n < G; ++n) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[w * 8 + n]);
+    float num = 0.f, den = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float mw = sm[w * 8 + n];
+        const float sc = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+        num = fmaf(so[(w * 8 + n) * 128 + t], sc, num);
+        den = fmaf(sl[w * 8 + n], sc, den);
+      }
+    }
+    const float val = (den > 0.f && !zero) ? num / den : 0.f;
+    const int64_t bh = int64_t(b) * p.H + kvh * G + n;
+    if (p.NP == 1) {
+      p.out[bh * 128 + t] = val;
+    } else {
+      const int64_t slot = bh * p.NP + part;
+      float* ws_m = p.ws;
+      float* ws_l = ws_m + int64_t(p.B) * p.H * p.NP;
+      float* ws_o = ws_l + int64_t(p.B) * p.H * p.NP;
+      ws_o[slot * 128 + t] = val;
+      if (t == 0) {
+        ws_m[slot] = M;
+        ws_l[slot] = zero ? -1.f : den;  // -1 poisons the whole row
+      }
+    }
+  }
+}
+
+cudaError_t launch_decode_q8(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.order) {
+    cudaError_t eo = launch_decode_order(a.kv_lens, a.B, a.order, stream);
+    if (eo != cudaSuccess) return eo;
+  }
+  const size_t smem = 128 + kQ8Stages * kQ8StageBytes + sizeof(Q8Tail);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_q8_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid(a.NP, a.Hkv, a.B);
+  decode_q8_kernel<<<grid, kQ8Threads, smem, stream>>>(a, a.scale * kLog2e);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || a.NP == 1) return e;
+  return launch_decode_combine(a.ws, a.B, a.H, a.NP, a.out, stream);
+}
+
+}  // namespace pa

@@ -50,11 +50,87 @@ __global__ void __launch_bounds__(256) cow_copy_kernel(
       if (c == 0) raise_err(err, PA_DEVERR_BLOCK_ID);
       continue;
     }
-    const V kv = k_cache[int64_t(s) * block_vecs + c];
-    const V vv = v_cache[int64_t(s) * block_vecs + c];
-    k_cache[int64_t(d) * block_vecs + c] = kv;
-    v_cache[int64_t(d) * block_vecs + c] = vv;
+    k_cache[int64_t(d) * block_vecs + c] = k_cache[int64_t(s) * block_vecs + c];
+    if (v_cache) v_cache[int64_t(d) * block_vecs + c] = v_cache[int64_t(s) * block_vecs + c];
   }
+}
+
+// int8 pools: one warp per (token, head) row of K and of V.  The row's
+// absmax is exact in float32 (bf16 inputs); scale = absmax / 127 and the
+// codes rint(x / scale), clipped to +-127, are decided in float64 as the
+// quantisation experiment of "vladkulikov.com modern-llms module 9 notebook"
+// states; the scale is stored as float32.  Returns this lane's 4 codes
+// (d = 4 lane .. 4 lane + 3) packed in a word; lane 0 also stores the scale.
+__device__ __forceinline__ uint32_t quantize_row(const __nv_bfloat16* __restrict__ src,
+                                                 float* scale_dst, int lane) {
+  const uint2 w = *reinterpret_cast<const uint2*>(src + 4 * lane);
+  float x[4];
+  x[0] = __uint_as_float(w.x << 16);
+  x[1] = __uint_as_float(w.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(w.y << 16);
+  x[3] = __uint_as_float(w.y & 0xFFFF0000u);
+  float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  double scale = double(amax) / 127.0;
+  if (scale == 0.0) scale = 1.0;
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const double q = fmin(fmax(rint(double(x[i]) / scale), -127.0), 127.0);
+    packed |= (uint32_t(int32_t(q)) & 0xFFu) << (8 * i);
+  }
+  if (lane == 0) *scale_dst = __double2float_rn(scale);
+  return packed;
+}
+
+// Writes each row into its packed (block, head) record: K codes at
+// token * 128 + ((chunk ^ (token & 7)) << 4) + byte, V codes at 2048 + d * 16
+// + token, scales at 4096 + 4 token (K) and 4160 + 4 token (V).
+__global__ void __launch_bounds__(256) reshape_and_cache_q8_kernel(
+    const __nv_bfloat16* __restrict__ key, const __nv_bfloat16* __restrict__ value,
+    uint8_t* __restrict__ records, const int64_t* __restrict__ slot_mapping, int32_t T,
+    int32_t Hkv, int64_t num_slots, int32_t* err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = int64_t(T) * Hkv;
+  const int64_t stride = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r = blockIdx.x * int64_t(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+       r += stride) {
+    const int64_t t = r / Hkv;
+    const int h = int(r - t * Hkv);
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot < 0) continue;                    // padding token
+    if (slot >= num_slots) {
+      if (lane == 0 && h == 0) raise_err(err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const int tok = int(slot & 15);
+    uint8_t* rec = records + ((slot >> 4) * Hkv + h) * kQ8RecordBytes;
+    const uint32_t kw =
+        quantize_row(key + r * 128, reinterpret_cast<float*>(rec + 4096) + tok, lane);
+    const uint32_t vw =
+        quantize_row(value + r * 128, reinterpret_cast<float*>(rec + 4160) + tok, lane);
+    // lane covers d = 4 lane .. + 3: chunk lane / 4, byte 4 (lane % 4)
+    *reinterpret_cast<uint32_t*>(rec + tok * 128 + (((lane >> 2) ^ (tok & 7)) << 4) +
+                                 4 * (lane & 3)) = kw;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) rec[2048 + (4 * lane + i) * 16 + tok] = uint8_t(vw >> (8 * i));
+  }
+}
+
+cudaError_t launch_reshape_and_cache_q8(const void* key, const void* value, void* records,
+                                        const int64_t* slots, int32_t T, int32_t Hkv,
+                                        int64_t num_slots, int32_t* err, int sms,
+                                        cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  const int64_t rows = int64_t(T) * Hkv;
+  int64_t g = (rows + 7) / 8;
+  g = g > int64_t(sms) * 8 ? int64_t(sms) * 8 : g;
+  reshape_and_cache_q8_kernel<<<int(g < 1 ? 1 : g), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value),
+      static_cast<uint8_t*>(records), slots, T, Hkv, num_slots, err);
+  return cudaGetLastError();
 }
 
 static int grid_for(int64_t work, int sms) {

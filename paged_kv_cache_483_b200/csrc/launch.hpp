@@ -63,6 +63,27 @@ cudaError_t launch_decode_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
                                const DecodeArgs& a, int sms,
                                cudaStream_t stream);
 size_t split_workspace_bytes(int32_t B, int32_t H, int32_t NP, int32_t d);
+// Shared by the bf16 and int8 decodes: the longest-first order prepass and
+// the log-sum-exp combine of split partitions.
+cudaError_t launch_decode_order(const int32_t* kv_lens, int32_t B, int32_t* order,
+                                cudaStream_t stream);
+cudaError_t launch_decode_combine(const float* ws, int32_t B, int32_t H, int32_t NP,
+                                  float* out, cudaStream_t stream);
+
+// int8 pools: one packed record of kQ8RecordBytes per (block, head),
+// [NB, Hkv, record]: K codes [16 tokens][128] with each token's 16-byte
+// chunks stored swizzled (chunk k at k ^ (token & 7)), V codes [128 d][16
+// tokens], 16 float32 K scales, 16 float32 V scales.
+constexpr int kQ8RecordBytes = 4224;
+// Append: key/value bf16 [T, Hkv, 128] are quantised per (token, head) row
+// (absmax / 127, round half to even, decided in float64) into their slots.
+cudaError_t launch_reshape_and_cache_q8(const void* key, const void* value, void* records,
+                                        const int64_t* slots, int32_t T, int32_t Hkv,
+                                        int64_t num_slots, int32_t* err, int sms,
+                                        cudaStream_t stream);
+// Decode over an int8 pool (G <= 8; a.k_cache = the records), dequantising
+// in the kernel.
+cudaError_t launch_decode_q8(const DecodeArgs& a, cudaStream_t stream);
 // Scratch for the longest-first order when the grid spans several waves.
 bool decode_wants_order(int32_t B, int32_t Hkv, int32_t NP, int sms);
 size_t order_workspace_bytes(int32_t B);

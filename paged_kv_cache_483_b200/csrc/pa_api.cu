@@ -71,7 +71,9 @@ pa_status from_mgr(MgrStatus s) {
   }
 }
 
-size_t elem_bytes(pa_dtype t) { return t == PA_BF16 ? 2 : 4; }
+static_assert(pa::kQ8RecordBytes == PA_INT8_RECORD_BYTES, "int8 record size");
+
+size_t elem_bytes(pa_dtype t) { return t == PA_INT8 ? 1 : t == PA_BF16 ? 2 : 4; }
 
 bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
@@ -100,13 +102,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 bool make_pool_map(CUtensorMap* map, void* base, const pa_pool* p) {
   auto fn = encode_fn();
   if (!fn) return false;
+  // int8 pools: one box = the block's 16 rows of 128 codes (128 bytes)
+  const bool q8 = p->dtype == PA_INT8;
+  const cuuint64_t eb = q8 ? 1 : 2;
   const cuuint64_t dims[3] = {cuuint64_t(p->head_dim), cuuint64_t(p->num_kv_heads),
                               cuuint64_t(p->num_blocks) * p->block_size};
-  const cuuint64_t strides[2] = {cuuint64_t(p->head_dim) * 2,
-                                 cuuint64_t(p->head_dim) * p->num_kv_heads * 2};
-  const cuuint32_t box[3] = {64, 1, cuuint32_t(p->block_size)};
+  const cuuint64_t strides[2] = {cuuint64_t(p->head_dim) * eb,
+                                 cuuint64_t(p->head_dim) * p->num_kv_heads * eb};
+  const cuuint32_t box[3] = {q8 ? 128u : 64u, 1, cuuint32_t(p->block_size)};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides,
+  CUresult r = fn(map, q8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  3, base, dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -138,6 +144,8 @@ bool decode_partitions(const pa_pool* p, int32_t B, int32_t MB,
 }
 
 bool use_fast_decode(const pa_pool* p, int32_t H) {
+  if (p->dtype == PA_INT8)   // packed records, no tensor maps
+    return p->device && H % p->num_kv_heads == 0 && H / p->num_kv_heads <= 8;
   return p->tmap_ok && H % p->num_kv_heads == 0 &&
          pa::decode_fast_supported(p->dtype == PA_BF16, p->head_dim,
                                    p->block_size, H / p->num_kv_heads);
@@ -163,17 +171,17 @@ void free_split(pa_pool* p) {
 
 extern "C" {
 
-pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
-                         int32_t num_kv_heads, int32_t head_dim,
-                         pa_dtype kv_dtype, void* k_cache, void* v_cache,
-                         const int32_t* alloc_order, pa_pool** out) {
+// int8 pools pass their packed records as k_cache and no v_cache.
+static pa_status create_pool(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                             int32_t head_dim, pa_dtype kv_dtype, void* k_cache, void* v_cache,
+                             const int32_t* alloc_order, pa_pool** out) {
   if (!out) return PA_ERR_INVALID_ARG;
   *out = nullptr;
   if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
     return PA_ERR_INVALID_ARG;
-  if (kv_dtype != PA_F32 && kv_dtype != PA_BF16) return PA_ERR_INVALID_ARG;
-  if ((k_cache == nullptr) != (v_cache == nullptr)) return PA_ERR_INVALID_ARG;
-  if (k_cache && (!aligned16(k_cache) || !aligned16(v_cache)))
+  if (kv_dtype != PA_INT8 && (k_cache == nullptr) != (v_cache == nullptr))
+    return PA_ERR_INVALID_ARG;
+  if (k_cache && (!aligned16(k_cache) || (v_cache && !aligned16(v_cache))))
     return PA_ERR_INVALID_ARG;
   if (int64_t(num_blocks) * block_size > (int64_t(1) << 31) - 1)
     return PA_ERR_INVALID_ARG;
@@ -220,6 +228,28 @@ pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
   }
   *out = p;
   return PA_OK;
+}
+
+pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
+                         int32_t num_kv_heads, int32_t head_dim,
+                         pa_dtype kv_dtype, void* k_cache, void* v_cache,
+                         const int32_t* alloc_order, pa_pool** out) {
+  if (kv_dtype != PA_F32 && kv_dtype != PA_BF16) {
+    if (out) *out = nullptr;
+    return PA_ERR_INVALID_ARG;
+  }
+  return create_pool(num_blocks, block_size, num_kv_heads, head_dim, kv_dtype, k_cache,
+                     v_cache, alloc_order, out);
+}
+
+pa_status pa_pool_create_int8(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                              int32_t head_dim, void* kv_records, const int32_t* alloc_order,
+                              pa_pool** out) {
+  if (out) *out = nullptr;
+  if (block_size != 16 || head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (!kv_records) return PA_ERR_INVALID_ARG;
+  return create_pool(num_blocks, block_size, num_kv_heads, head_dim, PA_INT8, kv_records,
+                     nullptr, alloc_order, out);
 }
 
 pa_status pa_free(pa_pool* p) {
@@ -365,6 +395,34 @@ pa_status pa_validate(const pa_pool* p) {
   return p->mgr.validate() ? PA_OK : PA_ERR_INTERNAL;
 }
 
+// K2 for any pool: whole blocks of codes/values (and, for int8 pools, of
+// their scales).
+static cudaError_t cow_blocks(pa_pool* p, const int32_t* d_src, const int32_t* d_dst, int32_t n,
+                              cudaStream_t s) {
+  if (p->dtype == PA_INT8)   // one array of packed records
+    return pa::launch_cow_copy(p->k_cache, nullptr, d_src, d_dst, n,
+                               int64_t(p->num_kv_heads) * pa::kQ8RecordBytes, p->num_blocks,
+                               p->d_err, p->sms, s);
+  const size_t eb = elem_bytes(p->dtype);
+  return pa::launch_cow_copy(
+      p->k_cache, p->v_cache, d_src, d_dst, n,
+      int64_t(p->block_size) * p->num_kv_heads * p->head_dim * eb, p->num_blocks, p->d_err,
+      p->sms, s);
+}
+
+// K1 for any pool: copies rows, or quantises bf16 rows into an int8 pool.
+static cudaError_t write_rows(pa_pool* p, const void* key, const void* value,
+                              const int64_t* d_slots, int32_t T, cudaStream_t s) {
+  const int64_t num_slots = int64_t(p->num_blocks) * p->block_size;
+  if (p->dtype == PA_INT8)
+    return pa::launch_reshape_and_cache_q8(key, value, p->k_cache, d_slots, T,
+                                           p->num_kv_heads, num_slots, p->d_err, p->sms, s);
+  return pa::launch_reshape_and_cache(key, value, p->k_cache, p->v_cache, d_slots, T,
+                                      int64_t(p->num_kv_heads) * p->head_dim *
+                                          elem_bytes(p->dtype),
+                                      num_slots, p->d_err, p->sms, s);
+}
+
 pa_status pa_append_kv(pa_pool* p, const int32_t* seqs, const int32_t* n_new,
                        int32_t n_seqs, const void* key, const void* value,
                        int64_t* slot_mapping_out, void* stream) {
@@ -418,16 +476,8 @@ pa_status pa_append_kv(pa_pool* p, const int32_t* seqs, const int32_t* n_new,
     return PA_ERR_CUDA;
   const int64_t* d_slots = static_cast<const int64_t*>(r.dev);
   const int32_t* d_cow = reinterpret_cast<const int32_t*>(d_slots + T);
-  const size_t eb = elem_bytes(p->dtype);
-  cudaError_t e = pa::launch_cow_copy(
-      p->k_cache, p->v_cache, d_cow, d_cow + n_cow, n_cow,
-      int64_t(p->block_size) * p->num_kv_heads * p->head_dim * eb, p->num_blocks,
-      p->d_err, p->sms, s);
-  if (e == cudaSuccess)
-    e = pa::launch_reshape_and_cache(
-        key, value, p->k_cache, p->v_cache, d_slots, int32_t(T),
-        int64_t(p->num_kv_heads) * p->head_dim * eb,
-        int64_t(p->num_blocks) * p->block_size, p->d_err, p->sms, s);
+  cudaError_t e = cow_blocks(p, d_cow, d_cow + n_cow, n_cow, s);
+  if (e == cudaSuccess) e = write_rows(p, key, value, d_slots, int32_t(T), s);
   if (e != cudaSuccess) return PA_ERR_CUDA;
   if (cudaEventRecord(r.done, s) != cudaSuccess) return PA_ERR_CUDA;
   r.pending = true;
@@ -441,12 +491,8 @@ pa_status pa_reshape_and_cache(pa_pool* p, const void* key, const void* value,
   if (!p) return PA_ERR_INVALID_ARG;
   if (!p->device) return PA_ERR_NO_DEVICE;
   if (T < 0 || (T > 0 && (!key || !value || !d_slot_mapping))) return PA_ERR_INVALID_ARG;
-  const size_t eb = elem_bytes(p->dtype);
-  return cuda_status(pa::launch_reshape_and_cache(
-      key, value, p->k_cache, p->v_cache, d_slot_mapping, T,
-      int64_t(p->num_kv_heads) * p->head_dim * eb,
-      int64_t(p->num_blocks) * p->block_size, p->d_err, p->sms,
-      static_cast<cudaStream_t>(stream)));
+  return cuda_status(write_rows(p, key, value, d_slot_mapping, T,
+                                static_cast<cudaStream_t>(stream)));
 }
 
 pa_status pa_cow_copy(pa_pool* p, const int32_t* d_src, const int32_t* d_dst,
@@ -454,11 +500,7 @@ pa_status pa_cow_copy(pa_pool* p, const int32_t* d_src, const int32_t* d_dst,
   if (!p) return PA_ERR_INVALID_ARG;
   if (!p->device) return PA_ERR_NO_DEVICE;
   if (n < 0 || (n > 0 && (!d_src || !d_dst))) return PA_ERR_INVALID_ARG;
-  const size_t eb = elem_bytes(p->dtype);
-  return cuda_status(pa::launch_cow_copy(
-      p->k_cache, p->v_cache, d_src, d_dst, n,
-      int64_t(p->block_size) * p->num_kv_heads * p->head_dim * eb, p->num_blocks,
-      p->d_err, p->sms, static_cast<cudaStream_t>(stream)));
+  return cuda_status(cow_blocks(p, d_src, d_dst, n, static_cast<cudaStream_t>(stream)));
 }
 
 size_t pa_decode_workspace_bytes(const pa_pool* p, int32_t B, int32_t H,
@@ -515,6 +557,8 @@ static pa_status decode_fast(pa_pool* p, const void* q, int32_t B, int32_t H,
   a.new_slots = new_slots;
   a.k_cache = p->k_cache;
   a.v_cache = p->v_cache;
+  if (p->dtype == PA_INT8)
+    return cuda_status(pa::launch_decode_q8(a, static_cast<cudaStream_t>(stream)));
   return cuda_status(pa::launch_decode_fast(&p->tmK, &p->tmV, a, p->sms,
                                             static_cast<cudaStream_t>(stream)));
 }
@@ -547,6 +591,7 @@ pa_status pa_decode(pa_pool* p, const void* q, int32_t B, int32_t H,
     return decode_fast(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale,
                        partition_tokens, workspace, workspace_bytes, out, stream, nullptr,
                        nullptr, nullptr);
+  if (p->dtype == PA_INT8) return PA_ERR_UNSUPPORTED;   // G > 8 on an int8 pool
   if (partition_tokens % p->block_size) return PA_ERR_INVALID_ARG;
   pa::GenericArgs g{q, p->k_cache, p->v_cache, d_block_tables, max_blocks,
                     d_kv_lens, B, 1, H, p->num_kv_heads, p->head_dim,
@@ -565,7 +610,7 @@ pa_status pa_decode_append(pa_pool* p, const void* q, const void* key, const voi
   if (B > 0 && (!key || !value || !d_slot_mapping)) return PA_ERR_INVALID_ARG;
   if (partition_tokens < 0) return PA_ERR_INVALID_ARG;
   if (B == 0) return PA_OK;
-  if (!use_fast_decode(p, H)) {
+  if (!use_fast_decode(p, H) || p->dtype == PA_INT8) {
     // same result in two launches on the other paths
     st = pa_reshape_and_cache(p, key, value, d_slot_mapping, B, stream);
     if (st != PA_OK) return st;
@@ -587,6 +632,7 @@ pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,
                                       d_kv_lens, out);
   if (st != PA_OK) return st;
   if (q_tokens <= 0 || q_tokens > 65535 || max_kv_splits < 0) return PA_ERR_INVALID_ARG;
+  if (p->dtype == PA_INT8) return PA_ERR_UNSUPPORTED;
   if (B == 0) return PA_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_fast_prefill(p, H)) {

@@ -12,7 +12,7 @@ import torch
 
 import paged_kv_cache_483_b200 as pa
 import workloads
-from oracle import KVPool, paged_attention
+from oracle import KVPool, paged_attention, stored_rows
 
 
 def torch_dtype(w):
@@ -20,15 +20,22 @@ def torch_dtype(w):
 
 
 class GpuRun:
-    def __init__(self, w, device="cuda", init="zeros"):
+    def __init__(self, w, device="cuda", init="zeros", q8=False):
+        """q8: an int8 pool (packed (block, head) records) fed the same bf16 rows."""
         self.w = w
-        dt = torch_dtype(w)
-        shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
         alloc = torch.zeros if init == "zeros" else torch.empty
-        self.k_cache = alloc(shape, dtype=dt, device=device)
-        self.v_cache = alloc(shape, dtype=dt, device=device)
-        self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.dtype,
-                            self.k_cache, self.v_cache, alloc_order=w.order)
+        if q8:
+            self.records = alloc((w.num_blocks, w.num_kv_heads, pa.PA_INT8_RECORD_BYTES),
+                                 dtype=torch.uint8, device=device)
+            self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, "int8",
+                                self.records, None, alloc_order=w.order)
+        else:
+            dt = torch_dtype(w)
+            shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
+            self.k_cache = alloc(shape, dtype=dt, device=device)
+            self.v_cache = alloc(shape, dtype=dt, device=device)
+            self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim,
+                                w.dtype, self.k_cache, self.v_cache, alloc_order=w.order)
         self.slots = {}
         self.device = device
 
@@ -74,12 +81,15 @@ class GpuRun:
 
 
 class OracleRun:
-    def __init__(self, w, heads="all"):
+    def __init__(self, w, heads="all", q8=False):
+        """q8: store each row as an int8 pool reads it back (codes x float32
+        scale, float64)."""
         self.w = w
+        self.q8 = q8
         self.heads = list(range(w.num_kv_heads)) if heads == "all" else list(heads)
         self.pool = KVPool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim,
                            w.order, store_heads=self.heads,
-                           dtype=np.float64 if w.dtype == "f32" else np.float32)
+                           dtype=np.float64 if (w.dtype == "f32" or q8) else np.float32)
         self.slots, self.cows = {}, {}
 
     def apply(self, ops):
@@ -93,8 +103,10 @@ class OracleRun:
             elif op.kind == "append":
                 k, v = self.w.kv_for(op)
                 dt = self.pool.keys.dtype
-                s, c = self.pool.append(op.args[0], op.args[1], k.to(torch.float64).numpy().astype(dt),
-                                        v.to(torch.float64).numpy().astype(dt))
+                k64, v64 = k.to(torch.float64).numpy(), v.to(torch.float64).numpy()
+                if self.q8:        # the rows an int8 pool reads back
+                    k64, v64 = stored_rows(k64)[2], stored_rows(v64)[2]
+                s, c = self.pool.append(op.args[0], op.args[1], k64.astype(dt), v64.astype(dt))
                 self.slots[op.index], self.cows[op.index] = s, c
         return self
 
