@@ -14,8 +14,8 @@
 // the bytes per token:
 //  * the pool keeps each (block, head) as one packed 4224-byte record
 //    [K codes 2 KB | V codes 2 KB | 16 K scales | 16 V scales], staged with a
-//    single bulk copy (one copy instruction per block: the producer thread's
-//    issue rate, not HBM, limited a design with one copy per array).  K rows
+//    single TMA load (the records viewed as [NB * Hkv][33][128 bytes], one
+//    33-row box per record; one copy instruction per block).  K rows
 //    are token-major with their 16-byte chunks stored pre-swizzled (chunk k of
 //    token t at k ^ (t & 7)); V is d-major (row d = the 16 tokens' codes);
 //  * S^T = K Q^T runs on the int8 tensor-core MMA (m16n8k32, s32
@@ -105,7 +105,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 }  // namespace
 
 __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
-    const DecodeArgs p, float scale_log2) {
+    const __grid_constant__ CUtensorMap tmR, const DecodeArgs p, float scale_log2) {
   extern __shared__ uint8_t q8_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(q8_raw) + 127) & ~uintptr_t(127));
@@ -170,10 +170,7 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
             tail->stage_bad[s] = 0;
             uint8_t* st = smem + s * kQ8StageBytes;
             mbar_arrive_expect_tx(&tail->full[s], kQ8StageBytes);
-            bulk_load(st,
-                      static_cast<const uint8_t*>(p.k_cache) +
-                          (int64_t(blk) * p.Hkv + kvh) * kQ8StageBytes,
-                      kQ8StageBytes, &tail->full[s], pol);
+            tma_load_3d(st, &tmR, &tail->full[s], 0, 0, blk * p.Hkv + kvh, pol);
           }
           issued = i + 1;
         }
@@ -251,47 +248,10 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
   float unit = 0.f;    // 2^-E of the warp's O (0 before its first block)
   const int tok_end = kv_len;
 
-  // S^T of one staged block (rows g, g + 8 = tokens tokA, tokB), already in
-  // log2 units, -inf where the slot is past the sequence end; also returns
-  // the two rows' V scales (0 past the end).
-  auto block_scores = [&](uint32_t kb, int tb, float (&sc)[4], float& vA, float& vB) {
-    int ih[4] = {0, 0, 0, 0}, il[4] = {0, 0, 0, 0};
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint32_t c0 = 2 * kk, c1 = 2 * kk + 1;
-      const uint32_t a0 = lds32(kb + rowA + ((c0 ^ keyA) << 4) + 4 * c);
-      const uint32_t a2 = lds32(kb + rowA + ((c1 ^ keyA) << 4) + 4 * c);
-      const uint32_t a1 = lds32(kb + rowB + ((c0 ^ keyB) << 4) + 4 * c);
-      const uint32_t a3 = lds32(kb + rowB + ((c1 ^ keyB) << 4) + 4 * c);
-      mma_s8_16832(ih, a0, a1, a2, a3, qh[kk][0], qh[kk][1]);
-      mma_s8_16832(il, a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
-    }
-    const float* scl = reinterpret_cast<const float*>(smem + (kb - smem_u32(smem)) + 4096);
-    const bool live0 = tb + tokA < tok_end, live1 = tb + tokB < tok_end;
-    const float kA = scl[tokA], kB = scl[tokB];
-    sc[0] = live0 ? fmaf(float(il[0]), 1.f / 254.f, float(ih[0])) * (kA * qs0) : -INFINITY;
-    sc[1] = live0 ? fmaf(float(il[1]), 1.f / 254.f, float(ih[1])) * (kA * qs1) : -INFINITY;
-    sc[2] = live1 ? fmaf(float(il[2]), 1.f / 254.f, float(ih[2])) * (kB * qs0) : -INFINITY;
-    sc[3] = live1 ? fmaf(float(il[3]), 1.f / 254.f, float(ih[3])) * (kB * qs1) : -INFINITY;
-    // past the end: the V scale is zeroed so the (finite) codes add exactly 0
-    vA = live0 ? scl[16 + tokA] : 0.f;
-    vB = live1 ? scl[16 + tokB] : 0.f;
-  };
-  // O^T += V^T P^T for one staged block (P^T as fp16 hi + lo fragments)
-  auto block_pv = [&](uint32_t vb, uint32_t hb0, uint32_t hb1, uint32_t lb0, uint32_t lb1) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t w0 = lds32(vb + (16 * j + g) * 16 + 4 * c) ^ 0x80808080u;
-      const uint32_t w1 = lds32(vb + (16 * j + g + 8) * 16 + 4 * c) ^ 0x80808080u;
-      const uint32_t a0 = codes_half2(w0, sel_a), a2 = codes_half2(w0, sel_b);
-      const uint32_t a1 = codes_half2(w1, sel_a), a3 = codes_half2(w1, sel_b);
-      mma_f16_16816(o[j], a0, a1, a2, a3, hb0, hb1);
-      mma_f16_16816(o[j], a0, a1, a2, a3, lb0, lb1);
-    }
-  };
-
   // Each warp takes its blocks two at a time (i and i + 4): one online-softmax
-  // step over 32 tokens, and two independent MMA chains to overlap.
+  // step over 32 tokens, and the two blocks' loads and MMAs interleaved.  A
+  // missing or unusable block runs the same code with every token dead: its
+  // scores are -inf and its V scales 0, so its (finite) codes add exactly 0.
   for (int i = warp; i < nblk; i += 8) {
     const int i2 = i + 4;
     const int sa = i % kQ8Stages, sb = i2 % kQ8Stages;
@@ -305,68 +265,116 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
       }
       break;
     }
-    const bool use1 = !tail->stage_bad[sa], use2 = has2 && !tail->stage_bad[sb];
-    if (use1 || use2) {
-      const uint32_t k1 = smem_u32(smem + sa * kQ8StageBytes);
-      const uint32_t k2 = smem_u32(smem + sb * kQ8StageBytes);
-      float s1[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      float s2[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      float v1A = 0.f, v1B = 0.f, v2A = 0.f, v2B = 0.f;
-      if (use1) block_scores(k1, (blk0 + i) * 16, s1, v1A, v1B);
-      if (use2) block_scores(k2, (blk0 + i2) * 16, s2, v2A, v2B);
-      float x0 = fmaxf(fmaxf(s1[0], s1[2]), fmaxf(s2[0], s2[2]));
-      float x1 = fmaxf(fmaxf(s1[1], s1[3]), fmaxf(s2[1], s2[3]));
-      float vmax = fmaxf(fmaxf(v1A, v1B), fmaxf(v2A, v2B));
+    const bool use[2] = {!tail->stage_bad[sa], has2 && !tail->stage_bad[sb]};
+    const uint32_t kb[2] = {smem_u32(smem + sa * kQ8StageBytes),
+                            smem_u32(smem + sb * kQ8StageBytes)};
+    const float* scl[2] = {reinterpret_cast<const float*>(smem + sa * kQ8StageBytes + 4096),
+                           reinterpret_cast<const float*>(smem + sb * kQ8StageBytes + 4096)};
+    const int tb[2] = {(blk0 + i) * 16, (blk0 + i2) * 16};
+    // ---- S^T = K Q^T on int8 codes: hi and lo parts of Q
+    int ih[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, il[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, off));
-        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, off));
-        vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
-      }
-      // a used block's first token is live, so x0 and x1 are finite here
-      const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
-      const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
-      float p1[4], p2[4];
-      p1[0] = exp2f(s1[0] - n0), p1[1] = exp2f(s1[1] - n1);
-      p1[2] = exp2f(s1[2] - n0), p1[3] = exp2f(s1[3] - n1);
-      p2[0] = exp2f(s2[0] - n0), p2[1] = exp2f(s2[1] - n1);
-      p2[2] = exp2f(s2[2] - n0), p2[3] = exp2f(s2[3] - n1);
-      l0 = l0 * al0 + ((p1[0] + p1[2]) + (p2[0] + p2[2]));
-      l1 = l1 * al1 + ((p1[1] + p1[3]) + (p2[1] + p2[3]));
-      m0 = n0;
-      m1 = n1;
-      // power-of-two V unit 2^(E+1) > the largest live V scale of the pair
-      const uint32_t e = min(max((__float_as_uint(vmax) >> 23) & 0xFFu, 1u), 252u);
-      const float bunit = __uint_as_float((253u - e) << 23);   // 2^-(E + 1)
-      const float ratio = unit == 0.f ? 1.f : bunit / unit;     // O in the new unit
-      unit = bunit;
-      const float r0 = al0 * ratio, r1 = al1 * ratio;
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint32_t c0 = 2 * kk, c1 = 2 * kk + 1;
+      uint32_t a[2][4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        o[j][0] *= r0;
-        o[j][1] *= r1;
-        o[j][2] *= r0;
-        o[j][3] *= r1;
+      for (int x = 0; x < 2; ++x) {
+        a[x][0] = lds32(kb[x] + rowA + ((c0 ^ keyA) << 4) + 4 * c);
+        a[x][2] = lds32(kb[x] + rowA + ((c1 ^ keyA) << 4) + 4 * c);
+        a[x][1] = lds32(kb[x] + rowB + ((c0 ^ keyB) << 4) + 4 * c);
+        a[x][3] = lds32(kb[x] + rowB + ((c1 ^ keyB) << 4) + 4 * c);
       }
-      auto frag = [&](const float (&pp)[4], float vA, float vB, uint32_t (&hb)[4]) {
-        const float q0 = pp[0] * (vA * bunit), q1 = pp[1] * (vA * bunit);
-        const float q2 = pp[2] * (vB * bunit), q3 = pp[3] * (vB * bunit);
-        const __half2 h01 = __floats2half2_rn(q0, q1), h23 = __floats2half2_rn(q2, q3);
-        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-        hb[0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
-        hb[1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
-        hb[2] = movmatrix_trans(pack_half2(q0 - f01.x, q1 - f01.y));
-        hb[3] = movmatrix_trans(pack_half2(q2 - f23.x, q3 - f23.y));
-      };
-      if (use1) {
-        uint32_t f[4];
-        frag(p1, v1A, v1B, f);
-        block_pv(k1 + 2048, f[0], f[1], f[2], f[3]);
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        mma_s8_16832(ih[x], a[x][0], a[x][1], a[x][2], a[x][3], qh[kk][0], qh[kk][1]);
+        mma_s8_16832(il[x], a[x][0], a[x][1], a[x][2], a[x][3], ql[kk][0], ql[kk][1]);
       }
-      if (use2) {
-        uint32_t f[4];
-        frag(p2, v2A, v2B, f);
-        block_pv(k2 + 2048, f[0], f[1], f[2], f[3]);
+    }
+    float sc[2][4], vA[2], vB[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const bool live0 = use[x] && tb[x] + tokA < tok_end;
+      const bool live1 = use[x] && tb[x] + tokB < tok_end;
+      const float kA = scl[x][tokA], kB = scl[x][tokB];
+      sc[x][0] = live0 ? fmaf(float(il[x][0]), 1.f / 254.f, float(ih[x][0])) * (kA * qs0) : -INFINITY;
+      sc[x][1] = live0 ? fmaf(float(il[x][1]), 1.f / 254.f, float(ih[x][1])) * (kA * qs1) : -INFINITY;
+      sc[x][2] = live1 ? fmaf(float(il[x][2]), 1.f / 254.f, float(ih[x][2])) * (kB * qs0) : -INFINITY;
+      sc[x][3] = live1 ? fmaf(float(il[x][3]), 1.f / 254.f, float(ih[x][3])) * (kB * qs1) : -INFINITY;
+      vA[x] = live0 ? scl[x][16 + tokA] : 0.f;
+      vB[x] = live1 ? scl[x][16 + tokB] : 0.f;
+    }
+    float x0 = fmaxf(fmaxf(sc[0][0], sc[0][2]), fmaxf(sc[1][0], sc[1][2]));
+    float x1 = fmaxf(fmaxf(sc[0][1], sc[0][3]), fmaxf(sc[1][1], sc[1][3]));
+    float vmax = fmaxf(fmaxf(vA[0], vB[0]), fmaxf(vA[1], vB[1]));
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, off));
+      x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, off));
+      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+    }
+    if (x0 == -INFINITY) {          // nothing usable in the pair (bad blocks)
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tail->empty[sa]);
+        if (has2) mbar_arrive(&tail->empty[sb]);
+      }
+      continue;
+    }
+    const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
+    const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
+    float pp[2][4];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      pp[x][0] = exp2f(sc[x][0] - n0);
+      pp[x][1] = exp2f(sc[x][1] - n1);
+      pp[x][2] = exp2f(sc[x][2] - n0);
+      pp[x][3] = exp2f(sc[x][3] - n1);
+    }
+    l0 = l0 * al0 + ((pp[0][0] + pp[0][2]) + (pp[1][0] + pp[1][2]));
+    l1 = l1 * al1 + ((pp[0][1] + pp[0][3]) + (pp[1][1] + pp[1][3]));
+    m0 = n0;
+    m1 = n1;
+    // power-of-two V unit 2^(E+1) > the largest live V scale of the pair
+    const uint32_t e = min(max((__float_as_uint(vmax) >> 23) & 0xFFu, 1u), 252u);
+    const float bunit = __uint_as_float((253u - e) << 23);   // 2^-(E + 1)
+    const float ratio = unit == 0.f ? 1.f : bunit / unit;     // O in the new unit
+    unit = bunit;
+    const float r0 = al0 * ratio, r1 = al1 * ratio;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      o[j][0] *= r0;
+      o[j][1] *= r1;
+      o[j][2] *= r0;
+      o[j][3] *= r1;
+    }
+    // P^T (times V scale and unit) as fp16 B fragments: hi + lo parts
+    uint32_t fb[2][4];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const float q0 = pp[x][0] * (vA[x] * bunit), q1 = pp[x][1] * (vA[x] * bunit);
+      const float q2 = pp[x][2] * (vB[x] * bunit), q3 = pp[x][3] * (vB[x] * bunit);
+      const __half2 h01 = __floats2half2_rn(q0, q1), h23 = __floats2half2_rn(q2, q3);
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      fb[x][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
+      fb[x][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
+      fb[x][2] = movmatrix_trans(pack_half2(q0 - f01.x, q1 - f01.y));
+      fb[x][3] = movmatrix_trans(pack_half2(q2 - f23.x, q3 - f23.y));
+    }
+    // ---- O^T += V^T P^T: d rows 16j + g and 16j + g + 8, tokens 4c .. 4c + 3
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t w[2][2];
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        w[x][0] = lds32(kb[x] + 2048 + (16 * j + g) * 16 + 4 * c) ^ 0x80808080u;
+        w[x][1] = lds32(kb[x] + 2048 + (16 * j + g + 8) * 16 + 4 * c) ^ 0x80808080u;
+      }
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const uint32_t a0 = codes_half2(w[x][0], sel_a), a2 = codes_half2(w[x][0], sel_b);
+        const uint32_t a1 = codes_half2(w[x][1], sel_a), a3 = codes_half2(w[x][1], sel_b);
+        mma_f16_16816(o[j], a0, a1, a2, a3, fb[x][0], fb[x][1]);
+        mma_f16_16816(o[j], a0, a1, a2, a3, fb[x][2], fb[x][3]);
       }
     }
     __syncwarp();
@@ -446,7 +454,8 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
   }
 }
 
-cudaError_t launch_decode_q8(const DecodeArgs& a, cudaStream_t stream) {
+cudaError_t launch_decode_q8(const CUtensorMap* tmR, const DecodeArgs& a,
+                             cudaStream_t stream) {
   if (a.order) {
     cudaError_t eo = launch_decode_order(a.kv_lens, a.B, a.order, stream);
     if (eo != cudaSuccess) return eo;
@@ -460,7 +469,7 @@ cudaError_t launch_decode_q8(const DecodeArgs& a, cudaStream_t stream) {
     attr_set = true;
   }
   dim3 grid(a.NP, a.Hkv, a.B);
-  decode_q8_kernel<<<grid, kQ8Threads, smem, stream>>>(a, a.scale * kLog2e);
+  decode_q8_kernel<<<grid, kQ8Threads, smem, stream>>>(*tmR, a, a.scale * kLog2e);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.NP == 1) return e;
   return launch_decode_combine(a.ws, a.B, a.H, a.NP, a.out, stream);

@@ -81,9 +81,9 @@ cudaError_t launch_reshape_and_cache_q8(const void* key, const void* value, void
                                         const int64_t* slots, int32_t T, int32_t Hkv,
                                         int64_t num_slots, int32_t* err, int sms,
                                         cudaStream_t stream);
-// Decode over an int8 pool (G <= 8; a.k_cache = the records), dequantising
-// in the kernel.
-cudaError_t launch_decode_q8(const DecodeArgs& a, cudaStream_t stream);
+// Decode over an int8 pool (G <= 8; tmR maps the records as
+// {128 bytes, 33 rows, NB * Hkv}), dequantising in the kernel.
+cudaError_t launch_decode_q8(const CUtensorMap* tmR, const DecodeArgs& a, cudaStream_t stream);
 // Scratch for the longest-first order when the grid spans several waves.
 bool decode_wants_order(int32_t B, int32_t Hkv, int32_t NP, int sms);
 size_t order_workspace_bytes(int32_t B);

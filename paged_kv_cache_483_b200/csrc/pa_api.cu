@@ -119,6 +119,22 @@ bool make_pool_map(CUtensorMap* map, void* base, const pa_pool* p) {
   return r == CUDA_SUCCESS;
 }
 
+// int8 pools: the packed records viewed as {128 bytes, 33 rows, NB * Hkv};
+// one box = one whole record.
+bool make_record_map(CUtensorMap* map, void* base, const pa_pool* p) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {128, pa::kQ8RecordBytes / 128,
+                              cuuint64_t(p->num_blocks) * p->num_kv_heads};
+  const cuuint64_t strides[2] = {128, pa::kQ8RecordBytes};
+  const cuuint32_t box[3] = {128, pa::kQ8RecordBytes / 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // Blocks per partition for the tensor-core decode.  partition_tokens > 0 is
 // taken as given; 0 picks enough partitions for about two resident CTAs per
 // SM when the batch has fewer (sequence, KV head) groups than that.
@@ -214,6 +230,11 @@ static pa_status create_pool(int32_t num_blocks, int32_t block_size, int32_t num
     if (kv_dtype == PA_BF16 && head_dim == 128 && block_size == 16)
       p->tmap_ok = make_pool_map(&p->tmK, k_cache, p) &&
                    make_pool_map(&p->tmV, v_cache, p);
+    if (kv_dtype == PA_INT8 && !make_record_map(&p->tmK, k_cache, p)) {
+      cudaFree(p->d_err);
+      delete p;
+      return PA_ERR_CUDA;
+    }
     if (p->tmap_ok) {
       // without it the prefill runs unsplit
       const size_t slots = size_t(p->sms);
@@ -558,7 +579,7 @@ static pa_status decode_fast(pa_pool* p, const void* q, int32_t B, int32_t H,
   a.k_cache = p->k_cache;
   a.v_cache = p->v_cache;
   if (p->dtype == PA_INT8)
-    return cuda_status(pa::launch_decode_q8(a, static_cast<cudaStream_t>(stream)));
+    return cuda_status(pa::launch_decode_q8(&p->tmK, a, static_cast<cudaStream_t>(stream)));
   return cuda_status(pa::launch_decode_fast(&p->tmK, &p->tmV, a, p->sms,
                                             static_cast<cudaStream_t>(stream)));
 }
