@@ -181,16 +181,23 @@ class Dist:
 class Setup:
     """A workload brought up on the GPU through the C ABI (untimed)."""
 
-    def __init__(self, w, device):
+    def __init__(self, w, device, q8=False):
         import torch
         import paged_kv_cache_483_b200 as pa
-        self.w, self.device = w, device
-        dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-        shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
-        self.k_cache = torch.empty(shape, dtype=dt, device=device)
-        self.v_cache = torch.empty(shape, dtype=dt, device=device)
-        self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.dtype,
-                            self.k_cache, self.v_cache, alloc_order=w.order)
+        self.w, self.device, self.q8 = w, device, q8
+        if q8:    # int8 pool: packed (block, head) records, bf16 rows quantised on append
+            self.k_cache = torch.empty((w.num_blocks, w.num_kv_heads, pa.PA_INT8_RECORD_BYTES),
+                                       dtype=torch.uint8, device=device)
+            self.v_cache = None
+            self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, "int8",
+                                self.k_cache, None, alloc_order=w.order)
+        else:
+            dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+            shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
+            self.k_cache = torch.empty(shape, dtype=dt, device=device)
+            self.v_cache = torch.empty(shape, dtype=dt, device=device)
+            self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.dtype,
+                                self.k_cache, self.v_cache, alloc_order=w.order)
         for op in w.setup:
             if op.kind == "create":
                 self.pool.create(op.args[0])
@@ -231,7 +238,9 @@ class Setup:
         self.n_cow = 0 if self.cow_src is None else int(self.cow_src.numel())
 
 
-def decode_bytes(w, lens):
+def decode_bytes(w, lens, q8=False):
+    if q8:    # int8 records: K and V codes plus two float32 scales per (token, head)
+        return int(np.sum(lens.astype(np.int64))) * w.num_kv_heads * (2 * w.head_dim + 8)
     eb = 2 if w.dtype == "bf16" else 4
     return int(np.sum(lens.astype(np.int64))) * w.num_kv_heads * w.head_dim * 2 * eb
 
@@ -250,7 +259,10 @@ def run_ours(args, dist):
     builder = workloads.ALL[args.config]
     w = builder(seed=workloads.seed_for({"decode32": 2, "ragged256": 3, "splitk128k": 4,
                                          "prefill": 5}[args.config]) + 1000 * dist.rank)
-    S = Setup(w, device)
+    q8 = args.kv == "int8"
+    if q8 and w.q_tokens > 1:
+        raise SystemExit("--kv int8 applies to the decode workloads")
+    S = Setup(w, device, q8=q8)
     pool = S.pool
     is_prefill = w.q_tokens > 1
     part = w.partition_tokens
@@ -260,8 +272,9 @@ def run_ours(args, dist):
         S.q.shape[0], S.q.shape[1], S.tables.shape[1], part)
     split = ws_bytes > 0                    # a second launch: order prepass or combine
     order_only = ws_bytes == 4 * S.q.shape[0]
-    # decode steps fuse the new token's append into the decode kernel
-    fused = (not is_prefill) and S.slots is not None
+    # decode steps fuse the new token's append into the decode kernel (bf16;
+    # on an int8 pool the append is its own quantising launch)
+    fused = (not is_prefill) and S.slots is not None and not q8
     per_step = ((1 if S.n_cow else 0) + (1 if (S.slots is not None and not fused) else 0)
                 + (2 if split else 1))
     launches = {"n": 0}
@@ -328,26 +341,32 @@ def run_ours(args, dist):
                 "peak_source": f"{peak_kind} bf16_tflops (burst)"}
         extra = {"tflops": round(value, 2)}
     else:
-        kv = decode_bytes(w, lens)
+        kv = decode_bytes(w, lens, q8)
         value = dist.world * kv / (ms_step_max * 1e-3) / 1e9
-        metric = "decode KV HBM GB/s (fraction of B200 peak) and seqs/s at 8K ctx, GQA 32/8"
+        metric = ("decode int8-KV HBM GB/s (codes + scales read) and seqs/s at 8K ctx, GQA 32/8"
+                  if q8 else
+                  "decode KV HBM GB/s (fraction of B200 peak) and seqs/s at 8K ctx, GQA 32/8")
         unit = "GB/s"
         achieved = kv / (kern_ms * 1e-3) / 1e9
+        kname = "decode_q8_kernel" if q8 else "decode_mma_kernel"
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4),
-                "traffic": profiled_traffic("decode_mma.cu", w.name),
-                "kernel": ("decode_order_kernel + decode_mma_kernel" if order_only else
-                           "decode_mma_kernel + decode_combine_kernel" if split else
-                           "decode_mma_kernel"),
+                "traffic": profiled_traffic("decode_q8.cu" if q8 else "decode_mma.cu",
+                                            w.name + ("_int8" if q8 else "")),
+                "kernel": (f"decode_order_kernel + {kname}" if order_only else
+                           f"{kname} + decode_combine_kernel" if split else kname),
                 "kernel_ms": round(kern_ms, 5),
                 "algorithmic_bytes_per_launch": kv, "peak_source": f"{peak_kind} hbm_gbs"}
         extra = {"seqs_per_s": round(dist.world * len(w.decode_seqs) / (ms_step_max * 1e-3), 1),
                  "frac_of_peak": round(value / hbm, 4)}
+        if q8:
+            extra["kv_bytes_vs_bf16"] = round(kv / decode_bytes(w, lens), 4)
     res = {
         "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": dist.world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded N(0,1), bf16-rounded)",
+        "dtype": "int8 KV codes (int8/fp16 MMA, fp32 softmax), bf16 Q" if q8 else "bf16",
+        "data": "synthetic (seeded N(0,1), bf16-rounded)",
         "config": config_of(w, args, dist),
         **extra,
         "host_plan_us": None if S.host_plan_us is None else round(S.host_plan_us, 1),
@@ -356,7 +375,7 @@ def run_ours(args, dist):
         "e2e": e2e,
         "clocks": clk.summary(),
     }
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and not q8:
         res["cpu_baseline"] = cpu_baseline(w, args)
     pool.close()
     return res
@@ -370,6 +389,7 @@ def config_of(w, args, dist):
             "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
             "q_tokens": w.q_tokens, "partition_tokens": w.partition_tokens,
             "parallelism": f"replicas x{dist.world} (no collective)",
+            "kv": getattr(args, "kv", "bf16"),
             "l2": "inputs larger than L2 (KV per step > 126 MB)" if w.name != "ragged256"
             else "KV per step ~0.5 GB > L2 (shared prefixes may hit in L2)"}
 
@@ -431,7 +451,7 @@ def run_e2e(args, S, dist, device, is_prefill, part):
         v = dist.world * prefill_flops(w, S.lens_h) / (ms * 1e-3) / 1e12
         unit = "TFLOP/s"
     else:
-        v = dist.world * decode_bytes(w, S.lens_h) / (ms * 1e-3) / 1e9
+        v = dist.world * decode_bytes(w, S.lens_h, S.q8) / (ms * 1e-3) / 1e9
         unit = "GB/s"
     return {"value": round(v, 2), "unit": unit, "h2d_bytes_per_step": int(bi),
             "d2h_bytes_per_step": int(bo), "ms_per_step": round(ms, 5), "steps": K}
@@ -549,6 +569,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv", choices=["bf16", "int8"], default="bf16",
+                    help="KV pool type for the decode workloads (int8: per-row absmax codes)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
