@@ -20,6 +20,8 @@ Pages this oracle follows (cited by title and section):
     ``PrefixCache``: content-keyed identity of full blocks.
   * "vladkulikov.com modern-llms module 9 notebook", KV quantisation --
     ``quantize_rows``: per-row absmax integer codes.
+  * "vladkulikov.com modern-llms module 9 notebook", streaming and
+    sliding-window caches -- ``visible_positions``: sink + recent window.
 
 Parity status: every function is pinned by a ``-m "not gpu"`` test in
 ``tests/test_oracle_pins.py`` (page-printed traces, closed forms, brute force
@@ -32,4 +34,5 @@ from .quant import quantize_rows, dequantize_rows, fake_quantize_rows, stored_ro
 from .attention import (  # noqa: F401
     attention_two_pass, paged_attention, attention_tiled, partition_stats,
     combine_partitions, attention_split_kv, online_softmax_stats,
+    visible_positions, attention_window,
 )

@@ -185,3 +185,25 @@ def attention_split_kv(q, k, v, partition, scale=None):
              for p in range(parts)]
     return combine_partitions([s[0] for s in stats], [s[1] for s in stats],
                               [s[2] for s in stats])
+
+
+def visible_positions(kv_len, window, sinks=0):
+    """Key positions one decode step sees under a sink + recent window.
+
+    "vladkulikov.com modern-llms module 9 notebook", ``streaming_keep_indices``
+    with budget = sinks + window: the first ``sinks`` positions and the most
+    recent ``window``; everything when kv_len <= budget.  With sinks = 0 this
+    is the sliding-window cache of the same page (``NumpyKVCacheExplicit``:
+    the last ``window`` positions survive)."""
+    kv_len, window, sinks = int(kv_len), int(window), int(sinks)
+    if window < 1 or sinks < 0:
+        raise ValueError("window must be >= 1 and sinks >= 0")
+    head = list(range(min(sinks, kv_len)))
+    start = max(len(head), kv_len - window)
+    return head + list(range(start, kv_len))
+
+
+def attention_window(q, k, v, window, sinks=0, scale=None):
+    """Decode attention (q_tokens = 1) over the visible positions only."""
+    idx = visible_positions(np.asarray(k).shape[0], window, sinks)
+    return attention_two_pass(q, np.asarray(k)[idx], np.asarray(v)[idx], scale)
