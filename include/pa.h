@@ -286,6 +286,26 @@ pa_status pa_decode(pa_pool* pool, const void* q, int32_t B, int32_t H,
                     int32_t partition_tokens, void* workspace,
                     size_t workspace_bytes, float* out, void* stream);
 
+/* Decode attention over a sink + recent window ([P2] streaming_keep_indices
+ * with budget = sinks + window, and its sliding-window cache for sinks = 0):
+ * key j of sequence b is visible iff j < kv_lens[b] and (j < sinks or
+ * j >= kv_lens[b] - window); with kv_lens[b] <= sinks + window every key is.
+ * The kernels walk only the blocks that hold a visible key, so a long
+ * sequence costs about sinks + window tokens.  Arguments, layouts and errors
+ * as pa_decode, plus window >= 1 and sinks >= 0 (else INVALID_ARG); the
+ * tensor-core paths only (bf16 or int8 pool, block 16, head_dim 128,
+ * H / Hkv <= 8), else PA_ERR_UNSUPPORTED.  partition_tokens splits the walked
+ * blocks; workspace: pa_decode_window_workspace_bytes bytes. */
+size_t pa_decode_window_workspace_bytes(const pa_pool* pool, int32_t B, int32_t H,
+                                        int32_t max_blocks, int32_t window,
+                                        int32_t sinks, int32_t partition_tokens);
+pa_status pa_decode_window(pa_pool* pool, const void* q, int32_t B, int32_t H,
+                           const int32_t* d_block_tables, int32_t max_blocks,
+                           const int32_t* d_kv_lens, float scale, int32_t window,
+                           int32_t sinks, int32_t partition_tokens,
+                           void* workspace, size_t workspace_bytes, float* out,
+                           void* stream);
+
 /* Decode step with the new token's append fused in: for each sequence b,
  * token kv_lens[b] - 1 is the one being decoded; its K/V rows
  * key[b]/value[b] (device [B, Hkv, head_dim], pool dtype) are written to pool

@@ -33,7 +33,8 @@ EXPORTS = ["pa_pool_create", "pa_free", "pa_seq_create", "pa_seq_fork", "pa_seq_
            "pa_cow_copy", "pa_decode_workspace_bytes", "pa_decode", "pa_prefill_chunk",
            "pa_get_error", "pa_status_string", "pa_decode_path", "pa_prefill_path",
            "pa_decode_static_scratch", "pa_decode_append", "pa_seq_create_cached",
-           "pa_prefix_publish", "pa_prefix_clear", "pa_prefix_entries", "pa_pool_create_int8"]
+           "pa_prefix_publish", "pa_prefix_clear", "pa_prefix_entries", "pa_pool_create_int8",
+           "pa_decode_window", "pa_decode_window_workspace_bytes"]
 
 
 class PAError(RuntimeError):
@@ -84,6 +85,9 @@ def lib():
         "pa_cow_copy": ([_P, _P, _P, _I32, _P], C.c_int),
         "pa_decode_workspace_bytes": ([_P, _I32, _I32, _I32, _I32], _SZ),
         "pa_decode": ([_P, _P, _I32, _I32, _P, _I32, _P, _F, _I32, _P, _SZ, _P, _P], C.c_int),
+        "pa_decode_window": ([_P, _P, _I32, _I32, _P, _I32, _P, _F, _I32, _I32, _I32, _P, _SZ,
+                              _P, _P], C.c_int),
+        "pa_decode_window_workspace_bytes": ([_P, _I32, _I32, _I32, _I32, _I32, _I32], _SZ),
         "pa_prefill_chunk": ([_P, _P, _I32, _I32, _I32, _P, _I32, _P, _F, _I32, _P, _P],
                              C.c_int),
         "pa_get_error": ([_P, _PI32], C.c_int),
@@ -340,6 +344,32 @@ class Pool:
                                workspace.numel() if need else 0,
                                _dev_ptr(out, torch.float32, "out"), _stream(stream)),
                "pa_decode")
+        return out
+
+    def decode_window(self, q, block_tables, kv_lens, window, sinks=0, out=None, scale=None,
+                      partition_tokens=0, workspace=None, stream=None):
+        """Decode over a sink + recent window: key j visible iff j < sinks or
+        j >= kv_len - window."""
+        import torch
+        B, H, d = q.shape
+        MB = block_tables.shape[1]
+        if out is None:
+            out = torch.empty((B, H, d), dtype=torch.float32, device=q.device)
+        scale = 1.0 / math.sqrt(self.head_dim) if scale is None else scale
+        need = int(lib().pa_decode_window_workspace_bytes(self._h, B, H, MB, int(window),
+                                                          int(sinks), int(partition_tokens)))
+        if need and workspace is None:
+            if self._ws is None or self._ws.numel() < need:
+                self._ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+            workspace = self._ws
+        wp = _dev_ptr(workspace, None, "workspace") if need else None
+        _check(lib().pa_decode_window(self._h, _dev_ptr(q, self._torch_dtype(), "q"), B, H,
+                                      _dev_ptr(block_tables, torch.int32, "block_tables"), MB,
+                                      _dev_ptr(kv_lens, torch.int32, "kv_lens"), float(scale),
+                                      int(window), int(sinks), int(partition_tokens), wp,
+                                      workspace.numel() if need else 0,
+                                      _dev_ptr(out, torch.float32, "out"), _stream(stream)),
+               "pa_decode_window")
         return out
 
     def decode_append(self, q, key, value, slot_mapping, block_tables, kv_lens, out=None,

@@ -77,8 +77,16 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
   const int kv_len = p.kv_lens[b];
   const bool len_bad = kv_len < 0 || kv_len > p.MB * 16;
   const int nblk_seq = len_bad ? 0 : (kv_len + 15) >> 4;
+  // Sink + recent window (window > 0): key j is visible iff j < sinks or
+  // j >= lo.  The CTAs walk the visible blocks only -- [0, sb) then [lb,
+  // nblk_seq) -- numbered 0 .. nvis - 1; with no window it is every block.
+  const int lo = (p.window > 0 && !len_bad) ? max(0, kv_len - p.window) : 0;
+  const int sb = (min(p.sinks, kv_len) + 15) >> 4, lb = lo >> 4;
+  const bool gap = lb > sb;
+  const int nvis = gap ? sb + (nblk_seq - lb) : nblk_seq;
+  auto vis_blk = [&](int v) { return (gap && v >= sb) ? lb + (v - sb) : v; };
   const int blk0 = part * p.part_blocks;
-  const int nblk = max(0, min(blk0 + p.part_blocks, nblk_seq) - blk0);
+  const int nblk = max(0, min(blk0 + p.part_blocks, nvis) - blk0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
@@ -98,12 +106,12 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
       const uint64_t pol = policy_evict_first();
-      const int32_t* trow = p.tables + int64_t(b) * p.MB + blk0;
+      const int32_t* trow = p.tables + int64_t(b) * p.MB;
       // Block ids in groups of 8, read one group ahead: an id read right
       // before its copies puts a table round trip on every block.
       auto load8 = [&](int base, int (&ids)[8]) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) ids[u] = base + u < nblk ? trow[base + u] : 0;
+        for (int u = 0; u < 8; ++u) ids[u] = base + u < nblk ? trow[vis_blk(blk0 + base + u)] : 0;
       };
       int cur[8], nxt[8];
       load8(0, cur);
@@ -155,7 +163,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
   // Fused append: the CTA whose partition holds token kv_len-1 writes that
   // token's K/V row of its KV head into the pool (and patches it into the
   // staged tile below, so the TMA copy of the stale slot is never used).
-  const bool appends = p.new_k != nullptr && nblk > 0 && blk0 + nblk == nblk_seq;
+  const bool appends = p.new_k != nullptr && nblk > 0 && blk0 + nblk == nvis;
   const int64_t new_slot = appends ? p.new_slots[b] : -1;
   if (appends && warp == 0) {
     if (new_slot >= int64_t(p.NB) * 16) {
@@ -209,8 +217,9 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
     if (!tail->stage_bad[s]) {
       const uint32_t kb = smem_u32(smem + s * kStageBytes);
       const uint32_t vb = kb + 4096;
-      const int valid = min(16, tok_end - (blk0 + i) * 16);
-      if (appends && new_slot >= 0 && new_slot < int64_t(p.NB) * 16 && blk0 + i == nblk_seq - 1) {
+      const int tb = vis_blk(blk0 + i) * 16;
+      const int valid = min(16, tok_end - tb);
+      if (appends && new_slot >= 0 && new_slot < int64_t(p.NB) * 16 && tb == (nblk_seq - 1) * 16) {
         // the new token's row: 2 x 128 bytes in each of the K and V tiles
         const int row = valid - 1, ch = lane & 15;
         const uint4* src = reinterpret_cast<const uint4*>(lane < 16 ? p.new_k : p.new_v) +
@@ -239,18 +248,19 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
         ldmatrix_x4(kb + (ch >> 3) * 2048 + swz128(ld_row, ch & 7), a0, a1, a2, a3);
         mma_bf16_16816(sc, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
       }
-      const int tb = (blk0 + i) * 16;
       float s0 = sc[0] * scale_log2, s1 = sc[1] * scale_log2;
       float s2 = sc[2] * scale_log2, s3 = sc[3] * scale_log2;
-      if (tb + g >= tok_end) s0 = s1 = -INFINITY;
-      if (tb + g + 8 >= tok_end) s2 = s3 = -INFINITY;
+      // past the end, or outside the window
+      auto hidden = [&](int t) { return t >= tok_end || (t < lo && t >= p.sinks); };
+      if (hidden(tb + g)) s0 = s1 = -INFINITY;
+      if (hidden(tb + g + 8)) s2 = s3 = -INFINITY;
       float x0 = fmaxf(s0, s2), x1 = fmaxf(s1, s3);
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
         x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, off));
         x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, off));
       }
-      // token tb < tok_end, so x0 and x1 are finite here
+      // every walked block holds a visible key, so x0 and x1 are finite here
       const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
       const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
       const float p0 = exp2f(s0 - n0), p2 = exp2f(s2 - n0);

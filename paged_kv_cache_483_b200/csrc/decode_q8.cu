@@ -118,8 +118,16 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
   const int kv_len = p.kv_lens[b];
   const bool len_bad = kv_len < 0 || kv_len > p.MB * 16;
   const int nblk_seq = len_bad ? 0 : (kv_len + 15) >> 4;
+  // Sink + recent window (window > 0): key j is visible iff j < sinks or
+  // j >= lo; the CTAs walk the visible blocks only ([0, sb), then [lb,
+  // nblk_seq)), numbered 0 .. nvis - 1.
+  const int lo = (p.window > 0 && !len_bad) ? max(0, kv_len - p.window) : 0;
+  const int sb = (min(p.sinks, kv_len) + 15) >> 4, lb = lo >> 4;
+  const bool gap = lb > sb;
+  const int nvis = gap ? sb + (nblk_seq - lb) : nblk_seq;
+  auto vis_blk = [&](int v) { return (gap && v >= sb) ? lb + (v - sb) : v; };
   const int blk0 = part * p.part_blocks;
-  const int nblk = max(0, min(blk0 + p.part_blocks, nblk_seq) - blk0);
+  const int nblk = max(0, min(blk0 + p.part_blocks, nvis) - blk0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQ8Stages; ++s) {
@@ -137,12 +145,12 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
     // ------------------------------------------------------------ producer
     if (lane == 0 && nblk > 0) {
       const uint64_t pol = policy_evict_first();
-      const int32_t* trow = p.tables + int64_t(b) * p.MB + blk0;
+      const int32_t* trow = p.tables + int64_t(b) * p.MB;
       // Block ids in groups of 8, read one group ahead: an id read right
       // before its copy puts a table round trip on every block.
       auto load8 = [&](int base, int (&ids)[8]) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) ids[u] = base + u < nblk ? trow[base + u] : 0;
+        for (int u = 0; u < 8; ++u) ids[u] = base + u < nblk ? trow[vis_blk(blk0 + base + u)] : 0;
       };
       int cur[8], nxt[8];
       load8(0, cur);
@@ -270,7 +278,7 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
                             smem_u32(smem + sb * kQ8StageBytes)};
     const float* scl[2] = {reinterpret_cast<const float*>(smem + sa * kQ8StageBytes + 4096),
                            reinterpret_cast<const float*>(smem + sb * kQ8StageBytes + 4096)};
-    const int tb[2] = {(blk0 + i) * 16, (blk0 + i2) * 16};
+    const int tb[2] = {vis_blk(blk0 + i) * 16, vis_blk(blk0 + i2) * 16};
     // ---- S^T = K Q^T on int8 codes: hi and lo parts of Q
     int ih[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, il[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
@@ -293,8 +301,9 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
     float sc[2][4], vA[2], vB[2];
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
-      const bool live0 = use[x] && tb[x] + tokA < tok_end;
-      const bool live1 = use[x] && tb[x] + tokB < tok_end;
+      const int t0 = tb[x] + tokA, t1 = tb[x] + tokB;
+      const bool live0 = use[x] && t0 < tok_end && (t0 >= lo || t0 < p.sinks);
+      const bool live1 = use[x] && t1 < tok_end && (t1 >= lo || t1 < p.sinks);
       const float kA = scl[x][tokA], kB = scl[x][tokB];
       sc[x][0] = live0 ? fmaf(float(il[x][0]), 1.f / 254.f, float(ih[x][0])) * (kA * qs0) : -INFINITY;
       sc[x][1] = live0 ? fmaf(float(il[x][1]), 1.f / 254.f, float(ih[x][1])) * (kA * qs1) : -INFINITY;

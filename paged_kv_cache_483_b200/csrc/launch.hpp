@@ -57,6 +57,10 @@ struct DecodeArgs {
   const int64_t* new_slots;
   void* k_cache;
   void* v_cache;
+  // sink + recent window (window <= 0: every key): key j of a sequence is
+  // visible iff j < sinks or j >= kv_len - window
+  int32_t window;
+  int32_t sinks;
 };
 bool decode_fast_supported(int dtype_bf16, int d, int bs, int G);
 cudaError_t launch_decode_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,

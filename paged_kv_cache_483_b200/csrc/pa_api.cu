@@ -135,6 +135,15 @@ bool make_record_map(CUtensorMap* map, void* base, const pa_pool* p) {
          CUDA_SUCCESS;
 }
 
+// Blocks a decode walks per sequence at most: all of them, or with a sink +
+// recent window the sink blocks plus the blocks the window can touch.
+int32_t window_blocks(const pa_pool* p, int32_t max_blocks, int32_t window, int32_t sinks) {
+  if (window <= 0) return max_blocks;
+  const int64_t bs = p->block_size;
+  const int64_t w = (sinks + bs - 1) / bs + (window + bs - 1) / bs + 1;
+  return int32_t(std::min<int64_t>(max_blocks, w));
+}
+
 // Blocks per partition for the tensor-core decode.  partition_tokens > 0 is
 // taken as given; 0 picks enough partitions for about two resident CTAs per
 // SM when the batch has fewer (sequence, KV head) groups than that.
@@ -549,10 +558,12 @@ static pa_status decode_fast(pa_pool* p, const void* q, int32_t B, int32_t H,
                              const int32_t* d_kv_lens, float scale, int32_t partition_tokens,
                              void* workspace, size_t workspace_bytes, float* out,
                              void* stream, const void* new_k, const void* new_v,
-                             const int64_t* new_slots) {
+                             const int64_t* new_slots, int32_t window = 0, int32_t sinks = 0) {
   if (!aligned16(q)) return PA_ERR_INVALID_ARG;
   pa::DecodeArgs a{};
-  if (!decode_partitions(p, B, max_blocks, partition_tokens, &a.part_blocks, &a.NP))
+  // partitions split the walked (visible) blocks
+  const int32_t walk = window_blocks(p, max_blocks, window, sinks);
+  if (!decode_partitions(p, B, walk, partition_tokens, &a.part_blocks, &a.NP))
     return PA_ERR_INVALID_ARG;
   const size_t split_bytes = pa::split_workspace_bytes(B, H, a.NP, p->head_dim);
   const bool order = pa::decode_wants_order(B, p->num_kv_heads, a.NP, p->sms);
@@ -578,6 +589,8 @@ static pa_status decode_fast(pa_pool* p, const void* q, int32_t B, int32_t H,
   a.new_slots = new_slots;
   a.k_cache = p->k_cache;
   a.v_cache = p->v_cache;
+  a.window = window;
+  a.sinks = sinks;
   if (p->dtype == PA_INT8)
     return cuda_status(pa::launch_decode_q8(&p->tmK, a, static_cast<cudaStream_t>(stream)));
   return cuda_status(pa::launch_decode_fast(&p->tmK, &p->tmV, a, p->sms,
@@ -619,6 +632,29 @@ pa_status pa_decode(pa_pool* p, const void* q, int32_t B, int32_t H,
                     p->block_size, p->num_blocks, scale, out, p->d_err,
                     p->dtype == PA_BF16};
   return cuda_status(pa::launch_attention_generic(g, s));
+}
+
+size_t pa_decode_window_workspace_bytes(const pa_pool* p, int32_t B, int32_t H,
+                                        int32_t max_blocks, int32_t window, int32_t sinks,
+                                        int32_t partition_tokens) {
+  if (!p || window < 1 || sinks < 0) return 0;
+  return pa_decode_workspace_bytes(p, B, H, window_blocks(p, max_blocks, window, sinks),
+                                   partition_tokens);
+}
+
+pa_status pa_decode_window(pa_pool* p, const void* q, int32_t B, int32_t H,
+                           const int32_t* d_block_tables, int32_t max_blocks,
+                           const int32_t* d_kv_lens, float scale, int32_t window, int32_t sinks,
+                           int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                           float* out, void* stream) {
+  pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, out);
+  if (st != PA_OK) return st;
+  if (partition_tokens < 0 || window < 1 || sinks < 0) return PA_ERR_INVALID_ARG;
+  if (!use_fast_decode(p, H)) return PA_ERR_UNSUPPORTED;
+  if (B == 0) return PA_OK;
+  return decode_fast(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale, partition_tokens,
+                     workspace, workspace_bytes, out, stream, nullptr, nullptr, nullptr, window,
+                     sinks);
 }
 
 pa_status pa_decode_append(pa_pool* p, const void* q, const void* key, const void* value,

@@ -1,0 +1,102 @@
+"""Sink + recent-window decode on the GPU (needs a B200) against the oracle's
+``attention_window`` ("vladkulikov.com modern-llms module 9 notebook",
+streaming and sliding-window caches), bf16 and int8 pools, max-abs <= 2e-3."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_483_b200 as pa
+import workloads
+from harness import GpuRun, OracleRun, q64
+from oracle import attention_window
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+LENS = [1, 3, 15, 16, 17, 40, 100, 255, 513, 1000, 2049, 0]
+WINDOWS = [(1, 0), (3, 0), (16, 0), (17, 4), (100, 16), (64, 1), (1000, 0), (5000, 0), (33, 40)]
+
+
+def _oracle_window(o, w, q, window, sinks):
+    G = w.num_heads // w.num_kv_heads
+    res = []
+    for i, seq in enumerate(w.decode_seqs):
+        k, v = o.pool.gather(seq)
+        rows = {}
+        for kvh in range(w.num_kv_heads):
+            hs = list(range(kvh * G, (kvh + 1) * G))
+            out = attention_window(q[i][:, hs], k[:, kvh:kvh + 1].astype(np.float64),
+                                   v[:, kvh:kvh + 1].astype(np.float64), window, sinks)
+            for j, h in enumerate(hs):
+                rows[h] = out[0, j]
+        res.append(rows)
+    return res
+
+
+@pytest.mark.parametrize("q8", [False, True])
+@pytest.mark.parametrize("part", [0, 64])
+def test_window_decode_parity(q8, part):
+    w = workloads.custom_decode("win", LENS, 32, 8, 128, 16, "bf16", seed=31 + part,
+                                spare_blocks=4)
+    g = GpuRun(w, q8=q8).apply(w.setup)
+    o = OracleRun(w, q8=q8).apply(w.setup)
+    tables, lens, _, _ = g.tables()
+    qd = w.queries()[:, 0].contiguous().cuda()
+    q = q64(w)
+    for window, sinks in WINDOWS:
+        out = g.pool.decode_window(qd, tables, lens, window, sinks,
+                                   partition_tokens=part).cpu().numpy()
+        ref = _oracle_window(o, w, q, window, sinks)
+        worst = max(float(np.abs(out[i, h] - r).max()) for i, rows in enumerate(ref)
+                    for h, r in rows.items())
+        assert worst <= TOL, (window, sinks, worst)
+        assert np.all(out[LENS.index(0)] == 0)
+    assert g.pool.get_error() == 0
+
+
+@pytest.mark.parametrize("q8", [False, True])
+def test_window_covering_everything_equals_decode(q8):
+    w = workloads.custom_decode("win2", [5, 300, 1111], 32, 8, 128, 16, "bf16", seed=3,
+                                spare_blocks=4)
+    g = GpuRun(w, q8=q8).apply(w.setup)
+    tables, lens, _, _ = g.tables()
+    qd = w.queries()[:, 0].contiguous().cuda()
+    full = g.pool.decode(qd, tables, lens).cpu().numpy()
+    for window, sinks in ((1111, 0), (2000, 7), (1, 1200)):
+        got = g.pool.decode_window(qd, tables, lens, window, sinks).cpu().numpy()
+        assert np.array_equal(got, full)                 # same blocks, same order
+
+
+def test_window_stale_slots_and_errors():
+    w = workloads.custom_decode("win3", [7, 70, 400], 32, 8, 128, 16, "bf16", seed=5,
+                                spare_blocks=4)
+    g = GpuRun(w, init="empty")
+    g.k_cache.fill_(float("nan"))
+    g.v_cache.fill_(float("inf"))
+    g.apply(w.setup)
+    o = OracleRun(w).apply(w.setup)
+    tables, lens, _, _ = g.tables()
+    qd = w.queries()[:, 0].contiguous().cuda()
+    out = g.pool.decode_window(qd, tables, lens, 20, 3).cpu().numpy()
+    ref = _oracle_window(o, w, q64(w), 20, 3)
+    assert np.isfinite(out).all()
+    assert max(float(np.abs(out[i, h] - r).max()) for i, rows in enumerate(ref)
+               for h, r in rows.items()) <= TOL
+    with pytest.raises(pa.PAError) as e:
+        g.pool.decode_window(qd, tables, lens, 0, 3)
+    assert e.value.code == 1
+    bad = tables.clone()
+    bad[2, -1] = w.num_blocks + 1                          # inside the window
+    out = g.pool.decode_window(qd, bad, lens, 20, 3)
+    assert g.pool.get_error() & pa.PA_DEVERR_BLOCK_ID and torch.all(out[2] == 0)
+    assert g.pool.get_error() == 0
+
+
+def test_window_unsupported_on_generic_path():
+    w = workloads.custom_decode("win4", [9, 40], 8, 2, 32, 8, "f32", seed=4, spare_blocks=4)
+    g = GpuRun(w).apply(w.setup)
+    tables, lens, _, _ = g.tables()
+    q = torch.zeros(2, 8, 32, dtype=torch.float32, device="cuda")
+    with pytest.raises(pa.PAError) as e:
+        g.pool.decode_window(q, tables, lens, 4, 0)
+    assert e.value.code == 7
