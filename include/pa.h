@@ -109,6 +109,30 @@ pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
                          pa_dtype kv_dtype, void* k_cache, void* v_cache,
                          const int32_t* alloc_order, pa_pool** out);
 
+/* A pool whose caches hold num_layers layers ([P3] paged_attention's
+ * `layer` argument: one block table per sequence serves every layer).
+ * k_cache/v_cache: [num_layers, <one layer as for pa_pool_create>] (bf16 /
+ * f32), or for PA_INT8 k_cache = [num_layers, num_blocks, num_kv_heads,
+ * PA_INT8_RECORD_BYTES] records and v_cache NULL.  The returned handle is
+ * layer 0; pa_pool_layer gives the others.  All layers share the host
+ * manager: sequence and plan calls on any of them act on the same tables.
+ * A step over L layers plans once (pa_plan_append), copies once
+ * (pa_cow_copy copies each pair in every layer), then writes and attends
+ * per layer (pa_reshape_and_cache, pa_decode, ... on each layer's handle);
+ * pa_append_kv on a layer plans, copies in every layer and writes only that
+ * layer.  Errors: as pa_pool_create / pa_pool_create_int8, INVALID_ARG for
+ * num_layers < 1 or a NULL k_cache. */
+pa_status pa_pool_create_layers(int32_t num_blocks, int32_t block_size,
+                                int32_t num_kv_heads, int32_t head_dim,
+                                pa_dtype kv_dtype, int32_t num_layers,
+                                void* k_cache, void* v_cache,
+                                const int32_t* alloc_order, pa_pool** out);
+
+/* Handle of layer `layer` of a pool (the pool itself for 0).  Layer handles
+ * belong to the pool: pa_free(pool) releases them, pa_free(layer handle)
+ * returns INVALID_ARG. */
+pa_status pa_pool_layer(pa_pool* pool, int32_t layer, pa_pool** layer_pool);
+
 /* Pool of int8 KV rows ([P2] KV quantisation experiment, 8 bits: per
  * (token, head) row, scale = max|x| / 127 (1 for a zero row), code =
  * round-half-even(x / scale) clipped to +-127, decided in float64; the

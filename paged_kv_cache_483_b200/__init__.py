@@ -34,7 +34,8 @@ EXPORTS = ["pa_pool_create", "pa_free", "pa_seq_create", "pa_seq_fork", "pa_seq_
            "pa_get_error", "pa_status_string", "pa_decode_path", "pa_prefill_path",
            "pa_decode_static_scratch", "pa_decode_append", "pa_seq_create_cached",
            "pa_prefix_publish", "pa_prefix_clear", "pa_prefix_entries", "pa_pool_create_int8",
-           "pa_decode_window", "pa_decode_window_workspace_bytes"]
+           "pa_decode_window", "pa_decode_window_workspace_bytes", "pa_pool_create_layers",
+           "pa_pool_layer"]
 
 
 class PAError(RuntimeError):
@@ -66,6 +67,9 @@ def lib():
     sig = {
         "pa_pool_create": ([_I32, _I32, _I32, _I32, C.c_int, _P, _P, _PI32, C.POINTER(_P)], C.c_int),
         "pa_free": ([_P], C.c_int),
+        "pa_pool_create_layers": ([_I32, _I32, _I32, _I32, C.c_int, _I32, _P, _P, _PI32,
+                                   C.POINTER(_P)], C.c_int),
+        "pa_pool_layer": ([_P, _I32, C.POINTER(_P)], C.c_int),
         "pa_pool_create_int8": ([_I32, _I32, _I32, _I32, _P, _PI32, C.POINTER(_P)], C.c_int),
         "pa_seq_create": ([_P, _I32], C.c_int),
         "pa_seq_fork": ([_P, _I32, _I32, _I32], C.c_int),
@@ -185,8 +189,45 @@ class Pool:
         self._h = h
         self._ws = None
 
+    @classmethod
+    def layered(cls, num_blocks, block_size, num_kv_heads, head_dim, dtype, num_layers,
+                k_cache, v_cache=None, alloc_order=None):
+        """A pool over caches holding ``num_layers`` layers (leading dimension);
+        ``layer(l)`` gives each layer's handle, all sharing one manager."""
+        import torch
+        self = cls.__new__(cls)
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+        self.num_kv_heads, self.head_dim = int(num_kv_heads), int(head_dim)
+        self.dtype, self.k_cache, self.v_cache = dtype, k_cache, v_cache
+        self._ws, self._view = None, False
+        code = {"bf16": PA_BF16, "f32": PA_F32, "int8": PA_INT8}[dtype]
+        want = {"bf16": torch.bfloat16, "f32": torch.float32, "int8": torch.uint8}[dtype]
+        order_arr, order_p = (None, None) if alloc_order is None else _i32(alloc_order)
+        h = C.c_void_p()
+        _check(lib().pa_pool_create_layers(num_blocks, block_size, num_kv_heads, head_dim, code,
+                                           num_layers, _dev_ptr(k_cache, want, "k_cache"),
+                                           _dev_ptr(v_cache, want, "v_cache"), order_p,
+                                           C.byref(h)), "pa_pool_create_layers")
+        self._h = h
+        self._layers = {0: self}
+        return self
+
+    def layer(self, index):
+        """Handle of one layer (borrowed: it lives as long as this pool)."""
+        if index in getattr(self, "_layers", {}):
+            return self._layers[index]
+        h = C.c_void_p()
+        _check(lib().pa_pool_layer(self._h, int(index), C.byref(h)), "pa_pool_layer")
+        v = Pool.__new__(Pool)
+        v.__dict__.update({k: val for k, val in self.__dict__.items() if k != "_layers"})
+        v._h, v._ws, v._view, v._parent = h, None, True, self
+        self._layers[index] = v
+        return v
+
     # -- lifetime ----------------------------------------------------------
     def close(self):
+        if getattr(self, "_view", False):
+            return                          # a layer handle: freed with its pool
         if getattr(self, "_h", None):
             lib().pa_free(self._h)
             self._h = None

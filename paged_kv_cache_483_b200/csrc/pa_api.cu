@@ -10,6 +10,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <memory>
 #include <new>
 #include <vector>
 
@@ -35,8 +36,16 @@ struct Staging {
 }  // namespace
 
 struct pa_pool {
-  BlockManager mgr;
+  // The host manager: owned by the pool that created it and shared by its
+  // layer views (one block table per sequence serves every layer).
+  std::unique_ptr<BlockManager> own_mgr;
+  BlockManager* mgr = nullptr;
   int32_t num_blocks, block_size, num_kv_heads, head_dim;
+  // multi-layer pools: caches [num_layers, ...]; a view addresses one layer
+  int32_t num_layers = 1, layer = 0;
+  int64_t layer_bytes = 0;        // bytes of one layer of one cache array
+  pa_pool* owner = nullptr;       // set on views 1 .. num_layers - 1
+  std::vector<pa_pool*> views;    // on the owner: views of layers 1 ..
   pa_dtype dtype;
   void* k_cache = nullptr;
   void* v_cache = nullptr;
@@ -56,7 +65,9 @@ struct pa_pool {
   std::vector<pa::CowPair> cow_tmp;
 
   pa_pool(int32_t nb, int32_t bs, const std::vector<int32_t>& order)
-      : mgr(nb, bs, order) {}
+      : own_mgr(new BlockManager(nb, bs, order)), mgr(own_mgr.get()) {}
+  pa_pool() = default;
+  pa_pool* base() { return owner ? owner : this; }
 };
 
 namespace {
@@ -260,6 +271,77 @@ static pa_status create_pool(int32_t num_blocks, int32_t block_size, int32_t num
   return PA_OK;
 }
 
+// Views of layers 1 .. L - 1 of a device pool whose caches hold L layers:
+// same manager, error word and prefill scratch; own base pointers, tensor
+// maps and append staging.
+static pa_status add_layer_views(pa_pool* p, int32_t num_layers) {
+  const size_t eb = p->dtype == PA_INT8 ? 1 : p->dtype == PA_BF16 ? 2 : 4;
+  p->num_layers = num_layers;
+  p->layer_bytes = p->dtype == PA_INT8
+                       ? int64_t(p->num_blocks) * p->num_kv_heads * pa::kQ8RecordBytes
+                       : int64_t(p->num_blocks) * p->block_size * p->num_kv_heads *
+                             p->head_dim * int64_t(eb);
+  for (int32_t l = 1; l < num_layers; ++l) {
+    pa_pool* v = new (std::nothrow) pa_pool();
+    if (!v) return PA_ERR_INVALID_ARG;
+    p->views.push_back(v);
+    v->mgr = p->mgr;
+    v->owner = p;
+    v->num_blocks = p->num_blocks;
+    v->block_size = p->block_size;
+    v->num_kv_heads = p->num_kv_heads;
+    v->head_dim = p->head_dim;
+    v->dtype = p->dtype;
+    v->num_layers = num_layers;
+    v->layer = l;
+    v->layer_bytes = p->layer_bytes;
+    v->device = p->device;
+    v->dev_id = p->dev_id;
+    v->sms = p->sms;
+    v->d_err = p->d_err;
+    v->split_o = p->split_o;
+    v->split_ml = p->split_ml;
+    v->tickets = p->tickets;
+    v->k_cache = static_cast<char*>(p->k_cache) + l * p->layer_bytes;
+    v->v_cache = p->v_cache ? static_cast<char*>(p->v_cache) + l * p->layer_bytes : nullptr;
+    if (p->dtype == PA_INT8) {
+      if (!make_record_map(&v->tmK, v->k_cache, v)) return PA_ERR_CUDA;
+    } else if (p->tmap_ok) {
+      v->tmap_ok = make_pool_map(&v->tmK, v->k_cache, v) && make_pool_map(&v->tmV, v->v_cache, v);
+      if (!v->tmap_ok) return PA_ERR_CUDA;
+    }
+  }
+  return PA_OK;
+}
+
+pa_status pa_pool_create_layers(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                                int32_t head_dim, pa_dtype kv_dtype, int32_t num_layers,
+                                void* k_cache, void* v_cache, const int32_t* alloc_order,
+                                pa_pool** out) {
+  if (out) *out = nullptr;
+  if (num_layers < 1 || !k_cache) return PA_ERR_INVALID_ARG;
+  if (kv_dtype == PA_INT8 && (block_size != 16 || head_dim != 128)) return PA_ERR_UNSUPPORTED;
+  if (kv_dtype == PA_INT8 && v_cache) return PA_ERR_INVALID_ARG;
+  pa_status st = create_pool(num_blocks, block_size, num_kv_heads, head_dim, kv_dtype, k_cache,
+                             v_cache, alloc_order, out);
+  if (st != PA_OK) return st;
+  st = add_layer_views(*out, num_layers);
+  if (st != PA_OK) {
+    pa_free(*out);
+    *out = nullptr;
+  }
+  return st;
+}
+
+pa_status pa_pool_layer(pa_pool* p, int32_t layer, pa_pool** view) {
+  if (!p || !view) return PA_ERR_INVALID_ARG;
+  *view = nullptr;
+  pa_pool* o = p->base();
+  if (layer < 0 || layer >= o->num_layers) return PA_ERR_INVALID_ARG;
+  *view = layer == 0 ? o : o->views[size_t(layer - 1)];
+  return PA_OK;
+}
+
 pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
                          int32_t num_kv_heads, int32_t head_dim,
                          pa_dtype kv_dtype, void* k_cache, void* v_cache,
@@ -282,36 +364,43 @@ pa_status pa_pool_create_int8(int32_t num_blocks, int32_t block_size, int32_t nu
                      nullptr, alloc_order, out);
 }
 
+static void free_ring(pa_pool* p) {
+  for (auto& r : p->ring) {
+    if (r.host) cudaFreeHost(r.host);
+    if (r.dev) cudaFree(r.dev);
+    if (r.done) cudaEventDestroy(r.done);
+  }
+}
+
 pa_status pa_free(pa_pool* p) {
   if (!p) return PA_OK;
+  if (p->owner) return PA_ERR_INVALID_ARG;   // a layer view: freed with its pool
   if (p->device) {
     cudaDeviceSynchronize();
-    for (auto& r : p->ring) {
-      if (r.host) cudaFreeHost(r.host);
-      if (r.dev) cudaFree(r.dev);
-      if (r.done) cudaEventDestroy(r.done);
-    }
+    for (pa_pool* v : p->views) free_ring(v);
+    free_ring(p);
     if (p->d_err) cudaFree(p->d_err);
     free_split(p);
   }
+  for (pa_pool* v : p->views) delete v;
   delete p;
   return PA_OK;
 }
 
 pa_status pa_seq_create(pa_pool* p, int32_t seq) {
   if (!p) return PA_ERR_INVALID_ARG;
-  return from_mgr(p->mgr.create(seq));
+  return from_mgr(p->mgr->create(seq));
 }
 
 pa_status pa_seq_fork(pa_pool* p, int32_t parent, int32_t child,
                       int32_t prefix_tokens) {
   if (!p || prefix_tokens < -1) return PA_ERR_INVALID_ARG;
-  return from_mgr(p->mgr.share_prefix(parent, child, prefix_tokens));
+  return from_mgr(p->mgr->share_prefix(parent, child, prefix_tokens));
 }
 
 pa_status pa_seq_release(pa_pool* p, int32_t seq) {
   if (!p) return PA_ERR_INVALID_ARG;
-  return from_mgr(p->mgr.release(seq));
+  return from_mgr(p->mgr->release(seq));
 }
 
 pa_status pa_seq_create_cached(pa_pool* p, int32_t seq, uint64_t scope,
@@ -319,7 +408,7 @@ pa_status pa_seq_create_cached(pa_pool* p, int32_t seq, uint64_t scope,
                                int32_t n_tokens, int32_t* hit_tokens) {
   if (!p) return PA_ERR_INVALID_ARG;
   int64_t hit = 0;
-  pa_status st = from_mgr(p->mgr.create_cached(seq, scope, revision, tokens, n_tokens, &hit));
+  pa_status st = from_mgr(p->mgr->create_cached(seq, scope, revision, tokens, n_tokens, &hit));
   if (st == PA_OK && hit_tokens) *hit_tokens = int32_t(hit);
   return st;
 }
@@ -329,27 +418,27 @@ pa_status pa_prefix_publish(pa_pool* p, int32_t seq, uint64_t scope,
                             int32_t n_tokens, int32_t* added_blocks) {
   if (!p) return PA_ERR_INVALID_ARG;
   int64_t added = 0;
-  pa_status st = from_mgr(p->mgr.publish(seq, scope, revision, tokens, n_tokens, &added));
+  pa_status st = from_mgr(p->mgr->publish(seq, scope, revision, tokens, n_tokens, &added));
   if (st == PA_OK && added_blocks) *added_blocks = int32_t(added);
   return st;
 }
 
 pa_status pa_prefix_clear(pa_pool* p, int32_t* freed_blocks) {
   if (!p) return PA_ERR_INVALID_ARG;
-  const int64_t freed = p->mgr.prefix_clear();
+  const int64_t freed = p->mgr->prefix_clear();
   if (freed_blocks) *freed_blocks = int32_t(freed);
   return PA_OK;
 }
 
-int64_t pa_prefix_entries(const pa_pool* p) { return p ? p->mgr.prefix_entries() : 0; }
+int64_t pa_prefix_entries(const pa_pool* p) { return p ? p->mgr->prefix_entries() : 0; }
 
 pa_status pa_seq_table(const pa_pool* p, int32_t seq, int32_t* blocks_out,
                        int32_t cap, int32_t* n_blocks, int32_t* length) {
   if (!p) return PA_ERR_INVALID_ARG;
-  const std::vector<int32_t>* t = p->mgr.table(seq);
+  const std::vector<int32_t>* t = p->mgr->table(seq);
   if (!t) return PA_ERR_UNKNOWN_SEQ;
   if (n_blocks) *n_blocks = int32_t(t->size());
-  if (length) *length = int32_t(p->mgr.length(seq));
+  if (length) *length = int32_t(p->mgr->length(seq));
   if (blocks_out) {
     if (cap < int32_t(t->size())) return PA_ERR_INVALID_ARG;
     std::copy(t->begin(), t->end(), blocks_out);
@@ -362,18 +451,18 @@ pa_status pa_block_tables(const pa_pool* p, const int32_t* seqs, int32_t n,
                           int32_t* kv_lens_out) {
   if (!p || n < 0 || width <= 0 || (n > 0 && !seqs)) return PA_ERR_INVALID_ARG;
   for (int32_t i = 0; i < n; ++i) {
-    const std::vector<int32_t>* t = p->mgr.table(seqs[i]);
+    const std::vector<int32_t>* t = p->mgr->table(seqs[i]);
     if (!t) return PA_ERR_UNKNOWN_SEQ;
     if (int32_t(t->size()) > width) return PA_ERR_INVALID_ARG;
   }
   for (int32_t i = 0; i < n; ++i) {
-    const std::vector<int32_t>* t = p->mgr.table(seqs[i]);
+    const std::vector<int32_t>* t = p->mgr->table(seqs[i]);
     if (tables_out) {
       int32_t* row = tables_out + int64_t(i) * width;
       std::fill(row, row + width, 0);
       std::copy(t->begin(), t->end(), row);
     }
-    if (kv_lens_out) kv_lens_out[i] = int32_t(p->mgr.length(seqs[i]));
+    if (kv_lens_out) kv_lens_out[i] = int32_t(p->mgr->length(seqs[i]));
   }
   return PA_OK;
 }
@@ -387,7 +476,7 @@ pa_status pa_plan_append(pa_pool* p, const int32_t* seqs, const int32_t* n_new,
   if ((cow_src_out || cow_dst_out) && cow_cap < n_seqs) return PA_ERR_INVALID_ARG;
   p->slots_tmp.clear();
   p->cow_tmp.clear();
-  pa_status st = from_mgr(p->mgr.append(seqs, n_new, n_seqs, &p->slots_tmp, &p->cow_tmp));
+  pa_status st = from_mgr(p->mgr->append(seqs, n_new, n_seqs, &p->slots_tmp, &p->cow_tmp));
   if (st != PA_OK) return st;
   if (slot_mapping_out)
     std::copy(p->slots_tmp.begin(), p->slots_tmp.end(), slot_mapping_out);
@@ -401,7 +490,7 @@ pa_status pa_plan_append(pa_pool* p, const int32_t* seqs, const int32_t* n_new,
 
 pa_status pa_pool_stats(const pa_pool* p, pa_stats* out) {
   if (!p || !out) return PA_ERR_INVALID_ARG;
-  pa::Snapshot s = p->mgr.snapshot();
+  pa::Snapshot s = p->mgr->snapshot();
   out->allocated_blocks = s.allocated;
   out->free_blocks = s.free;
   out->physical_capacity_tokens = s.capacity;
@@ -415,29 +504,37 @@ pa_status pa_pool_stats(const pa_pool* p, pa_stats* out) {
 
 pa_status pa_refcounts(const pa_pool* p, int32_t* out) {
   if (!p || !out) return PA_ERR_INVALID_ARG;
-  const auto& r = p->mgr.refcounts();
+  const auto& r = p->mgr->refcounts();
   std::copy(r.begin(), r.end(), out);
   return PA_OK;
 }
 
 pa_status pa_validate(const pa_pool* p) {
   if (!p) return PA_ERR_INVALID_ARG;
-  return p->mgr.validate() ? PA_OK : PA_ERR_INTERNAL;
+  return p->mgr->validate() ? PA_OK : PA_ERR_INTERNAL;
 }
 
 // K2 for any pool: whole blocks of codes/values (and, for int8 pools, of
 // their scales).
 static cudaError_t cow_blocks(pa_pool* p, const int32_t* d_src, const int32_t* d_dst, int32_t n,
                               cudaStream_t s) {
-  if (p->dtype == PA_INT8)   // one array of packed records
-    return pa::launch_cow_copy(p->k_cache, nullptr, d_src, d_dst, n,
-                               int64_t(p->num_kv_heads) * pa::kQ8RecordBytes, p->num_blocks,
-                               p->d_err, p->sms, s);
-  const size_t eb = elem_bytes(p->dtype);
-  return pa::launch_cow_copy(
-      p->k_cache, p->v_cache, d_src, d_dst, n,
-      int64_t(p->block_size) * p->num_kv_heads * p->head_dim * eb, p->num_blocks, p->d_err,
-      p->sms, s);
+  // the tables are shared by every layer: a copied block is copied in all
+  pa_pool* o = p->base();
+  cudaError_t e = cudaSuccess;
+  for (int32_t l = 0; l < o->num_layers && e == cudaSuccess; ++l) {
+    char* kc = static_cast<char*>(o->k_cache) + l * o->layer_bytes;
+    char* vc = o->v_cache ? static_cast<char*>(o->v_cache) + l * o->layer_bytes : nullptr;
+    if (o->dtype == PA_INT8)   // one array of packed records
+      e = pa::launch_cow_copy(kc, nullptr, d_src, d_dst, n,
+                              int64_t(o->num_kv_heads) * pa::kQ8RecordBytes, o->num_blocks,
+                              o->d_err, o->sms, s);
+    else
+      e = pa::launch_cow_copy(kc, vc, d_src, d_dst, n,
+                              int64_t(o->block_size) * o->num_kv_heads * o->head_dim *
+                                  elem_bytes(o->dtype),
+                              o->num_blocks, o->d_err, o->sms, s);
+  }
+  return e;
 }
 
 // K1 for any pool: copies rows, or quantises bf16 rows into an int8 pool.
@@ -489,7 +586,7 @@ pa_status pa_append_kv(pa_pool* p, const int32_t* seqs, const int32_t* n_new,
   // host plan (step a1): all-or-nothing
   p->slots_tmp.clear();
   p->cow_tmp.clear();
-  pa_status st = from_mgr(p->mgr.append(seqs, n_new, n_seqs, &p->slots_tmp, &p->cow_tmp));
+  pa_status st = from_mgr(p->mgr->append(seqs, n_new, n_seqs, &p->slots_tmp, &p->cow_tmp));
   if (st != PA_OK) return st;
   if (slot_mapping_out)
     std::copy(p->slots_tmp.begin(), p->slots_tmp.end(), slot_mapping_out);
