@@ -97,17 +97,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map,
       : "memory");
 }
 
-// Contiguous global -> shared copy (no tensor map, no multicast): both
-// addresses 16-byte aligned, bytes a multiple of 16; completes on `bar`.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-
 // Shared -> global tile store (no multicast); completion tracked per thread
 // with bulk async-groups.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src,

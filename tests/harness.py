@@ -12,7 +12,7 @@ import torch
 
 import paged_kv_cache_483_b200 as pa
 import workloads
-from oracle import KVPool, paged_attention, stored_rows
+from oracle import KVPool, stored_rows
 
 
 def torch_dtype(w):

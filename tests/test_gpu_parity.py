@@ -20,14 +20,6 @@ pytestmark = pytest.mark.gpu
 TOL_F32, TOL_DECODE, TOL_PREFILL = 1e-4, 2e-3, 5e-3
 
 
-def _max_err(gpu_out, oracle_rows, qt=None):
-    err = 0.0
-    for h, ref in oracle_rows.items():
-        got = gpu_out[:, h] if qt is None else gpu_out[qt, h]
-        err = max(err, float(np.abs(got - (ref[0] if qt is None else ref[0])).max()))
-    return err
-
-
 def _check_decode(g, o, w, tol, partition_tokens=0):
     out = g.decode(partition_tokens=partition_tokens)
     q = q64(w)
