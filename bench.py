@@ -238,11 +238,16 @@ class Setup:
         self.n_cow = 0 if self.cow_src is None else int(self.cow_src.numel())
 
 
-def decode_bytes(w, lens, q8=False):
+def decode_bytes(w, lens, q8=False, window=0, sinks=0):
+    """K/V bytes a decode step must read: every token, or with a window the
+    min(kv_len, sinks + window) visible ones."""
+    lens = lens.astype(np.int64)
+    if window > 0:
+        lens = np.minimum(lens, window + sinks)
     if q8:    # int8 records: K and V codes plus two float32 scales per (token, head)
-        return int(np.sum(lens.astype(np.int64))) * w.num_kv_heads * (2 * w.head_dim + 8)
+        return int(np.sum(lens)) * w.num_kv_heads * (2 * w.head_dim + 8)
     eb = 2 if w.dtype == "bf16" else 4
-    return int(np.sum(lens.astype(np.int64))) * w.num_kv_heads * w.head_dim * 2 * eb
+    return int(np.sum(lens)) * w.num_kv_heads * w.head_dim * 2 * eb
 
 
 def prefill_flops(w, lens):
@@ -260,21 +265,26 @@ def run_ours(args, dist):
     w = builder(seed=workloads.seed_for({"decode32": 2, "ragged256": 3, "splitk128k": 4,
                                          "prefill": 5}[args.config]) + 1000 * dist.rank)
     q8 = args.kv == "int8"
-    if q8 and w.q_tokens > 1:
-        raise SystemExit("--kv int8 applies to the decode workloads")
+    win, sinks = args.window, args.sinks
+    if (q8 or win) and w.q_tokens > 1:
+        raise SystemExit("--kv int8 and --window apply to the decode workloads")
     S = Setup(w, device, q8=q8)
     pool = S.pool
     is_prefill = w.q_tokens > 1
     part = w.partition_tokens
     stream = torch.cuda.current_stream(device)
 
-    ws_bytes = 0 if is_prefill else pool.decode_workspace_bytes(
-        S.q.shape[0], S.q.shape[1], S.tables.shape[1], part)
+    import paged_kv_cache_483_b200 as pa
+    ws_bytes = 0 if is_prefill else (
+        int(pa.lib().pa_decode_window_workspace_bytes(pool.handle, S.q.shape[0], S.q.shape[1],
+                                                      S.tables.shape[1], win, sinks, part))
+        if win else pool.decode_workspace_bytes(S.q.shape[0], S.q.shape[1],
+                                                S.tables.shape[1], part))
     split = ws_bytes > 0                    # a second launch: order prepass or combine
     order_only = ws_bytes == 4 * S.q.shape[0]
     # decode steps fuse the new token's append into the decode kernel (bf16;
     # on an int8 pool the append is its own quantising launch)
-    fused = (not is_prefill) and S.slots is not None and not q8
+    fused = (not is_prefill) and S.slots is not None and not q8 and not win
     per_step = ((1 if S.n_cow else 0) + (1 if (S.slots is not None and not fused) else 0)
                 + (2 if split else 1))
     launches = {"n": 0}
@@ -290,6 +300,9 @@ def run_ours(args, dist):
             pool.prefill_chunk(S.q, S.tables, S.lens, out=S.out, stream=stream)
         elif fused:
             pool.decode_append(S.q, S.step_k, S.step_v, S.slots, S.tables, S.lens, out=S.out,
+                               partition_tokens=part, stream=stream)
+        elif win:
+            pool.decode_window(S.q, S.tables, S.lens, win, sinks, out=S.out,
                                partition_tokens=part, stream=stream)
         else:
             pool.decode(S.q, S.tables, S.lens, out=S.out, partition_tokens=part, stream=stream)
@@ -341,11 +354,13 @@ def run_ours(args, dist):
                 "peak_source": f"{peak_kind} bf16_tflops (burst)"}
         extra = {"tflops": round(value, 2)}
     else:
-        kv = decode_bytes(w, lens, q8)
+        kv = decode_bytes(w, lens, q8, win, sinks)
         value = dist.world * kv / (ms_step_max * 1e-3) / 1e9
         metric = ("decode int8-KV HBM GB/s (codes + scales read) and seqs/s at 8K ctx, GQA 32/8"
                   if q8 else
                   "decode KV HBM GB/s (fraction of B200 peak) and seqs/s at 8K ctx, GQA 32/8")
+        if win:
+            metric += f", window {win} + {sinks} sinks (visible keys only)"
         unit = "GB/s"
         achieved = kv / (kern_ms * 1e-3) / 1e9
         kname = "decode_q8_kernel" if q8 else "decode_mma_kernel"
@@ -360,7 +375,10 @@ def run_ours(args, dist):
         extra = {"seqs_per_s": round(dist.world * len(w.decode_seqs) / (ms_step_max * 1e-3), 1),
                  "frac_of_peak": round(value / hbm, 4)}
         if q8:
-            extra["kv_bytes_vs_bf16"] = round(kv / decode_bytes(w, lens), 4)
+            extra["kv_bytes_vs_bf16"] = round(kv / decode_bytes(w, lens, False, win, sinks), 4)
+        if win:
+            extra["window"] = {"window": win, "sinks": sinks,
+                               "visible_fraction": round(kv / decode_bytes(w, lens, q8), 4)}
     res = {
         "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": dist.world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 5),
@@ -390,6 +408,7 @@ def config_of(w, args, dist):
             "q_tokens": w.q_tokens, "partition_tokens": w.partition_tokens,
             "parallelism": f"replicas x{dist.world} (no collective)",
             "kv": getattr(args, "kv", "bf16"),
+            "window": getattr(args, "window", 0), "sinks": getattr(args, "sinks", 0),
             "l2": "inputs larger than L2 (KV per step > 126 MB)" if w.name != "ragged256"
             else "KV per step ~0.5 GB > L2 (shared prefixes may hit in L2)"}
 
@@ -424,10 +443,13 @@ def run_e2e(args, S, dist, device, is_prefill, part):
             d_slots.copy_(h_slots, non_blocking=True)
             if S.n_cow:
                 pool.cow_copy(S.cow_src, S.cow_dst, stream)
-            if is_prefill:
+            if is_prefill or args.window:
                 pool.reshape_and_cache(d_k, d_v, d_slots, stream)
         if is_prefill:
             pool.prefill_chunk(d_q, S.tables, d_lens, out=S.out, stream=stream)
+        elif args.window:
+            pool.decode_window(d_q, S.tables, d_lens, args.window, args.sinks, out=S.out,
+                               partition_tokens=part, stream=stream)
         elif h_k is not None:
             pool.decode_append(d_q, d_k, d_v, d_slots, S.tables, d_lens, out=S.out,
                                partition_tokens=part, stream=stream)
@@ -451,7 +473,7 @@ def run_e2e(args, S, dist, device, is_prefill, part):
         v = dist.world * prefill_flops(w, S.lens_h) / (ms * 1e-3) / 1e12
         unit = "TFLOP/s"
     else:
-        v = dist.world * decode_bytes(w, S.lens_h, S.q8) / (ms * 1e-3) / 1e9
+        v = dist.world * decode_bytes(w, S.lens_h, S.q8, args.window, args.sinks) / (ms * 1e-3) / 1e9
         unit = "GB/s"
     return {"value": round(v, 2), "unit": unit, "h2d_bytes_per_step": int(bi),
             "d2h_bytes_per_step": int(bo), "ms_per_step": round(ms, 5), "steps": K}
@@ -571,6 +593,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kv", choices=["bf16", "int8"], default="bf16",
                     help="KV pool type for the decode workloads (int8: per-row absmax codes)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="decode over the last WINDOW keys (plus --sinks first keys); 0 = all")
+    ap.add_argument("--sinks", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

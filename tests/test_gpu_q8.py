@@ -218,3 +218,19 @@ def test_q8_unsupported_calls():
     with pytest.raises(pa.PAError):                       # int8 pools need block 16, d 128
         pa.Pool(4, 8, 1, 128, "int8",
                 torch.zeros(4, 1, pa.PA_INT8_RECORD_BYTES, dtype=torch.uint8, device="cuda"), None)
+
+
+def test_full_decode32_int8_sampled():
+    # the bench configuration (32 x 8192, GQA 32/8) over an int8 pool; the
+    # oracle stores two KV heads and checks three sequences against them
+    w = workloads.decode32()
+    g = GpuRun(w, q8=True).apply(w.setup)
+    o = OracleRun(w, heads=[0, 5], q8=True).apply(w.setup)
+    out = g.decode()
+    q = q64(w)
+    worst = 0.0
+    for i in (0, 13, 31):
+        for h, ref in o.attention(i, q[i]).items():
+            worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+    assert worst <= TOL_DECODE, worst
+    assert g.pool.get_error() == 0

@@ -100,3 +100,26 @@ def test_window_unsupported_on_generic_path():
     with pytest.raises(pa.PAError) as e:
         g.pool.decode_window(q, tables, lens, 4, 0)
     assert e.value.code == 7
+
+
+@pytest.mark.parametrize("q8", [False, True])
+def test_full_decode32_window_sampled(q8):
+    # 32 x 8192 with a 1024-token window and 4 sinks: three sequences, two KV heads
+    w = workloads.decode32()
+    g = GpuRun(w, q8=q8).apply(w.setup)
+    o = OracleRun(w, heads=[1, 6], q8=q8).apply(w.setup)
+    tables, lens, _, _ = g.tables()
+    qd = w.queries()[:, 0].contiguous().cuda()
+    out = g.pool.decode_window(qd, tables, lens, 1024, 4).cpu().numpy()
+    q = q64(w)
+    G = w.num_heads // w.num_kv_heads
+    worst = 0.0
+    for i in (0, 17, 31):
+        k, v = o.pool.gather(w.decode_seqs[i])
+        for j, kvh in enumerate(o.heads):
+            hs = list(range(kvh * G, (kvh + 1) * G))
+            ref = attention_window(q[i][:, hs], k[:, j:j + 1].astype(np.float64),
+                                   v[:, j:j + 1].astype(np.float64), 1024, 4)
+            worst = max(worst, float(np.abs(out[i, hs] - ref[0]).max()))
+    assert worst <= TOL, worst
+    assert g.pool.get_error() == 0
