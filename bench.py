@@ -43,6 +43,8 @@ import workloads  # noqa: E402
 
 MIB = 1 << 20
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+# datasheet figures, for the second fraction the measurement plan asks for
+NOMINAL_HBM_GBS, NOMINAL_BF16_TFLOPS = 8000.0, 2250.0
 
 
 # ------------------------------------------------------------------ helpers --
@@ -336,6 +338,23 @@ def run_ours(args, dist):
     ms_step_max = dist.max(ms_step, device)
     assert pool.get_error() == 0, "device error in the timed region"
 
+    # the chunk's own append (K1 at the planned slots), timed on its own
+    append = None
+    if is_prefill and S.slots is not None:
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(3):
+            pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
+        n_app = 20
+        a0.record(stream)
+        for _ in range(n_app):
+            pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        app_ms = a0.elapsed_time(a1) / n_app
+        moved = 2 * 2 * S.step_k.numel() * S.step_k.element_size()   # K and V, read + write
+        append = {"ms": round(app_ms, 5), "GB/s": round(moved / (app_ms * 1e-3) / 1e9, 1),
+                  "bytes": moved}
+
     # --------------------------------------------------------------- e2e --
     e2e = run_e2e(args, S, dist, device, is_prefill, part)
 
@@ -350,9 +369,11 @@ def run_ours(args, dist):
         roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": bf16,
                 "unit": "TFLOP/s", "frac": round(achieved / bf16, 4),
                 "traffic": profiled_traffic("prefill_tc.cu", w.name),
+                "frac_of_nominal": round(achieved / NOMINAL_BF16_TFLOPS, 4),
+                "frac_of_sustained": round(achieved / bf16_sus, 4),
                 "kernel": "prefill", "kernel_ms": round(kern_ms, 5),
                 "peak_source": f"{peak_kind} bf16_tflops (burst)"}
-        extra = {"tflops": round(value, 2)}
+        extra = {"tflops": round(value, 2), "append": append}
     else:
         kv = decode_bytes(w, lens, q8, win, sinks)
         value = dist.world * kv / (ms_step_max * 1e-3) / 1e9
@@ -366,6 +387,7 @@ def run_ours(args, dist):
         kname = "decode_q8_kernel" if q8 else "decode_mma_kernel"
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4),
+                "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
                 "traffic": profiled_traffic("decode_q8.cu" if q8 else "decode_mma.cu",
                                             w.name + ("_int8" if q8 else "")),
                 "kernel": (f"decode_order_kernel + {kname}" if order_only else
@@ -530,6 +552,14 @@ class OracleSampler:
         return work, spent, done
 
 
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return {i.get("internal_api", "?"): i.get("num_threads") for i in threadpool_info()}
+    except Exception:
+        return None
+
+
 def cpu_baseline(w, args):
     sampler = OracleSampler(w)
     work, spent, done = sampler.run(args.cpu_budget)
@@ -540,7 +570,8 @@ def cpu_baseline(w, args):
     else:
         val, unit = work / spent / 1e9, "GB/s"
     return {"value": round(val, 6), "unit": unit, "cores": oracle_threads(), "kind": "oracle",
-            "sample": desc, "seconds": round(spent, 2), "host_cpus": os.cpu_count()}
+            "sample": desc, "seconds": round(spent, 2), "host_cpus": os.cpu_count(),
+            "blas_threads": blas_threads()}
 
 
 def run_reference(args, dist):
