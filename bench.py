@@ -264,8 +264,11 @@ def run_ours(args, dist):
     torch.cuda.set_device(dist.local)
     device = torch.device("cuda", dist.local)
     builder = workloads.ALL[args.config]
-    w = builder(seed=workloads.seed_for({"decode32": 2, "ragged256": 3, "splitk128k": 4,
-                                         "prefill": 5}[args.config]) + 1000 * dist.rank)
+    base_seed = args.seed if args.seed is not None else (
+        workloads.SEED_TINY if args.config == "tiny" else
+        workloads.seed_for({"decode32": 2, "ragged256": 3, "splitk128k": 4,
+                            "prefill": 5}[args.config]))
+    w = builder(seed=base_seed + 1000 * dist.rank)
     q8 = args.kv == "int8"
     win, sinks = args.window, args.sinks
     if (q8 or win) and w.q_tokens > 1:
@@ -384,7 +387,8 @@ def run_ours(args, dist):
             metric += f", window {win} + {sinks} sinks (visible keys only)"
         unit = "GB/s"
         achieved = kv / (kern_ms * 1e-3) / 1e9
-        kname = "decode_q8_kernel" if q8 else "decode_mma_kernel"
+        kname = ("decode_q8_kernel" if q8 else "decode_mma_kernel"
+                 if pool.decode_path(w.num_heads) else "attention_generic_kernel")
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4),
                 "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
@@ -415,8 +419,8 @@ def run_ours(args, dist):
         "e2e": e2e,
         "clocks": clk.summary(),
     }
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and not q8:
-        res["cpu_baseline"] = cpu_baseline(w, args)
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and not q8 and not win:
+        res["cpu_baseline"] = cpu_baseline(w, args, S.out.float().cpu().numpy())
     pool.close()
     return res
 
@@ -431,8 +435,9 @@ def config_of(w, args, dist):
             "parallelism": f"replicas x{dist.world} (no collective)",
             "kv": getattr(args, "kv", "bf16"),
             "window": getattr(args, "window", 0), "sinks": getattr(args, "sinks", 0),
-            "l2": "inputs larger than L2 (KV per step > 126 MB)" if w.name != "ragged256"
-            else "KV per step ~0.5 GB > L2 (shared prefixes may hit in L2)"}
+            "l2": ("tiny: fits in L2 (correctness scale)" if w.name == "tiny" else
+                   "KV per step ~0.5 GB > L2 (shared prefixes may hit in L2)"
+                   if w.name == "ragged256" else "inputs larger than L2 (KV per step > 126 MB)")}
 
 
 def run_e2e(args, S, dist, device, is_prefill, part):
@@ -529,19 +534,23 @@ class OracleSampler:
         self.pool = p
         self.next = 0
 
-    def run(self, budget_s, max_units=None):
+    def run(self, budget_s, max_units=None, keep=0):
         """Decode (or prefill) whole sequences -- every head -- until the
-        budget is spent; returns (bytes or flops, seconds, sequences)."""
+        budget is spent; returns (bytes or flops, seconds, sequences).  The
+        outputs of the first ``keep`` sequences are kept in ``self.outs``."""
         from oracle import paged_attention
         w, p = self.w, self.pool
         work, spent, done = 0, 0.0, 0
+        self.outs = {}
         while spent < budget_s and (max_units is None or done < max_units):
             si = self.next % len(w.decode_seqs)
             self.next += 1
             seq = w.decode_seqs[si]
             t0 = time.perf_counter()
-            paged_attention(p, seq, self.q[si])        # gather + two-pass softmax
+            o = paged_attention(p, seq, self.q[si])    # gather + two-pass softmax
             spent += time.perf_counter() - t0
+            if len(self.outs) < keep:
+                self.outs[si] = o
             L = p.lengths[seq]
             if w.q_tokens > 1:
                 qn = w.q_tokens
@@ -560,18 +569,27 @@ def blas_threads():
         return None
 
 
-def cpu_baseline(w, args):
+def cpu_baseline(w, args, gpu_out=None):
     sampler = OracleSampler(w)
-    work, spent, done = sampler.run(args.cpu_budget)
+    work, spent, done = sampler.run(args.cpu_budget, keep=2 if gpu_out is not None else 0)
     desc = (f"{done} of the {len(w.decode_seqs)} sequences of {w.name} (all heads): oracle "
             f"paged gather + float64 two-pass softmax")
     if w.q_tokens > 1:
         val, unit = work / spent / 1e12, "TFLOP/s"
     else:
         val, unit = work / spent / 1e9, "GB/s"
-    return {"value": round(val, 6), "unit": unit, "cores": oracle_threads(), "kind": "oracle",
-            "sample": desc, "seconds": round(spent, 2), "host_cpus": os.cpu_count(),
-            "blas_threads": blas_threads()}
+    res = {"value": round(val, 6), "unit": unit, "cores": oracle_threads(), "kind": "oracle",
+           "sample": desc, "seconds": round(spent, 2), "host_cpus": os.cpu_count(),
+           "blas_threads": blas_threads()}
+    if gpu_out is not None and sampler.outs:
+        # the timed step's output against the oracle's, on the sequences it ran
+        err = 0.0
+        for si, o in sampler.outs.items():
+            got = gpu_out[si] if w.q_tokens > 1 else gpu_out[si][None]
+            err = max(err, float(np.abs(got - o).max()))
+        res["max_abs_err_vs_gpu"] = err
+        res["compared_sequences"] = sorted(int(i) for i in sampler.outs)
+    return res
 
 
 def run_reference(args, dist):
@@ -579,7 +597,7 @@ def run_reference(args, dist):
     if dist.rank != 0:
         return None
     builder = workloads.ALL[args.config]
-    w = builder()
+    w = builder() if args.seed is None else builder(seed=args.seed)
     sampler = OracleSampler(w)
     # each step: one bounded sample (whole groups) so the run stays ~2-3 minutes
     per_step = max(0.005, 120.0 / max(1, args.steps + args.warmup))
@@ -617,7 +635,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=["decode32", "ragged256", "splitk128k", "prefill"],
+    ap.add_argument("--config", choices=["tiny", "decode32", "ragged256", "splitk128k", "prefill"],
                     default="decode32")
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
@@ -627,6 +645,8 @@ def main():
     ap.add_argument("--window", type=int, default=0,
                     help="decode over the last WINDOW keys (plus --sinks first keys); 0 = all")
     ap.add_argument("--sinks", type=int, default=0)
+    ap.add_argument("--seed", type=int, default=None,
+                    help="workload seed (default: the configuration's own)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
