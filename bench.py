@@ -84,7 +84,7 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, cuda_index, period=0.02):
+    def __init__(self, cuda_index, period=0.005):
         self.samples, self.reasons, self.ok = [], set(), False
         self.period = period
         try:
@@ -289,7 +289,7 @@ def run_ours(args, dist):
     order_only = ws_bytes == 4 * S.q.shape[0]
     # decode steps fuse the new token's append into the decode kernel (bf16;
     # on an int8 pool the append is its own quantising launch)
-    fused = (not is_prefill) and S.slots is not None and not q8 and not win
+    fused = (not is_prefill) and S.slots is not None and not q8
     per_step = ((1 if S.n_cow else 0) + (1 if (S.slots is not None and not fused) else 0)
                 + (2 if split else 1))
     launches = {"n": 0}
@@ -303,6 +303,9 @@ def run_ours(args, dist):
             ev_pair[0].record(stream)
         if is_prefill:
             pool.prefill_chunk(S.q, S.tables, S.lens, out=S.out, stream=stream)
+        elif fused and win:
+            pool.decode_window_append(S.q, S.step_k, S.step_v, S.slots, S.tables, S.lens, win,
+                                      sinks, out=S.out, partition_tokens=part, stream=stream)
         elif fused:
             pool.decode_append(S.q, S.step_k, S.step_v, S.slots, S.tables, S.lens, out=S.out,
                                partition_tokens=part, stream=stream)
@@ -393,7 +396,8 @@ def run_ours(args, dist):
                 "frac": round(achieved / hbm, 4),
                 "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
                 "traffic": profiled_traffic("decode_q8.cu" if q8 else "decode_mma.cu",
-                                            w.name + ("_int8" if q8 else "")),
+                                            w.name + ("_int8" if q8 else "")
+                                            + (f"_window{win}_sinks{sinks}" if win else "")),
                 "kernel": (f"decode_order_kernel + {kname}" if order_only else
                            f"{kname} + decode_combine_kernel" if split else kname),
                 "kernel_ms": round(kern_ms, 5),
@@ -470,10 +474,14 @@ def run_e2e(args, S, dist, device, is_prefill, part):
             d_slots.copy_(h_slots, non_blocking=True)
             if S.n_cow:
                 pool.cow_copy(S.cow_src, S.cow_dst, stream)
-            if is_prefill or args.window:
+            if is_prefill:
                 pool.reshape_and_cache(d_k, d_v, d_slots, stream)
         if is_prefill:
             pool.prefill_chunk(d_q, S.tables, d_lens, out=S.out, stream=stream)
+        elif args.window and h_k is not None:
+            pool.decode_window_append(d_q, d_k, d_v, d_slots, S.tables, d_lens, args.window,
+                                      args.sinks, out=S.out, partition_tokens=part,
+                                      stream=stream)
         elif args.window:
             pool.decode_window(d_q, S.tables, d_lens, args.window, args.sinks, out=S.out,
                                partition_tokens=part, stream=stream)

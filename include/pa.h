@@ -348,6 +348,23 @@ pa_status pa_decode_append(pa_pool* pool, const void* q, const void* key,
                            void* workspace, size_t workspace_bytes, float* out,
                            void* stream);
 
+/* pa_decode_append over a sink + recent window: writes each sequence's new
+ * token (key/value [B, Hkv, head_dim] at d_slot_mapping[b], as
+ * pa_decode_append) and decodes over the window exactly as pa_decode_window
+ * -- the result equals pa_reshape_and_cache followed by pa_decode_window.
+ * The new token, at kv_lens[b] - 1, is always visible.  One kernel on a bf16
+ * pool; two launches (quantising append, then the windowed decode) on
+ * an int8 pool.  Workspace: pa_decode_window_workspace_bytes bytes.  Errors
+ * as pa_decode_window, plus INVALID_ARG for null or misaligned key / value /
+ * d_slot_mapping. */
+pa_status pa_decode_window_append(pa_pool* pool, const void* q, const void* key,
+                                  const void* value, const int64_t* d_slot_mapping,
+                                  int32_t B, int32_t H, const int32_t* d_block_tables,
+                                  int32_t max_blocks, const int32_t* d_kv_lens,
+                                  float scale, int32_t window, int32_t sinks,
+                                  int32_t partition_tokens, void* workspace,
+                                  size_t workspace_bytes, float* out, void* stream);
+
 /* Chunked prefill attention ([P3] with q_tokens > 1): for each sequence b
  * the chunk's q_tokens queries are its last q_tokens positions; query qt
  * sees cached positions j <= kv_lens[b] - q_tokens + qt.  The chunk's own

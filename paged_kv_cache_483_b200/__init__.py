@@ -35,7 +35,7 @@ EXPORTS = ["pa_pool_create", "pa_free", "pa_seq_create", "pa_seq_fork", "pa_seq_
            "pa_decode_static_scratch", "pa_decode_append", "pa_seq_create_cached",
            "pa_prefix_publish", "pa_prefix_clear", "pa_prefix_entries", "pa_pool_create_int8",
            "pa_decode_window", "pa_decode_window_workspace_bytes", "pa_pool_create_layers",
-           "pa_pool_layer"]
+           "pa_pool_layer", "pa_decode_window_append"]
 
 
 class PAError(RuntimeError):
@@ -92,6 +92,8 @@ def lib():
         "pa_decode_window": ([_P, _P, _I32, _I32, _P, _I32, _P, _F, _I32, _I32, _I32, _P, _SZ,
                               _P, _P], C.c_int),
         "pa_decode_window_workspace_bytes": ([_P, _I32, _I32, _I32, _I32, _I32, _I32], _SZ),
+        "pa_decode_window_append": ([_P, _P, _P, _P, _P, _I32, _I32, _P, _I32, _P, _F, _I32, _I32,
+                                     _I32, _P, _SZ, _P, _P], C.c_int),
         "pa_prefill_chunk": ([_P, _P, _I32, _I32, _I32, _P, _I32, _P, _F, _I32, _P, _P],
                              C.c_int),
         "pa_get_error": ([_P, _PI32], C.c_int),
@@ -411,6 +413,35 @@ class Pool:
                                       workspace.numel() if need else 0,
                                       _dev_ptr(out, torch.float32, "out"), _stream(stream)),
                "pa_decode_window")
+        return out
+
+    def decode_window_append(self, q, key, value, slot_mapping, block_tables, kv_lens, window,
+                             sinks=0, out=None, scale=None, partition_tokens=0, workspace=None,
+                             stream=None):
+        """decode_append over a sink + recent window: write each sequence's
+        new token, then decode with key j visible iff j < sinks or
+        j >= kv_len - window."""
+        import torch
+        B, H, d = q.shape
+        MB = block_tables.shape[1]
+        if out is None:
+            out = torch.empty((B, H, d), dtype=torch.float32, device=q.device)
+        scale = 1.0 / math.sqrt(self.head_dim) if scale is None else scale
+        need = int(lib().pa_decode_window_workspace_bytes(self._h, B, H, MB, int(window),
+                                                          int(sinks), int(partition_tokens)))
+        if need and workspace is None:
+            if self._ws is None or self._ws.numel() < need:
+                self._ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+            workspace = self._ws
+        wp = _dev_ptr(workspace, None, "workspace") if need else None
+        dt = self._torch_dtype()
+        _check(lib().pa_decode_window_append(
+            self._h, _dev_ptr(q, dt, "q"), _dev_ptr(key, dt, "key"), _dev_ptr(value, dt, "value"),
+            _dev_ptr(slot_mapping, torch.int64, "slot_mapping"), B, H,
+            _dev_ptr(block_tables, torch.int32, "block_tables"), MB,
+            _dev_ptr(kv_lens, torch.int32, "kv_lens"), float(scale), int(window), int(sinks),
+            int(partition_tokens), wp, workspace.numel() if need else 0,
+            _dev_ptr(out, torch.float32, "out"), _stream(stream)), "pa_decode_window_append")
         return out
 
     def decode_append(self, q, key, value, slot_mapping, block_tables, kv_lens, out=None,

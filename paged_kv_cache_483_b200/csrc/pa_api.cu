@@ -777,6 +777,33 @@ pa_status pa_decode_append(pa_pool* p, const void* q, const void* key, const voi
                      d_slot_mapping);
 }
 
+pa_status pa_decode_window_append(pa_pool* p, const void* q, const void* key,
+                                  const void* value, const int64_t* d_slot_mapping, int32_t B,
+                                  int32_t H, const int32_t* d_block_tables, int32_t max_blocks,
+                                  const int32_t* d_kv_lens, float scale, int32_t window,
+                                  int32_t sinks, int32_t partition_tokens, void* workspace,
+                                  size_t workspace_bytes, float* out, void* stream) {
+  pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, out);
+  if (st != PA_OK) return st;
+  if (B > 0 && (!key || !value || !d_slot_mapping)) return PA_ERR_INVALID_ARG;
+  if (partition_tokens < 0 || window < 1 || sinks < 0) return PA_ERR_INVALID_ARG;
+  if (!use_fast_decode(p, H)) return PA_ERR_UNSUPPORTED;
+  if (B == 0) return PA_OK;
+  if (p->dtype == PA_INT8) {
+    // the quantising append is its own launch on an int8 pool
+    st = pa_reshape_and_cache(p, key, value, d_slot_mapping, B, stream);
+    if (st != PA_OK) return st;
+    return pa_decode_window(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale, window,
+                            sinks, partition_tokens, workspace, workspace_bytes, out, stream);
+  }
+  if (!aligned16(key) || !aligned16(value)) return PA_ERR_INVALID_ARG;
+  // the newest key is always visible, so the CTA that walks the last
+  // visible block is the one that writes and patches the new row
+  return decode_fast(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale, partition_tokens,
+                     workspace, workspace_bytes, out, stream, key, value, d_slot_mapping, window,
+                     sinks);
+}
+
 pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,
                            int32_t q_tokens, int32_t H,
                            const int32_t* d_block_tables, int32_t max_blocks,

@@ -123,3 +123,66 @@ def test_full_decode32_window_sampled(q8):
             worst = max(worst, float(np.abs(out[i, hs] - ref[0]).max()))
     assert worst <= TOL, worst
     assert g.pool.get_error() == 0
+
+
+@pytest.mark.parametrize("q8", [False, True])
+@pytest.mark.parametrize("part", [0, 32])
+def test_window_append_equals_two_calls(q8, part):
+    # the fused step (write the new token, decode over the window) against
+    # reshape_and_cache followed by decode_window, and against the oracle
+    lens = [1, 2, 16, 17, 40, 300, 1000]
+    w = workloads.custom_decode("winf", lens, 32, 8, 128, 16, "bf16", seed=13 + part,
+                                spare_blocks=8, split_last=1)
+    windows = [(1, 0), (17, 4), (100, 16), (2000, 0)]
+    outs = {}
+    for fused in (True, False):
+        g = GpuRun(w, q8=q8).apply(w.setup)
+        seqs = [op.args[0] for op in w.step]
+        slots, cow = g.pool.plan_append(seqs, [1] * len(seqs))
+        assert not cow
+        ks, vs = zip(*[w.kv_for(op) for op in w.step])
+        key, val = torch.cat(ks).cuda(), torch.cat(vs).cuda()
+        d_slots = torch.tensor(slots, dtype=torch.int64, device="cuda")
+        tables, tl, _, _ = g.tables()
+        q = w.queries()[:, 0].contiguous().cuda()
+        if not fused:
+            g.pool.reshape_and_cache(key, val, d_slots)
+        for window, sinks in windows:
+            if fused:
+                out = g.pool.decode_window_append(q, key, val, d_slots, tables, tl, window,
+                                                  sinks, partition_tokens=part)
+            else:
+                out = g.pool.decode_window(q, tables, tl, window, sinks, partition_tokens=part)
+            outs[fused, window, sinks] = out.cpu().numpy()
+        assert g.pool.get_error() == 0
+    o = OracleRun(w, q8=q8).apply(w.setup + w.step)
+    qq = q64(w)
+    for window, sinks in windows:
+        assert np.array_equal(outs[True, window, sinks], outs[False, window, sinks])
+        ref = _oracle_window(o, w, qq, window, sinks)
+        worst = max(float(np.abs(outs[True, window, sinks][i, h] - r).max())
+                    for i, rows in enumerate(ref) for h, r in rows.items())
+        assert worst <= TOL, (window, sinks, worst)
+
+
+def test_window_append_argument_errors():
+    w = workloads.custom_decode("winf2", [5, 40], 32, 8, 128, 16, "bf16", seed=2,
+                                spare_blocks=4, split_last=1)
+    g = GpuRun(w).apply(w.setup)
+    seqs = [op.args[0] for op in w.step]
+    slots, _ = g.pool.plan_append(seqs, [1] * len(seqs))
+    ks, vs = zip(*[w.kv_for(op) for op in w.step])
+    key, val = torch.cat(ks).cuda(), torch.cat(vs).cuda()
+    d_slots = torch.tensor(slots, dtype=torch.int64, device="cuda")
+    tables, tl, _, _ = g.tables()
+    q = w.queries()[:, 0].contiguous().cuda()
+    for window, sinks in ((0, 0), (4, -1)):
+        with pytest.raises(pa.PAError) as e:
+            g.pool.decode_window_append(q, key, val, d_slots, tables, tl, window, sinks)
+        assert e.value.code == 1
+    bad = d_slots.clone()
+    bad[1] = w.num_blocks * 16                            # one past the pool
+    out = g.pool.decode_window_append(q, key, val, bad, tables, tl, 8, 2)
+    assert g.pool.get_error() & pa.PA_DEVERR_SLOT
+    assert torch.all(torch.isfinite(out))
+    assert g.pool.get_error() == 0
