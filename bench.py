@@ -187,11 +187,11 @@ class Setup:
         import torch
         import paged_kv_cache_483_b200 as pa
         self.w, self.device, self.q8 = w, device, q8
-        if q8:    # int8 pool: packed (block, head) records, bf16 rows quantised on append
+        if q8:    # "int8" / "fp8" pool: packed (block, head) records, bf16 rows quantised on append
             self.k_cache = torch.empty((w.num_blocks, w.num_kv_heads, pa.PA_INT8_RECORD_BYTES),
                                        dtype=torch.uint8, device=device)
             self.v_cache = None
-            self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, "int8",
+            self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, q8,
                                 self.k_cache, None, alloc_order=w.order)
         else:
             dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
@@ -246,7 +246,7 @@ def decode_bytes(w, lens, q8=False, window=0, sinks=0):
     lens = lens.astype(np.int64)
     if window > 0:
         lens = np.minimum(lens, window + sinks)
-    if q8:    # int8 records: K and V codes plus two float32 scales per (token, head)
+    if q8:    # int8 / fp8 records: K and V codes plus two float32 scales per (token, head)
         return int(np.sum(lens)) * w.num_kv_heads * (2 * w.head_dim + 8)
     eb = 2 if w.dtype == "bf16" else 4
     return int(np.sum(lens)) * w.num_kv_heads * w.head_dim * 2 * eb
@@ -269,10 +269,10 @@ def run_ours(args, dist):
         workloads.seed_for({"decode32": 2, "ragged256": 3, "splitk128k": 4,
                             "prefill": 5}[args.config]))
     w = builder(seed=base_seed + 1000 * dist.rank)
-    q8 = args.kv == "int8"
+    q8 = args.kv if args.kv in ("int8", "fp8") else False
     win, sinks = args.window, args.sinks
     if (q8 or win) and w.q_tokens > 1:
-        raise SystemExit("--kv int8 and --window apply to the decode workloads")
+        raise SystemExit("--kv int8/fp8 and --window apply to the decode workloads")
     S = Setup(w, device, q8=q8)
     pool = S.pool
     is_prefill = w.q_tokens > 1
@@ -383,20 +383,21 @@ def run_ours(args, dist):
     else:
         kv = decode_bytes(w, lens, q8, win, sinks)
         value = dist.world * kv / (ms_step_max * 1e-3) / 1e9
-        metric = ("decode int8-KV HBM GB/s (codes + scales read) and seqs/s at 8K ctx, GQA 32/8"
+        metric = (f"decode {q8}-KV HBM GB/s (codes + scales read) and seqs/s at 8K ctx, GQA 32/8"
                   if q8 else
                   "decode KV HBM GB/s (fraction of B200 peak) and seqs/s at 8K ctx, GQA 32/8")
         if win:
             metric += f", window {win} + {sinks} sinks (visible keys only)"
         unit = "GB/s"
         achieved = kv / (kern_ms * 1e-3) / 1e9
-        kname = ("decode_q8_kernel" if q8 else "decode_mma_kernel"
+        kname = (f"decode_q8_kernel<{'true' if q8 == 'fp8' else 'false'}>" if q8 else
+                 "decode_mma_kernel"
                  if pool.decode_path(w.num_heads) else "attention_generic_kernel")
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4),
                 "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
                 "traffic": profiled_traffic("decode_q8.cu" if q8 else "decode_mma.cu",
-                                            w.name + ("_int8" if q8 else "")
+                                            w.name + (f"_{q8}" if q8 else "")
                                             + (f"_window{win}_sinks{sinks}" if win else "")),
                 "kernel": (f"decode_order_kernel + {kname}" if order_only else
                            f"{kname} + decode_combine_kernel" if split else kname),
@@ -413,7 +414,8 @@ def run_ours(args, dist):
         "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": dist.world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8 KV codes (int8/fp16 MMA, fp32 softmax), bf16 Q" if q8 else "bf16",
+        "dtype": ("int8 KV codes (int8/fp16 MMA, fp32 softmax), bf16 Q" if q8 == "int8" else
+                  "fp8 e4m3 KV codes (fp16 MMA, fp32 softmax), bf16 Q" if q8 else "bf16"),
         "data": "synthetic (seeded N(0,1), bf16-rounded)",
         "config": config_of(w, args, dist),
         **extra,
@@ -648,8 +650,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kv", choices=["bf16", "int8"], default="bf16",
-                    help="KV pool type for the decode workloads (int8: per-row absmax codes)")
+    ap.add_argument("--kv", choices=["bf16", "int8", "fp8"], default="bf16",
+                    help="KV pool type for the decode workloads (int8 / fp8: per-row absmax "
+                         "integer / E4M3 codes)")
     ap.add_argument("--window", type=int, default=0,
                     help="decode over the last WINDOW keys (plus --sinks first keys); 0 = all")
     ap.add_argument("--sinks", type=int, default=0)

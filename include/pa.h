@@ -74,8 +74,10 @@ typedef enum pa_status {
 } pa_status;
 
 /* PA_INT8: int8 codes with one float32 scale per (token, head) row; only
- * through pa_pool_create_int8. */
-typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_INT8 = 2 } pa_dtype;
+ * through pa_pool_create_int8 (or pa_pool_create_layers).  PA_FP8: E4M3
+ * codes in the same record; only through pa_pool_create_fp8 (or
+ * pa_pool_create_layers). */
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_INT8 = 2, PA_FP8 = 3 } pa_dtype;
 
 /* Bits of the device error word. */
 #define PA_DEVERR_BLOCK_ID 1  /* block-table entry outside [0, num_blocks)   */
@@ -103,7 +105,7 @@ typedef struct pa_stats {
  * order.  Copied; the caller may free it after the call.
  * Errors: PA_ERR_INVALID_ARG (non-positive size, not a permutation, exactly
  * one of k_cache/v_cache NULL, cache pointer not 16-byte aligned, kv_dtype
- * PA_INT8: use pa_pool_create_int8). */
+ * PA_INT8 / PA_FP8: use pa_pool_create_int8 / pa_pool_create_fp8). */
 pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
                          int32_t num_kv_heads, int32_t head_dim,
                          pa_dtype kv_dtype, void* k_cache, void* v_cache,
@@ -112,8 +114,8 @@ pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
 /* A pool whose caches hold num_layers layers ([P3] paged_attention's
  * `layer` argument: one block table per sequence serves every layer).
  * k_cache/v_cache: [num_layers, <one layer as for pa_pool_create>] (bf16 /
- * f32), or for PA_INT8 k_cache = [num_layers, num_blocks, num_kv_heads,
- * PA_INT8_RECORD_BYTES] records and v_cache NULL.  The returned handle is
+ * f32), or for PA_INT8 / PA_FP8 k_cache = [num_layers, num_blocks,
+ * num_kv_heads, PA_INT8_RECORD_BYTES] records and v_cache NULL.  The returned handle is
  * layer 0; pa_pool_layer gives the others.  All layers share the host
  * manager: sequence and plan calls on any of them act on the same tables.
  * A step over L layers plans once (pa_plan_append), copies once
@@ -121,7 +123,7 @@ pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
  * per layer (pa_reshape_and_cache, pa_decode, ... on each layer's handle);
  * pa_append_kv on a layer plans, copies in every layer and writes only that
  * layer.  Errors: as pa_pool_create / pa_pool_create_int8, INVALID_ARG for
- * num_layers < 1 or a NULL k_cache. */
+ * num_layers < 1, a NULL k_cache or an unknown kv_dtype. */
 pa_status pa_pool_create_layers(int32_t num_blocks, int32_t block_size,
                                 int32_t num_kv_heads, int32_t head_dim,
                                 pa_dtype kv_dtype, int32_t num_layers,
@@ -159,6 +161,20 @@ pa_status pa_pool_create_int8(int32_t num_blocks, int32_t block_size,
                               int32_t num_kv_heads, int32_t head_dim,
                               void* kv_records, const int32_t* alloc_order,
                               pa_pool** out);
+
+/* Pool of FP8 KV rows: the per-row absmax recipe of pa_pool_create_int8 on
+ * the E4M3 grid of the OCP 8-bit floating point specification (exponent
+ * bias 7, 3 mantissa bits, subnormals, no infinities, largest finite 448):
+ * scale = max|x| / 448 (1 for a zero row); code = the E4M3 value nearest to
+ * x / scale, ties to the even code, decided in float64; a zero magnitude is
+ * stored as +0; the scale is stored as float32 and a row reads back as
+ * value(code) * scale.  The records, their layout (PA_INT8_RECORD_BYTES per
+ * (block, head), E4M3 bytes in place of the int8 codes), the calls that
+ * take them and the errors are those of pa_pool_create_int8. */
+pa_status pa_pool_create_fp8(int32_t num_blocks, int32_t block_size,
+                             int32_t num_kv_heads, int32_t head_dim,
+                             void* kv_records, const int32_t* alloc_order,
+                             pa_pool** out);
 
 /* Destroy the manager, its staging area and error word (synchronises the
  * device first).  Never frees k_cache/v_cache.  NULL is a no-op. */
@@ -317,7 +333,7 @@ pa_status pa_decode(pa_pool* pool, const void* q, int32_t B, int32_t H,
  * The kernels walk only the blocks that hold a visible key, so a long
  * sequence costs about sinks + window tokens.  Arguments, layouts and errors
  * as pa_decode, plus window >= 1 and sinks >= 0 (else INVALID_ARG); the
- * tensor-core paths only (bf16 or int8 pool, block 16, head_dim 128,
+ * tensor-core paths only (bf16, int8 or FP8 pool, block 16, head_dim 128,
  * H / Hkv <= 8), else PA_ERR_UNSUPPORTED.  partition_tokens splits the walked
  * blocks; workspace: pa_decode_window_workspace_bytes bytes. */
 size_t pa_decode_window_workspace_bytes(const pa_pool* pool, int32_t B, int32_t H,
@@ -354,7 +370,7 @@ pa_status pa_decode_append(pa_pool* pool, const void* q, const void* key,
  * -- the result equals pa_reshape_and_cache followed by pa_decode_window.
  * The new token, at kv_lens[b] - 1, is always visible.  One kernel on a bf16
  * pool; two launches (quantising append, then the windowed decode) on
- * an int8 pool.  Workspace: pa_decode_window_workspace_bytes bytes.  Errors
+ * an int8 or FP8 pool.  Workspace: pa_decode_window_workspace_bytes bytes.  Errors
  * as pa_decode_window, plus INVALID_ARG for null or misaligned key / value /
  * d_slot_mapping. */
 pa_status pa_decode_window_append(pa_pool* pool, const void* q, const void* key,

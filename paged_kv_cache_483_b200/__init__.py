@@ -20,8 +20,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
 
-PA_F32, PA_BF16, PA_INT8 = 0, 1, 2
-PA_INT8_RECORD_BYTES = 4224   # one (block, head) record of an int8 pool
+PA_F32, PA_BF16, PA_INT8, PA_FP8 = 0, 1, 2, 3
+PA_INT8_RECORD_BYTES = 4224   # one (block, head) record of an int8 or FP8 pool
 STATUS = {0: "ok", 1: "invalid argument", 2: "unknown sequence", 3: "duplicate sequence",
           4: "pool exhausted", 5: "CUDA error", 6: "device error", 7: "unsupported",
           8: "host-only pool", 9: "broken invariant", 10: "scratch limit"}
@@ -35,7 +35,7 @@ EXPORTS = ["pa_pool_create", "pa_free", "pa_seq_create", "pa_seq_fork", "pa_seq_
            "pa_decode_static_scratch", "pa_decode_append", "pa_seq_create_cached",
            "pa_prefix_publish", "pa_prefix_clear", "pa_prefix_entries", "pa_pool_create_int8",
            "pa_decode_window", "pa_decode_window_workspace_bytes", "pa_pool_create_layers",
-           "pa_pool_layer", "pa_decode_window_append"]
+           "pa_pool_layer", "pa_decode_window_append", "pa_pool_create_fp8"]
 
 
 class PAError(RuntimeError):
@@ -71,6 +71,7 @@ def lib():
                                    C.POINTER(_P)], C.c_int),
         "pa_pool_layer": ([_P, _I32, C.POINTER(_P)], C.c_int),
         "pa_pool_create_int8": ([_I32, _I32, _I32, _I32, _P, _PI32, C.POINTER(_P)], C.c_int),
+        "pa_pool_create_fp8": ([_I32, _I32, _I32, _I32, _P, _PI32, C.POINTER(_P)], C.c_int),
         "pa_seq_create": ([_P, _I32], C.c_int),
         "pa_seq_fork": ([_P, _I32, _I32, _I32], C.c_int),
         "pa_seq_release": ([_P, _I32], C.c_int),
@@ -147,10 +148,10 @@ class Pool:
     """A physical KV pool [num_blocks, block_size, num_kv_heads, head_dim]
     plus its host block manager.  ``k_cache``/``v_cache`` are borrowed CUDA
     tensors (kept alive here); pass ``None`` for both to get a host-only
-    manager (no GPU needed).  ``dtype="int8"``: ``k_cache`` is the uint8
-    tensor [num_blocks, num_kv_heads, PA_INT8_RECORD_BYTES] of packed
-    (block, head) records (layout in ``pa.h``) and ``v_cache`` is None;
-    appends and queries are bf16."""
+    manager (no GPU needed).  ``dtype="int8"`` or ``"fp8"`` (E4M3 codes):
+    ``k_cache`` is the uint8 tensor [num_blocks, num_kv_heads,
+    PA_INT8_RECORD_BYTES] of packed (block, head) records (layout in
+    ``pa.h``) and ``v_cache`` is None; appends and queries are bf16."""
 
     def __init__(self, num_blocks, block_size, num_kv_heads, head_dim, dtype="bf16",
                  k_cache=None, v_cache=None, alloc_order=None):
@@ -159,17 +160,18 @@ class Pool:
         self.num_kv_heads, self.head_dim = int(num_kv_heads), int(head_dim)
         self.dtype = dtype
         self.k_cache, self.v_cache = k_cache, v_cache
-        if dtype == "int8":
+        if dtype in ("int8", "fp8"):
             import torch
             rshape = (self.num_blocks, self.num_kv_heads, PA_INT8_RECORD_BYTES)
             if k_cache is None or tuple(k_cache.shape) != rshape or v_cache is not None:
-                raise ValueError(f"an int8 pool takes k_cache = uint8 records {rshape} "
+                raise ValueError(f"an {dtype} pool takes k_cache = uint8 records {rshape} "
                                  "and no v_cache")
             order_arr, order_p = (None, None) if alloc_order is None else _i32(alloc_order)
             h = C.c_void_p()
-            _check(L.pa_pool_create_int8(num_blocks, block_size, num_kv_heads, head_dim,
-                                         _dev_ptr(k_cache, torch.uint8, "k_cache"), order_p,
-                                         C.byref(h)), "pa_pool_create_int8")
+            fn = "pa_pool_create_int8" if dtype == "int8" else "pa_pool_create_fp8"
+            _check(getattr(L, fn)(num_blocks, block_size, num_kv_heads, head_dim,
+                                  _dev_ptr(k_cache, torch.uint8, "k_cache"), order_p,
+                                  C.byref(h)), fn)
             self._h = h
             self._ws = None
             return
@@ -202,8 +204,9 @@ class Pool:
         self.num_kv_heads, self.head_dim = int(num_kv_heads), int(head_dim)
         self.dtype, self.k_cache, self.v_cache = dtype, k_cache, v_cache
         self._ws, self._view = None, False
-        code = {"bf16": PA_BF16, "f32": PA_F32, "int8": PA_INT8}[dtype]
-        want = {"bf16": torch.bfloat16, "f32": torch.float32, "int8": torch.uint8}[dtype]
+        code = {"bf16": PA_BF16, "f32": PA_F32, "int8": PA_INT8, "fp8": PA_FP8}[dtype]
+        want = {"bf16": torch.bfloat16, "f32": torch.float32, "int8": torch.uint8,
+                "fp8": torch.uint8}[dtype]
         order_arr, order_p = (None, None) if alloc_order is None else _i32(alloc_order)
         h = C.c_void_p()
         _check(lib().pa_pool_create_layers(num_blocks, block_size, num_kv_heads, head_dim, code,
@@ -329,9 +332,9 @@ class Pool:
 
     # -- device hot path ------------------------------------------------------
     def _torch_dtype(self):
-        """Type of queries and of the K/V rows handed in (bf16 for int8 pools)."""
+        """Type of queries and of the K/V rows handed in (bf16 for int8 / fp8 pools)."""
         import torch
-        return torch.bfloat16 if self.dtype in ("bf16", "int8") else torch.float32
+        return torch.bfloat16 if self.dtype in ("bf16", "int8", "fp8") else torch.float32
 
     def append_kv(self, seqs, n_new, key, value, stream=None, return_slots=False):
         """Plan + copy-on-write + reshape_and_cache.  key/value [T, Hkv, d] CUDA."""

@@ -30,6 +30,12 @@
 //    keeps its precision; O is rescaled by the ratio of successive 2^E
 //    together with the online-softmax factor).  P goes in as fp16 hi + lo
 //    parts; l sums the unscaled p_j.
+// FP8 (E4M3) pools use the same record, with E4M3 codes and scales
+// absmax / 448.  The fp8 instance converts codes to fp16 with the E4M3 x2 ->
+// f16 x2 conversion (every E4M3 value is exact in fp16) and runs both
+// products on the fp16 MMA: Q enters as fp16 with a power-of-two scale (exact
+// for bf16 inputs), so S = K Q^T is exact up to fp32 accumulation; E4M3 has
+// NaN codes, so the V bytes of dead tokens are zeroed before conversion.
 // Token order: row r of a block's S^T tile holds token kPerm[r].  With it a
 // thread's P^T fragment covers tokens 4c .. 4c + 3 (two per register), the
 // four bytes of one 32-bit word of a V d-row, and the K rows a warp reads at
@@ -37,6 +43,7 @@
 #include <math.h>
 
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "launch.hpp"
@@ -97,6 +104,14 @@ __device__ __forceinline__ uint32_t codes_half2(uint32_t u, uint32_t sel) {
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
+// Two E4M3 codes (low byte, high byte of a 16-bit pair) as an exact half2
+// (low byte -> low half).
+__device__ __forceinline__ uint32_t e4m3x2_half2(uint32_t pair) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+      static_cast<__nv_fp8x2_storage_t>(pair & 0xFFFFu), __NV_E4M3);
+  return uint32_t(h.x) | (uint32_t(h.y) << 16);
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -104,6 +119,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 
 }  // namespace
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
     const __grid_constant__ CUtensorMap tmR, const DecodeArgs p, float scale_log2) {
   extern __shared__ uint8_t q8_raw[];
@@ -197,8 +213,11 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
 
   // ------------------------------------------------------------- consumers
   const int g = lane >> 2, c = lane & 3;
-  // Q of head g as int8 hi + lo parts in the B-fragment order of m16n8k32:
-  // word kk*2 + h covers d = 32 kk + 16 h + 4c .. + 3
+  // int8: Q of head g as int8 hi + lo parts in the B-fragment order of
+  // m16n8k32: word kk*2 + h covers d = 32 kk + 16 h + 4c .. + 3.
+  // fp8: Q / sq as fp16 B fragments of m16n8k16 over d chunk 2 kk + h, with
+  // MMA k (2c, 2c + 1) = d (4c, 4c + 1) in qh and k (2c + 8, 2c + 9) =
+  // d (4c + 2, 4c + 3) in ql, the order in which the K words unpack.
   uint32_t qh[4][2], ql[4][2];
   float qs0, qs1;   // sq * scale_log2 of heads 2c and 2c + 1 (S^T columns)
   {
@@ -221,7 +240,21 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
       }
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const float sq = amax > 0.f ? amax / 127.f : 1.f;
+    float sq;
+    if constexpr (kFp8) {
+      // sq = the power of two at or below amax: Q / sq is exact in fp16
+      const uint32_t e = min(max((__float_as_uint(amax) >> 23) & 0xFFu, 1u), 253u);
+      sq = __uint_as_float(e << 23);
+      const float inv = __uint_as_float((254u - e) << 23);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          qh[kk][h] = pack_half2(x[kk][h][0] * inv, x[kk][h][1] * inv);
+          ql[kk][h] = pack_half2(x[kk][h][2] * inv, x[kk][h][3] * inv);
+        }
+    } else {
+    sq = amax > 0.f ? amax / 127.f : 1.f;
     const float inv = amax > 0.f ? 127.f / amax : 0.f;
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
@@ -239,6 +272,7 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
         qh[kk][h] = hw;
         ql[kk][h] = lw;
       }
+    }
     qs0 = __shfl_sync(0xffffffffu, sq, 8 * c) * scale_log2;
     qs1 = __shfl_sync(0xffffffffu, sq, 8 * c + 4) * scale_log2;
   }
@@ -249,6 +283,9 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
   // for c < 2 and bytes (2,3) otherwise; kPerm[2c+8], kPerm[2c+9] the others
   const uint32_t sel_a = c < 2 ? 0x4140u : 0x4342u;
   const uint32_t sel_b = c < 2 ? 0x4342u : 0x4140u;
+  // fp8: the same pairs, as the low and high halves of the word rotated so
+  // that the pair of A fragment a0 comes first
+  const uint32_t vrot = c < 2 ? 0x3210u : 0x1032u;
   float o[8][4];
 #pragma unroll
   for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
@@ -281,6 +318,7 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
     const int tb[2] = {vis_blk(blk0 + i) * 16, vis_blk(blk0 + i2) * 16};
     // ---- S^T = K Q^T on int8 codes: hi and lo parts of Q
     int ih[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, il[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+    float fs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};   // fp8: S in fp32
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       const uint32_t c0 = 2 * kk, c1 = 2 * kk + 1;
@@ -294,8 +332,18 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
       }
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        mma_s8_16832(ih[x], a[x][0], a[x][1], a[x][2], a[x][3], qh[kk][0], qh[kk][1]);
-        mma_s8_16832(il[x], a[x][0], a[x][1], a[x][2], a[x][3], ql[kk][0], ql[kk][1]);
+        if constexpr (kFp8) {
+          // chunk 2kk: rows A, B in a[x][0], a[x][1]; chunk 2kk + 1: a[x][2], a[x][3]
+          mma_f16_16816(fs[x], e4m3x2_half2(a[x][0]), e4m3x2_half2(a[x][1]),
+                        e4m3x2_half2(a[x][0] >> 16), e4m3x2_half2(a[x][1] >> 16), qh[kk][0],
+                        ql[kk][0]);
+          mma_f16_16816(fs[x], e4m3x2_half2(a[x][2]), e4m3x2_half2(a[x][3]),
+                        e4m3x2_half2(a[x][2] >> 16), e4m3x2_half2(a[x][3] >> 16), qh[kk][1],
+                        ql[kk][1]);
+        } else {
+          mma_s8_16832(ih[x], a[x][0], a[x][1], a[x][2], a[x][3], qh[kk][0], qh[kk][1]);
+          mma_s8_16832(il[x], a[x][0], a[x][1], a[x][2], a[x][3], ql[kk][0], ql[kk][1]);
+        }
       }
     }
     float sc[2][4], vA[2], vB[2];
@@ -305,10 +353,14 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
       const bool live0 = use[x] && t0 < tok_end && (t0 >= lo || t0 < p.sinks);
       const bool live1 = use[x] && t1 < tok_end && (t1 >= lo || t1 < p.sinks);
       const float kA = scl[x][tokA], kB = scl[x][tokB];
-      sc[x][0] = live0 ? fmaf(float(il[x][0]), 1.f / 254.f, float(ih[x][0])) * (kA * qs0) : -INFINITY;
-      sc[x][1] = live0 ? fmaf(float(il[x][1]), 1.f / 254.f, float(ih[x][1])) * (kA * qs1) : -INFINITY;
-      sc[x][2] = live1 ? fmaf(float(il[x][2]), 1.f / 254.f, float(ih[x][2])) * (kB * qs0) : -INFINITY;
-      sc[x][3] = live1 ? fmaf(float(il[x][3]), 1.f / 254.f, float(ih[x][3])) * (kB * qs1) : -INFINITY;
+      float dot[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        dot[k] = kFp8 ? fs[x][k] : fmaf(float(il[x][k]), 1.f / 254.f, float(ih[x][k]));
+      sc[x][0] = live0 ? dot[0] * (kA * qs0) : -INFINITY;
+      sc[x][1] = live0 ? dot[1] * (kA * qs1) : -INFINITY;
+      sc[x][2] = live1 ? dot[2] * (kB * qs0) : -INFINITY;
+      sc[x][3] = live1 ? dot[3] * (kB * qs1) : -INFINITY;
       vA[x] = live0 ? scl[x][16 + tokA] : 0.f;
       vB[x] = live1 ? scl[x][16 + tokB] : 0.f;
     }
@@ -369,19 +421,43 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
       fb[x][2] = movmatrix_trans(pack_half2(q0 - f01.x, q1 - f01.y));
       fb[x][3] = movmatrix_trans(pack_half2(q2 - f23.x, q3 - f23.y));
     }
+    // fp8: byte mask of this thread's live tokens 4c .. 4c + 3 per block
+    uint32_t vmask[2] = {0u, 0u};
+    if constexpr (kFp8) {
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int t = tb[x] + 4 * c + u;
+          if (use[x] && t < tok_end && (t >= lo || t < p.sinks)) vmask[x] |= 0xFFu << (8 * u);
+        }
+    }
     // ---- O^T += V^T P^T: d rows 16j + g and 16j + g + 8, tokens 4c .. 4c + 3
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       uint32_t w[2][2];
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        w[x][0] = lds32(kb[x] + 2048 + (16 * j + g) * 16 + 4 * c) ^ 0x80808080u;
-        w[x][1] = lds32(kb[x] + 2048 + (16 * j + g + 8) * 16 + 4 * c) ^ 0x80808080u;
+        w[x][0] = lds32(kb[x] + 2048 + (16 * j + g) * 16 + 4 * c);
+        w[x][1] = lds32(kb[x] + 2048 + (16 * j + g + 8) * 16 + 4 * c);
       }
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        const uint32_t a0 = codes_half2(w[x][0], sel_a), a2 = codes_half2(w[x][0], sel_b);
-        const uint32_t a1 = codes_half2(w[x][1], sel_a), a3 = codes_half2(w[x][1], sel_b);
+        uint32_t a0, a1, a2, a3;
+        if constexpr (kFp8) {
+          const uint32_t u0 = __byte_perm(w[x][0] & vmask[x], 0u, vrot);
+          const uint32_t u1 = __byte_perm(w[x][1] & vmask[x], 0u, vrot);
+          a0 = e4m3x2_half2(u0);
+          a2 = e4m3x2_half2(u0 >> 16);
+          a1 = e4m3x2_half2(u1);
+          a3 = e4m3x2_half2(u1 >> 16);
+        } else {
+          const uint32_t b0 = w[x][0] ^ 0x80808080u, b1 = w[x][1] ^ 0x80808080u;
+          a0 = codes_half2(b0, sel_a);
+          a2 = codes_half2(b0, sel_b);
+          a1 = codes_half2(b1, sel_a);
+          a3 = codes_half2(b1, sel_b);
+        }
         mma_f16_16816(o[j], a0, a1, a2, a3, fb[x][0], fb[x][1]);
         mma_f16_16816(o[j], a0, a1, a2, a3, fb[x][2], fb[x][3]);
       }
@@ -463,22 +539,23 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
   }
 }
 
-cudaError_t launch_decode_q8(const CUtensorMap* tmR, const DecodeArgs& a,
+cudaError_t launch_decode_q8(const CUtensorMap* tmR, const DecodeArgs& a, bool fp8,
                              cudaStream_t stream) {
   if (a.order) {
     cudaError_t eo = launch_decode_order(a.kv_lens, a.B, a.order, stream);
     if (eo != cudaSuccess) return eo;
   }
   const size_t smem = 128 + kQ8Stages * kQ8StageBytes + sizeof(Q8Tail);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_q8_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  auto* kern = fp8 ? decode_q8_kernel<true> : decode_q8_kernel<false>;
+  static bool attr_set[2] = {false, false};
+  if (!attr_set[fp8]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(smem));
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[fp8] = true;
   }
   dim3 grid(a.NP, a.Hkv, a.B);
-  decode_q8_kernel<<<grid, kQ8Threads, smem, stream>>>(*tmR, a, a.scale * kLog2e);
+  kern<<<grid, kQ8Threads, smem, stream>>>(*tmR, a, a.scale * kLog2e);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.NP == 1) return e;
   return launch_decode_combine(a.ws, a.B, a.H, a.NP, a.out, stream);

@@ -55,12 +55,32 @@ __global__ void __launch_bounds__(256) cow_copy_kernel(
   }
 }
 
-// int8 pools: one warp per (token, head) row of K and of V.  The row's
-// absmax is exact in float32 (bf16 inputs); scale = absmax / 127 and the
-// codes rint(x / scale), clipped to +-127, are decided in float64 as the
-// quantisation experiment of "vladkulikov.com modern-llms module 9 notebook"
-// states; the scale is stored as float32.  Returns this lane's 4 codes
-// (d = 4 lane .. 4 lane + 3) packed in a word; lane 0 also stores the scale.
+// E4M3 code of y, |y| <= 448 (float64): the nearest value of the E4M3 grid
+// of the OCP 8-bit floating point specification (exponent bias 7, 3 mantissa
+// bits, subnormals, largest finite 448), ties to the even code; a zero
+// magnitude gives +0.  Inside binade e (floored at -6, the subnormal range)
+// the grid step is 2^(e - 3), so m = rint(|y| / 2^(e - 3)) lies in [8, 16]
+// ([0, 8] for subnormals) and the code is (e + 7) * 8 + m - 8 -- which is
+// also right when m rounds up to 16, the next binade's first value.
+__device__ __forceinline__ uint32_t e4m3_code(double y) {
+  const double a = fmin(fabs(y), 448.0);
+  const int e = max(int((__double_as_longlong(a) >> 52) & 0x7FF) - 1023, -6);
+  const double m = rint(a * __longlong_as_double(int64_t(1023 + 3 - e) << 52));
+  const uint32_t mag = uint32_t((e + 7) * 8 + int(m) - 8);
+  return (mag != 0u && y < 0.0) ? (mag | 0x80u) : mag;
+}
+
+// Quantised pools: one warp per (token, head) row of K and of V.  The row's
+// absmax is exact in float32 (bf16 inputs); the codes are decided in float64
+// as the quantisation experiment of "vladkulikov.com modern-llms module 9
+// notebook" states:
+//  * int8: scale = absmax / 127, code = rint(x / scale) clipped to +-127;
+//  * fp8 (E4M3): scale = absmax / 448, code = the nearest E4M3 value to
+//    x / scale (the same per-row recipe on the 8-bit float grid).
+// A zero row takes scale 1.  The scale is stored as float32.  Returns this
+// lane's 4 codes (d = 4 lane .. 4 lane + 3) packed in a word; lane 0 also
+// stores the scale.
+template <bool kFp8>
 __device__ __forceinline__ uint32_t quantize_row(const __nv_bfloat16* __restrict__ src,
                                                  float* scale_dst, int lane) {
   const uint2 w = *reinterpret_cast<const uint2*>(src + 4 * lane);
@@ -73,13 +93,15 @@ __device__ __forceinline__ uint32_t quantize_row(const __nv_bfloat16* __restrict
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1)
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  double scale = double(amax) / 127.0;
+  const double limit = kFp8 ? 448.0 : 127.0;
+  double scale = double(amax) / limit;
   if (scale == 0.0) scale = 1.0;
   uint32_t packed = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const double q = fmin(fmax(rint(double(x[i]) / scale), -127.0), 127.0);
-    packed |= (uint32_t(int32_t(q)) & 0xFFu) << (8 * i);
+    const double t = fmin(fmax(double(x[i]) / scale, -limit), limit);
+    const uint32_t code = kFp8 ? e4m3_code(t) : (uint32_t(int32_t(rint(t))) & 0xFFu);
+    packed |= code << (8 * i);
   }
   if (lane == 0) *scale_dst = __double2float_rn(scale);
   return packed;
@@ -88,6 +110,7 @@ __device__ __forceinline__ uint32_t quantize_row(const __nv_bfloat16* __restrict
 // Writes each row into its packed (block, head) record: K codes at
 // token * 128 + ((chunk ^ (token & 7)) << 4) + byte, V codes at 2048 + d * 16
 // + token, scales at 4096 + 4 token (K) and 4160 + 4 token (V).
+template <bool kFp8>
 __global__ void __launch_bounds__(256) reshape_and_cache_q8_kernel(
     const __nv_bfloat16* __restrict__ key, const __nv_bfloat16* __restrict__ value,
     uint8_t* __restrict__ records, const int64_t* __restrict__ slot_mapping, int32_t T,
@@ -108,9 +131,9 @@ __global__ void __launch_bounds__(256) reshape_and_cache_q8_kernel(
     const int tok = int(slot & 15);
     uint8_t* rec = records + ((slot >> 4) * Hkv + h) * kQ8RecordBytes;
     const uint32_t kw =
-        quantize_row(key + r * 128, reinterpret_cast<float*>(rec + 4096) + tok, lane);
+        quantize_row<kFp8>(key + r * 128, reinterpret_cast<float*>(rec + 4096) + tok, lane);
     const uint32_t vw =
-        quantize_row(value + r * 128, reinterpret_cast<float*>(rec + 4160) + tok, lane);
+        quantize_row<kFp8>(value + r * 128, reinterpret_cast<float*>(rec + 4160) + tok, lane);
     // lane covers d = 4 lane .. + 3: chunk lane / 4, byte 4 (lane % 4)
     *reinterpret_cast<uint32_t*>(rec + tok * 128 + (((lane >> 2) ^ (tok & 7)) << 4) +
                                  4 * (lane & 3)) = kw;
@@ -121,13 +144,15 @@ __global__ void __launch_bounds__(256) reshape_and_cache_q8_kernel(
 
 cudaError_t launch_reshape_and_cache_q8(const void* key, const void* value, void* records,
                                         const int64_t* slots, int32_t T, int32_t Hkv,
-                                        int64_t num_slots, int32_t* err, int sms,
+                                        int64_t num_slots, bool fp8, int32_t* err, int sms,
                                         cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
   const int64_t rows = int64_t(T) * Hkv;
   int64_t g = (rows + 7) / 8;
   g = g > int64_t(sms) * 8 ? int64_t(sms) * 8 : g;
-  reshape_and_cache_q8_kernel<<<int(g < 1 ? 1 : g), 256, 0, stream>>>(
+  const int grid = int(g < 1 ? 1 : g);
+  auto* kern = fp8 ? reshape_and_cache_q8_kernel<true> : reshape_and_cache_q8_kernel<false>;
+  kern<<<grid, 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value),
       static_cast<uint8_t*>(records), slots, T, Hkv, num_slots, err);
   return cudaGetLastError();

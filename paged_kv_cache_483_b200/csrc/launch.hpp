@@ -79,15 +79,18 @@ cudaError_t launch_decode_combine(const float* ws, int32_t B, int32_t H, int32_t
 // chunks stored swizzled (chunk k at k ^ (token & 7)), V codes [128 d][16
 // tokens], 16 float32 K scales, 16 float32 V scales.
 constexpr int kQ8RecordBytes = 4224;
+// The same record holds int8 codes or FP8 (E4M3) codes.
 // Append: key/value bf16 [T, Hkv, 128] are quantised per (token, head) row
-// (absmax / 127, round half to even, decided in float64) into their slots.
+// (int8: absmax / 127, round half to even; fp8: absmax / 448, nearest E4M3
+// value, ties to even; decided in float64) into their slots.
 cudaError_t launch_reshape_and_cache_q8(const void* key, const void* value, void* records,
                                         const int64_t* slots, int32_t T, int32_t Hkv,
-                                        int64_t num_slots, int32_t* err, int sms,
+                                        int64_t num_slots, bool fp8, int32_t* err, int sms,
                                         cudaStream_t stream);
-// Decode over an int8 pool (G <= 8; tmR maps the records as
+// Decode over an int8 or FP8 pool (G <= 8; tmR maps the records as
 // {128 bytes, 33 rows, NB * Hkv}), dequantising in the kernel.
-cudaError_t launch_decode_q8(const CUtensorMap* tmR, const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_q8(const CUtensorMap* tmR, const DecodeArgs& a, bool fp8,
+                             cudaStream_t stream);
 // Scratch for the longest-first order when the grid spans several waves.
 bool decode_wants_order(int32_t B, int32_t Hkv, int32_t NP, int sms);
 size_t order_workspace_bytes(int32_t B);

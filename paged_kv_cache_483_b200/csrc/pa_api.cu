@@ -84,7 +84,10 @@ pa_status from_mgr(MgrStatus s) {
 
 static_assert(pa::kQ8RecordBytes == PA_INT8_RECORD_BYTES, "int8 record size");
 
-size_t elem_bytes(pa_dtype t) { return t == PA_INT8 ? 1 : t == PA_BF16 ? 2 : 4; }
+// int8 and FP8 pools share one packed record layout
+bool is_q8(pa_dtype t) { return t == PA_INT8 || t == PA_FP8; }
+
+size_t elem_bytes(pa_dtype t) { return is_q8(t) ? 1 : t == PA_BF16 ? 2 : 4; }
 
 bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
@@ -114,7 +117,7 @@ bool make_pool_map(CUtensorMap* map, void* base, const pa_pool* p) {
   auto fn = encode_fn();
   if (!fn) return false;
   // int8 pools: one box = the block's 16 rows of 128 codes (128 bytes)
-  const bool q8 = p->dtype == PA_INT8;
+  const bool q8 = is_q8(p->dtype);
   const cuuint64_t eb = q8 ? 1 : 2;
   const cuuint64_t dims[3] = {cuuint64_t(p->head_dim), cuuint64_t(p->num_kv_heads),
                               cuuint64_t(p->num_blocks) * p->block_size};
@@ -180,7 +183,7 @@ bool decode_partitions(const pa_pool* p, int32_t B, int32_t MB,
 }
 
 bool use_fast_decode(const pa_pool* p, int32_t H) {
-  if (p->dtype == PA_INT8)   // packed records, no tensor maps
+  if (is_q8(p->dtype))   // packed records, no tensor maps
     return p->device && H % p->num_kv_heads == 0 && H / p->num_kv_heads <= 8;
   return p->tmap_ok && H % p->num_kv_heads == 0 &&
          pa::decode_fast_supported(p->dtype == PA_BF16, p->head_dim,
@@ -215,7 +218,7 @@ static pa_status create_pool(int32_t num_blocks, int32_t block_size, int32_t num
   *out = nullptr;
   if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
     return PA_ERR_INVALID_ARG;
-  if (kv_dtype != PA_INT8 && (k_cache == nullptr) != (v_cache == nullptr))
+  if (!is_q8(kv_dtype) && (k_cache == nullptr) != (v_cache == nullptr))
     return PA_ERR_INVALID_ARG;
   if (k_cache && (!aligned16(k_cache) || (v_cache && !aligned16(v_cache))))
     return PA_ERR_INVALID_ARG;
@@ -250,7 +253,7 @@ static pa_status create_pool(int32_t num_blocks, int32_t block_size, int32_t num
     if (kv_dtype == PA_BF16 && head_dim == 128 && block_size == 16)
       p->tmap_ok = make_pool_map(&p->tmK, k_cache, p) &&
                    make_pool_map(&p->tmV, v_cache, p);
-    if (kv_dtype == PA_INT8 && !make_record_map(&p->tmK, k_cache, p)) {
+    if (is_q8(kv_dtype) && !make_record_map(&p->tmK, k_cache, p)) {
       cudaFree(p->d_err);
       delete p;
       return PA_ERR_CUDA;
@@ -275,9 +278,9 @@ static pa_status create_pool(int32_t num_blocks, int32_t block_size, int32_t num
 // same manager, error word and prefill scratch; own base pointers, tensor
 // maps and append staging.
 static pa_status add_layer_views(pa_pool* p, int32_t num_layers) {
-  const size_t eb = p->dtype == PA_INT8 ? 1 : p->dtype == PA_BF16 ? 2 : 4;
+  const size_t eb = is_q8(p->dtype) ? 1 : p->dtype == PA_BF16 ? 2 : 4;
   p->num_layers = num_layers;
-  p->layer_bytes = p->dtype == PA_INT8
+  p->layer_bytes = is_q8(p->dtype)
                        ? int64_t(p->num_blocks) * p->num_kv_heads * pa::kQ8RecordBytes
                        : int64_t(p->num_blocks) * p->block_size * p->num_kv_heads *
                              p->head_dim * int64_t(eb);
@@ -304,7 +307,7 @@ static pa_status add_layer_views(pa_pool* p, int32_t num_layers) {
     v->tickets = p->tickets;
     v->k_cache = static_cast<char*>(p->k_cache) + l * p->layer_bytes;
     v->v_cache = p->v_cache ? static_cast<char*>(p->v_cache) + l * p->layer_bytes : nullptr;
-    if (p->dtype == PA_INT8) {
+    if (is_q8(p->dtype)) {
       if (!make_record_map(&v->tmK, v->k_cache, v)) return PA_ERR_CUDA;
     } else if (p->tmap_ok) {
       v->tmap_ok = make_pool_map(&v->tmK, v->k_cache, v) && make_pool_map(&v->tmV, v->v_cache, v);
@@ -320,8 +323,9 @@ pa_status pa_pool_create_layers(int32_t num_blocks, int32_t block_size, int32_t 
                                 pa_pool** out) {
   if (out) *out = nullptr;
   if (num_layers < 1 || !k_cache) return PA_ERR_INVALID_ARG;
-  if (kv_dtype == PA_INT8 && (block_size != 16 || head_dim != 128)) return PA_ERR_UNSUPPORTED;
-  if (kv_dtype == PA_INT8 && v_cache) return PA_ERR_INVALID_ARG;
+  if (kv_dtype != PA_F32 && kv_dtype != PA_BF16 && !is_q8(kv_dtype)) return PA_ERR_INVALID_ARG;
+  if (is_q8(kv_dtype) && (block_size != 16 || head_dim != 128)) return PA_ERR_UNSUPPORTED;
+  if (is_q8(kv_dtype) && v_cache) return PA_ERR_INVALID_ARG;
   pa_status st = create_pool(num_blocks, block_size, num_kv_heads, head_dim, kv_dtype, k_cache,
                              v_cache, alloc_order, out);
   if (st != PA_OK) return st;
@@ -361,6 +365,16 @@ pa_status pa_pool_create_int8(int32_t num_blocks, int32_t block_size, int32_t nu
   if (block_size != 16 || head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (!kv_records) return PA_ERR_INVALID_ARG;
   return create_pool(num_blocks, block_size, num_kv_heads, head_dim, PA_INT8, kv_records,
+                     nullptr, alloc_order, out);
+}
+
+pa_status pa_pool_create_fp8(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                             int32_t head_dim, void* kv_records, const int32_t* alloc_order,
+                             pa_pool** out) {
+  if (out) *out = nullptr;
+  if (block_size != 16 || head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (!kv_records) return PA_ERR_INVALID_ARG;
+  return create_pool(num_blocks, block_size, num_kv_heads, head_dim, PA_FP8, kv_records,
                      nullptr, alloc_order, out);
 }
 
@@ -524,7 +538,7 @@ static cudaError_t cow_blocks(pa_pool* p, const int32_t* d_src, const int32_t* d
   for (int32_t l = 0; l < o->num_layers && e == cudaSuccess; ++l) {
     char* kc = static_cast<char*>(o->k_cache) + l * o->layer_bytes;
     char* vc = o->v_cache ? static_cast<char*>(o->v_cache) + l * o->layer_bytes : nullptr;
-    if (o->dtype == PA_INT8)   // one array of packed records
+    if (is_q8(o->dtype))   // one array of packed records
       e = pa::launch_cow_copy(kc, nullptr, d_src, d_dst, n,
                               int64_t(o->num_kv_heads) * pa::kQ8RecordBytes, o->num_blocks,
                               o->d_err, o->sms, s);
@@ -537,13 +551,15 @@ static cudaError_t cow_blocks(pa_pool* p, const int32_t* d_src, const int32_t* d
   return e;
 }
 
-// K1 for any pool: copies rows, or quantises bf16 rows into an int8 pool.
+// K1 for any pool: copies rows, or quantises bf16 rows into an int8 or FP8
+// pool.
 static cudaError_t write_rows(pa_pool* p, const void* key, const void* value,
                               const int64_t* d_slots, int32_t T, cudaStream_t s) {
   const int64_t num_slots = int64_t(p->num_blocks) * p->block_size;
-  if (p->dtype == PA_INT8)
+  if (is_q8(p->dtype))
     return pa::launch_reshape_and_cache_q8(key, value, p->k_cache, d_slots, T,
-                                           p->num_kv_heads, num_slots, p->d_err, p->sms, s);
+                                           p->num_kv_heads, num_slots, p->dtype == PA_FP8,
+                                           p->d_err, p->sms, s);
   return pa::launch_reshape_and_cache(key, value, p->k_cache, p->v_cache, d_slots, T,
                                       int64_t(p->num_kv_heads) * p->head_dim *
                                           elem_bytes(p->dtype),
@@ -688,8 +704,9 @@ static pa_status decode_fast(pa_pool* p, const void* q, int32_t B, int32_t H,
   a.v_cache = p->v_cache;
   a.window = window;
   a.sinks = sinks;
-  if (p->dtype == PA_INT8)
-    return cuda_status(pa::launch_decode_q8(&p->tmK, a, static_cast<cudaStream_t>(stream)));
+  if (is_q8(p->dtype))
+    return cuda_status(pa::launch_decode_q8(&p->tmK, a, p->dtype == PA_FP8,
+                                            static_cast<cudaStream_t>(stream)));
   return cuda_status(pa::launch_decode_fast(&p->tmK, &p->tmV, a, p->sms,
                                             static_cast<cudaStream_t>(stream)));
 }
@@ -722,7 +739,7 @@ pa_status pa_decode(pa_pool* p, const void* q, int32_t B, int32_t H,
     return decode_fast(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale,
                        partition_tokens, workspace, workspace_bytes, out, stream, nullptr,
                        nullptr, nullptr);
-  if (p->dtype == PA_INT8) return PA_ERR_UNSUPPORTED;   // G > 8 on an int8 pool
+  if (is_q8(p->dtype)) return PA_ERR_UNSUPPORTED;   // G > 8 on an int8 / FP8 pool
   if (partition_tokens % p->block_size) return PA_ERR_INVALID_ARG;
   pa::GenericArgs g{q, p->k_cache, p->v_cache, d_block_tables, max_blocks,
                     d_kv_lens, B, 1, H, p->num_kv_heads, p->head_dim,
@@ -764,7 +781,7 @@ pa_status pa_decode_append(pa_pool* p, const void* q, const void* key, const voi
   if (B > 0 && (!key || !value || !d_slot_mapping)) return PA_ERR_INVALID_ARG;
   if (partition_tokens < 0) return PA_ERR_INVALID_ARG;
   if (B == 0) return PA_OK;
-  if (!use_fast_decode(p, H) || p->dtype == PA_INT8) {
+  if (!use_fast_decode(p, H) || is_q8(p->dtype)) {
     // same result in two launches on the other paths
     st = pa_reshape_and_cache(p, key, value, d_slot_mapping, B, stream);
     if (st != PA_OK) return st;
@@ -789,8 +806,8 @@ pa_status pa_decode_window_append(pa_pool* p, const void* q, const void* key,
   if (partition_tokens < 0 || window < 1 || sinks < 0) return PA_ERR_INVALID_ARG;
   if (!use_fast_decode(p, H)) return PA_ERR_UNSUPPORTED;
   if (B == 0) return PA_OK;
-  if (p->dtype == PA_INT8) {
-    // the quantising append is its own launch on an int8 pool
+  if (is_q8(p->dtype)) {
+    // the quantising append is its own launch on an int8 / FP8 pool
     st = pa_reshape_and_cache(p, key, value, d_slot_mapping, B, stream);
     if (st != PA_OK) return st;
     return pa_decode_window(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale, window,
@@ -813,7 +830,7 @@ pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,
                                       d_kv_lens, out);
   if (st != PA_OK) return st;
   if (q_tokens <= 0 || q_tokens > 65535 || max_kv_splits < 0) return PA_ERR_INVALID_ARG;
-  if (p->dtype == PA_INT8) return PA_ERR_UNSUPPORTED;
+  if (is_q8(p->dtype)) return PA_ERR_UNSUPPORTED;
   if (B == 0) return PA_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_fast_prefill(p, H)) {

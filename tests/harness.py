@@ -12,7 +12,7 @@ import torch
 
 import paged_kv_cache_483_b200 as pa
 import workloads
-from oracle import KVPool, stored_rows
+from oracle import KVPool, stored_rows, stored_rows_fp8
 
 
 def torch_dtype(w):
@@ -21,14 +21,16 @@ def torch_dtype(w):
 
 class GpuRun:
     def __init__(self, w, device="cuda", init="zeros", q8=False):
-        """q8: an int8 pool (packed (block, head) records) fed the same bf16 rows."""
+        """q8: True / "int8" for an int8 pool, "fp8" for an FP8 (E4M3) pool
+        (packed (block, head) records), fed the same bf16 rows."""
         self.w = w
         alloc = torch.zeros if init == "zeros" else torch.empty
         if q8:
             self.records = alloc((w.num_blocks, w.num_kv_heads, pa.PA_INT8_RECORD_BYTES),
                                  dtype=torch.uint8, device=device)
-            self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, "int8",
-                                self.records, None, alloc_order=w.order)
+            self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim,
+                                "fp8" if q8 == "fp8" else "int8", self.records, None,
+                                alloc_order=w.order)
         else:
             dt = torch_dtype(w)
             shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
@@ -82,8 +84,8 @@ class GpuRun:
 
 class OracleRun:
     def __init__(self, w, heads="all", q8=False):
-        """q8: store each row as an int8 pool reads it back (codes x float32
-        scale, float64)."""
+        """q8: True / "int8" / "fp8": store each row as that pool reads it
+        back (value of the code x float32 scale, float64)."""
         self.w = w
         self.q8 = q8
         self.heads = list(range(w.num_kv_heads)) if heads == "all" else list(heads)
@@ -104,8 +106,9 @@ class OracleRun:
                 k, v = self.w.kv_for(op)
                 dt = self.pool.keys.dtype
                 k64, v64 = k.to(torch.float64).numpy(), v.to(torch.float64).numpy()
-                if self.q8:        # the rows an int8 pool reads back
-                    k64, v64 = stored_rows(k64)[2], stored_rows(v64)[2]
+                if self.q8:        # the rows an int8 / FP8 pool reads back
+                    rows = stored_rows_fp8 if self.q8 == "fp8" else stored_rows
+                    k64, v64 = rows(k64)[2], rows(v64)[2]
                 s, c = self.pool.append(op.args[0], op.args[1], k64.astype(dt), v64.astype(dt))
                 self.slots[op.index], self.cows[op.index] = s, c
         return self

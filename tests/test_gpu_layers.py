@@ -11,7 +11,7 @@ import torch
 import paged_kv_cache_483_b200 as pa
 import workloads
 from harness import q64
-from oracle import KVPool, attention_two_pass, stored_rows
+from oracle import KVPool, attention_two_pass, stored_rows, stored_rows_fp8
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +27,8 @@ def _run(w, L, q8):
     NB, bs, Hkv, d = w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim
     if q8:
         kc = torch.zeros((L, NB, Hkv, pa.PA_INT8_RECORD_BYTES), dtype=torch.uint8, device="cuda")
-        pool = pa.Pool.layered(NB, bs, Hkv, d, "int8", L, kc, None, alloc_order=w.order)
+        pool = pa.Pool.layered(NB, bs, Hkv, d, "fp8" if q8 == "fp8" else "int8", L, kc, None,
+                               alloc_order=w.order)
     else:
         kc = torch.zeros((L, NB, bs, Hkv, d), dtype=torch.bfloat16, device="cuda")
         vc = torch.zeros_like(kc)
@@ -62,7 +63,8 @@ def _run(w, L, q8):
                 pool.layer(layer).reshape_and_cache(kl.cuda(), vl.cuda(), d_slots)
                 k64, v64 = kl.double().numpy(), vl.double().numpy()
                 if q8:
-                    k64, v64 = stored_rows(k64)[2], stored_rows(v64)[2]
+                    rows = stored_rows_fp8 if q8 == "fp8" else stored_rows
+                    k64, v64 = rows(k64)[2], rows(v64)[2]
                 got, _ = refs[layer].append(seq, n, k64, v64)
                 assert got == slots
     assert pool.refcounts() == refs[0].refs
@@ -84,7 +86,7 @@ def _run(w, L, q8):
     return pool, n_cow
 
 
-@pytest.mark.parametrize("q8", [False, True])
+@pytest.mark.parametrize("q8", [False, True, "fp8"])
 def test_layers_share_tables_and_copy_on_write(q8):
     w = workloads.ragged256(groups=2, per_group=3, prefix=40, spare_blocks=16)
     pool, n_cow = _run(w, 3, q8)

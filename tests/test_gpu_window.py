@@ -33,7 +33,7 @@ def _oracle_window(o, w, q, window, sinks):
     return res
 
 
-@pytest.mark.parametrize("q8", [False, True])
+@pytest.mark.parametrize("q8", [False, True, "fp8"])
 @pytest.mark.parametrize("part", [0, 64])
 def test_window_decode_parity(q8, part):
     w = workloads.custom_decode("win", LENS, 32, 8, 128, 16, "bf16", seed=31 + part,
@@ -54,7 +54,7 @@ def test_window_decode_parity(q8, part):
     assert g.pool.get_error() == 0
 
 
-@pytest.mark.parametrize("q8", [False, True])
+@pytest.mark.parametrize("q8", [False, True, "fp8"])
 def test_window_covering_everything_equals_decode(q8):
     w = workloads.custom_decode("win2", [5, 300, 1111], 32, 8, 128, 16, "bf16", seed=3,
                                 spare_blocks=4)
@@ -102,7 +102,7 @@ def test_window_unsupported_on_generic_path():
     assert e.value.code == 7
 
 
-@pytest.mark.parametrize("q8", [False, True])
+@pytest.mark.parametrize("q8", [False, True, "fp8"])
 def test_full_decode32_window_sampled(q8):
     # 32 x 8192 with a 1024-token window and 4 sinks: three sequences, two KV heads
     w = workloads.decode32()
@@ -125,7 +125,7 @@ def test_full_decode32_window_sampled(q8):
     assert g.pool.get_error() == 0
 
 
-@pytest.mark.parametrize("q8", [False, True])
+@pytest.mark.parametrize("q8", [False, True, "fp8"])
 @pytest.mark.parametrize("part", [0, 32])
 def test_window_append_equals_two_calls(q8, part):
     # the fused step (write the new token, decode over the window) against
