@@ -31,11 +31,16 @@
 //    together with the online-softmax factor).  P goes in as fp16 hi + lo
 //    parts; l sums the unscaled p_j.
 // FP8 (E4M3) pools use the same record, with E4M3 codes and scales
-// absmax / 448.  The fp8 instance converts codes to fp16 with the E4M3 x2 ->
-// f16 x2 conversion (every E4M3 value is exact in fp16) and runs both
-// products on the fp16 MMA: Q enters as fp16 with a power-of-two scale (exact
-// for bf16 inputs), so S = K Q^T is exact up to fp32 accumulation; E4M3 has
-// NaN codes, so the V bytes of dead tokens are zeroed before conversion.
+// absmax / 448.  The fp8 instance runs both products on the fp16 MMA (every
+// E4M3 value is exact in fp16).  V codes go through the E4M3 x2 -> f16 x2
+// conversion; K codes, to spare that conversion unit, through integer ops:
+// a code b in a 16-bit lane, (b + (b & 0x80)) << 7, is the fp16 pattern of
+// value(b) * 2^-8 (sign to bit 15, exponent and mantissa bits shifted in
+// place, subnormals included), taken as pairs (d0, d2) and (d1, d3) of each
+// 4-byte word, with Q packed to match and the 2^8 folded into the score
+// scale.  Q enters as fp16 with a power-of-two scale (exact for bf16
+// inputs), so S = K Q^T is exact up to fp32 accumulation.  E4M3 has NaN
+// codes, so the V bytes of dead tokens are zeroed before conversion.
 // Token order: row r of a block's S^T tile holds token kPerm[r].  With it a
 // thread's P^T fragment covers tokens 4c .. 4c + 3 (two per register), the
 // four bytes of one 32-bit word of a V d-row, and the K rows a warp reads at
@@ -110,6 +115,15 @@ __device__ __forceinline__ uint32_t e4m3x2_half2(uint32_t pair) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
       static_cast<__nv_fp8x2_storage_t>(pair & 0xFFFFu), __NV_E4M3);
   return uint32_t(h.x) | (uint32_t(h.y) << 16);
+}
+
+// Two E4M3 codes at bits 0-7 and 16-23 of y (other bits zero) as a half2
+// of their values times 2^-8: y * 128 moves each code's magnitude bits to
+// 7-13 (fp16 exponent and mantissa) and its sign to bit 14; adding that bit
+// again carries it up to bit 15.
+__device__ __forceinline__ uint32_t e4m3x2_half2_div256(uint32_t y) {
+  const uint32_t z = y * 128u;
+  return z + (z & 0x40004000u);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
@@ -216,8 +230,8 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
   // int8: Q of head g as int8 hi + lo parts in the B-fragment order of
   // m16n8k32: word kk*2 + h covers d = 32 kk + 16 h + 4c .. + 3.
   // fp8: Q / sq as fp16 B fragments of m16n8k16 over d chunk 2 kk + h, with
-  // MMA k (2c, 2c + 1) = d (4c, 4c + 1) in qh and k (2c + 8, 2c + 9) =
-  // d (4c + 2, 4c + 3) in ql, the order in which the K words unpack.
+  // MMA k (2c, 2c + 1) = d (4c, 4c + 2) in qh and k (2c + 8, 2c + 9) =
+  // d (4c + 1, 4c + 3) in ql, the order in which the K words unpack.
   uint32_t qh[4][2], ql[4][2];
   float qs0, qs1;   // sq * scale_log2 of heads 2c and 2c + 1 (S^T columns)
   {
@@ -250,8 +264,8 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
       for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          qh[kk][h] = pack_half2(x[kk][h][0] * inv, x[kk][h][1] * inv);
-          ql[kk][h] = pack_half2(x[kk][h][2] * inv, x[kk][h][3] * inv);
+          qh[kk][h] = pack_half2(x[kk][h][0] * inv, x[kk][h][2] * inv);
+          ql[kk][h] = pack_half2(x[kk][h][1] * inv, x[kk][h][3] * inv);
         }
     } else {
     sq = amax > 0.f ? amax / 127.f : 1.f;
@@ -273,8 +287,10 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
         ql[kk][h] = lw;
       }
     }
-    qs0 = __shfl_sync(0xffffffffu, sq, 8 * c) * scale_log2;
-    qs1 = __shfl_sync(0xffffffffu, sq, 8 * c + 4) * scale_log2;
+    // fp8: K enters the MMA as value * 2^-8
+    const float ks = kFp8 ? 256.f * scale_log2 : scale_log2;
+    qs0 = __shfl_sync(0xffffffffu, sq, 8 * c) * ks;
+    qs1 = __shfl_sync(0xffffffffu, sq, 8 * c + 4) * ks;
   }
   const int tokA = kPerm[g], tokB = kPerm[g + 8];       // tokens of S^T rows g, g + 8
   const uint32_t rowA = tokA * 128, rowB = tokB * 128;
@@ -334,12 +350,15 @@ __global__ void __launch_bounds__(kQ8Threads, 3) decode_q8_kernel(
       for (int x = 0; x < 2; ++x) {
         if constexpr (kFp8) {
           // chunk 2kk: rows A, B in a[x][0], a[x][1]; chunk 2kk + 1: a[x][2], a[x][3]
-          mma_f16_16816(fs[x], e4m3x2_half2(a[x][0]), e4m3x2_half2(a[x][1]),
-                        e4m3x2_half2(a[x][0] >> 16), e4m3x2_half2(a[x][1] >> 16), qh[kk][0],
-                        ql[kk][0]);
-          mma_f16_16816(fs[x], e4m3x2_half2(a[x][2]), e4m3x2_half2(a[x][3]),
-                        e4m3x2_half2(a[x][2] >> 16), e4m3x2_half2(a[x][3] >> 16), qh[kk][1],
-                        ql[kk][1]);
+          // even bytes (d0, d2) -> MMA k (2c, 2c + 1); odd (d1, d3) -> (2c + 8, 2c + 9)
+          mma_f16_16816(fs[x], e4m3x2_half2_div256(a[x][0] & 0x00FF00FFu),
+                        e4m3x2_half2_div256(a[x][1] & 0x00FF00FFu),
+                        e4m3x2_half2_div256((a[x][0] >> 8) & 0x00FF00FFu),
+                        e4m3x2_half2_div256((a[x][1] >> 8) & 0x00FF00FFu), qh[kk][0], ql[kk][0]);
+          mma_f16_16816(fs[x], e4m3x2_half2_div256(a[x][2] & 0x00FF00FFu),
+                        e4m3x2_half2_div256(a[x][3] & 0x00FF00FFu),
+                        e4m3x2_half2_div256((a[x][2] >> 8) & 0x00FF00FFu),
+                        e4m3x2_half2_div256((a[x][3] >> 8) & 0x00FF00FFu), qh[kk][1], ql[kk][1]);
         } else {
           mma_s8_16832(ih[x], a[x][0], a[x][1], a[x][2], a[x][3], qh[kk][0], qh[kk][1]);
           mma_s8_16832(il[x], a[x][0], a[x][1], a[x][2], a[x][3], ql[kk][0], ql[kk][1]);
