@@ -19,7 +19,7 @@ def torch_dtype(w):
     return torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
 
-class GpuRun:
+class DeviceRun:
     def __init__(self, w, device="cuda", init="zeros", q8=False):
         """q8: True / "int8" for an int8 pool, "fp8" for an FP8 (E4M3) pool
         (packed (block, head) records), fed the same bf16 rows."""

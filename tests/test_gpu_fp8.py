@@ -11,7 +11,7 @@ import torch
 
 import paged_kv_cache_483_b200 as pa
 import workloads
-from harness import GpuRun, OracleRun, q64
+from harness import DeviceRun, OracleRun, q64
 from oracle import e4m3_values, stored_rows_fp8
 from test_gpu_q8 import _pool_rows, _worst
 
@@ -32,7 +32,7 @@ def _codes(g, slot):
 
 def test_fp8_append_codes_and_scales_bit_exact():
     w = _small([1, 15, 16, 17, 100, 300], 32, 8, seed=3)
-    g = GpuRun(w, q8="fp8").apply(w.setup)
+    g = DeviceRun(w, q8="fp8").apply(w.setup)
     torch.cuda.synchronize()
     n = 0
     for op in w.setup:
@@ -54,7 +54,7 @@ def test_fp8_append_special_rows():
     # a zero row (scale 1, codes 0) and a row whose absmax is 448 (scale 1)
     # holding exact E4M3 ties and subnormals
     w = _small([2], 8, 8, seed=4)
-    g = GpuRun(w, q8="fp8")
+    g = DeviceRun(w, q8="fp8")
     g.pool.create(0)
     k = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
     vals = [448.0, 1.0625, 432.0, 400.0, 2.0 ** -10, 3 * 2.0 ** -10, -1.0625, -(2.0 ** -11),
@@ -79,7 +79,7 @@ LENS = [1, 15, 16, 17, 33, 100, 255, 256, 513, 1000, 0, 2]
 @pytest.mark.parametrize("part", [0, 16, 256])
 def test_fp8_decode_parity(H, Hkv, part):
     w = _small(LENS, H, Hkv, seed=H * 7 + Hkv + part)
-    g = GpuRun(w, q8="fp8").apply(w.setup)
+    g = DeviceRun(w, q8="fp8").apply(w.setup)
     assert g.pool.decode_path(H) == 1
     o = OracleRun(w, q8="fp8").apply(w.setup)
     worst, out = _worst(g, o, w, part)
@@ -92,7 +92,7 @@ def test_fp8_stale_slots_hold_nan_codes():
     # never-written slots hold the E4M3 NaN code (0x7F) and NaN / Inf scales;
     # dead tokens must add exactly nothing
     w = _small([3, 17, 31, 64], 32, 8, seed=6)
-    g = GpuRun(w, q8="fp8", init="empty")
+    g = DeviceRun(w, q8="fp8", init="empty")
     g.records.fill_(0x7F)
     sc = g.records[:, :, 4096:].view(torch.float32)
     sc[:, :, :16].fill_(float("nan"))
@@ -106,7 +106,7 @@ def test_fp8_stale_slots_hold_nan_codes():
 
 def test_fp8_decode_with_sharing_and_copy_on_write():
     w = workloads.ragged256(groups=3, per_group=4, prefix=40, spare_blocks=16)
-    g = GpuRun(w, q8="fp8").apply(w.setup + w.step)
+    g = DeviceRun(w, q8="fp8").apply(w.setup + w.step)
     o = OracleRun(w, q8="fp8").apply(w.setup + w.step)
     assert any(o.cows.values())
     worst, _ = _worst(g, o, w)
@@ -119,8 +119,8 @@ def test_fp8_within_grid_bound_of_bf16_decode():
     # every stored element is within 2^-4 of its value (relative), so the
     # decode stays within that of the unquantised one
     w = _small([64, 300, 1000, 2048], 32, 8, seed=7)
-    out_f8 = GpuRun(w, q8="fp8").apply(w.setup).decode()
-    out_bf = GpuRun(w).apply(w.setup).decode()
+    out_f8 = DeviceRun(w, q8="fp8").apply(w.setup).decode()
+    out_bf = DeviceRun(w).apply(w.setup).decode()
     for i in range(4):
         rel = np.linalg.norm(out_f8[i] - out_bf[i]) / np.linalg.norm(out_bf[i])
         assert rel < 2.0 ** -4, rel
@@ -132,7 +132,7 @@ def test_fp8_two_calls_equal_decode_append():
                                 spare_blocks=8, split_last=1)
     outs = []
     for fused in (True, False):
-        g = GpuRun(w, q8="fp8").apply(w.setup)
+        g = DeviceRun(w, q8="fp8").apply(w.setup)
         seqs = [op.args[0] for op in w.step]
         slots, cow = g.pool.plan_append(seqs, [1] * len(seqs))
         assert not cow
@@ -160,7 +160,7 @@ def test_fp8_two_calls_equal_decode_append():
 
 def test_fp8_device_errors_and_unsupported_calls():
     w = _small([40, 70], 32, 8, seed=10)
-    g = GpuRun(w, q8="fp8").apply(w.setup)
+    g = DeviceRun(w, q8="fp8").apply(w.setup)
     tables, lens, _, _ = g.tables()
     q = w.queries()[:, 0].contiguous().cuda()
     bad = tables.clone()
@@ -185,7 +185,7 @@ def test_fp8_device_errors_and_unsupported_calls():
 
 def test_full_decode32_fp8_sampled():
     w = workloads.decode32()
-    g = GpuRun(w, q8="fp8").apply(w.setup)
+    g = DeviceRun(w, q8="fp8").apply(w.setup)
     o = OracleRun(w, heads=[2, 7], q8="fp8").apply(w.setup)
     out = g.decode()
     q = q64(w)

@@ -13,7 +13,7 @@ import torch
 
 import paged_kv_cache_483_b200 as pa
 import workloads
-from harness import GpuRun, OracleRun, q64
+from harness import DeviceRun, OracleRun, q64
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +34,7 @@ def _check_decode(g, o, w, tol, partition_tokens=0):
 
 def test_tiny_trace_fp32():
     w = workloads.tiny()
-    g = GpuRun(w).apply(w.setup)
+    g = DeviceRun(w).apply(w.setup)
     o = OracleRun(w).apply(w.setup)
     assert g.slots == o.slots                                 # bit-exact plan
     assert g.pool.refcounts() == o.pool.refs
@@ -59,7 +59,7 @@ LENS = [1, 15, 16, 17, 33, 100, 255, 256, 513, 1000, 0, 2]
 @pytest.mark.parametrize("part", [0, 16, 64, 256])
 def test_decode_fast_parity(H, Hkv, part):
     w = _small(LENS, H, Hkv, seed=H * 7 + Hkv + part)
-    g = GpuRun(w).apply(w.setup)
+    g = DeviceRun(w).apply(w.setup)
     assert g.pool.decode_path(H) == 1
     o = OracleRun(w).apply(w.setup)
     _check_decode(g, o, w, TOL_DECODE, part)
@@ -69,7 +69,7 @@ def test_decode_fast_parity(H, Hkv, part):
 def test_decode_uninitialised_pool_is_safe():
     # stale slots past a sequence end must not leak into the result
     w = _small([3, 17, 31], 32, 8, seed=5)
-    g = GpuRun(w, init="empty")
+    g = DeviceRun(w, init="empty")
     g.k_cache.fill_(float("nan"))
     g.v_cache.fill_(float("inf"))
     g.apply(w.setup)
@@ -82,27 +82,27 @@ def test_decode_is_invariant_under_block_permutation():
     outs = []
     for k in range(3):
         wk = dataclasses.replace(w, order=workloads.permutation(w.num_blocks, 100 + k))
-        outs.append(GpuRun(wk).apply(wk.setup).decode())
+        outs.append(DeviceRun(wk).apply(wk.setup).decode())
     assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
 
 
 def test_generic_path_bf16_head_dim_64():
     w = _small([5, 70, 129], 8, 2, d=64, seed=3)
-    g = GpuRun(w).apply(w.setup)
+    g = DeviceRun(w).apply(w.setup)
     assert g.pool.decode_path(8) == 0
     _check_decode(g, OracleRun(w).apply(w.setup), w, TOL_DECODE)
 
 
 def test_generic_path_fp32_gqa():
     w = _small([9, 40, 64], 8, 2, d=32, bs=8, dtype="f32", seed=4)
-    g = GpuRun(w).apply(w.setup)
+    g = DeviceRun(w).apply(w.setup)
     _check_decode(g, OracleRun(w).apply(w.setup), w, TOL_F32)
 
 
 def test_append_with_sharing_is_bit_exact():
     # groups sharing prefixes, private tails, a copy-on-write in the step
     w = workloads.ragged256(groups=3, per_group=4, prefix=40, spare_blocks=8)
-    g = GpuRun(w).apply(w.setup + w.step)
+    g = DeviceRun(w).apply(w.setup + w.step)
     o = OracleRun(w).apply(w.setup + w.step)
     assert g.slots == o.slots
     assert any(o.cows.values())
@@ -119,7 +119,7 @@ def test_append_with_sharing_is_bit_exact():
 
 def test_reshape_and_cache_and_cow_entry_points():
     w = workloads.custom_decode("rc", [40], 8, 8, 128, 16, "bf16", 9, spare_blocks=4)
-    g = GpuRun(w)
+    g = DeviceRun(w)
     T = 20
     key = torch.randn(T, 8, 128, device="cuda").to(torch.bfloat16)
     val = torch.randn(T, 8, 128, device="cuda").to(torch.bfloat16)
@@ -138,7 +138,7 @@ def test_reshape_and_cache_and_cow_entry_points():
 
 def test_device_bounds_errors_zero_rows():
     w = _small([40, 40], 32, 8, seed=21)
-    g = GpuRun(w).apply(w.setup)
+    g = DeviceRun(w).apply(w.setup)
     tables, lens, _, _ = g.tables()
     q = w.queries()[:, 0].contiguous().cuda()
     bad = tables.clone()
@@ -166,7 +166,7 @@ def test_prefill_parity_small(batch, cached, chunk, H, Hkv, splits):
     # over its keys (up to 4 parts, some of them empty), splits=1 never does
     w = workloads.prefill(seed=batch * 100 + cached + chunk + H, batch=batch, cached=cached,
                           chunk=chunk, num_heads=H, num_kv_heads=Hkv)
-    g = GpuRun(w).apply(w.setup + w.step)
+    g = DeviceRun(w).apply(w.setup + w.step)
     assert g.pool.prefill_path(H) == 1
     o = OracleRun(w).apply(w.setup + w.step)
     out = g.prefill(max_kv_splits=splits)
@@ -182,7 +182,7 @@ def test_prefill_parity_small(batch, cached, chunk, H, Hkv, splits):
 
 # ---------------------------------------------------------------- full sizes
 def _full(w, kv_heads, sample_seqs, decode=True, partition_tokens=0, check_slots=True):
-    g = GpuRun(w).apply(w.setup + w.step)
+    g = DeviceRun(w).apply(w.setup + w.step)
     o = OracleRun(w, heads=kv_heads).apply(w.setup + w.step)
     if check_slots:
         assert g.slots == o.slots
@@ -246,7 +246,7 @@ def test_full_prefill_sampled():
 @pytest.mark.parametrize("splits", [0, 1])
 def test_prefill_device_errors_zero_rows(splits):
     w = workloads.prefill(seed=41, batch=2, cached=100, chunk=70)
-    g = GpuRun(w).apply(w.setup + w.step)
+    g = DeviceRun(w).apply(w.setup + w.step)
     tables, lens, _, _ = g.tables()
     q = w.queries().contiguous().cuda()
     assert g.pool.prefill_path(32) == 1
@@ -271,7 +271,7 @@ def test_prefill_tail_split(splits):
     # full waves on 148 SMs and a tail of 24 that is split over its keys; a
     # second call must give the same bits (the merge tickets reset themselves)
     w = workloads.prefill(seed=47, batch=10, cached=500, chunk=256)
-    g = GpuRun(w).apply(w.setup + w.step)
+    g = DeviceRun(w).apply(w.setup + w.step)
     o = OracleRun(w).apply(w.setup + w.step)
     out = g.prefill(max_kv_splits=splits)
     again = g.prefill(max_kv_splits=splits)
@@ -289,7 +289,7 @@ def test_prefill_tail_split(splits):
 
 def test_prefill_split_arg_checked():
     w = workloads.prefill(seed=48, batch=1, cached=20, chunk=30)
-    g = GpuRun(w).apply(w.setup + w.step)
+    g = DeviceRun(w).apply(w.setup + w.step)
     with pytest.raises(pa.PAError):
         g.prefill(max_kv_splits=-1)
 
@@ -297,7 +297,7 @@ def test_prefill_split_arg_checked():
 def test_prefill_uninitialised_pool_is_safe():
     # stale slots past the sequence end (NaN / Inf bit patterns) must not leak
     w = workloads.prefill(seed=43, batch=2, cached=37, chunk=60)
-    g = GpuRun(w, init="empty")
+    g = DeviceRun(w, init="empty")
     g.k_cache.fill_(float("nan"))
     g.v_cache.fill_(float("inf"))
     g.apply(w.setup + w.step)
@@ -315,7 +315,7 @@ def test_prefill_uninitialised_pool_is_safe():
 def _fused_step(w, fused=True, init="zeros"):
     """Setup through the library, then the step's one-token appends either
     fused into the decode or as reshape_and_cache + decode."""
-    g = GpuRun(w, init=init).apply(w.setup)
+    g = DeviceRun(w, init=init).apply(w.setup)
     seqs = [op.args[0] for op in w.step]
     slots, cow = g.pool.plan_append(seqs, [1] * len(seqs))
     if cow:

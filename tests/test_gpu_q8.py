@@ -10,7 +10,7 @@ import torch
 
 import paged_kv_cache_483_b200 as pa
 import workloads
-from harness import GpuRun, OracleRun, q64
+from harness import DeviceRun, OracleRun, q64
 from oracle import stored_rows
 
 pytestmark = pytest.mark.gpu
@@ -65,7 +65,7 @@ def _pool_rows(g, slot):
 
 def test_q8_append_codes_and_scales_bit_exact():
     w = _small([1, 15, 16, 17, 100, 300], 32, 8, seed=3)
-    g = GpuRun(w, q8=True).apply(w.setup)
+    g = DeviceRun(w, q8=True).apply(w.setup)
     torch.cuda.synchronize()
     want = _expect_rows(g, w, w.setup)
     assert len(want) == sum([1, 15, 16, 17, 100, 300])
@@ -80,7 +80,7 @@ def test_q8_append_special_rows():
     # a zero row (scale 1, codes 0), exact half-way ties (round half to even)
     # and a row whose absmax is negative
     w = _small([3], 8, 8, seed=4)
-    g = GpuRun(w, q8=True)
+    g = DeviceRun(w, q8=True)
     g.pool.create(0)
     k = torch.zeros(3, 8, 128, dtype=torch.bfloat16)
     k[1, :, 0] = 127.0
@@ -107,7 +107,7 @@ LENS = [1, 15, 16, 17, 33, 100, 255, 256, 513, 1000, 0, 2]
 @pytest.mark.parametrize("part", [0, 16, 64, 256])
 def test_q8_decode_parity(H, Hkv, part):
     w = _small(LENS, H, Hkv, seed=H * 5 + Hkv + part)
-    g = GpuRun(w, q8=True).apply(w.setup)
+    g = DeviceRun(w, q8=True).apply(w.setup)
     assert g.pool.decode_path(H) == 1
     o = OracleRun(w, q8=True).apply(w.setup)
     worst, out = _worst(g, o, w, part)
@@ -120,7 +120,7 @@ def test_q8_decode_with_sharing_and_copy_on_write():
     # shared prefixes, a released root, one-token appends that copy shared
     # partial tails (codes and scales must both move)
     w = workloads.ragged256(groups=3, per_group=4, prefix=40, spare_blocks=16)
-    g = GpuRun(w, q8=True).apply(w.setup + w.step)
+    g = DeviceRun(w, q8=True).apply(w.setup + w.step)
     o = OracleRun(w, q8=True).apply(w.setup + w.step)
     assert any(o.cows.values())
     worst, _ = _worst(g, o, w)
@@ -132,7 +132,7 @@ def test_q8_decode_with_sharing_and_copy_on_write():
 def test_q8_stale_slots_do_not_leak():
     # never-written slots hold arbitrary codes and NaN / Inf scales
     w = _small([3, 17, 31, 64], 32, 8, seed=6)
-    g = GpuRun(w, q8=True, init="empty")
+    g = DeviceRun(w, q8=True, init="empty")
     g.records.random_(0, 256)
     sc = g.records[:, :, 4096:].view(torch.float32)         # every scale slot
     sc[:, :, :16].fill_(float("nan"))
@@ -145,8 +145,8 @@ def test_q8_stale_slots_do_not_leak():
 
 def test_q8_within_page_bound_of_bf16_decode():
     w = _small([64, 300, 1000, 2048], 32, 8, seed=7)
-    out_q8 = GpuRun(w, q8=True).apply(w.setup).decode()
-    out_bf = GpuRun(w).apply(w.setup).decode()
+    out_q8 = DeviceRun(w, q8=True).apply(w.setup).decode()
+    out_bf = DeviceRun(w).apply(w.setup).decode()
     for i in range(4):
         rel = np.linalg.norm(out_q8[i] - out_bf[i]) / np.linalg.norm(out_bf[i])
         assert rel < 0.03, rel
@@ -158,7 +158,7 @@ def test_q8_two_calls_equal_decode_append():
                                 spare_blocks=8, split_last=1)
     outs = []
     for fused in (True, False):
-        g = GpuRun(w, q8=True).apply(w.setup)
+        g = DeviceRun(w, q8=True).apply(w.setup)
         seqs = [op.args[0] for op in w.step]
         slots, cow = g.pool.plan_append(seqs, [1] * len(seqs))
         assert not cow
@@ -186,7 +186,7 @@ def test_q8_two_calls_equal_decode_append():
 
 def test_q8_device_errors_zero_rows():
     w = _small([40, 70], 32, 8, seed=10)
-    g = GpuRun(w, q8=True).apply(w.setup)
+    g = DeviceRun(w, q8=True).apply(w.setup)
     tables, lens, _, _ = g.tables()
     q = w.queries()[:, 0].contiguous().cuda()
     bad = tables.clone()
@@ -204,7 +204,7 @@ def test_q8_device_errors_zero_rows():
 
 def test_q8_unsupported_calls():
     w = _small([20], 128, 8, seed=11)                     # group 16 > 8
-    g = GpuRun(w, q8=True).apply(w.setup)
+    g = DeviceRun(w, q8=True).apply(w.setup)
     tables, lens, _, _ = g.tables()
     q = torch.zeros(1, 128, 128, dtype=torch.bfloat16, device="cuda")
     assert g.pool.decode_path(128) == 0
@@ -224,7 +224,7 @@ def test_full_decode32_int8_sampled():
     # the bench configuration (32 x 8192, GQA 32/8) over an int8 pool; the
     # oracle stores two KV heads and checks three sequences against them
     w = workloads.decode32()
-    g = GpuRun(w, q8=True).apply(w.setup)
+    g = DeviceRun(w, q8=True).apply(w.setup)
     o = OracleRun(w, heads=[0, 5], q8=True).apply(w.setup)
     out = g.decode()
     q = q64(w)

@@ -7,7 +7,7 @@ import torch
 
 import paged_kv_cache_483_b200 as pa
 import workloads
-from harness import GpuRun, OracleRun, q64
+from harness import DeviceRun, OracleRun, q64
 from oracle import attention_window
 
 pytestmark = pytest.mark.gpu
@@ -38,7 +38,7 @@ def _oracle_window(o, w, q, window, sinks):
 def test_window_decode_parity(q8, part):
     w = workloads.custom_decode("win", LENS, 32, 8, 128, 16, "bf16", seed=31 + part,
                                 spare_blocks=4)
-    g = GpuRun(w, q8=q8).apply(w.setup)
+    g = DeviceRun(w, q8=q8).apply(w.setup)
     o = OracleRun(w, q8=q8).apply(w.setup)
     tables, lens, _, _ = g.tables()
     qd = w.queries()[:, 0].contiguous().cuda()
@@ -58,7 +58,7 @@ def test_window_decode_parity(q8, part):
 def test_window_covering_everything_equals_decode(q8):
     w = workloads.custom_decode("win2", [5, 300, 1111], 32, 8, 128, 16, "bf16", seed=3,
                                 spare_blocks=4)
-    g = GpuRun(w, q8=q8).apply(w.setup)
+    g = DeviceRun(w, q8=q8).apply(w.setup)
     tables, lens, _, _ = g.tables()
     qd = w.queries()[:, 0].contiguous().cuda()
     full = g.pool.decode(qd, tables, lens).cpu().numpy()
@@ -70,7 +70,7 @@ def test_window_covering_everything_equals_decode(q8):
 def test_window_stale_slots_and_errors():
     w = workloads.custom_decode("win3", [7, 70, 400], 32, 8, 128, 16, "bf16", seed=5,
                                 spare_blocks=4)
-    g = GpuRun(w, init="empty")
+    g = DeviceRun(w, init="empty")
     g.k_cache.fill_(float("nan"))
     g.v_cache.fill_(float("inf"))
     g.apply(w.setup)
@@ -94,7 +94,7 @@ def test_window_stale_slots_and_errors():
 
 def test_window_unsupported_on_generic_path():
     w = workloads.custom_decode("win4", [9, 40], 8, 2, 32, 8, "f32", seed=4, spare_blocks=4)
-    g = GpuRun(w).apply(w.setup)
+    g = DeviceRun(w).apply(w.setup)
     tables, lens, _, _ = g.tables()
     q = torch.zeros(2, 8, 32, dtype=torch.float32, device="cuda")
     with pytest.raises(pa.PAError) as e:
@@ -106,7 +106,7 @@ def test_window_unsupported_on_generic_path():
 def test_full_decode32_window_sampled(q8):
     # 32 x 8192 with a 1024-token window and 4 sinks: three sequences, two KV heads
     w = workloads.decode32()
-    g = GpuRun(w, q8=q8).apply(w.setup)
+    g = DeviceRun(w, q8=q8).apply(w.setup)
     o = OracleRun(w, heads=[1, 6], q8=q8).apply(w.setup)
     tables, lens, _, _ = g.tables()
     qd = w.queries()[:, 0].contiguous().cuda()
@@ -136,7 +136,7 @@ def test_window_append_equals_two_calls(q8, part):
     windows = [(1, 0), (17, 4), (100, 16), (2000, 0)]
     outs = {}
     for fused in (True, False):
-        g = GpuRun(w, q8=q8).apply(w.setup)
+        g = DeviceRun(w, q8=q8).apply(w.setup)
         seqs = [op.args[0] for op in w.step]
         slots, cow = g.pool.plan_append(seqs, [1] * len(seqs))
         assert not cow
@@ -168,7 +168,7 @@ def test_window_append_equals_two_calls(q8, part):
 def test_window_append_argument_errors():
     w = workloads.custom_decode("winf2", [5, 40], 32, 8, 128, 16, "bf16", seed=2,
                                 spare_blocks=4, split_last=1)
-    g = GpuRun(w).apply(w.setup)
+    g = DeviceRun(w).apply(w.setup)
     seqs = [op.args[0] for op in w.step]
     slots, _ = g.pool.plan_append(seqs, [1] * len(seqs))
     ks, vs = zip(*[w.kv_for(op) for op in w.step])

@@ -17,7 +17,7 @@ import torch
 
 import paged_kv_cache_483_b200 as pa
 import workloads
-from harness import GpuRun
+from harness import DeviceRun
 
 pytestmark = pytest.mark.gpu
 
@@ -36,7 +36,7 @@ def _call(L, g, q, tables, lens, part, out):
 def test_static_scratch_matches_workspace_decode_twice():
     w = workloads.custom_decode("noalloc", [700, 1234, 40, 4097, 1, 0, 333], 64, 8, 128, 16,
                                 "bf16", seed=99, spare_blocks=4)
-    g = GpuRun(w).apply(w.setup)
+    g = DeviceRun(w).apply(w.setup)
     tables, lens, _, _ = g.tables()
     q = w.queries()[:, 0].contiguous().cuda()
     part = 256     # several partitions per sequence, so the scratch is used
@@ -56,7 +56,7 @@ def test_static_scratch_matches_workspace_decode_twice():
 def test_static_scratch_refuses_oversized_requests():
     w = workloads.custom_decode("noalloc_big", [64] * 8, 64, 8, 128, 16, "bf16", seed=5,
                                 spare_blocks=4)
-    g = GpuRun(w).apply(w.setup)
+    g = DeviceRun(w).apply(w.setup)
     q = w.queries()[:, 0].contiguous().cuda()
     wide = torch.zeros((8, 4096), dtype=torch.int32, device="cuda")
     lens = torch.full((8,), 64, dtype=torch.int32, device="cuda")
