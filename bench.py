@@ -369,7 +369,7 @@ def run_ours(args, dist):
     if is_prefill:
         flops = prefill_flops(w, lens)
         value = dist.world * flops / (ms_step_max * 1e-3) / 1e12
-        metric = "chunked prefill attention TFLOP/s (causal pairs), 8 x 512 over 4608, GQA 32/8"
+        metric = metric_name(w, q8, win, sinks)
         unit = "TFLOP/s"
         achieved = flops / (kern_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": bf16,
@@ -383,11 +383,7 @@ def run_ours(args, dist):
     else:
         kv = decode_bytes(w, lens, q8, win, sinks)
         value = dist.world * kv / (ms_step_max * 1e-3) / 1e9
-        metric = (f"decode {q8}-KV HBM GB/s (codes + scales read) and seqs/s at 8K ctx, GQA 32/8"
-                  if q8 else
-                  "decode KV HBM GB/s (fraction of B200 peak) and seqs/s at 8K ctx, GQA 32/8")
-        if win:
-            metric += f", window {win} + {sinks} sinks (visible keys only)"
+        metric = metric_name(w, q8, win, sinks)
         unit = "GB/s"
         achieved = kv / (kern_ms * 1e-3) / 1e9
         kname = (f"decode_q8_kernel<{'true' if q8 == 'fp8' else 'false'}>" if q8 else
@@ -425,8 +421,8 @@ def run_ours(args, dist):
         "e2e": e2e,
         "clocks": clk.summary(),
     }
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and not q8 and not win:
-        res["cpu_baseline"] = cpu_baseline(w, args, S.out.float().cpu().numpy())
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, args, S.out.float().cpu().numpy(), q8)
     pool.close()
     return res
 
@@ -521,16 +517,22 @@ class OracleSampler:
     """The float64 oracle (paged gather, then two-pass softmax) run on
     (sequence, KV head) groups of a workload.  The oracle pool is built once
     (untimed, data stored as float32 holding the bf16 values exactly); only the
-    attention calls are timed."""
+    gather and attention calls are timed.  ``q8`` ("int8" / "fp8"): the
+    oracle pool holds, in float64, the value that pool type stores for each
+    appended row (quantised once, untimed); ``window`` / ``sinks``: the
+    windowed decode over the visible keys only."""
 
-    def __init__(self, w):
+    def __init__(self, w, q8=False, window=0, sinks=0):
         import torch
         from oracle import KVPool
         self.w = w
+        self.q8, self.window, self.sinks = q8, window, sinks
         self.G = w.num_heads // w.num_kv_heads
         self.q = w.queries().to(torch.float64).numpy()
+        from oracle import stored_rows, stored_rows_fp8
+        rows = stored_rows_fp8 if q8 == "fp8" else stored_rows
         p = KVPool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.order,
-                   store_heads="all", dtype=np.float32)
+                   store_heads="all", dtype=np.float64 if q8 else np.float32)
         for op in w.setup + w.step:
             if op.kind == "create":
                 p.create(op.args[0])
@@ -540,7 +542,11 @@ class OracleSampler:
                 p.release(op.args[0])
             else:
                 k, v = w.kv_for(op)
-                p.append(op.args[0], op.args[1], k.float().numpy(), v.float().numpy())
+                if q8:
+                    kr, vr = rows(k.double().numpy())[2], rows(v.double().numpy())[2]
+                else:
+                    kr, vr = k.float().numpy(), v.float().numpy()
+                p.append(op.args[0], op.args[1], kr, vr)
         self.pool = p
         self.next = 0
 
@@ -548,8 +554,10 @@ class OracleSampler:
         """Decode (or prefill) whole sequences -- every head -- until the
         budget is spent; returns (bytes or flops, seconds, sequences).  The
         outputs of the first ``keep`` sequences are kept in ``self.outs``."""
-        from oracle import paged_attention
+        from oracle import attention_window, paged_attention
         w, p = self.w, self.pool
+        tok_bytes = 2 * w.head_dim + 8 if self.q8 else \
+            w.head_dim * 2 * (2 if w.dtype == "bf16" else 4)
         work, spent, done = 0, 0.0, 0
         self.outs = {}
         while spent < budget_s and (max_units is None or done < max_units):
@@ -557,7 +565,11 @@ class OracleSampler:
             self.next += 1
             seq = w.decode_seqs[si]
             t0 = time.perf_counter()
-            o = paged_attention(p, seq, self.q[si])    # gather + two-pass softmax
+            if self.window:
+                k, v = p.gather(seq)
+                o = attention_window(self.q[si], k, v, self.window, self.sinks)
+            else:
+                o = paged_attention(p, seq, self.q[si])    # gather + two-pass softmax
             spent += time.perf_counter() - t0
             if len(self.outs) < keep:
                 self.outs[si] = o
@@ -566,7 +578,8 @@ class OracleSampler:
                 qn = w.q_tokens
                 work += 4 * w.head_dim * w.num_heads * (qn * (L - qn) + qn * (qn + 1) // 2)
             else:
-                work += L * w.num_kv_heads * w.head_dim * 2 * (2 if w.dtype == "bf16" else 4)
+                vis = min(L, self.window + self.sinks) if self.window else L
+                work += vis * w.num_kv_heads * tok_bytes
             done += 1
         return work, spent, done
 
@@ -579,11 +592,18 @@ def blas_threads():
         return None
 
 
-def cpu_baseline(w, args, gpu_out=None):
-    sampler = OracleSampler(w)
+def oracle_desc(q8, window, sinks):
+    return ("oracle paged gather + float64 two-pass softmax"
+            + (f" over the window {window} + {sinks} sinks" if window else "")
+            + (f", pool holding the rows an {q8} pool stores (quantised once, untimed)"
+               if q8 else ""))
+
+
+def cpu_baseline(w, args, gpu_out=None, q8=False):
+    sampler = OracleSampler(w, q8, args.window, args.sinks)
     work, spent, done = sampler.run(args.cpu_budget, keep=2 if gpu_out is not None else 0)
-    desc = (f"{done} of the {len(w.decode_seqs)} sequences of {w.name} (all heads): oracle "
-            f"paged gather + float64 two-pass softmax")
+    desc = (f"{done} of the {len(w.decode_seqs)} sequences of {w.name} (all heads): "
+            + oracle_desc(q8, args.window, args.sinks))
     if w.q_tokens > 1:
         val, unit = work / spent / 1e12, "TFLOP/s"
     else:
@@ -602,13 +622,27 @@ def cpu_baseline(w, args, gpu_out=None):
     return res
 
 
+def metric_name(w, q8=False, window=0, sinks=0):
+    """The metric both arms report for a workload and pool type."""
+    if w.q_tokens > 1:
+        return "chunked prefill attention TFLOP/s (causal pairs), 8 x 512 over 4608, GQA 32/8"
+    m = (f"decode {q8}-KV HBM GB/s (codes + scales read) and seqs/s at 8K ctx, GQA 32/8" if q8
+         else "decode KV HBM GB/s (fraction of B200 peak) and seqs/s at 8K ctx, GQA 32/8")
+    if window:
+        m += f", window {window} + {sinks} sinks (visible keys only)"
+    return m
+
+
 def run_reference(args, dist):
     """The float64 oracle as the reference arm, on this host's cores."""
     if dist.rank != 0:
         return None
     builder = workloads.ALL[args.config]
     w = builder() if args.seed is None else builder(seed=args.seed)
-    sampler = OracleSampler(w)
+    q8 = args.kv if args.kv in ("int8", "fp8") else False
+    if (q8 or args.window) and w.q_tokens > 1:
+        raise SystemExit("--kv int8/fp8 and --window apply to the decode workloads")
+    sampler = OracleSampler(w, q8, args.window, args.sinks)
     # each step: one bounded sample (whole groups) so the run stays ~2-3 minutes
     per_step = max(0.005, 120.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
@@ -619,20 +653,19 @@ def run_reference(args, dist):
         work, spent, groups, steps = work + wk, spent + sp, groups + n, steps + 1
         if spent > 150:
             break
-    desc = (f"{groups} sequences (all heads) of {w.name} over {steps} steps: oracle paged "
-            f"gather + float64 two-pass softmax")
+    desc = (f"{groups} sequences (all heads) of {w.name} over {steps} steps: "
+            + oracle_desc(q8, args.window, args.sinks))
+    metric = metric_name(w, q8, args.window, args.sinks)
     if w.q_tokens > 1:
-        val, unit, metric = work / spent / 1e12, "TFLOP/s", \
-            "chunked prefill attention TFLOP/s (causal pairs), 8 x 512 over 4608, GQA 32/8"
+        val, unit = work / spent / 1e12, "TFLOP/s"
     else:
-        val, unit, metric = work / spent / 1e9, "GB/s", \
-            "decode KV HBM GB/s (fraction of B200 peak) and seqs/s at 8K ctx, GQA 32/8"
+        val, unit = work / spent / 1e9, "GB/s"
     ms = spent / max(1, steps) * 1e3
     return {"impl": "reference", "metric": metric, "value": round(val, 6), "unit": unit,
             "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), bf16-rounded)",
-            "config": {"workload": w.name, "sample": desc},
+            "config": {**config_of(w, args, dist), "sample": desc},
             "cpu_baseline": {"value": round(val, 6), "unit": unit, "cores": oracle_threads(),
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": round(val, 6), "unit": unit, "h2d_bytes_per_step": 0,
