@@ -53,6 +53,40 @@ def test_create_rejects_bad_arguments():
                             C.byref(h)) == 1
 
 
+def test_quantised_and_layered_creation_checks():
+    # argument checks that return before any device call
+    L = pa.lib()
+    import ctypes as C
+    h = C.c_void_p()
+    fake = C.c_void_p(16)                       # never dereferenced: rejected first
+    for fn in (L.pa_pool_create_int8, L.pa_pool_create_fp8):
+        assert fn(4, 8, 1, 128, fake, None, C.byref(h)) == 7      # block_size != 16
+        assert fn(4, 16, 1, 64, fake, None, C.byref(h)) == 7      # head_dim != 128
+        assert fn(4, 16, 1, 128, None, None, C.byref(h)) == 1     # no records
+        assert h.value is None
+    # quantised dtypes only through their own entry points or the layered one
+    for dt in (pa.PA_INT8, pa.PA_FP8, 9):
+        assert L.pa_pool_create(4, 16, 1, 128, dt, None, None, None, C.byref(h)) == 1
+    assert L.pa_pool_create_layers(4, 16, 1, 128, 9, 2, fake, fake, None, C.byref(h)) == 1
+    assert L.pa_pool_create_layers(4, 16, 1, 128, pa.PA_FP8, 0, fake, None, None,
+                                   C.byref(h)) == 1                # no layers
+    assert L.pa_pool_create_layers(4, 16, 1, 128, pa.PA_FP8, 2, fake, fake, None,
+                                   C.byref(h)) == 1                # records take no v_cache
+    assert L.pa_pool_create_layers(4, 8, 1, 128, pa.PA_FP8, 2, fake, None, None,
+                                   C.byref(h)) == 7
+
+
+def test_window_calls_reject_bad_arguments_on_host_pools():
+    # a host-only pool answers NO_DEVICE before looking at device pointers
+    p = pa.Pool(4, 16, 1, 128, "bf16")
+    L = pa.lib()
+    assert L.pa_decode_window(p.handle, None, 1, 1, None, 1, None, 1.0, 4, 0, 0, None, 0, None,
+                              None) == 8
+    assert L.pa_decode_window_append(p.handle, None, None, None, None, 1, 1, None, 1, None, 1.0,
+                                     4, 0, 0, None, 0, None, None) == 8
+    assert L.pa_decode_window_workspace_bytes(p.handle, 1, 1, 4, 0, 0, 0) == 0   # window < 1
+
+
 def _mirror(oracle, pool, op):
     kind, args = op[0], op[1:]
     if kind == "create":
