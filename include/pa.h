@@ -32,6 +32,11 @@
  *     borrows k_cache/v_cache; pa_free never frees them.  The pool owns its
  *     manager state (free list, refcounts, tables), a small device staging
  *     area for append plans and a device error word.
+ *   - Devices: a device pool belongs to the device that was current when it
+ *     was created.  Every device call runs there: the library makes that
+ *     device current for the call, when it is not already, and restores the
+ *     caller's device before returning.  Streams, buffers and workspaces
+ *     passed in must belong to the pool's device.
  *   - Streams: device work is queued asynchronously on the caller's stream
  *     (cudaStream_t passed as void*; NULL = legacy default stream).  Calls on
  *     one pool must be issued from one host thread and on one stream, or be
@@ -413,7 +418,7 @@ pa_status pa_prefill_chunk(pa_pool* pool, const void* q, int32_t B,
  * PA_STATIC_SCRATCH_BYTES (16 MiB) that every GPU loading the library holds
  * until the process exits, and calls no cudaMalloc, cudaFree or other
  * allocating routine.  Arguments and results are those of pa_decode without
- * the workspace pair; the current device must be the pool's device.
+ * the workspace pair; it runs on the pool's device like every device call.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.

@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "../../include/pa.h"
+#include "launch.hpp"
 
 namespace {
 
@@ -48,6 +49,7 @@ extern "C" pa_status pa_decode_static_scratch(pa_pool* pool, const void* q, int3
                                               float scale, int32_t partition_tokens,
                                               float* out, void* stream) {
   if (!pool) return PA_ERR_INVALID_ARG;
+  pa::DeviceScope on_pool_device(pa::pool_device(pool));   // the scratch of the pool's device
   void* scratch = nullptr;
   pa_status st = scratch_for_current_device(&scratch);
   if (st != PA_OK) return st;

@@ -5,7 +5,31 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+struct pa_pool;
+
 namespace pa {
+
+// The device a pool's memory lives on (-1 for a host-only pool).
+int pool_device(const pa_pool* p);
+
+// Makes `dev` current for the lifetime of one entry-point call (when it is
+// not already) and restores the caller's device afterwards; dev < 0 = no-op.
+class DeviceScope {
+ public:
+  explicit DeviceScope(int dev) {
+    if (dev >= 0 && cudaGetDevice(&prev_) == cudaSuccess && prev_ != dev)
+      switched_ = cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceScope() {
+    if (switched_) cudaSetDevice(prev_);
+  }
+  DeviceScope(const DeviceScope&) = delete;
+  DeviceScope& operator=(const DeviceScope&) = delete;
+
+ private:
+  int prev_ = -1;
+  bool switched_ = false;
+};
 
 cudaError_t launch_reshape_and_cache(const void* key, const void* value,
                                      void* k_cache, void* v_cache,

@@ -16,6 +16,7 @@
 
 #include "../../include/pa.h"
 #include "block_manager.hpp"
+#include "common.cuh"
 #include "launch.hpp"
 
 using pa::BlockManager;
@@ -70,6 +71,8 @@ struct pa_pool {
   pa_pool* base() { return owner ? owner : this; }
 };
 
+int pa::pool_device(const pa_pool* p) { return (p && p->device) ? p->dev_id : -1; }
+
 namespace {
 
 pa_status from_mgr(MgrStatus s) {
@@ -93,22 +96,7 @@ bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
-// library needs no link-time dependency on libcuda.
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault,
-                                &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() { return pa::tensor_map_encoder(); }
 
 // The pool viewed as a 3-D tensor {head_dim, num_kv_heads, num_blocks *
 // block_size}; one box = one block's 16 tokens x 64 columns of one KV head,
@@ -389,6 +377,7 @@ static void free_ring(pa_pool* p) {
 pa_status pa_free(pa_pool* p) {
   if (!p) return PA_OK;
   if (p->owner) return PA_ERR_INVALID_ARG;   // a layer view: freed with its pool
+  pa::DeviceScope on_pool_device(pa::pool_device(p));
   if (p->device) {
     cudaDeviceSynchronize();
     for (pa_pool* v : p->views) free_ring(v);
@@ -571,6 +560,7 @@ pa_status pa_append_kv(pa_pool* p, const int32_t* seqs, const int32_t* n_new,
                        int64_t* slot_mapping_out, void* stream) {
   if (!p) return PA_ERR_INVALID_ARG;
   if (!p->device) return PA_ERR_NO_DEVICE;
+  pa::DeviceScope on_pool_device(p->dev_id);
   if (n_seqs < 0 || (n_seqs > 0 && (!seqs || !n_new))) return PA_ERR_INVALID_ARG;
   int64_t T = 0;
   for (int32_t i = 0; i < n_seqs; ++i) T += std::max<int32_t>(0, n_new[i]);
@@ -634,6 +624,7 @@ pa_status pa_reshape_and_cache(pa_pool* p, const void* key, const void* value,
   if (!p) return PA_ERR_INVALID_ARG;
   if (!p->device) return PA_ERR_NO_DEVICE;
   if (T < 0 || (T > 0 && (!key || !value || !d_slot_mapping))) return PA_ERR_INVALID_ARG;
+  pa::DeviceScope on_pool_device(p->dev_id);
   return cuda_status(write_rows(p, key, value, d_slot_mapping, T,
                                 static_cast<cudaStream_t>(stream)));
 }
@@ -642,6 +633,7 @@ pa_status pa_cow_copy(pa_pool* p, const int32_t* d_src, const int32_t* d_dst,
                       int32_t n, void* stream) {
   if (!p) return PA_ERR_INVALID_ARG;
   if (!p->device) return PA_ERR_NO_DEVICE;
+  pa::DeviceScope on_pool_device(p->dev_id);
   if (n < 0 || (n > 0 && (!d_src || !d_dst))) return PA_ERR_INVALID_ARG;
   return cuda_status(cow_blocks(p, d_src, d_dst, n, static_cast<cudaStream_t>(stream)));
 }
@@ -732,6 +724,7 @@ pa_status pa_decode(pa_pool* p, const void* q, int32_t B, int32_t H,
   pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks,
                                       d_kv_lens, out);
   if (st != PA_OK) return st;
+  pa::DeviceScope on_pool_device(p->dev_id);
   if (partition_tokens < 0) return PA_ERR_INVALID_ARG;
   if (B == 0) return PA_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -763,6 +756,7 @@ pa_status pa_decode_window(pa_pool* p, const void* q, int32_t B, int32_t H,
                            float* out, void* stream) {
   pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, out);
   if (st != PA_OK) return st;
+  pa::DeviceScope on_pool_device(p->dev_id);
   if (partition_tokens < 0 || window < 1 || sinks < 0) return PA_ERR_INVALID_ARG;
   if (!use_fast_decode(p, H)) return PA_ERR_UNSUPPORTED;
   if (B == 0) return PA_OK;
@@ -778,6 +772,7 @@ pa_status pa_decode_append(pa_pool* p, const void* q, const void* key, const voi
                            void* workspace, size_t workspace_bytes, float* out, void* stream) {
   pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, out);
   if (st != PA_OK) return st;
+  pa::DeviceScope on_pool_device(p->dev_id);
   if (B > 0 && (!key || !value || !d_slot_mapping)) return PA_ERR_INVALID_ARG;
   if (partition_tokens < 0) return PA_ERR_INVALID_ARG;
   if (B == 0) return PA_OK;
@@ -802,6 +797,7 @@ pa_status pa_decode_window_append(pa_pool* p, const void* q, const void* key,
                                   size_t workspace_bytes, float* out, void* stream) {
   pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, out);
   if (st != PA_OK) return st;
+  pa::DeviceScope on_pool_device(p->dev_id);
   if (B > 0 && (!key || !value || !d_slot_mapping)) return PA_ERR_INVALID_ARG;
   if (partition_tokens < 0 || window < 1 || sinks < 0) return PA_ERR_INVALID_ARG;
   if (!use_fast_decode(p, H)) return PA_ERR_UNSUPPORTED;
@@ -829,6 +825,7 @@ pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,
   pa_status st = check_attention_args(p, q, B, H, d_block_tables, max_blocks,
                                       d_kv_lens, out);
   if (st != PA_OK) return st;
+  pa::DeviceScope on_pool_device(p->dev_id);
   if (q_tokens <= 0 || q_tokens > 65535 || max_kv_splits < 0) return PA_ERR_INVALID_ARG;
   if (is_q8(p->dtype)) return PA_ERR_UNSUPPORTED;
   if (B == 0) return PA_OK;
@@ -852,6 +849,7 @@ pa_status pa_get_error(pa_pool* p, int32_t* device_code) {
   if (!p || !device_code) return PA_ERR_INVALID_ARG;
   *device_code = 0;
   if (!p->device) return PA_ERR_NO_DEVICE;
+  pa::DeviceScope on_pool_device(p->dev_id);
   if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
   if (cudaMemcpy(device_code, p->d_err, sizeof(int32_t), cudaMemcpyDeviceToHost) !=
       cudaSuccess)
