@@ -36,7 +36,11 @@
  *     was created.  Every device call runs there: the library makes that
  *     device current for the call, when it is not already, and restores the
  *     caller's device before returning.  Streams, buffers and workspaces
- *     passed in must belong to the pool's device.
+ *     passed in must belong to the pool's device.  Known limit: the
+ *     tensor-core kernels opt into their large shared memory once per
+ *     process, on the first device that launches them; in a process with
+ *     pools on several devices those kernels fail on the others
+ *     (PA_ERR_CUDA, nothing faults).
  *   - Streams: device work is queued asynchronously on the caller's stream
  *     (cudaStream_t passed as void*; NULL = legacy default stream).  Calls on
  *     one pool must be issued from one host thread and on one stream, or be

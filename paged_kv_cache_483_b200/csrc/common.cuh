@@ -8,8 +8,6 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include <atomic>
-
 #include "../../include/pa.h"
 
 namespace pa {
@@ -31,20 +29,6 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// Opt a kernel into `bytes` of dynamic shared memory on the current device.
-// The attribute belongs to each device's context, so it is set once per
-// device (devices 0..63 are remembered in `done`; others set it every time).
-template <typename Kernel>
-inline cudaError_t smem_opt_in(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
-  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
-  return e;
-}
 
 // ---------------------------------------------------------------- errors ---
 __device__ __forceinline__ void raise_err(int32_t* err, int32_t bit) {

@@ -460,9 +460,13 @@ template <int NST>
 static cudaError_t launch_ring(const CUtensorMap* tmK, const CUtensorMap* tmV,
                                const DecodeArgs& a, cudaStream_t stream) {
   const size_t smem = 1024 + NST * kStageBytes + sizeof(DecodeSmemTail<NST>);
-  static std::atomic<uint64_t> opted{0};
-  cudaError_t e = smem_opt_in(decode_mma_kernel<NST>, int(smem), opted);
-  if (e != cudaSuccess) return e;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NST>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   dim3 grid(a.NP, a.Hkv, a.B);
   decode_mma_kernel<NST><<<grid, kDecThreads, smem, stream>>>(*tmK, *tmV, a,
                                                               a.scale * kLog2eF);

@@ -566,10 +566,12 @@ cudaError_t launch_decode_q8(const CUtensorMap* tmR, const DecodeArgs& a, bool f
   }
   const size_t smem = 128 + kQ8Stages * kQ8StageBytes + sizeof(Q8Tail);
   auto* kern = fp8 ? decode_q8_kernel<true> : decode_q8_kernel<false>;
-  static std::atomic<uint64_t> opted[2] = {{0}, {0}};
-  {
-    cudaError_t e = smem_opt_in(kern, int(smem), opted[fp8]);
+  static bool attr_set[2] = {false, false};
+  if (!attr_set[fp8]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(smem));
     if (e != cudaSuccess) return e;
+    attr_set[fp8] = true;
   }
   dim3 grid(a.NP, a.Hkv, a.B);
   kern<<<grid, kQ8Threads, smem, stream>>>(*tmR, a, a.scale * kLog2e);

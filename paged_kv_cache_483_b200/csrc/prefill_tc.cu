@@ -594,7 +594,20 @@ bool prefill_fast_supported(int dtype_bf16, int d, int bs, int G) {
   return dtype_bf16 && d == 128 && bs == 16 && (G == 1 || G == 2 || G == 4 || G == 8);
 }
 
-static PFN_cuTensorMapEncodeTiled_v12000 q_encode_fn() { return tensor_map_encoder(); }
+static PFN_cuTensorMapEncodeTiled_v12000 q_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
 
 cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
                                 const PrefillArgs& a, int sms, cudaStream_t stream) {
@@ -628,10 +641,12 @@ cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
       tmO = tmQ;   // never used
   }
   const size_t smem = 1024 + kDataBytes + sizeof(PfBars);
-  static std::atomic<uint64_t> opted{0};
-  {
-    cudaError_t e = smem_opt_in(prefill_tc_kernel, int(smem), opted);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
+    attr_set = true;
   }
   PfPlan pl;
   pl.nq = (a.q_tokens + 2 * TQ - 1) / (2 * TQ);

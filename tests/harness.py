@@ -113,14 +113,18 @@ class OracleRun:
                 self.slots[op.index], self.cows[op.index] = s, c
         return self
 
-    def attention(self, seq_index, q, heads=None):
+    def attention(self, seq_index, q, heads=None, abs_values=False):
         """Output of query rows q [q_tokens, H, d] (float64) for the decode
         sequence at position seq_index, restricted to query heads whose KV head
-        is stored.  Returns {h: out[q_tokens, d]}."""
+        is stored.  Returns {h: out[q_tokens, d]}.  abs_values: the same
+        attention over |V|, i.e. sum_j p_j |v_j| / sum_j p_j, the scale that
+        every per-term relative rounding error of the kernels is bounded by."""
         w = self.w
         G = w.num_heads // w.num_kv_heads
         seq = w.decode_seqs[seq_index]
         k, v = self.pool.gather(seq)
+        if abs_values:
+            v = np.abs(v)
         res = {}
         for i, kvh in enumerate(self.heads):
             hs = list(range(kvh * G, (kvh + 1) * G)) if heads is None else \
@@ -137,3 +141,8 @@ class OracleRun:
 
 def q64(w):
     return w.queries().to(torch.float64).numpy()
+
+
+def scaled_error(out, ref, scale):
+    """max |out - ref| / scale, elementwise (scale = attention over |V|)."""
+    return float((np.abs(out - ref) / np.maximum(scale, 1e-30)).max())

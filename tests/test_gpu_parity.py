@@ -13,11 +13,19 @@ import torch
 
 import paged_kv_cache_483_b200 as pa
 import workloads
-from harness import DeviceRun, OracleRun, q64
+from harness import DeviceRun, OracleRun, q64, scaled_error
 
 pytestmark = pytest.mark.gpu
 
 TOL_F32, TOL_DECODE, TOL_PREFILL = 1e-4, 2e-3, 5e-3
+# Relative bars: error / (attention over |V|), elementwise.  Every rounding in
+# the kernels is a relative error per term p_j v_j, so the error of an output
+# element is bounded by that relative error times sum_j p_j |v_j| / sum_j p_j.
+# Decode: fp32 scores of exact bf16 products (~6e-5 of a score) and fp32
+# sums, P carried as bf16 hi + lo (2^-16): bar 1e-3.  Prefill: P rounded to
+# bf16 for PV (bf16's unit roundoff 2^-8 per weight, 3.9e-3 if every error
+# aligned; the row sum l stays fp32): bar 8e-3.
+REL_DECODE, REL_PREFILL = 1e-3, 8e-3
 
 
 def _check_decode(g, o, w, tol, partition_tokens=0):
@@ -197,11 +205,14 @@ def _full(w, kv_heads, sample_seqs, decode=True, partition_tokens=0, check_slots
 def test_full_decode32_sampled():
     w = workloads.decode32()
     g, o, out, q = _full(w, [0, 5], None)
-    worst = 0.0
+    worst = rel = 0.0
     for i in (0, 13, 31):
+        scale = o.attention(i, q[i], abs_values=True)
         for h, ref in o.attention(i, q[i]).items():
             worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+            rel = max(rel, scaled_error(out[i, h], ref[0], scale[h][0]))
     assert worst <= TOL_DECODE, worst
+    assert rel <= REL_DECODE, rel
     assert g.pool.get_error() == 0
 
 
@@ -211,35 +222,44 @@ def test_full_ragged256_sampled():
     assert any(o.cows.values())
     lens = [o.pool.lengths[s] for s in w.decode_seqs]
     pick = sorted(set([int(np.argmin(lens)), int(np.argmax(lens))] + list(range(0, 256, 37))))
-    worst = 0.0
+    worst = rel = 0.0
     for i in pick:
+        scale = o.attention(i, q[i], abs_values=True)
         for h, ref in o.attention(i, q[i]).items():
             worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+            rel = max(rel, scaled_error(out[i, h], ref[0], scale[h][0]))
     assert worst <= TOL_DECODE, worst
+    assert rel <= REL_DECODE, rel
     assert g.pool.get_error() == 0
 
 
 def test_full_splitk128k_sampled():
     w = workloads.splitk128k()
     g, o, out, q = _full(w, [2], None, partition_tokens=w.partition_tokens)
-    worst = 0.0
+    worst = rel = 0.0
     for i in (0, 3):
+        scale = o.attention(i, q[i], abs_values=True)
         for h, ref in o.attention(i, q[i]).items():
             worst = max(worst, float(np.abs(out[i, h] - ref[0]).max()))
+            rel = max(rel, scaled_error(out[i, h], ref[0], scale[h][0]))
     assert worst <= TOL_DECODE, worst
+    assert rel <= REL_DECODE, rel
     assert g.pool.get_error() == 0
 
 
 def test_full_prefill_sampled():
     w = workloads.prefill()
     g, o, out, q = _full(w, [1], None, decode=False)
-    worst = 0.0
+    worst = rel = 0.0
     rows = [0, 1, 127, 128, 255, 511]
     for i in (0, 7):
         ref = o.attention(i, q[i])
+        scale = o.attention(i, q[i], abs_values=True)
         for h, r in ref.items():
             worst = max(worst, float(np.abs(out[i, rows, h] - r[rows]).max()))
+            rel = max(rel, scaled_error(out[i, rows, h], r[rows], scale[h][rows]))
     assert worst <= TOL_PREFILL, worst
+    assert rel <= REL_PREFILL, rel
     assert g.pool.get_error() == 0
 
 
