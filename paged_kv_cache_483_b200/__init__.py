@@ -336,11 +336,43 @@ class Pool:
         import torch
         return torch.bfloat16 if self.dtype in ("bf16", "int8", "fp8") else torch.float32
 
+    # -- size checks: the C ABI cannot see device array sizes, so a short table,
+    # kv_lens or row buffer would be read past its end by the kernels --------
+    def _attn_sizes(self, q, block_tables, kv_lens, out, dims):
+        """(B, H, d, max_blocks) of an attention call, checked against the pool
+        and against each other."""
+        if q.dim() != dims:
+            raise ValueError(f"q must have {dims} dimensions, got shape {tuple(q.shape)}")
+        B, H, d = int(q.shape[0]), int(q.shape[-2]), int(q.shape[-1])
+        if d != self.head_dim:
+            raise ValueError(f"q head_dim {d} != pool head_dim {self.head_dim}")
+        if H % self.num_kv_heads:
+            raise ValueError(f"num_heads {H} is not a multiple of num_kv_heads "
+                             f"{self.num_kv_heads}")
+        if block_tables.dim() != 2 or int(block_tables.shape[0]) < B:
+            raise ValueError(f"block_tables must be [>= {B}, max_blocks], got "
+                             f"{tuple(block_tables.shape)}")
+        if kv_lens.numel() < B:
+            raise ValueError(f"kv_lens needs {B} entries, got {kv_lens.numel()}")
+        if out is not None and tuple(out.shape) != tuple(q.shape):
+            raise ValueError(f"out must have shape {tuple(q.shape)}, got {tuple(out.shape)}")
+        return B, H, d, int(block_tables.shape[1])
+
+    def _row_sizes(self, key, value, n):
+        """key / value must be [n, num_kv_heads, head_dim]."""
+        want = (n, self.num_kv_heads, self.head_dim)
+        for name, t in (("key", key), ("value", value)):
+            if t is None or tuple(t.shape) != want:
+                raise ValueError(f"{name} must have shape {want}, got "
+                                 f"{None if t is None else tuple(t.shape)}")
+
     def append_kv(self, seqs, n_new, key, value, stream=None, return_slots=False):
         """Plan + copy-on-write + reshape_and_cache.  key/value [T, Hkv, d] CUDA."""
         seqs_a, sp = _i32(seqs)
         n_a, np_ = _i32(n_new)
         T = int(np.maximum(n_a, 0).sum())
+        if T > 0:
+            self._row_sizes(key, value, T)
         dt = self._torch_dtype()
         slots = np.zeros(max(T, 1), np.int64) if return_slots else None
         _check(lib().pa_append_kv(self._h, sp, np_, len(seqs_a),
@@ -351,6 +383,7 @@ class Pool:
 
     def reshape_and_cache(self, key, value, slot_mapping, stream=None):
         import torch
+        self._row_sizes(key, value, int(slot_mapping.numel()))
         dt = self._torch_dtype()
         _check(lib().pa_reshape_and_cache(self._h, _dev_ptr(key, dt, "key"),
                                           _dev_ptr(value, dt, "value"),
@@ -360,6 +393,8 @@ class Pool:
 
     def cow_copy(self, src, dst, stream=None):
         import torch
+        if src.numel() != dst.numel():
+            raise ValueError(f"src and dst must pair up: {src.numel()} vs {dst.numel()}")
         _check(lib().pa_cow_copy(self._h, _dev_ptr(src, torch.int32, "src"),
                                  _dev_ptr(dst, torch.int32, "dst"), int(src.numel()),
                                  _stream(stream)), "pa_cow_copy")
@@ -372,8 +407,7 @@ class Pool:
                workspace=None, stream=None):
         """q [B, H, d] CUDA (pool dtype) -> out [B, H, d] float32."""
         import torch
-        B, H, d = q.shape
-        MB = block_tables.shape[1]
+        B, H, d, MB = self._attn_sizes(q, block_tables, kv_lens, out, 3)
         if out is None:
             out = torch.empty((B, H, d), dtype=torch.float32, device=q.device)
         scale = 1.0 / math.sqrt(self.head_dim) if scale is None else scale
@@ -397,8 +431,7 @@ class Pool:
         """Decode over a sink + recent window: key j visible iff j < sinks or
         j >= kv_len - window."""
         import torch
-        B, H, d = q.shape
-        MB = block_tables.shape[1]
+        B, H, d, MB = self._attn_sizes(q, block_tables, kv_lens, out, 3)
         if out is None:
             out = torch.empty((B, H, d), dtype=torch.float32, device=q.device)
         scale = 1.0 / math.sqrt(self.head_dim) if scale is None else scale
@@ -425,8 +458,10 @@ class Pool:
         new token, then decode with key j visible iff j < sinks or
         j >= kv_len - window."""
         import torch
-        B, H, d = q.shape
-        MB = block_tables.shape[1]
+        B, H, d, MB = self._attn_sizes(q, block_tables, kv_lens, out, 3)
+        self._row_sizes(key, value, B)
+        if slot_mapping.numel() < B:
+            raise ValueError(f"slot_mapping needs {B} entries, got {slot_mapping.numel()}")
         if out is None:
             out = torch.empty((B, H, d), dtype=torch.float32, device=q.device)
         scale = 1.0 / math.sqrt(self.head_dim) if scale is None else scale
@@ -452,8 +487,10 @@ class Pool:
         """Fused step: write each sequence's new token (key/value [B, Hkv, d]
         at slot_mapping [B] int64) and decode q [B, H, d] over kv_lens."""
         import torch
-        B, H, d = q.shape
-        MB = block_tables.shape[1]
+        B, H, d, MB = self._attn_sizes(q, block_tables, kv_lens, out, 3)
+        self._row_sizes(key, value, B)
+        if slot_mapping.numel() < B:
+            raise ValueError(f"slot_mapping needs {B} entries, got {slot_mapping.numel()}")
         if out is None:
             out = torch.empty((B, H, d), dtype=torch.float32, device=q.device)
         scale = 1.0 / math.sqrt(self.head_dim) if scale is None else scale
@@ -482,8 +519,8 @@ class Pool:
         max_kv_splits: 0 = split the last wave's query tiles over their keys
         as the library chooses, 1 = never split, n = at most n parts."""
         import torch
-        B, T, H, d = q.shape
-        MB = block_tables.shape[1]
+        B, H, d, MB = self._attn_sizes(q, block_tables, kv_lens, out, 4)
+        T = int(q.shape[1])
         if out is None:
             out = torch.empty((B, T, H, d), dtype=torch.float32, device=q.device)
         scale = 1.0 / math.sqrt(self.head_dim) if scale is None else scale

@@ -5,6 +5,7 @@ import os
 import re
 
 import numpy as np
+import torch
 import pytest
 
 import paged_kv_cache_483_b200 as pa
@@ -262,3 +263,39 @@ def test_workload_scripts_match_oracle(name):
     tables, lens = pool.block_tables(w.decode_seqs, max(len(o.tables[s]) for s in w.decode_seqs))
     assert np.array_equal(tables, o.block_table(w.decode_seqs, tables.shape[1]))
     assert lens.tolist() == [o.lengths[s] for s in w.decode_seqs]
+
+
+def test_binding_checks_sizes_before_any_device_pointer():
+    # the C ABI cannot see device array sizes: the binding rejects a short
+    # table / kv_lens / row buffer, a wrong head_dim or output shape first
+    p = pa.Pool(8, 16, 2, 128, "bf16")
+    bf = torch.bfloat16
+    q = torch.zeros(3, 8, 128, dtype=bf)
+    t = torch.zeros(3, 4, dtype=torch.int32)
+    lens = torch.zeros(3, dtype=torch.int32)
+    cases = [
+        (lambda: p.decode(torch.zeros(3, 8, 64, dtype=bf), t, lens), "head_dim"),
+        (lambda: p.decode(torch.zeros(3, 7, 128, dtype=bf), t, lens), "multiple"),
+        (lambda: p.decode(q, t[:2], lens), "block_tables"),
+        (lambda: p.decode(q, t, lens[:2]), "kv_lens"),
+        (lambda: p.decode(q, t, lens, out=torch.zeros(3, 8, 64)), "out must have shape"),
+        (lambda: p.decode(q[0], t, lens), "dimensions"),
+        (lambda: p.prefill_chunk(torch.zeros(3, 5, 8, 128, dtype=bf), t[:1], lens), "block_tables"),
+        (lambda: p.decode_append(q, torch.zeros(3, 2, 128, dtype=bf), torch.zeros(2, 2, 128, dtype=bf),
+                                 torch.zeros(3, dtype=torch.int64), t, lens), "value must have shape"),
+        (lambda: p.decode_append(q, torch.zeros(3, 2, 128, dtype=bf), torch.zeros(3, 2, 128, dtype=bf),
+                                 torch.zeros(2, dtype=torch.int64), t, lens), "slot_mapping"),
+        (lambda: p.decode_window_append(q, torch.zeros(3, 1, 128, dtype=bf),
+                                        torch.zeros(3, 1, 128, dtype=bf),
+                                        torch.zeros(3, dtype=torch.int64), t, lens, 4), "key must"),
+        (lambda: p.reshape_and_cache(torch.zeros(4, 2, 128, dtype=bf), torch.zeros(4, 2, 128, dtype=bf),
+                                     torch.zeros(5, dtype=torch.int64)), "key must"),
+        (lambda: p.cow_copy(torch.zeros(2, dtype=torch.int32), torch.zeros(3, dtype=torch.int32)),
+         "pair up"),
+    ]
+    for call, msg in cases:
+        with pytest.raises(ValueError, match=msg):
+            call()
+    # sizes that fit get as far as the device-pointer check
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        p.decode(q, t, lens)
