@@ -115,7 +115,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map,
       : "memory");
 }
 
-// Shared -> global tile store (no multicast); completion tracked per thread
+// Shared -> global tile store (plain, this CTA only); completion tracked per thread
 // with bulk async-groups.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src,
                                              int32_t x, int32_t y, int32_t z) {
