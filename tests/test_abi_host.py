@@ -299,3 +299,20 @@ def test_binding_checks_sizes_before_any_device_pointer():
     # sizes that fit get as far as the device-pointer check
     with pytest.raises(ValueError, match="CUDA tensor"):
         p.decode(q, t, lens)
+
+
+def test_manager_preflight_counts_the_copy_of_a_shared_partial_tail():
+    # the same case as the oracle pin: one free block covers the new block
+    # but not the copy of the shared partial tail, so the plan must fail
+    # whole and change nothing
+    pool = pa.Pool(3, 4, 1, 1, "f32")
+    pool.create(0)
+    pool.plan_append([0], [6])
+    pool.fork(0, 1, 6)
+    before = (pool.refcounts(), pool.table(0), pool.table(1), pool.stats())
+    with pytest.raises(pa.PAError) as e:
+        pool.plan_append([1], [3])
+    assert e.value.code == 4                             # PA_ERR_POOL_EXHAUSTED
+    assert (pool.refcounts(), pool.table(0), pool.table(1), pool.stats()) == before
+    slots, cow = pool.plan_append([1], [2])              # the copy alone fits
+    assert len(cow) == 1 and pool.validate()

@@ -54,6 +54,24 @@ MISTAKES = {
                                     "return (scope, tuple(tokens[:end]))"),
     "prefix key without context": (C, "prefix_key", "tuple(tokens[:end])",
                                    "tuple(tokens[max(0, end - 16):end])"),
+    "split partition sees one key fewer": (A, "partition_stats",
+                                           "hi = min(stop, max_visible + 1)",
+                                           "hi = min(stop, max_visible)"),
+    "split partition not normalised": (A, "partition_stats",
+                                       "o[qt, h] = (p @ v[start:hi, kv_h, :]) / l[qt, h]",
+                                       "o[qt, h] = p @ v[start:hi, kv_h, :]"),
+    "share_prefix one block short": (P, "KVPool.share_prefix",
+                                     "[:math.ceil(prefix / self.block_size)]",
+                                     "[:prefix // self.block_size]"),
+    "preflight ignores the shared tail": (P, "KVPool.blocks_needed",
+                                          "need += 1", "need += 0"),
+    "waste counted from logical tokens": (P, "KVPool.snapshot",
+                                          '"internal_waste_tokens": capacity - payload',
+                                          '"internal_waste_tokens": capacity - logical'),
+    "int8 scale kept in float64": (Q, "stored_rows", "s32 = scale.astype(np.float32)",
+                                   "s32 = scale"),
+    "cached blocks not referenced": (C, "PrefixCache.create_cached",
+                                     "pool.refs[blk] += 1", "pool.refs[blk] += 0"),
 }
 
 

@@ -74,6 +74,28 @@ def test_p2_negative_contract():
     pool.validate()
 
 
+def test_preflight_counts_the_copy_of_a_shared_partial_tail():
+    # the notebook's preflight (PagedKVPool._blocks_needed_for_append): a
+    # partial tail block with more than one reference needs one extra block,
+    # for its copy, before the room left in it can be used
+    pool = KVPool(3, 4, store_heads=None)
+    pool.create("a")
+    pool.append("a", 6)                       # 2 blocks, tail 2 of 4 used; 1 free
+    pool.share_prefix("a", "b", 6)            # both blocks shared, tail partial
+    assert pool.blocks_needed("b", 1) == 1    # the copy; the token fits its room
+    assert pool.blocks_needed("b", 2) == 1
+    assert pool.blocks_needed("b", 3) == 2    # the copy and one new block
+    assert pool.blocks_needed("a", 0) == 0
+    # one free block covers the new block but not the copy: all or nothing
+    before = pool.snapshot()
+    with pytest.raises(PoolExhausted):
+        pool.append("b", 3)
+    assert pool.snapshot() == before
+    pool.release("a")                          # now b's tail is private
+    assert pool.blocks_needed("b", 3) == 1
+    pool.validate()
+
+
 @pytest.mark.parametrize("action,payload", [("release", 1), ("append", 5)])
 def test_p2_short_child_survives_parent(action, payload):
     pool = KVPool(4, 4, store_heads=None)
