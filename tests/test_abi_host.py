@@ -316,3 +316,13 @@ def test_manager_preflight_counts_the_copy_of_a_shared_partial_tail():
     assert (pool.refcounts(), pool.table(0), pool.table(1), pool.stats()) == before
     slots, cow = pool.plan_append([1], [2])              # the copy alone fits
     assert len(cow) == 1 and pool.validate()
+
+
+def test_manager_payload_takes_the_largest_fill_among_sharers():
+    pool = pa.Pool(4, 4, 1, 1, "f32")
+    pool.create(0)
+    pool.plan_append([0], [6])
+    pool.fork(0, 1, 5)                                   # child sees the tail with 1 slot
+    st = pool.stats()
+    assert st["physical_payload_tokens"] == 6 and st["logical_tokens"] == 11
+    assert st["internal_waste_tokens"] == 2 and st["sharing_savings_tokens"] == 5

@@ -70,6 +70,23 @@ MISTAKES = {
                                           '"internal_waste_tokens": capacity - logical'),
     "int8 scale kept in float64": (Q, "stored_rows", "s32 = scale.astype(np.float32)",
                                    "s32 = scale"),
+    "int8 zero row scale 0.5": (Q, "quantize_rows", "scale = np.where(scale == 0.0, 1.0, scale)",
+                                "scale = np.where(scale == 0.0, 0.5, scale)"),
+    "E4M3 negative zero kept": (Q, "e4m3_round", "neg = (y.ravel() < 0) & (mag != 0)",
+                                "neg = (y.ravel() < 0)"),
+    "E4M3 subnormal exponent": (Q, "e4m3_values", "2.0 ** (1 - 7)", "2.0 ** (0 - 7)"),
+    "tiled causal mask one late": (A, "attention_tiled", "np.arange(s0, s1) > max_visible",
+                                   "np.arange(s0, s1) > max_visible + 1"),
+    "split drops the tail partition": (A, "attention_split_kv",
+                                       "parts = max(1, -(-kv_len // partition))",
+                                       "parts = max(1, kv_len // partition)"),
+    "fill takes the smallest sharer": (P, "KVPool.fills", "fill[blk] = max(fill[blk], min(",
+                                       "fill[blk] = min(fill[blk] or self.block_size, min("),
+    "prefix hit stops a block early": (C, "PrefixCache.hit_tokens",
+                                       "(run + 1) * bs <= len(tokens)",
+                                       "(run + 2) * bs <= len(tokens)"),
+    "prefix cache last writer wins": (C, "PrefixCache.publish", "if key not in self.blocks:",
+                                      "if True:"),
     "cached blocks not referenced": (C, "PrefixCache.create_cached",
                                      "pool.refs[blk] += 1", "pool.refs[blk] += 0"),
 }

@@ -74,6 +74,24 @@ def test_p2_negative_contract():
     pool.validate()
 
 
+def test_payload_takes_the_largest_fill_among_sharers():
+    # both pages count a shared block's live slots as the largest fill any
+    # sharer gives it ("abhik.ai examples/pagedattention.py", the ownership
+    # snapshot's occupied slots; "vladkulikov.com modern-llms module 9
+    # notebook", PagedKVPool._refresh_fills, unequal prefixes sharing a block)
+    pool = KVPool(4, 4, store_heads=None)
+    pool.create("parent")
+    pool.append("parent", 6)                  # blocks [b0: 4, b1: 2]
+    pool.share_prefix("parent", "child", 5)   # child sees b1 with 1 slot
+    assert pool.fills()[pool.tables["parent"][1]] == 2
+    snap = pool.snapshot()
+    assert snap["physical_payload_tokens"] == 6
+    assert snap["logical_tokens"] == 11
+    assert snap["internal_waste_tokens"] == 8 - 6
+    assert snap["sharing_savings_tokens"] == 11 - 6
+    pool.validate()
+
+
 def test_preflight_counts_the_copy_of_a_shared_partial_tail():
     # the notebook's preflight (PagedKVPool._blocks_needed_for_append): a
     # partial tail block with more than one reference needs one extra block,
