@@ -92,13 +92,23 @@ MISTAKES = {
 }
 
 
+# the pin suites that cover each oracle module (the control runs them all)
+SUITES_FOR = {
+    A: ["tests/test_oracle_pins.py", "tests/test_window_pins.py"],
+    Q: ["tests/test_quant_pins.py"],
+    P: ["tests/test_oracle_pins.py", "tests/test_prefix_cache.py"],
+    C: ["tests/test_prefix_cache.py"],
+}
+
+
 def _run(mistake):
     env = dict(os.environ, PYTHONPATH=os.pathsep.join([ROOT, os.path.join(ROOT, "tests")]))
     env.pop("ORACLE_MUTATION", None)
     if mistake is not None:
         env["ORACLE_MUTATION"] = json.dumps(mistake)
+    suites = PIN_SUITES if mistake is None else SUITES_FOR[mistake[0]]
     cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-m", "not gpu", "-p", "oracle_mutation",
-           "-p", "no:cacheprovider", *PIN_SUITES]
+           "-p", "no:cacheprovider", *suites]
     return subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
 
 
