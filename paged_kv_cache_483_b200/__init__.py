@@ -236,6 +236,9 @@ class Pool:
         if getattr(self, "_h", None):
             lib().pa_free(self._h)
             self._h = None
+            # the pool's layer handles went with it
+            for v in getattr(self, "_layers", {}).values():
+                v._h = None
 
     def __del__(self):
         try:
