@@ -72,7 +72,8 @@ def attention_two_pass(q, k, v, scale=None):
 
 def paged_attention(pool, seq, q, kv_len=None, scale=None):
     """Attention of ``q`` [q_tokens, H, d] over sequence ``seq`` of an oracle
-    ``KVPool``: gather through the block table, then ``attention_two_pass``.
+    ``KVPool``: gather through the block table, then ``attention_two_pass``
+    ("docs.rs ferrum-kv 0.4.0 src/attention.rs", ``paged_attention``; "abhik.ai examples/pagedattention.py", ``KVPool.attention``).
 
     The pool must store every KV head (``store_heads='all'``) unless H equals
     the number of stored heads times the group size of those heads; for a pool
@@ -83,7 +84,8 @@ def paged_attention(pool, seq, q, kv_len=None, scale=None):
 
 
 def online_softmax_stats(score_blocks):
-    """(m, l) of a score vector seen block by block; softmax_i = e^(x_i - m) / l."""
+    """(m, l) of a score vector seen block by block; softmax_i = e^(x_i - m) / l
+    ("semidirectx cmu11-667 lecture19 infer_world.py", section 3, ``online_softmax_stats``)."""
     m, l = -math.inf, 0.0
     for blk in score_blocks:
         blk = np.asarray(blk, np.float64)
@@ -96,7 +98,8 @@ def online_softmax_stats(score_blocks):
 
 
 def attention_tiled(q, k, v, tile=16, scale=None):
-    """The one-pass (m, l, acc) recurrence over key tiles, causal offset rule.
+    """The one-pass (m, l, acc) recurrence over key tiles, causal offset rule
+    ("semidirectx cmu11-667 lecture19 infer_world.py", section 3, ``tiled_attention``).
 
     Same contract as ``attention_two_pass``; each query keeps running
     max m, sum l and unnormalised accumulator acc, rescaled by e^(m - m') when a
@@ -132,7 +135,8 @@ def attention_tiled(q, k, v, tile=16, scale=None):
 
 
 def partition_stats(q, k, v, start, stop, scale=None):
-    """Per (qt, h): (m, l, o) over keys [start, stop) with the causal rule of
+    """Reading (split-K is not on the pages): the recurrence of "semidirectx cmu11-667 lecture19 infer_world.py",
+    section 3, over one key range.  Per (qt, h): (m, l, o) over keys [start, stop) with the causal rule of
     the whole sequence; o = acc / l, or zeros with m = -inf, l = 0 when no key
     of the partition is visible."""
     q, k, v = _check(q, k, v)
@@ -160,7 +164,8 @@ def partition_stats(q, k, v, start, stop, scale=None):
 
 
 def combine_partitions(ms, ls, os):
-    """Merge partition statistics: M = max_p m_p, w_p = l_p e^(m_p - M),
+    """Reading: the rescale of "semidirectx cmu11-667 lecture19 infer_world.py", section 3, applied once
+    across partitions.  Merge partition statistics: M = max_p m_p, w_p = l_p e^(m_p - M),
     o = sum_p w_p o_p / sum_p w_p.  ms, ls: [P, ...]; os: [P, ..., d]."""
     ms = np.asarray(ms, np.float64)
     ls = np.asarray(ls, np.float64)
@@ -178,7 +183,8 @@ def combine_partitions(ms, ls, os):
 
 
 def attention_split_kv(q, k, v, partition, scale=None):
-    """Attention computed as partitions of ``partition`` keys plus the merge."""
+    """Attention computed as partitions of ``partition`` keys plus the merge
+    (``partition_stats`` and ``combine_partitions``, readings of "semidirectx cmu11-667 lecture19 infer_world.py", section 3)."""
     kv_len = np.asarray(k).shape[0]
     parts = max(1, -(-kv_len // partition))
     stats = [partition_stats(q, k, v, p * partition, (p + 1) * partition, scale)
@@ -204,6 +210,7 @@ def visible_positions(kv_len, window, sinks=0):
 
 
 def attention_window(q, k, v, window, sinks=0, scale=None):
-    """Decode attention (q_tokens = 1) over the visible positions only."""
+    """Decode attention (q_tokens = 1) over the visible positions only
+    ("vladkulikov.com modern-llms module 9 notebook", ``streaming_keep_indices``; see ``visible_positions``)."""
     idx = visible_positions(np.asarray(k).shape[0], window, sinks)
     return attention_two_pass(q, np.asarray(k)[idx], np.asarray(v)[idx], scale)

@@ -37,6 +37,10 @@ class PoolExhausted(MemoryError):
 
 
 class KVPool:
+    """The physical pool, its tables and refcounts ("abhik.ai examples/pagedattention.py", ``KVPool``; the
+    multi-token append, sharing and accounting of "vladkulikov.com modern-llms module 9 notebook",
+    ``PagedKVPool``)."""
+
     def __init__(self, num_blocks, block_size, num_kv_heads=1, head_dim=1,
                  allocation_order=None, store_heads="all", dtype=np.float64):
         for name, v in (("num_blocks", num_blocks), ("block_size", block_size),
@@ -196,6 +200,8 @@ class KVPool:
 
     # -- addressing ("abhik.ai ... region logical_address") -------------------
     def address(self, seq, token):
+        """(block, offset) of a live token: divmod(token, block_size) through
+        the table ("abhik.ai examples/pagedattention.py", region logical_address)."""
         self._require(seq)
         if not 0 <= token < self.lengths[seq]:
             raise PoolError("token index must address a live token")
@@ -203,11 +209,14 @@ class KVPool:
         return self.tables[seq][logical], offset
 
     def slot(self, seq, token):
+        """Flat slot block * block_size + offset: the slot mapping the append
+        writes through ("docs.rs ferrum-kv 0.4.0 src/attention.rs"'s per-token layout stored block by block)."""
         blk, off = self.address(seq, token)
         return blk * self.block_size + off
 
     def gather(self, seq, kv_len=None):
-        """Live K, V rows in logical order: two arrays [kv_len, stored heads, d]."""
+        """Live K, V rows in logical order: two arrays [kv_len, stored heads, d]
+        ("abhik.ai examples/pagedattention.py", the gather of ``KVPool.attention``)."""
         self._require(seq)
         n = self.lengths[seq] if kv_len is None else int(kv_len)
         k = np.empty((n, len(self.heads), self.head_dim), self.keys.dtype)
@@ -219,7 +228,8 @@ class KVPool:
         return k, v
 
     def block_table(self, seqs, width=None, pad=0):
-        """Tables of ``seqs`` as an int32 matrix padded with ``pad``."""
+        """Tables of ``seqs`` as an int32 matrix padded with ``pad`` (the block
+        tables "docs.rs ferrum-kv 0.4.0 src/attention.rs"'s ``paged_attention`` reads, one row per sequence)."""
         width = width or max([len(self.tables[s]) for s in seqs] + [1])
         out = np.full((len(seqs), width), pad, np.int32)
         for i, s in enumerate(seqs):
@@ -229,6 +239,10 @@ class KVPool:
 
     # -- accounting ("vladkulikov.com ... _refresh_fills, snapshot") -----------
     def fills(self):
+        """Live slots per physical block: the largest fill any sharer gives it
+        ("vladkulikov.com modern-llms module 9 notebook", ``PagedKVPool._refresh_fills``; "abhik.ai examples/pagedattention.py", the
+        ownership snapshot's occupied slots); a block a prefix cache maps is
+        full."""
         fill = [0] * self.num_blocks
         for blk in self.external:              # blocks a prefix cache maps are full
             fill[blk] = self.block_size
@@ -240,6 +254,7 @@ class KVPool:
 
     @property
     def free_blocks(self):
+        """Number of free physical blocks ("vladkulikov.com modern-llms module 9 notebook", ``free_blocks``)."""
         return len(self._free)
 
     def snapshot(self):

@@ -18,7 +18,8 @@ import numpy as np
 
 
 def quantize_rows(x, bits=8):
-    """Codes (int8) and float64 scales (one per row of the last axis)."""
+    """Codes (int8) and float64 scales (one per row of the last axis), as
+    "vladkulikov.com modern-llms module 9 notebook"'s ``fake_quantize_rows`` decides them."""
     limit = float(2 ** (bits - 1) - 1)
     x = np.asarray(x, dtype=np.float64)
     scale = np.abs(x).max(axis=-1) / limit
@@ -29,7 +30,7 @@ def quantize_rows(x, bits=8):
 
 
 def dequantize_rows(codes, scale):
-    """code * scale, float64."""
+    """code * scale, float64 ("vladkulikov.com modern-llms module 9 notebook", ``fake_quantize_rows``)."""
     return np.asarray(codes, dtype=np.float64) * np.asarray(scale, dtype=np.float64)[..., None]
 
 
@@ -40,7 +41,8 @@ def fake_quantize_rows(x, bits=8):
 
 
 def stored_rows(x):
-    """A row as an int8 pool holds it: (codes, float32 scale, value read back)."""
+    """A row as an int8 pool holds it: (codes, float32 scale, value read back);
+    the float32 scale is the reading stated in the module header."""
     codes, scale = quantize_rows(x, 8)
     s32 = scale.astype(np.float32)
     return codes, s32, dequantize_rows(codes, s32.astype(np.float64))
@@ -63,7 +65,7 @@ E4M3_MAX = 448.0
 
 def e4m3_values():
     """Value of each of the 256 codes (NaN for 0x7F and 0xFF), float64,
-    straight from the format definition."""
+    straight from the format definition (the E4M3 format of the OCP 8-bit floating point specification)."""
     vals = np.empty(256, dtype=np.float64)
     for code in range(256):
         s, e, m = code >> 7, (code >> 3) & 15, code & 7
@@ -79,7 +81,7 @@ def e4m3_values():
 
 def e4m3_round(y):
     """Codes (uint8) of the E4M3 values nearest to y (|y| <= 448), ties to the
-    even code; magnitude zero gives 0x00."""
+    even code; magnitude zero gives 0x00 (round to nearest even on the E4M3 format of the OCP 8-bit floating point specification)."""
     y = np.asarray(y, dtype=np.float64)
     if np.any(np.abs(y) > E4M3_MAX) or np.any(np.isnan(y)):
         raise ValueError("e4m3_round: |y| must be <= 448")
@@ -96,7 +98,8 @@ def e4m3_round(y):
 
 
 def quantize_rows_fp8(x):
-    """E4M3 codes (uint8 bit patterns) and float64 scales, one per row."""
+    """E4M3 codes (uint8 bit patterns) and float64 scales, one per row: the
+    per-row recipe of "vladkulikov.com modern-llms module 9 notebook"'s ``fake_quantize_rows`` on the E4M3 format of the OCP 8-bit floating point specification (a reading)."""
     x = np.asarray(x, dtype=np.float64)
     scale = np.abs(x).max(axis=-1) / E4M3_MAX
     scale = np.where(scale == 0.0, 1.0, scale)
@@ -105,13 +108,14 @@ def quantize_rows_fp8(x):
 
 
 def dequantize_rows_fp8(codes, scale):
-    """value(code) * scale, float64."""
+    """value(code) * scale, float64 (the E4M3 format of the OCP 8-bit floating point specification)."""
     return e4m3_values()[np.asarray(codes, dtype=np.uint8)] * \
         np.asarray(scale, dtype=np.float64)[..., None]
 
 
 def stored_rows_fp8(x):
-    """A row as an FP8 pool holds it: (codes, float32 scale, value read back)."""
+    """A row as an FP8 pool holds it: (codes, float32 scale, value read back);
+    the float32 scale as for the int8 pool."""
     codes, scale = quantize_rows_fp8(x)
     s32 = scale.astype(np.float32)
     return codes, s32, dequantize_rows_fp8(codes, s32.astype(np.float64))
