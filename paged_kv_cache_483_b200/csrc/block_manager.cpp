@@ -31,6 +31,7 @@ bool BlockManager::is_permutation(const int32_t* order, int32_t n) {
   return true;
 }
 
+// The first free id in the allocation order ("abhik.ai examples/pagedattention.py", KVPool._allocate).
 int32_t BlockManager::take_block() {
   int32_t r = free_heap_.top();
   free_heap_.pop();
@@ -53,6 +54,8 @@ MgrStatus BlockManager::create(int32_t seq) {
   return MgrStatus::ok;
 }
 
+// Share the blocks of the first `prefix` tokens ("vladkulikov.com modern-llms module 9 notebook",
+// PagedKVPool.share_prefix; fork is the whole length, "abhik.ai examples/pagedattention.py").
 MgrStatus BlockManager::share_prefix(int32_t parent, int32_t child,
                                      int64_t prefix) {
   auto it = seqs_.find(parent);
@@ -69,6 +72,8 @@ MgrStatus BlockManager::share_prefix(int32_t parent, int32_t child,
   return MgrStatus::ok;
 }
 
+// One reference less per block; zero-reference blocks become free ("abhik.ai examples/pagedattention.py",
+// KVPool.release).
 MgrStatus BlockManager::release(int32_t seq) {
   auto it = seqs_.find(seq);
   if (it == seqs_.end()) return MgrStatus::unknown_seq;
@@ -78,6 +83,9 @@ MgrStatus BlockManager::release(int32_t seq) {
   return MgrStatus::ok;
 }
 
+// Preflight ("vladkulikov.com modern-llms module 9 notebook", PagedKVPool._blocks_needed_for_append), then
+// the copy of a shared partial tail and token placement ("abhik.ai examples/pagedattention.py",
+// KVPool.append and copy_on_write).
 MgrStatus BlockManager::append(const int32_t* seqs, const int32_t* n_new,
                                int32_t n, std::vector<int64_t>* slots,
                                std::vector<CowPair>* cow) {
@@ -145,6 +153,8 @@ int64_t BlockManager::length(int32_t seq) const {
   return it == seqs_.end() ? -1 : it->second.length;
 }
 
+// Live slots per block: the largest fill any sharer gives it ("vladkulikov.com modern-llms module 9 notebook",
+// PagedKVPool._refresh_fills); a block the prefix cache maps counts as full.
 std::vector<int64_t> BlockManager::fills() const {
   std::vector<int64_t> fill(num_blocks_, 0);
   for (int32_t b = 0; b < num_blocks_; ++b)
@@ -159,6 +169,7 @@ std::vector<int64_t> BlockManager::fills() const {
   return fill;
 }
 
+// The state summary of "vladkulikov.com modern-llms module 9 notebook", PagedKVPool.snapshot.
 Snapshot BlockManager::snapshot() const {
   Snapshot r{};
   std::vector<int64_t> fill = fills();
@@ -174,6 +185,7 @@ Snapshot BlockManager::snapshot() const {
   return r;
 }
 
+// The invariants of "vladkulikov.com modern-llms module 9 notebook", PagedKVPool.validate.
 bool BlockManager::validate() const {
   if (int64_t(free_heap_.size()) != n_free_) return false;
   std::vector<int32_t> expect(num_blocks_, 0);
@@ -245,6 +257,8 @@ int32_t BlockManager::pfind(int32_t parent, uint64_t scope, uint64_t revision,
   return -1;
 }
 
+// Prefix reuse ("vladkulikov.com modern-llms module 9 notebook", prefix-hash trace): the new sequence starts
+// with the longest run of cached leading full blocks.
 MgrStatus BlockManager::create_cached(int32_t seq, uint64_t scope, uint64_t revision,
                                       const int32_t* tokens, int64_t n,
                                       int64_t* hit_tokens) {
@@ -265,6 +279,7 @@ MgrStatus BlockManager::create_cached(int32_t seq, uint64_t scope, uint64_t revi
   return MgrStatus::ok;
 }
 
+// Key every full block of a sequence; the first publisher of a key wins.
 MgrStatus BlockManager::publish(int32_t seq, uint64_t scope, uint64_t revision,
                                 const int32_t* tokens, int64_t n, int64_t* added) {
   auto it = seqs_.find(seq);
