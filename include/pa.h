@@ -124,8 +124,8 @@ pa_status pa_pool_create(int32_t num_blocks, int32_t block_size,
  * `layer` argument: one block table per sequence serves every layer).
  * k_cache/v_cache: [num_layers, <one layer as for pa_pool_create>] (bf16 /
  * f32), or for PA_INT8 / PA_FP8 k_cache = [num_layers, num_blocks,
- * num_kv_heads, PA_INT8_RECORD_BYTES] records and v_cache NULL.  The returned handle is
- * layer 0; pa_pool_layer gives the others.  All layers share the host
+ * num_kv_heads, PA_INT8_RECORD_BYTES] records and v_cache NULL.  The
+ * returned handle is layer 0; pa_pool_layer gives the others.  All layers share the host
  * manager: sequence and plan calls on any of them act on the same tables.
  * A step over L layers plans once (pa_plan_append), copies once
  * (pa_cow_copy copies each pair in every layer), then writes and attends
@@ -155,12 +155,13 @@ pa_status pa_pool_layer(pa_pool* pool, int32_t layer, pa_pool** layer_pool);
  *     [2048, 4096)  V codes, 128 rows d of 16 bytes (token t at d * 16 + t)
  *     [4096, 4160)  16 float32 K scales, token order
  *     [4160, 4224)  16 float32 V scales
- *   A block's record moves with one bulk copy.  Only block_size 16 and
- *   head_dim 128.
+ *   The decode loads a (block, head) record with one copy.  Only
+ *   block_size 16 and head_dim 128.
  * On such a pool pa_append_kv / pa_reshape_and_cache take bf16 key/value
  * [T, Hkv, 128] and quantise them into their slots; pa_cow_copy copies whole
- * records; pa_decode (and pa_decode_append, as two launches) dequantise in
- * the kernel for H / Hkv <= 8.  pa_prefill_chunk and groups above 8 return
+ * records; pa_decode and pa_decode_window (and pa_decode_append /
+ * pa_decode_window_append, as two launches) dequantise in the kernel for
+ * H / Hkv <= 8.  pa_prefill_chunk and groups above 8 return
  * PA_ERR_UNSUPPORTED.
  * Errors: PA_ERR_UNSUPPORTED (block_size != 16 or head_dim != 128),
  * PA_ERR_INVALID_ARG (NULL or misaligned kv_records, bad size or order),
@@ -317,8 +318,8 @@ size_t pa_decode_workspace_bytes(const pa_pool* pool, int32_t B, int32_t H,
  * q_tokens = 1, [P1] Eq. 3): out[b, h, :] = sum_j softmax_j(q[b,h].k_j *
  * scale) v_j over j < kv_lens[b], k_j/v_j of KV head h / (H / Hkv) read
  * through block_tables[b].
- *   q: device [B, H, head_dim], pool dtype.  out: device [B, H, head_dim]
- *   float32.  d_block_tables: device [B, max_blocks] int32.  d_kv_lens:
+ *   q: device [B, H, head_dim], pool dtype (bf16 on an int8 or FP8 pool).
+ *   out: device [B, H, head_dim] float32.  d_block_tables: device [B, max_blocks] int32.  d_kv_lens:
  *   device [B] int32 (0 gives a zero row).  scale: usually 1/sqrt(head_dim).
  *   partition_tokens: 0 = automatic, > 0 = split each sequence into
  *   partitions of that many tokens (a multiple of block_size) whose softmax
@@ -377,11 +378,11 @@ pa_status pa_decode_append(pa_pool* pool, const void* q, const void* key,
  * token (key/value [B, Hkv, head_dim] at d_slot_mapping[b], as
  * pa_decode_append) and decodes over the window exactly as pa_decode_window
  * -- the result equals pa_reshape_and_cache followed by pa_decode_window.
- * The new token, at kv_lens[b] - 1, is always visible.  One kernel on a bf16
- * pool; two launches (quantising append, then the windowed decode) on
- * an int8 or FP8 pool.  Workspace: pa_decode_window_workspace_bytes bytes.  Errors
- * as pa_decode_window, plus INVALID_ARG for null or misaligned key / value /
- * d_slot_mapping. */
+ * The new token, at kv_lens[b] - 1, is always visible.  One kernel on a
+ * bf16 pool; two launches (quantising append, then the windowed decode) on
+ * an int8 or FP8 pool.  Workspace: pa_decode_window_workspace_bytes bytes.
+ * Errors as pa_decode_window, plus INVALID_ARG for null or misaligned key /
+ * value / d_slot_mapping. */
 pa_status pa_decode_window_append(pa_pool* pool, const void* q, const void* key,
                                   const void* value, const int64_t* d_slot_mapping,
                                   int32_t B, int32_t H, const int32_t* d_block_tables,
