@@ -101,6 +101,23 @@ def test_generic_path_bf16_head_dim_64():
     _check_decode(g, OracleRun(w).apply(w.setup), w, TOL_DECODE)
 
 
+@pytest.mark.parametrize("d,bs,H,Hkv,dtype", [
+    (512, 16, 4, 2, "f32"),      # the largest head_dim the generic kernel takes
+    (80, 4, 6, 3, "bf16"),       # head_dim not a multiple of 32
+    (128, 1, 16, 1, "bf16"),     # one-token blocks, group 16
+    (128, 32, 32, 2, "bf16"),    # group 16 at head_dim 128 (beyond the fast path)
+    (256, 7, 2, 2, "f32"),       # odd block size
+])
+def test_generic_path_edge_shapes(d, bs, H, Hkv, dtype):
+    w = _small([1, 2, 31, 130, 0], H, Hkv, d=d, bs=bs, dtype=dtype, seed=d + bs + H)
+    g = DeviceRun(w).apply(w.setup)
+    assert g.pool.decode_path(H) == 0
+    out = _check_decode(g, OracleRun(w).apply(w.setup), w,
+                        TOL_F32 if dtype == "f32" else TOL_DECODE)
+    assert np.all(out[4] == 0)                             # the empty sequence
+    assert g.pool.get_error() == 0
+
+
 def test_generic_path_fp32_gqa():
     w = _small([9, 40, 64], 8, 2, d=32, bs=8, dtype="f32", seed=4)
     g = DeviceRun(w).apply(w.setup)
