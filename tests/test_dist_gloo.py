@@ -73,3 +73,16 @@ def test_single_process_dist_is_identity():
     assert d.world == 1 and d.max(4.2) == 4.2
     d.barrier()
     d.close()
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    # under torchrun every rank starts bench.py --impl reference; ranks other
+    # than 0 must exit 0 at once, with no output and no collective
+    import subprocess
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1",
+               MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--config", "tiny", "--steps", "3", "--warmup", "3"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
