@@ -10,7 +10,8 @@ BlockManager::BlockManager(int32_t num_blocks, int32_t block_size,
                            const std::vector<int32_t>& order)
     : num_blocks_(num_blocks), block_size_(block_size),
       order_(order), rank_(num_blocks), refs_(num_blocks, 0),
-      is_free_(num_blocks, 1), n_free_(num_blocks), cache_refs_(num_blocks, 0) {
+      is_free_(num_blocks, 1), n_free_(num_blocks), tail_drop_(num_blocks, 0),
+      cache_refs_(num_blocks, 0) {
   if (order_.empty()) {
     order_.resize(num_blocks);
     for (int32_t i = 0; i < num_blocks; ++i) order_[i] = i;
@@ -90,37 +91,50 @@ MgrStatus BlockManager::append(const int32_t* seqs, const int32_t* n_new,
                                int32_t n, std::vector<int64_t>* slots,
                                std::vector<CowPair>* cow) {
   // -- preflight: nothing below this block changes state until it passes.
-  std::unordered_set<int32_t> seen;
-  std::unordered_map<int32_t, int32_t> ref_drop;  // copies made earlier in batch
+  // A sequence named twice in the batch is caught by its batch stamp; a
+  // shared tail copied earlier in the batch holds one reference less for the
+  // sequences after it (tail_drop_, reset before returning).
+  ++batch_;
+  batch_seqs_.clear();
+  tail_touched_.clear();
+  MgrStatus verdict = MgrStatus::ok;
   int64_t need = 0, total_tokens = 0;
   for (int32_t i = 0; i < n; ++i) {
     auto it = seqs_.find(seqs[i]);
-    if (it == seqs_.end()) return MgrStatus::unknown_seq;
-    if (n_new[i] < 0 || !seen.insert(seqs[i]).second) return MgrStatus::invalid;
-    const Seq& s = it->second;
+    if (it == seqs_.end()) {
+      verdict = MgrStatus::unknown_seq;
+      break;
+    }
+    Seq& s = it->second;
+    if (n_new[i] < 0 || s.batch == batch_) {
+      verdict = MgrStatus::invalid;
+      break;
+    }
+    s.batch = batch_;
+    batch_seqs_.push_back(&s);
     int64_t cnt = n_new[i];
     total_tokens += cnt;
     if (cnt == 0) continue;
     int64_t used = s.length % block_size_, room = 0;
     if (!s.blocks.empty() && used) {
       room = block_size_ - used;
-      int32_t tail = s.blocks.back();
-      auto d = ref_drop.find(tail);
-      int32_t ref = refs_[tail] - (d == ref_drop.end() ? 0 : d->second);
-      if (ref > 1) {
+      const int32_t tail = s.blocks.back();
+      if (refs_[tail] - tail_drop_[tail] > 1) {
         need += 1;
-        ++ref_drop[tail];
+        if (tail_drop_[tail]++ == 0) tail_touched_.push_back(tail);
       }
     }
     int64_t beyond = std::max<int64_t>(0, cnt - room);
     need += (beyond + block_size_ - 1) / block_size_;
   }
+  for (int32_t b : tail_touched_) tail_drop_[b] = 0;
+  if (verdict != MgrStatus::ok) return verdict;
   if (need > n_free_) return MgrStatus::exhausted;
 
   // -- apply: per sequence, copy a shared partial tail, then place tokens.
   if (slots) slots->reserve(slots->size() + total_tokens);
   for (int32_t i = 0; i < n; ++i) {
-    Seq& s = seqs_[seqs[i]];
+    Seq& s = *batch_seqs_[size_t(i)];
     int64_t cnt = n_new[i];
     if (cnt == 0) continue;
     if (!s.blocks.empty() && (s.length % block_size_) &&

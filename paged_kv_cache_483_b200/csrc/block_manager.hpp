@@ -71,6 +71,7 @@ class BlockManager {
   struct Seq {
     int64_t length = 0;
     std::vector<int32_t> blocks;
+    uint64_t batch = 0;   // the last append batch that named this sequence
   };
   int32_t take_block();            // first free id in the order
   void give_back(int32_t block);   // refcount reached zero
@@ -83,6 +84,11 @@ class BlockManager {
   // min-heap of the free blocks' positions in the allocation order
   std::priority_queue<int32_t, std::vector<int32_t>, std::greater<int32_t>> free_heap_;
   std::unordered_map<int32_t, Seq> seqs_;
+  // append scratch, reused by every call (no allocation per call once warm)
+  uint64_t batch_ = 0;                  // stamp of the current append batch
+  std::vector<Seq*> batch_seqs_;        // the batch's sequences, in order
+  std::vector<int32_t> tail_drop_;      // per block: copies planned earlier in the batch
+  std::vector<int32_t> tail_touched_;   // blocks whose tail_drop_ is non-zero
 
   // A key is stored as (its parent's entry, the block's own tokens): two
   // keys are equal exactly when their parents are and their last
