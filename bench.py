@@ -5,9 +5,10 @@ Default workload (the headline metric): decode batch 32 at 8K context, GQA
 32/8, head_dim 128, block 16, bf16 K/V/Q, a 16384-block pool in a seeded
 permuted order.  One step = append of every sequence's new token (K/V written
 at the slots the host manager planned for position 8191) and paged decode
-attention at kv_len 8192, fused in one kernel (pa_decode_append).  The host plan itself is
-timed separately (``host_plan_us``) because a repeated step must rewrite the
-same slots.
+attention at kv_len 8192, fused in one kernel (pa_decode_append).  The device
+step replays one plan (a repeated step must rewrite the same slots); the host
+plan is timed on its own (``host_plan_us``, median of warm calls) and inside
+every ``e2e`` step, which plans, copies, runs and rolls the step back.
 
 Metric: effective KV bytes read by decode per second (sum_b kv_len_b * Hkv *
 head_dim * 2 (K and V) * 2 bytes), whole job over all ranks; ``seqs_per_s``
@@ -15,7 +16,9 @@ is the same time expressed as sequences decoded per second.
 
 Other workloads (``--config``): ragged256 (copy-on-write + append + decode),
 splitk128k (split-K decode + log-sum-exp combine), prefill (512-token chunk
-append + causal chunked prefill; metric TFLOP/s of causal pairs).
+append + causal chunked prefill; metric TFLOP/s of causal pairs).  The
+default run also measures each of them, and decode32 over int8 and FP8
+pools, under ``configs`` (each with its own roofline, e2e and clocks).
 
 Multi-GPU: one process per GPU (torchrun); every rank decodes its own replica
 batch (different seeds), no collective on the data path ("scaling": "weak");
@@ -181,9 +184,12 @@ class Dist:
 
 # --------------------------------------------------------- our CUDA path ----
 class Setup:
-    """A workload brought up on the GPU through the C ABI (untimed)."""
+    """A workload brought up on the GPU through the C ABI (untimed).
 
-    def __init__(self, w, device, q8=False):
+    ``memo`` (optional dict) keeps each append op's host K/V so that another
+    pool type over the same workload reuses them instead of drawing again."""
+
+    def __init__(self, w, device, q8=False, memo=None):
         import torch
         import paged_kv_cache_483_b200 as pa
         self.w, self.device, self.q8 = w, device, q8
@@ -200,6 +206,14 @@ class Setup:
             self.v_cache = torch.empty(shape, dtype=dt, device=device)
             self.pool = pa.Pool(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.dtype,
                                 self.k_cache, self.v_cache, alloc_order=w.order)
+
+        def kv(op):
+            if memo is None:
+                return w.kv_for(op)
+            if op.index not in memo:
+                memo[op.index] = w.kv_for(op)
+            return memo[op.index]
+
         for op in w.setup:
             if op.kind == "create":
                 self.pool.create(op.args[0])
@@ -208,21 +222,19 @@ class Setup:
             elif op.kind == "release":
                 self.pool.release(op.args[0])
             else:
-                k, v = w.kv_for(op)
+                k, v = kv(op)
                 self.pool.append_kv([op.args[0]], [op.args[1]], k.to(device), v.to(device))
         torch.cuda.synchronize()
-        # the step's appends: planned once by the host manager (timed alone)
+        # the step's appends: planned once by the host manager (the plan's own
+        # cost is measured separately, on warm calls)
         self.step_k = self.step_v = None
         self.slots = None
         self.cow_src = self.cow_dst = None
-        self.host_plan_us = None
         if w.step:
             seqs = [op.args[0] for op in w.step]
             n_new = [op.args[1] for op in w.step]
-            t0 = time.perf_counter()
             slots, cow = self.pool.plan_append(seqs, n_new)
-            self.host_plan_us = (time.perf_counter() - t0) * 1e6
-            ks, vs = zip(*[w.kv_for(op) for op in w.step])
+            ks, vs = zip(*[kv(op) for op in w.step])
             self.step_k = torch.cat(ks).to(device)
             self.step_v = torch.cat(vs).to(device)
             self.slots = torch.tensor(slots, dtype=torch.int64, device=device)
@@ -259,21 +271,27 @@ def prefill_flops(w, lens):
                    for L in lens))
 
 
-def run_ours(args, dist):
+def default_seed(config):
+    return (workloads.SEED_TINY if config == "tiny" else
+            workloads.seed_for({"decode32": 2, "ragged256": 3, "splitk128k": 4,
+                                "prefill": 5}[config]))
+
+
+def run_workload(args, dist, config, kv="bf16", win=0, sinks=0, *, steps, min_ms=0.0,
+                 clock_period=0.001, cpu=False, memo=None):
+    """Bring one workload up, time its step on the device and end to end.
+
+    steps: timed steps; with min_ms > 0 the count grows until the timed region
+    lasts about min_ms (long enough for the clock sampler to see the run)."""
     import torch
-    torch.cuda.set_device(dist.local)
     device = torch.device("cuda", dist.local)
-    builder = workloads.ALL[args.config]
-    base_seed = args.seed if args.seed is not None else (
-        workloads.SEED_TINY if args.config == "tiny" else
-        workloads.seed_for({"decode32": 2, "ragged256": 3, "splitk128k": 4,
-                            "prefill": 5}[args.config]))
+    builder = workloads.ALL[config]
+    base_seed = args.seed if args.seed is not None else default_seed(config)
     w = builder(seed=base_seed + 1000 * dist.rank)
-    q8 = args.kv if args.kv in ("int8", "fp8") else False
-    win, sinks = args.window, args.sinks
+    q8 = kv if kv in ("int8", "fp8") else False
     if (q8 or win) and w.q_tokens > 1:
         raise SystemExit("--kv int8/fp8 and --window apply to the decode workloads")
-    S = Setup(w, device, q8=q8)
+    S = Setup(w, device, q8=q8, memo=memo)
     pool = S.pool
     is_prefill = w.q_tokens > 1
     part = w.partition_tokens
@@ -318,20 +336,28 @@ def run_ours(args, dist):
             ev_pair[1].record(stream)
         launches["n"] += per_step
 
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
     for _ in range(args.warmup):
         step()
+    w1.record(stream)
     torch.cuda.synchronize()
     assert pool.get_error() == 0, "device error during warm-up"
+    K = steps
+    if min_ms > 0:
+        est = w0.elapsed_time(w1) / max(1, args.warmup)
+        K = max(K, int(math.ceil(min_ms / max(est, 1e-3))))
+        K = dist.max(K, device) if dist.world > 1 else K
+        K = int(K)
 
     # ------------------------------------------------------ timed region --
-    K = args.steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches["n"] = 0
     dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    with ClockSampler(torch.cuda.current_device(), clock_period) as clk:
         t_start.record(stream)
         for i in range(K):
             step(evs[i])
@@ -344,25 +370,14 @@ def run_ours(args, dist):
     ms_step_max = dist.max(ms_step, device)
     assert pool.get_error() == 0, "device error in the timed region"
 
-    # the chunk's own append (K1 at the planned slots), timed on its own
+    # the chunk's own append (K1 at the planned slots), timed on its own with
+    # L2 flushed between launches (its 32 MiB of traffic would fit in L2)
     append = None
     if is_prefill and S.slots is not None:
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        for _ in range(3):
-            pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
-        n_app = 20
-        a0.record(stream)
-        for _ in range(n_app):
-            pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
-        a1.record(stream)
-        torch.cuda.synchronize()
-        app_ms = a0.elapsed_time(a1) / n_app
-        moved = 2 * 2 * S.step_k.numel() * S.step_k.element_size()   # K and V, read + write
-        append = {"ms": round(app_ms, 5), "GB/s": round(moved / (app_ms * 1e-3) / 1e9, 1),
-                  "bytes": moved}
+        append = time_append(S, stream, torch.cuda.current_device())
 
     # --------------------------------------------------------------- e2e --
-    e2e = run_e2e(args, S, dist, device, is_prefill, part)
+    e2e = run_e2e(args, S, dist, device, is_prefill, part, win, sinks)
 
     hbm, bf16, bf16_sus, peak_kind = peaks()
     lens = S.lens_h
@@ -377,15 +392,16 @@ def run_ours(args, dist):
                 "traffic": profiled_traffic("prefill_tc.cu", w.name),
                 "frac_of_nominal": round(achieved / NOMINAL_BF16_TFLOPS, 4),
                 "frac_of_sustained": round(achieved / bf16_sus, 4),
-                "kernel": "prefill", "kernel_ms": round(kern_ms, 5),
+                "kernel": "prefill_tc_kernel", "kernel_ms": round(kern_ms, 5),
+                "algorithmic_flops_per_launch": flops,
                 "peak_source": f"{peak_kind} bf16_tflops (burst)"}
         extra = {"tflops": round(value, 2), "append": append}
     else:
-        kv = decode_bytes(w, lens, q8, win, sinks)
-        value = dist.world * kv / (ms_step_max * 1e-3) / 1e9
+        kvb = decode_bytes(w, lens, q8, win, sinks)
+        value = dist.world * kvb / (ms_step_max * 1e-3) / 1e9
         metric = metric_name(w, q8, win, sinks)
         unit = "GB/s"
-        achieved = kv / (kern_ms * 1e-3) / 1e9
+        achieved = kvb / (kern_ms * 1e-3) / 1e9
         kname = (f"decode_q8_kernel<{'true' if q8 == 'fp8' else 'false'}>" if q8 else
                  "decode_mma_kernel"
                  if pool.decode_path(w.num_heads) else "attention_generic_kernel")
@@ -398,14 +414,14 @@ def run_ours(args, dist):
                 "kernel": (f"decode_order_kernel + {kname}" if order_only else
                            f"{kname} + decode_combine_kernel" if split else kname),
                 "kernel_ms": round(kern_ms, 5),
-                "algorithmic_bytes_per_launch": kv, "peak_source": f"{peak_kind} hbm_gbs"}
+                "algorithmic_bytes_per_launch": kvb, "peak_source": f"{peak_kind} hbm_gbs"}
         extra = {"seqs_per_s": round(dist.world * len(w.decode_seqs) / (ms_step_max * 1e-3), 1),
                  "frac_of_peak": round(value / hbm, 4)}
         if q8:
-            extra["kv_bytes_vs_bf16"] = round(kv / decode_bytes(w, lens, False, win, sinks), 4)
+            extra["kv_bytes_vs_bf16"] = round(kvb / decode_bytes(w, lens, False, win, sinks), 4)
         if win:
             extra["window"] = {"window": win, "sinks": sinks,
-                               "visible_fraction": round(kv / decode_bytes(w, lens, q8), 4)}
+                               "visible_fraction": round(kvb / decode_bytes(w, lens, q8), 4)}
     res = {
         "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": dist.world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 5),
@@ -413,21 +429,76 @@ def run_ours(args, dist):
         "dtype": ("int8 KV codes (int8/fp16 MMA, fp32 softmax), bf16 Q" if q8 == "int8" else
                   "fp8 e4m3 KV codes (fp16 MMA, fp32 softmax), bf16 Q" if q8 else "bf16"),
         "data": "synthetic (seeded N(0,1), bf16-rounded)",
-        "config": config_of(w, args, dist),
+        "config": config_of(w, kv, win, sinks, dist),
         **extra,
-        "host_plan_us": None if S.host_plan_us is None else round(S.host_plan_us, 1),
+        "host_plan_us": host_plan_us(S) if S.slots is not None else None,
         "gpu_launches": gpu_launches,
         "roofline": roof,
         "e2e": e2e,
         "clocks": clk.summary(),
     }
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, args, S.out.float().cpu().numpy(), q8)
+    if cpu and dist.rank == 0 and dist.world == 1:
+        res["cpu_baseline"] = cpu_baseline(w, args, S.out.float().cpu().numpy(), q8, win, sinks)
     pool.close()
+    del S
+    torch.cuda.empty_cache()
     return res
 
 
-def config_of(w, args, dist):
+def time_append(S, stream, cuda_index, n_app=300):
+    """reshape_and_cache of the step's rows at their planned slots, one launch
+    at a time with L2 flushed (a 256 MiB write) between launches."""
+    import torch
+    pool = S.pool
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=S.device)
+    for _ in range(3):
+        pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_app)]
+    torch.cuda.synchronize()
+    with ClockSampler(cuda_index, 0.0005) as clk:
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+    assert pool.get_error() == 0
+    app_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    moved = 2 * 2 * S.step_k.numel() * S.step_k.element_size()   # K and V, read + write
+    hbm, _, _, peak_kind = peaks()
+    gbs = moved / (app_ms * 1e-3) / 1e9
+    return {"kernel": "reshape_and_cache_kernel<uint4>", "launches": n_app,
+            "kernel_ms": round(app_ms, 5), "bytes_per_launch": moved,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4),
+                         "traffic": profiled_traffic("kv_write.cu", "prefill_append"),
+                         "peak_source": f"{peak_kind} hbm_gbs"},
+            "l2": "flushed between launches (256 MiB write, untimed)",
+            "clocks": clk.summary()}
+
+
+def host_plan_us(S, n=200):
+    """Median wall time of one warm pa_plan_append of the step's appends (host
+    manager, through ctypes), each followed by an untimed rollback
+    (pa_seq_truncate) so that every call plans the same step."""
+    pool = S.pool
+    seqs = [op.args[0] for op in S.w.step]
+    n_new = [op.args[1] for op in S.w.step]
+    base = [pool.table(s)[1] for s in seqs]           # lengths after the step's plan
+    start = [b - k for b, k in zip(base, n_new)]
+    pool.truncate(seqs, start)
+    t = []
+    for _ in range(n):
+        t0 = time.perf_counter()
+        pool.plan_append(seqs, n_new)
+        t.append(time.perf_counter() - t0)
+        pool.truncate(seqs, start)
+    pool.plan_append(seqs, n_new)                     # the state the step assumes
+    return round(statistics.median(t) * 1e6, 2)
+
+
+def config_of(w, kv, win, sinks, dist):
     G = w.num_heads // w.num_kv_heads
     return {"workload": w.name, "batch_per_gpu": len(w.decode_seqs),
             "global_batch": len(w.decode_seqs) * dist.world,
@@ -435,65 +506,112 @@ def config_of(w, args, dist):
             "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
             "q_tokens": w.q_tokens, "partition_tokens": w.partition_tokens,
             "parallelism": f"replicas x{dist.world} (no collective)",
-            "kv": getattr(args, "kv", "bf16"),
-            "window": getattr(args, "window", 0), "sinks": getattr(args, "sinks", 0),
+            "kv": kv, "window": win, "sinks": sinks,
             "l2": ("tiny: fits in L2 (correctness scale)" if w.name == "tiny" else
                    "KV per step ~0.5 GB > L2 (shared prefixes may hit in L2)"
                    if w.name == "ragged256" else "inputs larger than L2 (KV per step > 126 MB)")}
 
 
-def run_e2e(args, S, dist, device, is_prefill, part):
-    """Same metric through the public API with host buffers: every step copies
-    its inputs (queries, new K/V, slot mapping, kv_lens) from pinned host memory
-    and reads the output back; copies are inside the timed region."""
+class _PinnedRing:
+    """Pinned host buffers reused round-robin; a buffer is rewritten only after
+    the copy that last read it has run."""
+
+    def __init__(self, make, depth=8):
+        import torch
+        self.bufs = [make() for _ in range(depth)]
+        self.evs = [torch.cuda.Event() for _ in range(depth)]
+        self.used = [False] * depth
+        self.i = 0
+
+    def take(self):
+        i = self.i
+        self.i = (i + 1) % len(self.bufs)
+        if self.used[i]:
+            self.evs[i].synchronize()
+        self.used[i] = True
+        return self.bufs[i], self.evs[i]
+
+
+def run_e2e(args, S, dist, device, is_prefill, part, win, sinks):
+    """Same metric through the public API with host buffers.  Every step
+    plans its appends on the host manager (pa_plan_append), copies its inputs
+    (queries, new K/V, slot mapping, copy-on-write pairs, kv_lens) from pinned
+    host memory, runs the step's kernels and reads the output back; then the
+    step's tokens are rolled back (pa_seq_truncate) so that every step is the
+    same step.  Plans, copies and the rollback are inside the timed region.
+    A copy-on-write of a shared partial tail happens in the first planned
+    step only (the tail is private afterwards), as in serving."""
     import torch
     pool = S.pool
     stream = torch.cuda.current_stream(device)
+    w = S.w
     h_q = S.q.cpu().pin_memory()
     h_out = torch.empty(S.out.shape, dtype=torch.float32).pin_memory()
     h_lens = S.lens.cpu().pin_memory()
     d_q, d_lens = torch.empty_like(S.q), torch.empty_like(S.lens)
-    h_k = h_v = h_slots = None
     bi = h_q.numel() * h_q.element_size() + h_lens.numel() * 4
-    if S.slots is not None:
+    seqs = [op.args[0] for op in w.step]
+    n_new = [op.args[1] for op in w.step]
+    plan = bool(w.step)
+    if plan:
         h_k, h_v = S.step_k.cpu().pin_memory(), S.step_v.cpu().pin_memory()
-        h_slots = S.slots.cpu().pin_memory()
-        d_k, d_v, d_slots = torch.empty_like(S.step_k), torch.empty_like(S.step_v), torch.empty_like(S.slots)
-        bi += 2 * h_k.numel() * h_k.element_size() + h_slots.numel() * 8
+        d_k, d_v = torch.empty_like(S.step_k), torch.empty_like(S.step_v)
+        T = int(S.slots.numel())
+        d_slots = torch.empty_like(S.slots)
+        d_cow = torch.empty(2 * len(seqs), dtype=torch.int32, device=device)
+        ring = _PinnedRing(lambda: (torch.empty(T, dtype=torch.int64).pin_memory(),
+                                    torch.empty(2 * len(seqs), dtype=torch.int32).pin_memory()))
+        bi += 2 * h_k.numel() * h_k.element_size() + T * 8
+        lens_now = [pool.table(s)[1] for s in seqs]
+        start = [L - k for L, k in zip(lens_now, n_new)]
+        pool.truncate(seqs, start)                       # undo the set-up's plan
     bo = h_out.numel() * 4
     K = max(1, min(args.steps, args.e2e_steps))
+    fused = (not is_prefill) and plan and not S.q8
+    cow_bytes = [0]
 
     def step():
         d_q.copy_(h_q, non_blocking=True)
         d_lens.copy_(h_lens, non_blocking=True)
-        if h_k is not None:
+        if plan:
+            slots, cow = pool.plan_append(seqs, n_new)            # step a1, on the host
+            (hs, hc), ev = ring.take()
+            hs.numpy()[:] = slots
+            d_slots.copy_(hs, non_blocking=True)
             d_k.copy_(h_k, non_blocking=True)
             d_v.copy_(h_v, non_blocking=True)
-            d_slots.copy_(h_slots, non_blocking=True)
-            if S.n_cow:
-                pool.cow_copy(S.cow_src, S.cow_dst, stream)
-            if is_prefill:
+            if cow:
+                n = len(cow)
+                hc.numpy()[:n] = [c[0] for c in cow]
+                hc.numpy()[n:2 * n] = [c[1] for c in cow]
+                d_cow[:2 * n].copy_(hc[:2 * n], non_blocking=True)
+                pool.cow_copy(d_cow[:n], d_cow[n:2 * n], stream)
+                cow_bytes[0] += 8 * n
+            ev.record(stream)
+            if not fused:
                 pool.reshape_and_cache(d_k, d_v, d_slots, stream)
         if is_prefill:
             pool.prefill_chunk(d_q, S.tables, d_lens, out=S.out, stream=stream)
-        elif args.window and h_k is not None:
-            pool.decode_window_append(d_q, d_k, d_v, d_slots, S.tables, d_lens, args.window,
-                                      args.sinks, out=S.out, partition_tokens=part,
-                                      stream=stream)
-        elif args.window:
-            pool.decode_window(d_q, S.tables, d_lens, args.window, args.sinks, out=S.out,
-                               partition_tokens=part, stream=stream)
-        elif h_k is not None:
+        elif fused and win:
+            pool.decode_window_append(d_q, d_k, d_v, d_slots, S.tables, d_lens, win, sinks,
+                                      out=S.out, partition_tokens=part, stream=stream)
+        elif fused:
             pool.decode_append(d_q, d_k, d_v, d_slots, S.tables, d_lens, out=S.out,
+                               partition_tokens=part, stream=stream)
+        elif win:
+            pool.decode_window(d_q, S.tables, d_lens, win, sinks, out=S.out,
                                partition_tokens=part, stream=stream)
         else:
             pool.decode(d_q, S.tables, d_lens, out=S.out, partition_tokens=part, stream=stream)
         h_out.copy_(S.out, non_blocking=True)
+        if plan:
+            pool.truncate(seqs, start)                            # roll the step back
 
     for _ in range(3):
         step()
     torch.cuda.synchronize()
     dist.barrier()
+    cow_bytes[0] = 0
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(K):
@@ -501,15 +619,17 @@ def run_e2e(args, S, dist, device, is_prefill, part):
     b.record(stream)
     torch.cuda.synchronize()
     ms = dist.max(a.elapsed_time(b) / K, device)
-    w = S.w
+    if plan:
+        pool.plan_append(seqs, n_new)                 # back to the state the step assumes
     if is_prefill:
         v = dist.world * prefill_flops(w, S.lens_h) / (ms * 1e-3) / 1e12
         unit = "TFLOP/s"
     else:
-        v = dist.world * decode_bytes(w, S.lens_h, S.q8, args.window, args.sinks) / (ms * 1e-3) / 1e9
+        v = dist.world * decode_bytes(w, S.lens_h, S.q8, win, sinks) / (ms * 1e-3) / 1e9
         unit = "GB/s"
-    return {"value": round(v, 2), "unit": unit, "h2d_bytes_per_step": int(bi),
-            "d2h_bytes_per_step": int(bo), "ms_per_step": round(ms, 5), "steps": K}
+    return {"value": round(v, 2), "unit": unit, "h2d_bytes_per_step": int(bi + cow_bytes[0] / K),
+            "d2h_bytes_per_step": int(bo), "ms_per_step": round(ms, 5), "steps": K,
+            "host_plan_in_step": plan}
 
 
 # --------------------------------------------------------------- oracle ----
@@ -599,11 +719,12 @@ def oracle_desc(q8, window, sinks):
                if q8 else ""))
 
 
-def cpu_baseline(w, args, gpu_out=None, q8=False):
-    sampler = OracleSampler(w, q8, args.window, args.sinks)
+def cpu_baseline(w, args, gpu_out=None, q8=False, window=0, sinks=0):
+    sampler = OracleSampler(w, q8, window, sinks)
     work, spent, done = sampler.run(args.cpu_budget, keep=2 if gpu_out is not None else 0)
-    desc = (f"{done} of the {len(w.decode_seqs)} sequences of {w.name} (all heads): "
-            + oracle_desc(q8, args.window, args.sinks))
+    distinct = min(done, len(w.decode_seqs))
+    desc = (f"{done} sequence decodes (all heads) over {distinct} distinct sequences of "
+            f"{w.name}: " + oracle_desc(q8, window, sinks))
     if w.q_tokens > 1:
         val, unit = work / spent / 1e12, "TFLOP/s"
     else:
@@ -665,7 +786,7 @@ def run_reference(args, dist):
             "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), bf16-rounded)",
-            "config": {**config_of(w, args, dist), "sample": desc},
+            "config": {**config_of(w, args.kv, args.window, args.sinks, dist), "sample": desc},
             "cpu_baseline": {"value": round(val, 6), "unit": unit, "cores": oracle_threads(),
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": round(val, 6), "unit": unit, "h2d_bytes_per_step": 0,
@@ -691,6 +812,9 @@ def main():
     ap.add_argument("--sinks", type=int, default=0)
     ap.add_argument("--seed", type=int, default=None,
                     help="workload seed (default: the configuration's own)")
+    ap.add_argument("--configs", choices=["auto", "all", "none"], default="auto",
+                    help="also measure every other workload under 'configs' (auto: on the "
+                         "default decode32 run at one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -702,11 +826,48 @@ def main():
         return
     dist.init("nccl")
     try:
-        res = run_ours(args, dist)
+        import torch
+        torch.cuda.set_device(dist.local)
+        memo = {}
+        # the headline: exactly --steps timed steps; the clock sampler runs fast
+        # enough to see a few milliseconds
+        res = run_workload(args, dist, args.config, args.kv, args.window, args.sinks,
+                           steps=args.steps, clock_period=0.0002,
+                           cpu=not args.no_cpu_baseline, memo=memo)
+        default_run = (args.config == "decode32" and args.kv == "bf16" and not args.window)
+        extras = args.configs == "all" or (args.configs == "auto" and default_run
+                                           and dist.world == 1)
+        if extras:
+            res["configs"] = run_extras(args, dist, memo)
         if dist.rank == 0:
             print(json.dumps(res), flush=True)
     finally:
         dist.close()
+
+
+EXTRAS = [("ragged256", "ragged256", "bf16"), ("splitk128k", "splitk128k", "bf16"),
+          ("prefill", "prefill", "bf16"), ("decode32_int8", "decode32", "int8"),
+          ("decode32_fp8", "decode32", "fp8")]
+
+
+def run_extras(args, dist, memo):
+    """Every other workload, each timed for at least ~100 ms (so the clock
+    sampler sees it), with its own roofline, e2e and clocks.  No CPU baseline
+    here (the headline line carries it)."""
+    out = {}
+    keep = ("metric", "value", "unit", "steps", "ms_per_step", "dtype", "config", "seqs_per_s",
+            "tflops", "kv_bytes_vs_bf16", "host_plan_us", "gpu_launches", "roofline", "e2e",
+            "clocks", "frac_of_peak")
+    for name, config, kv in EXTRAS:
+        r = run_workload(args, dist, config, kv, steps=args.steps, min_ms=100.0,
+                         clock_period=0.001, memo=memo if config == "decode32" else None)
+        out[name] = {k: r[k] for k in keep if k in r}
+        if r.get("append"):
+            out["prefill_append"] = {"workload": "prefill chunk append: 8 x 512 tokens, 8 KV "
+                                                 "heads, head_dim 128, bf16 (reshape_and_cache)",
+                                     **r["append"]}
+    memo.clear()
+    return out
 
 
 if __name__ == "__main__":

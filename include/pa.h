@@ -36,11 +36,10 @@
  *     was created.  Every device call runs there: the library makes that
  *     device current for the call, when it is not already, and restores the
  *     caller's device before returning.  Streams, buffers and workspaces
- *     passed in must belong to the pool's device.  Known limit: the
- *     tensor-core kernels opt into their large shared memory once per
- *     process, on the first device that launches them; in a process with
- *     pools on several devices those kernels fail on the others
- *     (PA_ERR_CUDA, nothing faults).
+ *     passed in must belong to the pool's device.  The tensor-core kernels
+ *     opt into their large shared memory once per device, the first time
+ *     they launch there (any host thread may be the first), so pools on
+ *     several devices of one process all work.
  *   - Streams: device work is queued asynchronously on the caller's stream
  *     (cudaStream_t passed as void*; NULL = legacy default stream).  Calls on
  *     one pool must be issued from one host thread and on one stream, or be
@@ -205,6 +204,19 @@ pa_status pa_seq_fork(pa_pool* pool, int32_t parent, int32_t child,
 /* Drop one reference per block of `seq`; blocks reaching zero return to the
  * free list ([P1] release, [P2] release). */
 pa_status pa_seq_release(pa_pool* pool, int32_t seq);
+
+/* Keep the first lengths[i] tokens of sequence seqs[i], for n distinct
+ * sequences (a rollback of their newest tokens, e.g. drafted tokens that were
+ * not accepted).  Not on the pages: it is [P1] release applied to the dropped
+ * tail -- every block wholly past lengths[i] loses this sequence's reference
+ * and returns to the free list at zero -- and equals [P2] share_prefix of the
+ * kept tokens into a new sequence followed by release of the old one.  A
+ * kept partial tail block is left as it is (a copy-on-write already made is
+ * not undone).  seqs, lengths: host [n].  All-or-nothing: UNKNOWN_SEQ, or
+ * INVALID_ARG (length < 0 or beyond the sequence, an id named twice, NULL
+ * arrays with n > 0), before any change. */
+pa_status pa_seq_truncate(pa_pool* pool, const int32_t* seqs,
+                          const int32_t* lengths, int32_t n);
 
 /* Prefix cache ([P2] prefix-hash trace, "complete block boundaries"): the
  * block that ends at token `end` is identified by (scope, revision, every

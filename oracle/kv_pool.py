@@ -198,6 +198,27 @@ class KVPool:
         del self.tables[seq]
         del self.lengths[seq]
 
+    def truncate(self, seq, length):
+        """Keep the first ``length`` tokens of ``seq`` (a rollback of its
+        newest tokens).  Not on the pages; it is the pages' release applied
+        to the dropped tail ("abhik.ai ... KVPool.release"): every block
+        wholly past ``length`` loses this sequence's reference and is freed at
+        zero, and the result equals share_prefix(seq, tmp, length) followed by
+        release(seq), with tmp then named seq.  A kept partial block stays as
+        it is, so a copy-on-write already made is not undone."""
+        self._require(seq)
+        length = int(length)
+        if length < 0 or length > self.lengths[seq]:
+            raise PoolError("length must lie within the sequence")
+        table = self.tables[seq]
+        keep = math.ceil(length / self.block_size)
+        for blk in table[keep:]:
+            self.refs[blk] -= 1
+            if self.refs[blk] == 0:
+                self._give_back(blk)
+        del table[keep:]
+        self.lengths[seq] = length
+
     # -- addressing ("abhik.ai ... region logical_address") -------------------
     def address(self, seq, token):
         """(block, offset) of a live token: divmod(token, block_size) through

@@ -35,7 +35,7 @@ EXPORTS = ["pa_pool_create", "pa_free", "pa_seq_create", "pa_seq_fork", "pa_seq_
            "pa_decode_static_scratch", "pa_decode_append", "pa_seq_create_cached",
            "pa_prefix_publish", "pa_prefix_clear", "pa_prefix_entries", "pa_pool_create_int8",
            "pa_decode_window", "pa_decode_window_workspace_bytes", "pa_pool_create_layers",
-           "pa_pool_layer", "pa_decode_window_append", "pa_pool_create_fp8"]
+           "pa_pool_layer", "pa_decode_window_append", "pa_pool_create_fp8", "pa_seq_truncate"]
 
 
 class PAError(RuntimeError):
@@ -75,6 +75,7 @@ def lib():
         "pa_seq_create": ([_P, _I32], C.c_int),
         "pa_seq_fork": ([_P, _I32, _I32, _I32], C.c_int),
         "pa_seq_release": ([_P, _I32], C.c_int),
+        "pa_seq_truncate": ([_P, _PI32, _PI32, _I32], C.c_int),
         "pa_seq_table": ([_P, _I32, _PI32, _I32, _PI32, _PI32], C.c_int),
         "pa_seq_create_cached": ([_P, _I32, C.c_uint64, C.c_uint64, _PI32, _I32, _PI32], C.c_int),
         "pa_prefix_publish": ([_P, _I32, C.c_uint64, C.c_uint64, _PI32, _I32, _PI32], C.c_int),
@@ -260,6 +261,15 @@ class Pool:
 
     def release(self, seq):
         _check(lib().pa_seq_release(self._h, int(seq)), "pa_seq_release")
+
+    def truncate(self, seqs, lengths):
+        """Keep the first lengths[i] tokens of seqs[i] (rollback of the newest
+        tokens; all-or-nothing)."""
+        seqs_a, sp = _i32(seqs)
+        lens_a, lp = _i32(lengths)
+        if len(seqs_a) != len(lens_a):
+            raise ValueError("seqs and lengths must pair up")
+        _check(lib().pa_seq_truncate(self._h, sp, lp, len(seqs_a)), "pa_seq_truncate")
 
     # -- prefix cache (content-keyed full blocks) ----------------------------
     def create_cached(self, seq, tokens, scope=0, revision=0):

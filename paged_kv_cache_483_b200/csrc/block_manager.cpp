@@ -84,6 +84,29 @@ MgrStatus BlockManager::release(int32_t seq) {
   return MgrStatus::ok;
 }
 
+// A rollback of each sequence's newest tokens; equal to share_prefix of the
+// kept tokens into a new sequence followed by release of the old one.
+MgrStatus BlockManager::truncate(const int32_t* seqs, const int32_t* lengths, int32_t n) {
+  if (n < 0 || (n > 0 && (!seqs || !lengths))) return MgrStatus::invalid;
+  const uint64_t stamp = ++batch_;
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = seqs_.find(seqs[i]);
+    if (it == seqs_.end()) return MgrStatus::unknown_seq;
+    if (lengths[i] < 0 || lengths[i] > it->second.length) return MgrStatus::invalid;
+    if (it->second.batch == stamp) return MgrStatus::invalid;   // named twice
+    it->second.batch = stamp;
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    Seq& s = seqs_.find(seqs[i])->second;
+    const size_t keep = size_t((int64_t(lengths[i]) + block_size_ - 1) / block_size_);
+    for (size_t j = keep; j < s.blocks.size(); ++j)
+      if (--refs_[s.blocks[j]] == 0) give_back(s.blocks[j]);
+    if (keep < s.blocks.size()) s.blocks.resize(keep);
+    s.length = lengths[i];
+  }
+  return MgrStatus::ok;
+}
+
 // Preflight ("vladkulikov.com modern-llms module 9 notebook", PagedKVPool._blocks_needed_for_append), then
 // the copy of a shared partial tail and token placement ("abhik.ai examples/pagedattention.py",
 // KVPool.append and copy_on_write).

@@ -36,6 +36,11 @@ class BlockManager {
   MgrStatus create(int32_t seq);
   MgrStatus share_prefix(int32_t parent, int32_t child, int64_t prefix);
   MgrStatus release(int32_t seq);
+  // Keep the first lengths[i] tokens of seqs[i] (distinct ids): blocks
+  // wholly past them lose that sequence's reference, freed at zero -- the
+  // release of "abhik.ai examples/pagedattention.py" applied to the dropped
+  // tail.  All-or-nothing: every pair is checked before any change.
+  MgrStatus truncate(const int32_t* seqs, const int32_t* lengths, int32_t n);
 
   // Batch append plan; all-or-nothing (preflight over the whole batch with
   // the refcount changes earlier members of the batch make).

@@ -34,6 +34,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "device_once.hpp"
 #include "launch.hpp"
 
 namespace pa {
@@ -460,13 +461,15 @@ template <int NST>
 static cudaError_t launch_ring(const CUtensorMap* tmK, const CUtensorMap* tmV,
                                const DecodeArgs& a, cudaStream_t stream) {
   const size_t smem = 1024 + NST * kStageBytes + sizeof(DecodeSmemTail<NST>);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NST>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = static_cast<cudaError_t>(attr.run(dev, [&] {
+    return int(cudaFuncSetAttribute(decode_mma_kernel<NST>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+  }));
+  if (e != cudaSuccess) return e;
   dim3 grid(a.NP, a.Hkv, a.B);
   decode_mma_kernel<NST><<<grid, kDecThreads, smem, stream>>>(*tmK, *tmV, a,
                                                               a.scale * kLog2eF);

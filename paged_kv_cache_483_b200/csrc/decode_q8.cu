@@ -51,6 +51,7 @@
 #include <cuda_fp8.h>
 
 #include "common.cuh"
+#include "device_once.hpp"
 #include "launch.hpp"
 
 namespace pa {
@@ -566,13 +567,15 @@ cudaError_t launch_decode_q8(const CUtensorMap* tmR, const DecodeArgs& a, bool f
   }
   const size_t smem = 128 + kQ8Stages * kQ8StageBytes + sizeof(Q8Tail);
   auto* kern = fp8 ? decode_q8_kernel<true> : decode_q8_kernel<false>;
-  static bool attr_set[2] = {false, false};
-  if (!attr_set[fp8]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(smem));
-    if (e != cudaSuccess) return e;
-    attr_set[fp8] = true;
-  }
+  static PerDeviceOnce attr[2];
+  int dev = 0;
+  cudaError_t ea = cudaGetDevice(&dev);
+  if (ea != cudaSuccess) return ea;
+  ea = static_cast<cudaError_t>(attr[fp8].run(dev, [&] {
+    return int(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(smem)));
+  }));
+  if (ea != cudaSuccess) return ea;
   dim3 grid(a.NP, a.Hkv, a.B);
   kern<<<grid, kQ8Threads, smem, stream>>>(*tmR, a, a.scale * kLog2e);
   cudaError_t e = cudaGetLastError();

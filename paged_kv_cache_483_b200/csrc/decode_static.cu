@@ -49,6 +49,9 @@ extern "C" pa_status pa_decode_static_scratch(pa_pool* pool, const void* q, int3
                                               float scale, int32_t partition_tokens,
                                               float* out, void* stream) {
   if (!pool) return PA_ERR_INVALID_ARG;
+  // a host-only pool answers like every other device call, before any CUDA
+  // call could create a context on whatever device is current
+  if (pa::pool_device(pool) < 0) return PA_ERR_NO_DEVICE;
   pa::DeviceScope on_pool_device(pa::pool_device(pool));   // the scratch of the pool's device
   void* scratch = nullptr;
   pa_status st = scratch_for_current_device(&scratch);

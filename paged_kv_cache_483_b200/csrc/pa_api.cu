@@ -406,6 +406,12 @@ pa_status pa_seq_release(pa_pool* p, int32_t seq) {
   return from_mgr(p->mgr->release(seq));
 }
 
+pa_status pa_seq_truncate(pa_pool* p, const int32_t* seqs, const int32_t* lengths,
+                          int32_t n) {
+  if (!p) return PA_ERR_INVALID_ARG;
+  return from_mgr(p->mgr->truncate(seqs, lengths, n));
+}
+
 pa_status pa_seq_create_cached(pa_pool* p, int32_t seq, uint64_t scope,
                                uint64_t revision, const int32_t* tokens,
                                int32_t n_tokens, int32_t* hit_tokens) {

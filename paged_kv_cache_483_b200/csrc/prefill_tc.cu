@@ -34,6 +34,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "device_once.hpp"
 #include "launch.hpp"
 #include "tcgen05.cuh"
 
@@ -594,27 +595,12 @@ bool prefill_fast_supported(int dtype_bf16, int d, int bs, int G) {
   return dtype_bf16 && d == 128 && bs == 16 && (G == 1 || G == 2 || G == 4 || G == 8);
 }
 
-static PFN_cuTensorMapEncodeTiled_v12000 q_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    cudaDriverEntryPointQueryResult q;
-    void* ptr = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
 cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
                                 const PrefillArgs& a, int sms, cudaStream_t stream) {
   const int G = a.H / a.Hkv, TQ = 128 / G;
   // Q viewed as {head_dim, H, B * q_tokens}; one box = TQ tokens x G heads x 64
   CUtensorMap tmQ;
-  auto fn = q_encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return cudaErrorNotSupported;
   const cuuint64_t dims[3] = {128, cuuint64_t(a.H), cuuint64_t(a.B) * a.q_tokens};
   const cuuint64_t strides[2] = {128 * 2, cuuint64_t(a.H) * 128 * 2};
@@ -641,13 +627,15 @@ cudaError_t launch_prefill_fast(const CUtensorMap* tmK, const CUtensorMap* tmV,
       tmO = tmQ;   // never used
   }
   const size_t smem = 1024 + kDataBytes + sizeof(PfBars);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr;
+  int dev = 0;
+  cudaError_t ea = cudaGetDevice(&dev);
+  if (ea != cudaSuccess) return ea;
+  ea = static_cast<cudaError_t>(attr.run(dev, [&] {
+    return int(cudaFuncSetAttribute(prefill_tc_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+  }));
+  if (ea != cudaSuccess) return ea;
   PfPlan pl;
   pl.nq = (a.q_tokens + 2 * TQ - 1) / (2 * TQ);
   const int64_t units = int64_t(pl.nq) * a.Hkv * a.B;

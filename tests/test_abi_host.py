@@ -88,6 +88,17 @@ def test_window_calls_reject_bad_arguments_on_host_pools():
     assert L.pa_decode_window_workspace_bytes(p.handle, 1, 1, 4, 0, 0, 0) == 0   # window < 1
 
 
+def test_static_scratch_decode_answers_no_device_on_host_pools():
+    # answered before the scratch array's address is looked up, so no CUDA
+    # call runs (on a host without a GPU it would fail with PA_ERR_CUDA)
+    p = pa.Pool(4, 16, 1, 128, "bf16")
+    L = pa.lib()
+    assert L.pa_decode_static_scratch(p.handle, None, 1, 1, None, 1, None, 1.0, 0, None,
+                                      None) == 8
+    assert L.pa_decode_static_scratch(None, None, 1, 1, None, 1, None, 1.0, 0, None,
+                                      None) == 1
+
+
 def _mirror(oracle, pool, op):
     kind, args = op[0], op[1:]
     if kind == "create":
@@ -243,12 +254,37 @@ def test_random_traces_match_oracle_bit_exactly():
                     src = live[rng.integers(len(live))]
                     p = int(rng.integers(0, o.lengths[src] + 1))
                     _mirror(o, pool, ("share", src, nxt, p)); live.append(nxt); nxt += 1
-                else:
+                elif r < 0.9:
                     s = live.pop(rng.integers(len(live)))
                     _mirror(o, pool, ("release", s))
+                else:
+                    # a rollback of one or two sequences' newest tokens
+                    ss = list(rng.choice(live, size=min(len(live), 2), replace=False))
+                    keep = [int(rng.integers(0, o.lengths[s] + 1)) for s in ss]
+                    for s, k in zip(ss, keep):
+                        o.truncate(int(s), k)
+                    pool.truncate(ss, keep)
             except PoolError:
                 raise
             _same_state(o, pool)
+
+
+def test_truncate_checks_before_changing_anything():
+    pool = pa.Pool(8, 4, 1, 1, "f32")
+    pool.create(0); pool.create(1)
+    pool.plan_append([0, 1], [9, 5])
+    before = (pool.stats(), pool.refcounts(), pool.table(0), pool.table(1))
+    for seqs, lens, code in (([0, 7], [1, 1], 2),      # unknown sequence
+                             ([0, 1], [1, 6], 1),      # beyond the length
+                             ([0, 1], [-1, 0], 1),     # negative
+                             ([1, 1], [2, 1], 1)):     # named twice
+        with pytest.raises(pa.PAError) as e:
+            pool.truncate(seqs, lens)
+        assert e.value.code == code
+        assert (pool.stats(), pool.refcounts(), pool.table(0), pool.table(1)) == before
+    pool.truncate([0, 1], [4, 0])
+    assert pool.table(0) == ([0, 1][:1], 4) and pool.table(1) == ([], 0)
+    assert pool.stats()["free_blocks"] == 7 and pool.validate()
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged256", "prefill"])

@@ -205,6 +205,36 @@ def test_prefill_parity_small(batch, cached, chunk, H, Hkv, splits):
     assert g.pool.get_error() == 0
 
 
+@pytest.mark.parametrize("dtype,H,Hkv,d,bs", [
+    ("f32", 8, 2, 128, 16),      # fp32 pool: the 1e-4 bar
+    ("f32", 4, 4, 64, 8),        # fp32, no grouping, head_dim 64
+    ("bf16", 32, 2, 128, 16),    # group 16 (beyond the tensor-core kernel's 8)
+    ("bf16", 8, 2, 64, 16),      # head_dim 64
+    ("bf16", 6, 3, 80, 4),       # head_dim 80, block 4
+])
+@pytest.mark.parametrize("cached,chunk", [(0, 1), (1, 37), (130, 129)])
+def test_prefill_generic_path(dtype, H, Hkv, d, bs, cached, chunk):
+    # q_tokens > 1 on the CUDA-core kernel: the causal offset rule
+    # j <= kv_len - q_tokens + qt for every query row of the chunk
+    w = workloads.prefill(seed=d * 31 + H + cached + chunk, batch=2, cached=cached,
+                          chunk=chunk, num_heads=H, num_kv_heads=Hkv, head_dim=d,
+                          dtype=dtype, block_size=bs)
+    g = DeviceRun(w).apply(w.setup + w.step)
+    assert g.pool.prefill_path(H) == 0
+    o = OracleRun(w).apply(w.setup + w.step)
+    assert g.slots == o.slots
+    out = g.prefill()
+    q = q64(w)
+    worst = 0.0
+    for i in range(2):
+        rows = o.attention(i, q[i])
+        assert sorted(rows) == list(range(H))
+        for h, ref in rows.items():
+            worst = max(worst, float(np.abs(out[i, :, h] - ref).max()))
+    assert worst <= (TOL_F32 if dtype == "f32" else TOL_PREFILL), worst
+    assert g.pool.get_error() == 0
+
+
 # ---------------------------------------------------------------- full sizes
 def _full(w, kv_heads, sample_seqs, decode=True, partition_tokens=0, check_slots=True):
     g = DeviceRun(w).apply(w.setup + w.step)
@@ -220,8 +250,9 @@ def _full(w, kv_heads, sample_seqs, decode=True, partition_tokens=0, check_slots
 
 
 def test_full_decode32_sampled():
+    # three sequences, every head of every KV head
     w = workloads.decode32()
-    g, o, out, q = _full(w, [0, 5], None)
+    g, o, out, q = _full(w, "all", None)
     worst = rel = 0.0
     for i in (0, 13, 31):
         scale = o.attention(i, q[i], abs_values=True)
@@ -265,16 +296,18 @@ def test_full_splitk128k_sampled():
 
 
 def test_full_prefill_sampled():
+    # KV heads 1 and 6 of sequences 0, 3 and 7: all 512 query rows of each of
+    # their query heads
     w = workloads.prefill()
-    g, o, out, q = _full(w, [1], None, decode=False)
+    g, o, out, q = _full(w, [1, 6], None, decode=False)
     worst = rel = 0.0
-    rows = [0, 1, 127, 128, 255, 511]
-    for i in (0, 7):
+    for i in (0, 3, 7):
         ref = o.attention(i, q[i])
         scale = o.attention(i, q[i], abs_values=True)
+        assert len(ref) == 8
         for h, r in ref.items():
-            worst = max(worst, float(np.abs(out[i, rows, h] - r[rows]).max()))
-            rel = max(rel, scaled_error(out[i, rows, h], r[rows], scale[h][rows]))
+            worst = max(worst, float(np.abs(out[i, :, h] - r).max()))
+            rel = max(rel, scaled_error(out[i, :, h], r, scale[h]))
     assert worst <= TOL_PREFILL, worst
     assert rel <= REL_PREFILL, rel
     assert g.pool.get_error() == 0

@@ -89,6 +89,11 @@ MISTAKES = {
                                       "if True:"),
     "cached blocks not referenced": (C, "PrefixCache.create_cached",
                                      "pool.refs[blk] += 1", "pool.refs[blk] += 0"),
+    "truncate keeps a dropped block": (P, "KVPool.truncate",
+                                       "keep = math.ceil(length / self.block_size)",
+                                       "keep = length // self.block_size + 1"),
+    "truncate frees a shared block": (P, "KVPool.truncate", "if self.refs[blk] == 0:",
+                                      "if self.refs[blk] <= 1:"),
 }
 
 

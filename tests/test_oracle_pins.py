@@ -213,6 +213,68 @@ def test_cow_copies_whole_block_and_only_partial_shared_tails():
     assert cow == [] and pool.tables[2] == [0, 3]      # full block: no copy
 
 
+def _rename(pool, old, new):
+    pool.tables[new] = pool.tables.pop(old)
+    pool.lengths[new] = pool.lengths.pop(old)
+
+
+def test_truncate_equals_share_prefix_then_release():
+    # truncate(s, n) is the pages' share_prefix of the first n tokens into a
+    # new sequence followed by release of s: same tables, refcounts, free
+    # blocks, statistics and next allocations, on random traces with sharing
+    rng = np.random.default_rng(23)
+    for trial in range(60):
+        nb, bs = 48, int(rng.integers(1, 7))
+        order = rng.permutation(nb)
+        a, b = (KVPool(nb, bs, allocation_order=order, store_heads=None) for _ in range(2))
+        for p in (a, b):
+            p.create(0)
+        n0 = int(rng.integers(1, 30))
+        a.append(0, n0); b.append(0, n0)
+        for child in (1, 2):                       # sharers of various prefixes
+            src = int(rng.integers(0, child))
+            pre = int(rng.integers(0, a.lengths[src] + 1))
+            a.share_prefix(src, child, pre); b.share_prefix(src, child, pre)
+            k = int(rng.integers(0, 9))
+            a.append(child, k); b.append(child, k)
+        victim = int(rng.integers(0, 3))
+        n = int(rng.integers(0, a.lengths[victim] + 1))
+        a.truncate(victim, n)
+        b.share_prefix(victim, "tmp", n)
+        b.release(victim)
+        _rename(b, "tmp", victim)
+        assert a.tables == b.tables and a.lengths == b.lengths and a.refs == b.refs
+        assert a.free_blocks == b.free_blocks and a.snapshot() == b.snapshot()
+        a.validate(); b.validate()
+        grow = int(rng.integers(0, 2 * bs + 1))   # the next allocations agree too
+        if a.blocks_needed(victim, grow) <= a.free_blocks:
+            assert a.append(victim, grow) == b.append(victim, grow)
+            assert a.tables == b.tables and a.refs == b.refs
+
+
+def test_truncate_special_cases():
+    pool = KVPool(8, 4, store_heads=None)
+    pool.create(0); pool.append(0, 10)             # blocks 0, 1, 2 (2 tokens in 2)
+    pool.truncate(0, 10)                           # to its own length: nothing changes
+    assert pool.tables[0] == [0, 1, 2] and pool.free_blocks == 5
+    pool.truncate(0, 8)                            # a whole block dropped, freed
+    assert pool.tables[0] == [0, 1] and pool.refs[2] == 0 and pool.free_blocks == 6
+    pool.truncate(0, 5)                            # partial block kept
+    assert pool.tables[0] == [0, 1] and pool.lengths[0] == 5
+    pool.share_prefix(0, 1, 5)
+    pool.truncate(0, 0)                            # shared blocks survive their sharer
+    assert pool.tables[0] == [] and pool.refs[:2] == [1, 1] and pool.free_blocks == 6
+    slots, cow = pool.append(1, 1)                 # sole holder now: no copy-on-write
+    assert cow == [] and slots == [1 * 4 + 1]
+    with pytest.raises(PoolError):
+        pool.truncate(1, 7)                        # beyond the length
+    with pytest.raises(PoolError):
+        pool.truncate(1, -1)
+    with pytest.raises(PoolError):
+        pool.truncate(5, 0)                        # unknown sequence
+    pool.validate()
+
+
 # ---------------------------------------------------------------------------
 # Attention: "docs.rs ferrum-kv 0.4.0 src/attention.rs" unit tests, closed forms
 # ---------------------------------------------------------------------------
@@ -446,9 +508,12 @@ def test_random_op_fuzz_keeps_invariants():
                 src = live[rng.integers(len(live))]
                 pool.share_prefix(src, nxt, int(rng.integers(0, pool.lengths[src] + 1)))
                 live.append(nxt); nxt += 1
-            else:
+            elif r < 0.9:
                 s = live.pop(rng.integers(len(live)))
                 pool.release(s)
+            else:
+                s = live[rng.integers(len(live))]
+                pool.truncate(s, int(rng.integers(0, pool.lengths[s] + 1)))
         except PoolExhausted:
             pass
         pool.validate()

@@ -192,22 +192,18 @@ def splitk128k(seed: int = seed_for(4)) -> Workload:
 
 
 def prefill(seed: int = seed_for(5), batch: int = 8, cached: int = 4096,
-            chunk: int = 512, num_heads: int = 32, num_kv_heads: int = 8) -> Workload:
+            chunk: int = 512, num_heads: int = 32, num_kv_heads: int = 8,
+            head_dim: int = 128, dtype: str = "bf16", block_size: int = 16) -> Workload:
     """Chunked prefill: cached tokens, then a chunk appended and attended causally."""
-    bs = 16
+    bs = block_size
     ops = [("create", b) for b in range(batch)]
     ops += [("append", b, cached) for b in range(batch) if cached > 0]
     setup = _script(ops)
     step = [Op("append", (b, chunk), len(ops) + b) for b in range(batch)]
     nb = batch * (-(-(cached + chunk) // bs)) + 64
-    return Workload("prefill", nb, bs, num_heads, num_kv_heads, 128, "bf16", seed,
+    return Workload("prefill", nb, bs, num_heads, num_kv_heads, head_dim, dtype, seed,
                     permutation(nb, seed), setup=setup, step=step,
                     decode_seqs=list(range(batch)), q_tokens=chunk)
-
-
-def scaled(w_fn, **kw) -> Workload:
-    """A smaller instance of a workload family (for parity at oracle-friendly sizes)."""
-    return w_fn(**kw)
 
 
 def custom_decode(name: str, lens, num_heads: int, num_kv_heads: int, head_dim: int,
