@@ -34,7 +34,6 @@ import math
 import os
 import statistics
 import sys
-import threading
 import time
 
 import numpy as np
@@ -78,66 +77,114 @@ def profiled_traffic(kernel_file, workload):
     return d.get("dram_bytes_per_launch")
 
 
-class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML in a thread."""
-    REASONS = {
-        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
-        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
-        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
-        0x100: "display_clock_setting",
-    }
+SAMPLER = None                # the bench run's clock sampler (main)
 
-    def __init__(self, cuda_index, period=0.005):
-        self.samples, self.reasons, self.ok = [], set(), False
-        self.period = period
+CLOCK_REASONS = {
+    0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+    0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+def _clock_sampler_main(uuid, index, period, conn):
+    """Child process: after 'begin', samples (time, SM MHz, reason bits)
+    every `period` seconds until 'end', then sends the samples back."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
         try:
-            import pynvml
-            import torch
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            try:
-                uuid = str(torch.cuda.get_device_properties(cuda_index).uuid)
-                self.h = pynvml.nvmlDeviceGetHandleByUUID(
-                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
-            except Exception:
-                self.h = pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-            self.ok = True
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
         except Exception:
-            self.max_mhz = None
-        self._stop = threading.Event()
-        self._t = None
-
-    def _run(self):
-        nv = self.nv
-        while not self._stop.is_set():
+            h = pynvml.nvmlDeviceGetHandleByIndex(index)
+        conn.send(("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)))
+    except Exception as e:            # no NVML: report it, sample nothing
+        conn.send(("error", repr(e)))
+        return
+    while True:
+        msg = conn.recv()
+        if msg == "quit":
+            return
+        buf = []
+        first = True
+        while not conn.poll():
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit and bit != 0x1:
-                        self.reasons.add(name)
+                buf.append((time.time(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                            pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
             except Exception:
                 pass
-            time.sleep(self.period)
+            if first:
+                conn.send("sampling")      # the window opens after the first sample
+                first = False
+            time.sleep(period)
+        conn.recv()                    # 'end'
+        conn.send(buf)
+
+
+class ClockSampler:
+    """SM clock and clock-event reasons sampled through NVML by a separate
+    process (no contention with the launch loop for the interpreter lock).
+    ``with sampler.window() as w:`` brackets a timed region; ``w.summary()``
+    then covers only the samples taken between its two time stamps."""
+
+    def __init__(self, cuda_index, period=0.0002):
+        import multiprocessing as mp
+        import torch
+        self.max_mhz, self.error = None, None
+        uuid = str(torch.cuda.get_device_properties(cuda_index).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        ctx = mp.get_context("spawn")
+        self.conn, child = ctx.Pipe()
+        self.proc = ctx.Process(target=_clock_sampler_main, args=(uuid, cuda_index, period, child),
+                                daemon=True)
+        self.proc.start()
+        try:
+            kind, val = self.conn.recv() if self.conn.poll(120) else ("error", "no answer")
+        except (EOFError, OSError) as e:
+            kind, val = "error", repr(e)
+        if kind == "max":
+            self.max_mhz = val
+        else:
+            self.error = val
+
+    def window(self):
+        return _ClockWindow(self)
+
+    def close(self):
+        if self.proc.is_alive():
+            try:
+                self.conn.send("quit")
+            except Exception:
+                pass
+            self.proc.join(timeout=5)
+
+
+class _ClockWindow:
+    def __init__(self, sampler):
+        self.s, self.samples, self.t0, self.t1 = sampler, [], None, None
 
     def __enter__(self):
-        if self.ok:
-            self._t = threading.Thread(target=self._run, daemon=True)
-            self._t.start()
+        if self.s.error is None:
+            self.s.conn.send("begin")
+            self.s.conn.recv()         # 'sampling': the sampler is running
+        self.t0 = time.time()
         return self
 
     def __exit__(self, *a):
-        if self._t:
-            self._stop.set()
-            self._t.join()
+        self.t1 = time.time()
+        if self.s.error is None:
+            time.sleep(0.001)
+            self.s.conn.send("end")
+            self.samples = self.s.conn.recv()
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                    "samples": 0}
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        inside = [(t, mhz, r) for t, mhz, r in self.samples if self.t0 <= t <= self.t1]
+        reasons = sorted({name for _, _, r in inside for bit, name in CLOCK_REASONS.items()
+                          if r & bit})
+        out = {"sm_mhz": float(statistics.median(m for _, m, _ in inside)) if inside else None,
+               "sm_max_mhz": self.s.max_mhz, "reasons": reasons, "samples": len(inside)}
+        if self.s.error:
+            out["error"] = self.s.error
+        return out
 
 
 def oracle_threads():
@@ -278,11 +325,11 @@ def default_seed(config):
 
 
 def run_workload(args, dist, config, kv="bf16", win=0, sinks=0, *, steps, min_ms=0.0,
-                 clock_period=0.001, cpu=False, memo=None):
+                 cpu=False, memo=None):
     """Bring one workload up, time its step on the device and end to end.
 
     steps: timed steps; with min_ms > 0 the count grows until the timed region
-    lasts about min_ms (long enough for the clock sampler to see the run)."""
+    lasts about min_ms."""
     import torch
     device = torch.device("cuda", dist.local)
     builder = workloads.ALL[config]
@@ -357,7 +404,7 @@ def run_workload(args, dist, config, kv="bf16", win=0, sinks=0, *, steps, min_ms
     launches["n"] = 0
     dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device(), clock_period) as clk:
+    with SAMPLER.window() as clk:
         t_start.record(stream)
         for i in range(K):
             step(evs[i])
@@ -447,18 +494,21 @@ def run_workload(args, dist, config, kv="bf16", win=0, sinks=0, *, steps, min_ms
 
 def time_append(S, stream, cuda_index, n_app=300):
     """reshape_and_cache of the step's rows at their planned slots, one launch
-    at a time with L2 flushed (a 256 MiB write) between launches."""
+    at a time with L2 flushed (a 256 MiB read) between launches."""
     import torch
     pool = S.pool
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=S.device)
+    # the flush reads a buffer larger than L2, leaving it full of clean lines
+    # (a write flush would leave dirty lines for the timed kernel to evict)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=S.device)
+    sink = torch.empty(1, dtype=torch.float32, device=S.device)
     for _ in range(3):
         pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(n_app)]
     torch.cuda.synchronize()
-    with ClockSampler(cuda_index, 0.0005) as clk:
+    with SAMPLER.window() as clk:
         for a, b in evs:
-            flush.zero_()
+            torch.sum(flush, dim=0, keepdim=True, out=sink)
             a.record(stream)
             pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
             b.record(stream)
@@ -474,7 +524,7 @@ def time_append(S, stream, cuda_index, n_app=300):
                          "frac": round(gbs / hbm, 4),
                          "traffic": profiled_traffic("kv_write.cu", "prefill_append"),
                          "peak_source": f"{peak_kind} hbm_gbs"},
-            "l2": "flushed between launches (256 MiB write, untimed)",
+            "l2": "flushed between launches (a 256 MiB read, untimed)",
             "clocks": clk.summary()}
 
 
@@ -825,14 +875,16 @@ def main():
             print(json.dumps(res), flush=True)
         return
     dist.init("nccl")
+    global SAMPLER
     try:
         import torch
         torch.cuda.set_device(dist.local)
+        SAMPLER = ClockSampler(dist.local)
         memo = {}
         # the headline: exactly --steps timed steps; the clock sampler runs fast
         # enough to see a few milliseconds
         res = run_workload(args, dist, args.config, args.kv, args.window, args.sinks,
-                           steps=args.steps, clock_period=0.0002,
+                           steps=args.steps,
                            cpu=not args.no_cpu_baseline, memo=memo)
         default_run = (args.config == "decode32" and args.kv == "bf16" and not args.window)
         extras = args.configs == "all" or (args.configs == "auto" and default_run
@@ -842,6 +894,8 @@ def main():
         if dist.rank == 0:
             print(json.dumps(res), flush=True)
     finally:
+        if SAMPLER is not None:
+            SAMPLER.close()
         dist.close()
 
 
@@ -860,7 +914,7 @@ def run_extras(args, dist, memo):
             "clocks", "frac_of_peak")
     for name, config, kv in EXTRAS:
         r = run_workload(args, dist, config, kv, steps=args.steps, min_ms=100.0,
-                         clock_period=0.001, memo=memo if config == "decode32" else None)
+                         memo=memo if config == "decode32" else None)
         out[name] = {k: r[k] for k in keep if k in r}
         if r.get("append"):
             out["prefill_append"] = {"workload": "prefill chunk append: 8 x 512 tokens, 8 KV "

@@ -115,6 +115,11 @@ cudaError_t launch_reshape_and_cache_q8(const void* key, const void* value, void
 // {128 bytes, 33 rows, NB * Hkv}), dequantising in the kernel.
 cudaError_t launch_decode_q8(const CUtensorMap* tmR, const DecodeArgs& a, bool fp8,
                              cudaStream_t stream);
+// The same decode on tcgen05 tensor cores straight from the codes: tmRK maps
+// the records with a {128, 16, 1} box (K codes), tmRV with a {128, 17, 1}
+// box (V codes and the two scale rows, read at row 16).
+cudaError_t launch_decode_q8tc(const CUtensorMap* tmRK, const CUtensorMap* tmRV,
+                               const DecodeArgs& a, bool fp8, cudaStream_t stream);
 // Scratch for the longest-first order when the grid spans several waves.
 bool decode_wants_order(int32_t B, int32_t Hkv, int32_t NP, int sms);
 size_t order_workspace_bytes(int32_t B);

@@ -56,6 +56,8 @@ struct pa_pool {
   int32_t* d_err = nullptr;
   bool tmap_ok = false;
   CUtensorMap tmK, tmV;
+  // int8 / FP8 pools: the records with a K-codes box and a V-codes + scales box
+  CUtensorMap tmRK, tmRV;
   // tensor-core prefill: key-split scratch for one wave (one slot per SM)
   float* split_o = nullptr;
   float* split_ml = nullptr;
@@ -122,19 +124,27 @@ bool make_pool_map(CUtensorMap* map, void* base, const pa_pool* p) {
 }
 
 // int8 pools: the packed records viewed as {128 bytes, 33 rows, NB * Hkv};
-// one box = one whole record.
-bool make_record_map(CUtensorMap* map, void* base, const pa_pool* p) {
+// one box = `rows` rows of a record (33: the whole record).
+bool make_record_map(CUtensorMap* map, void* base, const pa_pool* p, uint32_t rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {128, pa::kQ8RecordBytes / 128,
                               cuuint64_t(p->num_blocks) * p->num_kv_heads};
   const cuuint64_t strides[2] = {128, pa::kQ8RecordBytes};
-  const cuuint32_t box[3] = {128, pa::kQ8RecordBytes / 128, 1};
+  const cuuint32_t box[3] = {128, rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
+}
+
+// All three record maps of an int8 / FP8 pool (or layer): the whole record,
+// the K codes (rows 0-15), the V codes with the scale row (rows 16-32).
+bool make_record_maps(pa_pool* p) {
+  return make_record_map(&p->tmK, p->k_cache, p, pa::kQ8RecordBytes / 128) &&
+         make_record_map(&p->tmRK, p->k_cache, p, 16) &&
+         make_record_map(&p->tmRV, p->k_cache, p, 17);
 }
 
 // Blocks a decode walks per sequence at most: all of them, or with a sink +
@@ -241,7 +251,7 @@ static pa_status create_pool(int32_t num_blocks, int32_t block_size, int32_t num
     if (kv_dtype == PA_BF16 && head_dim == 128 && block_size == 16)
       p->tmap_ok = make_pool_map(&p->tmK, k_cache, p) &&
                    make_pool_map(&p->tmV, v_cache, p);
-    if (is_q8(kv_dtype) && !make_record_map(&p->tmK, k_cache, p)) {
+    if (is_q8(kv_dtype) && !make_record_maps(p)) {
       cudaFree(p->d_err);
       delete p;
       return PA_ERR_CUDA;
@@ -296,7 +306,7 @@ static pa_status add_layer_views(pa_pool* p, int32_t num_layers) {
     v->k_cache = static_cast<char*>(p->k_cache) + l * p->layer_bytes;
     v->v_cache = p->v_cache ? static_cast<char*>(p->v_cache) + l * p->layer_bytes : nullptr;
     if (is_q8(p->dtype)) {
-      if (!make_record_map(&v->tmK, v->k_cache, v)) return PA_ERR_CUDA;
+      if (!make_record_maps(v)) return PA_ERR_CUDA;
     } else if (p->tmap_ok) {
       v->tmap_ok = make_pool_map(&v->tmK, v->k_cache, v) && make_pool_map(&v->tmV, v->v_cache, v);
       if (!v->tmap_ok) return PA_ERR_CUDA;
@@ -703,8 +713,8 @@ static pa_status decode_fast(pa_pool* p, const void* q, int32_t B, int32_t H,
   a.window = window;
   a.sinks = sinks;
   if (is_q8(p->dtype))
-    return cuda_status(pa::launch_decode_q8(&p->tmK, a, p->dtype == PA_FP8,
-                                            static_cast<cudaStream_t>(stream)));
+    return cuda_status(pa::launch_decode_q8tc(&p->tmRK, &p->tmRV, a, p->dtype == PA_FP8,
+                                              static_cast<cudaStream_t>(stream)));
   return cuda_status(pa::launch_decode_fast(&p->tmK, &p->tmV, a, p->sms,
                                             static_cast<cudaStream_t>(stream)));
 }

@@ -103,7 +103,7 @@ def test_q8_append_special_rows():
 LENS = [1, 15, 16, 17, 33, 100, 255, 256, 513, 1000, 0, 2]
 
 
-@pytest.mark.parametrize("H,Hkv", [(32, 8), (64, 8), (8, 8), (16, 8), (8, 1)])
+@pytest.mark.parametrize("H,Hkv", [(32, 8), (64, 8), (8, 8), (16, 8), (8, 1), (24, 8), (48, 8)])
 @pytest.mark.parametrize("part", [0, 16, 64, 256])
 def test_q8_decode_parity(H, Hkv, part):
     w = _small(LENS, H, Hkv, seed=H * 5 + Hkv + part)
