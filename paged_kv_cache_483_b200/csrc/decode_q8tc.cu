@@ -1,5 +1,5 @@
 // Paged decode attention over an int8 or FP8 (E4M3) KV pool on the 5th-
-// generation tensor cores: head_dim 128, block_size 16, GQA group G <= 8.
+// generation tensor cores: head_dim 128, block_size 16, GQA group G <= 4.
 // One CTA per (partition, KV head, sequence).
 //
 // What it computes: the decode of "docs.rs ferrum-kv 0.4.0 src/attention.rs"
@@ -14,8 +14,10 @@
 // [16 tokens][128] with token t's 16-byte chunks pre-swizzled (chunk c at
 // c ^ (t & 7)), V codes [128 d][16 tokens], 16 K scales, 16 V scales.  Work
 // goes in groups of eight blocks (128 keys):
-//  * warp 0 copies each block with two TMA boxes: the K codes (16 rows of
-//    128 B) into the group's K tile, where eight blocks' K rows form one
+//  * warp 0 copies each block with two TMA boxes (lane i of the warp copies
+//    block i of a group: one thread's copy-issue rate is too low for two
+//    boxes per block): the K codes (16 rows of 128 B) into the group's K
+//    tile, where eight blocks' K rows form one
 //    128 x 128 operand in the 128-byte-swizzle K-major layout (the record's
 //    own swizzle is that layout), and the V codes + scales (17 rows) into the
 //    group's V tile, where block b's V rows sit 2176 B after block b - 1:
@@ -25,14 +27,21 @@
 //    S^T[128 keys x N] = K Q~^T and, once the softmax has written P~,
 //    O_g^T[128 d x N] = V^T P~^T, both straight from the codes in shared
 //    memory, fp32 (s32) accumulators in tensor memory;
-//  * warps 2-5 (one thread per key of the group, and per d row in the fold)
-//    read S, form the scores, take the group's max per head (warp max, then
-//    across the four warps through shared memory), write P, and fold the
-//    previous group's O_g into fp32 registers: o = o * alpha + O_g * unit,
-//    alpha = 2^(m_old - m_new) -- the exact online-softmax recurrence, no
-//    stale maximum, no rescale of tensor memory.
-// Q and P enter the 8-bit MMA as sums of 8-bit terms (columns n = term * G +
-// head of the B operands):
+//  * two softmax warpgroups take alternate groups (one thread per key of the
+//    group, and per d row in the fold): each reads S, forms the scores, takes
+//    the group's max per head (warp max, then across its four warps through
+//    shared memory), writes P, and folds the group's O_g into fp32 registers:
+//    o = o * alpha + O_g * unit, alpha = 2^(m_old - m_new) -- the exact
+//    online-softmax recurrence, no stale maximum, no rescale of tensor
+//    memory; the two warpgroups' (m, l, o) are merged at the end;
+//  * K tiles (two) are handed back when their QK completes, V tiles (four)
+//    when their PV does; S, P and O have four buffers each, so QK runs up to
+//    three groups ahead of the softmax.
+// Groups of more than 4 heads go to the warp-level kernel (decode_q8.cu):
+// the per-byte softmax work here grows with the group, while its 8-column
+// MMA tiles are full at G = 8.
+// Q and P enter the 8-bit MMA as sums of 8-bit terms (columns n = term * Gp +
+// head of the B operands, Gp = G rounded up to a power of two):
 //  * FP8: Q / sq (sq a power of two with max |Q / sq| <= 448) as three E4M3
 //    terms q1 + q2 / 16 + q3 / 256, each the E4M3 rounding of the remainder of
 //    the previous ones times 16 (relative error ~2^-12); P as three E4M3 terms
@@ -58,29 +67,30 @@ namespace pa {
 
 namespace {
 
-// Threads: a producer warp, an MMA warp and kWG softmax warpgroups (two when
-// G <= 4, which leaves the registers for it at two CTAs per SM; one above).
-__host__ __device__ constexpr int q8tc_wgs(int gp) { return gp <= 4 ? 2 : 1; }
+// Threads: a producer warp, an MMA warp and two softmax warpgroups that take
+// alternate groups.
+constexpr int kWG = 2;
 constexpr int kGroupBlocks = 8;          // 128 keys per group = the MMA's M
 constexpr uint32_t kKTile = kGroupBlocks * 2048;       // K codes of a group
 constexpr uint32_t kVSlot = 2176;                     // one block's V codes + scales
 constexpr uint32_t kVTile = kGroupBlocks * kVSlot;    // 17408
 constexpr int kKStages = 2;              // K tiles: free again once their QK is done
 constexpr int kMaxVStages = 4;           // V tiles: free again once their PV is done
-constexpr uint32_t kTmemCols = 128;      // S x 2, O x 2, 32 columns each
+constexpr int kBufs = 4;                 // S, P and O buffers (QK runs up to 3 groups ahead)
+constexpr uint32_t kTmemCols = 256;      // S x 4, O x 4, 32 columns each
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct TcTail {
   uint64_t kfull[kKStages], kempty[kKStages];
   uint64_t vfull[kMaxVStages], vempty[kMaxVStages];
-  uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t s_full[kBufs], p_full[kBufs], o_full[kBufs];
   uint64_t q_ready;
   uint32_t tmem_base;
   int badmask[kMaxVStages];  // per V stage: bit i = block i of the group missing or unusable
   int any_bad;
   int abort;
   float qs[8];         // per head: sq * scale_log2
-  float red[2][4][10]; // per group parity, softmax warp: G maxima, V-scale max, ok flag
+  float red[2][2][4][10];  // per iteration parity, warpgroup, warp: head maxima, V-scale max, ok
 };
 
 // Columns of the B operands (Q~ and P~): T terms of kGp heads, padded to the
@@ -89,18 +99,16 @@ __host__ __device__ constexpr int q8tc_cols(bool fp8, int gp) {
   return ((gp * (fp8 ? 3 : 2) + 15) / 16) * 16;
 }
 
-// V stages: four at 16 columns, three at 32 (two CTAs per SM either way).
-__host__ __device__ constexpr int q8tc_vstages(int N) { return N <= 16 ? 4 : 3; }
 
 // Shared-memory layout of a CTA for N columns (a multiple of 16) and vst V
 // stages: K tiles [2][128 keys x 128 B] | V tiles [vst][8 blocks x 2176 B] |
-// Q terms (N rows of 128 B, swizzled) | P terms x 2 (N rows of 128 keys, core
+// Q terms (N rows of 128 B, swizzled) | P terms x 4 (N rows of 128 keys, core
 // matrices) | tail.
 __host__ __device__ constexpr uint32_t v_off() { return uint32_t(kKStages) * kKTile; }
 __host__ __device__ constexpr uint32_t q_off(int vst) { return v_off() + uint32_t(vst) * kVTile; }
 __host__ __device__ constexpr uint32_t p_off(int vst, int N) { return q_off(vst) + uint32_t(N) * 128; }
 __host__ __device__ constexpr uint32_t tail_off(int vst, int N) {
-  return p_off(vst, N) + 2u * uint32_t(N / 8) * 1024u;
+  return p_off(vst, N) + uint32_t(kBufs) * uint32_t(N / 8) * 1024u;
 }
 
 // 128-byte-swizzle-free K-major descriptor: core matrices of 8 rows x 16 B,
@@ -184,6 +192,44 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
     tmem_ld32(taddr, r);
 }
 
+// Columns [c, c + 4) of each of T terms (term k at column addr + k * stride)
+// of this thread's TMEM lane, then one wait for all of them.
+template <int T>
+__device__ __forceinline__ void tmem_ld_terms(uint32_t addr, uint32_t stride,
+                                              uint32_t (&r)[3][4]) {
+  if constexpr (T == 3)
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%12];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4,%5,%6,%7}, [%13];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8,%9,%10,%11}, [%14];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[1][0]),
+          "=r"(r[1][1]), "=r"(r[1][2]), "=r"(r[1][3]), "=r"(r[2][0]), "=r"(r[2][1]),
+          "=r"(r[2][2]), "=r"(r[2][3])
+        : "r"(addr), "r"(addr + stride), "r"(addr + 2 * stride)
+        : "memory");
+  else
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%8];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4,%5,%6,%7}, [%9];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[1][0]),
+          "=r"(r[1][1]), "=r"(r[1][2]), "=r"(r[1][3])
+        : "r"(addr), "r"(addr + stride)
+        : "memory");
+}
+
+// The value a head's T accumulator columns stand for: FP8 t0 + t1 / 16 +
+// t2 / 256 (f32 sums), int8 t0 + t1 / 254 (s32 sums).
+template <bool kFp8>
+__device__ __forceinline__ float terms_value(const uint32_t (&r)[3][4], int h) {
+  if constexpr (kFp8)
+    return __uint_as_float(r[0][h]) + __uint_as_float(r[1][h]) * 0.0625f +
+           __uint_as_float(r[2][h]) * 0.00390625f;
+  else
+    return float(int32_t(r[0][h])) + float(int32_t(r[1][h])) * (1.f / 254.f);
+}
+
 __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, TcTail* tail,
                                              int32_t* err) {
   if (mbar_wait(bar, parity)) return true;
@@ -194,7 +240,7 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, TcT
 
 }  // namespace
 
-template <bool kFp8, int kGp, int kWG>
+template <bool kFp8, int kGp>
 __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
     const __grid_constant__ CUtensorMap tmRK, const __grid_constant__ CUtensorMap tmRV,
     const DecodeArgs p, float scale_log2) {
@@ -202,7 +248,8 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
   // n = term * kGp + head, so every register index is a compile-time one
   constexpr int T = kFp8 ? 3 : 2;          // 8-bit terms of Q and of P
   constexpr int N = q8tc_cols(kFp8, kGp);
-  constexpr int kVStages = q8tc_vstages(N);
+  constexpr int kVStages = kMaxVStages;
+  static_assert(N == 16, "G <= 4: 16 columns");
   extern __shared__ uint8_t tc_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(tc_raw) + 1023) & ~uintptr_t(1023));
@@ -241,7 +288,7 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
       mbar_init(&tail->vempty[s], 1);
       tail->badmask[s] = 0;
     }
-    for (int x = 0; x < 2; ++x) {
+    for (int x = 0; x < kBufs; ++x) {
       mbar_init(&tail->s_full[x], 1);
       mbar_init(&tail->p_full[x], 128);
       mbar_init(&tail->o_full[x], 1);
@@ -346,8 +393,8 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
       uint32_t polls = 0;
       while (ok && npv < ngroups) {
         bool progressed = false;
-        if (nq < ngroups && nq <= npv + 1) {
-          const int s = nq % kKStages, x = nq & 1;
+        if (nq < ngroups && nq <= npv + kBufs - 1) {
+          const int s = nq % kKStages, x = nq % kBufs;
           if (mbar_try_wait(&tail->kfull[s], (nq / kKStages) & 1)) {
             tc_fence_after();
             const uint32_t kb = smem_u32(smem + s * kKTile);
@@ -362,14 +409,14 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
           }
         }
         if (npv < nq) {
-          const int s = npv % kVStages, x = npv & 1;
-          if (mbar_try_wait(&tail->p_full[x], (npv >> 1) & 1)) {
+          const int s = npv % kVStages, x = npv % kBufs;
+          if (mbar_try_wait(&tail->p_full[x], (npv / kBufs) & 1)) {
             tc_fence_after();
             const uint32_t vb = smem_u32(vtile + s * kVTile);
             const uint32_t pb = smem_u32(pterm + x * p_bytes);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)             // O_x = V^T(npv) P~(npv)^T
-              umma_8bit<kFp8>(tbase + 64 + 32 * x,
+              umma_8bit<kFp8>(tbase + 32 * kBufs + 32 * x,
                               desc_kmajor_plain(vb + 2 * kk * kVSlot, kVSlot, 128),
                               desc_kmajor_plain(pb + 256 * kk, 128, 1024), idesc,
                               kk > 0 ? 1u : 0u);
@@ -391,8 +438,9 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
     }
   } else {
     // ------------------------------------------- softmax, fold, epilogue
-    // kWG warpgroups; warpgroup wg takes groups wg, wg + kWG, ... (with two,
-    // one group's softmax runs while the other's is waiting on its MMAs)
+    // Two warpgroups: warpgroup wg takes groups wg, wg + 2, ... (one group's
+    // softmax runs while the other's waits on its MMAs).
+    constexpr int kH = kGp;                           // heads per thread
     const int wg = (warp - 2) >> 2;
     const int sw = (warp - 2) & 3;                    // softmax warp of its warpgroup
     const int quarter = warp & 3;                     // its TMEM lane quarter
@@ -406,7 +454,7 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
     // padding columns are never read, but the MMA reads their bytes
     for (int n = st >> 5; n < N; n += kSm / 32)
       reinterpret_cast<uint32_t*>(qterm + (n >> 3) * 1024 + (n & 7) * 128)[lane] = 0u;
-    for (uint32_t o = st * 16; o < 2 * p_bytes; o += kSm * 16)
+    for (uint32_t o = st * 16; o < kBufs * p_bytes; o += kSm * 16)
       *reinterpret_cast<uint4*>(pterm + o) = make_uint4(0u, 0u, 0u, 0u);
     named_bar_sync(kBarAll, kSm);                     // zeros before the terms
     // ---- Q terms, one warp per head: lane covers d = 4 lane .. 4 lane + 3
@@ -446,23 +494,22 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
     fence_proxy_async_smem();
     named_bar_sync(kBarAll, kSm);                     // Q~ and qs[] of every head
     mbar_arrive(&tail->q_ready);
-    float qs[kGp];
+    float qs[kH];
 #pragma unroll
-    for (int h = 0; h < kGp; ++h) qs[h] = h < G ? tail->qs[h] : 0.f;
+    for (int h = 0; h < kH; ++h) qs[h] = h < G ? tail->qs[h] : 0.f;
 
-    float m[kGp], l[kGp], o[kGp], alpha_prev[kGp], unit_prev = 0.f;
+    float m[kH], l[kH], o[kH];
 #pragma unroll
-    for (int h = 0; h < kGp; ++h) {
+    for (int h = 0; h < kH; ++h) {
       m[h] = -INFINITY;
       l[h] = 0.f;
       o[h] = 0.f;
-      alpha_prev[h] = 0.f;
     }
     // fold group jf's O_g into the registers (this thread's d row = tg):
     // o = o * alpha + O_g * unit; false if its wait gave up
-    auto fold = [&](int jf, const float (&alpha)[kGp], float unit_f) -> bool {
-      const int xf = jf & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&tail->o_full[xf], (jf >> 1) & 1))) {
+    auto fold = [&](int jf, const float (&alpha)[kH], float unit_f) -> bool {
+      const int xf = jf % kBufs;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tail->o_full[xf], (jf / kBufs) & 1))) {
         if (lane == 0) {
           raise_err(p.err, PA_DEVERR_TIMEOUT);
           atomicExch(&tail->abort, 1);
@@ -470,36 +517,28 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
         return false;
       }
       tc_fence_after();
-      uint32_t v[N];
-      tmem_ld_cols<N>(tbase + lane_off + 64 + 32 * xf, v);
+      uint32_t v[3][4];
+      tmem_ld_terms<T>(tbase + lane_off + 32 * kBufs + 32 * xf, kGp, v);
 #pragma unroll
-      for (int h = 0; h < kGp; ++h) {
-        if (h < G) {
-          float g;
-          if constexpr (kFp8)
-            g = __uint_as_float(v[h]) + __uint_as_float(v[kGp + h]) * 0.0625f +
-                __uint_as_float(v[2 * kGp + h]) * 0.00390625f;
-          else
-            g = float(int32_t(v[h])) + float(int32_t(v[kGp + h])) * (1.f / 254.f);
-          o[h] = fmaf(o[h], alpha[h], g * unit_f);
-        }
-      }
+      for (int h = 0; h < kH; ++h)
+        if (h < G) o[h] = fmaf(o[h], alpha[h], terms_value<kFp8>(v, h) * unit_f);
       return true;
     };
 
     // The four warps of a warpgroup leave the loop together: each group's
     // exchange carries every warp's "all waits succeeded" flag.
     bool ok = true, fold_ok = true;
-    int jprev = -1;
+    int it = -1;
     for (int j = wg; j < ngroups; j += kWG) {
-      const int x = j & 1, s = j % kVStages;
+      ++it;
+      const int x = j % kBufs, s = j % kVStages;
       // S(j), and the group's V tile (its scales, its block mask)
       const bool mine = fold_ok &&
-                        __all_sync(0xffffffffu, mbar_wait(&tail->s_full[x], (j >> 1) & 1) &&
+                        __all_sync(0xffffffffu, mbar_wait(&tail->s_full[x], (j / kBufs) & 1) &&
                                                     mbar_wait(&tail->vfull[s], (j / kVStages) & 1));
       tc_fence_after();
-      uint32_t raw[N];
-      if (mine) tmem_ld_cols<N>(tbase + lane_off + 32 * x, raw);
+      uint32_t raw[3][4];
+      if (mine) tmem_ld_terms<T>(tbase + lane_off + 32 * x, kGp, raw);
       const int mask = tail->badmask[s];
       const int i = tg >> 4, r = tg & 15;             // block of the group, key in the block
       const bool present = !((mask >> i) & 1);
@@ -509,23 +548,16 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
       const uint8_t* vs = vt + i * kVSlot;
       const float kscale = live ? reinterpret_cast<const float*>(vs + 2048)[r] : 0.f;
       const float vscale = live ? reinterpret_cast<const float*>(vs + 2112)[r] : 0.f;
-      float sc[kGp];
+      float sc[kH];
 #pragma unroll
-      for (int h = 0; h < kGp; ++h) {
-        float raw_s = 0.f;
-        if (h < G && live) {
-          if constexpr (kFp8)
-            raw_s = __uint_as_float(raw[h]) + __uint_as_float(raw[kGp + h]) * 0.0625f +
-                    __uint_as_float(raw[2 * kGp + h]) * 0.00390625f;
-          else
-            raw_s = float(int32_t(raw[h])) + float(int32_t(raw[kGp + h])) * (1.f / 254.f);
-        }
-        sc[h] = (live && h < G) ? raw_s * kscale * qs[h] : -INFINITY;
-      }
+      for (int h = 0; h < kH; ++h)
+        sc[h] = (live && h < G) ? terms_value<kFp8>(raw, h) * kscale * qs[h] : -INFINITY;
       // group maxima per head and of the live V scales: warp, then the 4 warps
-      float* red = tail->red[x][sw];
+      // exchange buffers alternate by this warpgroup's iteration, so a warp
+      // ahead by one group never writes the slot another is still reading
+      float* red = tail->red[it & 1][wg][sw];
 #pragma unroll
-      for (int h = 0; h < kGp; ++h) {
+      for (int h = 0; h < kH; ++h) {
         if (h < G) {
           const float mx = warp_max(sc[h]);
           if (lane == 0) red[h] = mx;
@@ -537,7 +569,7 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
         red[9] = mine ? 1.f : 0.f;
       }
       named_bar_sync(bar_wg, 128);
-      const float* rr = tail->red[x][0];
+      const float* rr = tail->red[it & 1][wg][0];
       ok = rr[9] != 0.f && rr[19] != 0.f && rr[29] != 0.f && rr[39] != 0.f;
       if (!ok) break;
       const float gv = fmaxf(fmaxf(rr[8], rr[18]), fmaxf(rr[28], rr[38]));
@@ -545,10 +577,10 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
       const float unit =
           gv > 0.f ? __uint_as_float(((__float_as_uint(gv) >> 23) + 1) << 23) : 1.f;
       const float v_over_unit = vscale * (1.f / unit);   // exact scaling by a power of two
-      float alpha[kGp];
-      uint32_t pw[3][kGp];
+      float alpha[kH];
+      uint32_t pw[3][kH];
 #pragma unroll
-      for (int h = 0; h < kGp; ++h) {
+      for (int h = 0; h < kH; ++h) {
         alpha[h] = 1.f;
         pw[0][h] = pw[1][h] = pw[2][h] = 0u;
         if (h < G) {
@@ -570,7 +602,7 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
 #pragma unroll
       for (int k = 0; k < T; ++k)
 #pragma unroll
-        for (int h = 0; h < kGp; ++h)
+        for (int h = 0; h < kH; ++h)
           if (h < G) {
             const int n = k * kGp + h;
             pb[(n >> 3) * 1024 + (n & 7) * 16] = uint8_t(pw[k][h]);
@@ -600,29 +632,17 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&tail->p_full[x]);
-      const float unit_f = unit * (kFp8 ? (1.f / 256.f) : (1.f / 127.f));
-      if constexpr (kWG == 2) {
-        // this warpgroup's O buffer is reused by its next group: fold now
-        // (the other warpgroup's softmax covers the wait)
-        fold_ok = fold(j, alpha, unit_f);
-      } else {
-        // fold the previous group while this group's PV runs
-        if (jprev >= 0) fold_ok = fold(jprev, alpha_prev, unit_prev);
-#pragma unroll
-        for (int h = 0; h < kGp; ++h) alpha_prev[h] = alpha[h];
-        unit_prev = unit_f;
-        jprev = j;
-      }
+      // fold now (the other warpgroup's softmax covers the wait for PV)
+      fold_ok = fold(j, alpha, kFp8 ? unit * (1.f / 256.f) : unit * (1.f / 127.f));
     }
-    if (kWG == 1 && ok && fold_ok && jprev >= 0) fold_ok = fold(jprev, alpha_prev, unit_prev);
     ok = ok && fold_ok;
 
     // ------------------------------------------------------------ epilogue
     // l per head: sum over the warpgroup's 128 keys' partial sums; flags too
-    float* er = tail->red[wg][sw];
+    float* er = tail->red[0][wg][sw];
     named_bar_sync(bar_wg, 128);                      // the last exchange's reads are done
 #pragma unroll
-    for (int h = 0; h < kGp; ++h) {
+    for (int h = 0; h < kH; ++h) {
       if (h < G) {
         float v = l[h];
 #pragma unroll
@@ -632,41 +652,42 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
     }
     if (lane == 0) er[9] = ok ? 1.f : 0.f;
     named_bar_sync(bar_wg, 128);
-    const float* rr = tail->red[wg][0];
+    const float* rr = tail->red[0][wg][0];
     bool all_ok = rr[9] != 0.f && rr[19] != 0.f && rr[29] != 0.f && rr[39] != 0.f;
-    float L[kGp];
+    float L[kH];
 #pragma unroll
-    for (int h = 0; h < kGp; ++h) L[h] = h < G ? (rr[h] + rr[10 + h]) + (rr[20 + h] + rr[30 + h]) : 0.f;
-    if constexpr (kWG == 2) {
+    for (int h = 0; h < kH; ++h)
+      L[h] = h < G ? (rr[h] + rr[10 + h]) + (rr[20 + h] + rr[30 + h]) : 0.f;
+    {
       // merge the two warpgroups' (m, l, o) through shared memory, in the K
       // tiles: once both warpgroups are past their loops every MMA of the CTA
       // has completed (each folded its last PV, and every QK precedes a PV)
-      float* mo = reinterpret_cast<float*>(smem);     // [kGp][128] o of warpgroup 1
-      float* mml = mo + kGp * 128;                    // [kGp] m, [kGp] l, ok
+      float* mo = reinterpret_cast<float*>(smem);     // [kH][128] o of warpgroup 1
+      float* mml = mo + kH * 128;                    // [kH] m, [kH] l, ok
       named_bar_sync(kBarAll, kSm);
       if (wg == 1) {
 #pragma unroll
-        for (int h = 0; h < kGp; ++h) mo[h * 128 + tg] = o[h];
+        for (int h = 0; h < kH; ++h) mo[h * 128 + tg] = o[h];
         if (tg == 0) {
 #pragma unroll
-          for (int h = 0; h < kGp; ++h) {
+          for (int h = 0; h < kH; ++h) {
             mml[h] = m[h];
-            mml[kGp + h] = L[h];
+            mml[kH + h] = L[h];
           }
-          mml[2 * kGp] = all_ok ? 1.f : 0.f;
+          mml[2 * kH] = all_ok ? 1.f : 0.f;
         }
       }
       named_bar_sync(kBarAll, kSm);
       if (wg == 0) {
-        all_ok = all_ok && mml[2 * kGp] != 0.f;
+        all_ok = all_ok && mml[2 * kH] != 0.f;
 #pragma unroll
-        for (int h = 0; h < kGp; ++h) {
+        for (int h = 0; h < kH; ++h) {
           const float m1 = mml[h];
           const float M = fmaxf(m[h], m1);
           const float w0 = m[h] == -INFINITY ? 0.f : exp2f(m[h] - M);
           const float w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
           o[h] = o[h] * w0 + mo[h * 128 + tg] * w1;
-          L[h] = L[h] * w0 + mml[kGp + h] * w1;
+          L[h] = L[h] * w0 + mml[kH + h] * w1;
           m[h] = M;
         }
       }
@@ -674,7 +695,7 @@ __global__ void __launch_bounds__(64 + 128 * kWG, 2) decode_q8tc_kernel(
     if (wg == 0) {
       const bool zero = tail->any_bad != 0 || !all_ok || tail->abort;
 #pragma unroll
-      for (int h = 0; h < kGp; ++h) {
+      for (int h = 0; h < kH; ++h) {
         if (h >= G) break;
         const float val = (L[h] > 0.f && !zero) ? o[h] / L[h] : 0.f;
         const int64_t bh = int64_t(b) * p.H + kvh * G + h;
@@ -705,13 +726,12 @@ namespace {
 template <bool kFp8, int kGp>
 cudaError_t launch_tc(const CUtensorMap* tmRK, const CUtensorMap* tmRV, const DecodeArgs& a,
                       cudaStream_t stream) {
-  // two K tiles and four V tiles (three at 32 columns): two CTAs per SM
+  // two K tiles and four V tiles: two CTAs per SM
   constexpr int N = q8tc_cols(kFp8, kGp);
-  const size_t smem = 1024 + tail_off(q8tc_vstages(N), N) + sizeof(TcTail);
-  static_assert(1024 + tail_off(q8tc_vstages(N), N) + sizeof(TcTail) <= 113 * 1024,
+  const size_t smem = 1024 + tail_off(kMaxVStages, N) + sizeof(TcTail);
+  static_assert(1024 + tail_off(kMaxVStages, N) + sizeof(TcTail) <= 113 * 1024,
                 "two CTAs per SM");
-  constexpr int kWG = q8tc_wgs(kGp);
-  auto* kern = decode_q8tc_kernel<kFp8, kGp, kWG>;
+  auto* kern = decode_q8tc_kernel<kFp8, kGp>;
   static PerDeviceOnce attr;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -731,8 +751,7 @@ cudaError_t launch_tc_g(const CUtensorMap* tmRK, const CUtensorMap* tmRV, const 
                         int G, cudaStream_t stream) {
   if (G <= 1) return launch_tc<kFp8, 1>(tmRK, tmRV, a, stream);
   if (G <= 2) return launch_tc<kFp8, 2>(tmRK, tmRV, a, stream);
-  if (G <= 4) return launch_tc<kFp8, 4>(tmRK, tmRV, a, stream);
-  return launch_tc<kFp8, 8>(tmRK, tmRV, a, stream);
+  return launch_tc<kFp8, 4>(tmRK, tmRV, a, stream);
 }
 
 }  // namespace
@@ -740,7 +759,7 @@ cudaError_t launch_tc_g(const CUtensorMap* tmRK, const CUtensorMap* tmRV, const 
 cudaError_t launch_decode_q8tc(const CUtensorMap* tmRK, const CUtensorMap* tmRV,
                                const DecodeArgs& a, bool fp8, cudaStream_t stream) {
   const int G = a.H / a.Hkv;
-  if (G < 1 || G > 8) return cudaErrorInvalidValue;
+  if (G < 1 || G > 4) return cudaErrorInvalidValue;
   if (a.order) {
     cudaError_t eo = launch_decode_order(a.kv_lens, a.B, a.order, stream);
     if (eo != cudaSuccess) return eo;

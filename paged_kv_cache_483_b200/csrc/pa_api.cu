@@ -712,9 +712,16 @@ static pa_status decode_fast(pa_pool* p, const void* q, int32_t B, int32_t H,
   a.v_cache = p->v_cache;
   a.window = window;
   a.sinks = sinks;
-  if (is_q8(p->dtype))
-    return cuda_status(pa::launch_decode_q8tc(&p->tmRK, &p->tmRV, a, p->dtype == PA_FP8,
-                                              static_cast<cudaStream_t>(stream)));
+  if (is_q8(p->dtype)) {
+    // Groups of up to 4 heads: tcgen05 MMAs straight from the codes (a 128-key
+    // group per MMA; the per-byte softmax work grows with the group).  Larger
+    // groups: the warp-level kernel, whose 8-column MMA tiles they fill.
+    const bool fp8 = p->dtype == PA_FP8;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return cuda_status(H / p->num_kv_heads <= 4
+                           ? pa::launch_decode_q8tc(&p->tmRK, &p->tmRV, a, fp8, s)
+                           : pa::launch_decode_q8(&p->tmK, a, fp8, s));
+  }
   return cuda_status(pa::launch_decode_fast(&p->tmK, &p->tmV, a, p->sms,
                                             static_cast<cudaStream_t>(stream)));
 }

@@ -181,14 +181,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
   regs_dealloc<kCtrlRegs>();
   if (warp == 0 || warp == 2) {
     // ------------------------------------- TMA producers: Q and K (warp 0), V (warp 2)
-    // Two threads issue the copies: one thread's TMA issue rate does not
-    // keep up with the K and V tiles of both query tiles.
+    // Two warps issue the copies, eight lanes each (lane i copies block i of
+    // a tile): one thread's TMA issue rate does not keep up with the K and V
+    // tiles of both query tiles.
     const bool is_k = warp == 0;
-    if (lane == 0 && n_tiles > 0) {
+    if (n_tiles > 0) {
       const CUtensorMap* map = is_k ? &tmK : &tmV;
-      prefetch_tensormap(map);
+      if (lane == 0) prefetch_tensormap(map);
       const uint64_t pol_kv = policy_evict_last();
-      if (is_k) {
+      if (is_k && lane == 0) {
         prefetch_tensormap(&tmQ);
         const uint64_t pol_q = policy_evict_first();
         mbar_arrive_expect_tx(&bars->q_full, 2 * kTile);
@@ -199,45 +200,44 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
                       pol_q);
         }
       }
-      // Block ids of a tile, read one tile ahead of their use: the TMA
-      // issues are ordered with every memory access, so an id read next to
-      // its copy would cost one global-memory round trip per block.
-      auto tile_ids = [&](int j, int (&ids)[8]) {
+      // This lane's block id of a tile, read one tile ahead of its use: the
+      // TMA issues are ordered with every memory access, so an id read next
+      // to its copy would cost one global-memory round trip per block.
+      auto tile_id = [&](int j) {
         const int nb = min(8, n_blk - (j0 + j) * 8);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          int blk = i < nb ? trow[(j0 + j) * 8 + i] : 0;
-          ids[i] = (blk < 0 || blk >= p.NB) ? 0 : blk;   // reported and zeroed by the softmax
-        }
+        const int blk = lane < nb ? trow[(j0 + j) * 8 + lane] : 0;
+        return (blk < 0 || blk >= p.NB) ? 0 : blk;   // reported and zeroed by the softmax
       };
       uint64_t* full = is_k ? bars->k_full : bars->v_full;
       uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
       uint8_t* ring = smem + (is_k ? kOffK : kOffV);
       const int stages = is_k ? kKStages : kVStages;
-      int ids[8];
-      tile_ids(0, ids);
+      int id = tile_id(0);
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % stages, round = j / stages;
-        if (round > 0 && !wait_or_abort(&empty[s], (round - 1) & 1, bars, p.err)) break;
-        if (bars->abort) break;
+        bool go = true;
+        if (lane == 0)
+          go = (round == 0 || wait_or_abort(&empty[s], (round - 1) & 1, bars, p.err)) &&
+               !bars->abort;
+        if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) break;
         uint8_t* dst = ring + s * kTile;
         const int nb = min(8, n_blk - (j0 + j) * 8);
-        mbar_arrive_expect_tx(&full[s], nb * 4096);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (i < nb) {
-            tma_load_3d(dst + i * 2048, map, &full[s], 0, kvh, ids[i] * 16, pol_kv);
-            tma_load_3d(dst + kHalf + i * 2048, map, &full[s], 64, kvh, ids[i] * 16, pol_kv);
-          }
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], nb * 4096);
+        __syncwarp();                                  // the bytes are expected first
+        if (lane < nb) {
+          tma_load_3d(dst + lane * 2048, map, &full[s], 0, kvh, id * 16, pol_kv);
+          tma_load_3d(dst + kHalf + lane * 2048, map, &full[s], 64, kvh, id * 16, pol_kv);
         }
         issued = j + 1;
-        if (j + 1 < n_tiles) tile_ids(j + 1, ids);
+        if (j + 1 < n_tiles) id = tile_id(j + 1);
       }
       // drain: every issued copy has landed before the CTA may exit
-      if (is_k) mbar_wait(&bars->q_full, 0);
-      for (int s = 0; s < stages; ++s)
-        if (s < issued) mbar_wait(&full[s], ((issued - 1 - s) / stages) & 1);
+      if (lane == 0) {
+        if (is_k) mbar_wait(&bars->q_full, 0);
+        for (int s = 0; s < stages; ++s)
+          if (s < issued) mbar_wait(&full[s], ((issued - 1 - s) / stages) & 1);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
