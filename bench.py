@@ -583,7 +583,75 @@ class _PinnedRing:
 
 
 def run_e2e(args, S, dist, device, is_prefill, part, win, sinks):
-    """Same metric through the public API with host buffers.  Every step
+    """Same metric through the public API with host buffers (see run_e2e_steps
+    and run_e2e_batch): decode steps that append one token per sequence go
+    through the prepared batch, the rest through the separate calls."""
+    w = S.w
+    one_token = (not is_prefill) and bool(w.step) and all(op.args[1] == 1 for op in w.step) \
+        and not win and [op.args[0] for op in w.step] == list(w.decode_seqs)
+    if one_token:
+        return run_e2e_batch(args, S, dist, device, part)
+    return run_e2e_steps(args, S, dist, device, is_prefill, part, win, sinks)
+
+
+def run_e2e_batch(args, S, dist, device, part):
+    """The serving decode loop through pa_batch_step: each step is one C call
+    that plans the step's appends on the host manager (step a1), uploads the
+    plan, the changed table entries, the queries and the new K/V from pinned
+    host memory, runs copy-on-write copies and the fused append + decode, and
+    downloads the output; pa_batch_rollback then gives every sequence's token
+    back (host-only) so that every step is the same step.  The timed region
+    holds K steps and the final wait for the last output.  Copies of
+    consecutive steps overlap their neighbours' kernels (two buffer sets, two
+    copy streams).  A copy-on-write of a shared partial tail happens in the
+    first step only (the tail is private afterwards), as in serving."""
+    import torch
+    import paged_kv_cache_483_b200 as pa
+    pool, w = S.pool, S.w
+    stream = torch.cuda.current_stream(device)
+    seqs = list(w.decode_seqs)
+    n = len(seqs)
+    h_q = S.q.cpu().pin_memory()
+    h_k, h_v = S.step_k.cpu().pin_memory(), S.step_v.cpu().pin_memory()
+    h_out = torch.empty(S.out.shape, dtype=torch.float32).pin_memory()
+    lens_now = [pool.table(s)[1] for s in seqs]
+    pool.truncate(seqs, [L - 1 for L in lens_now])        # undo the set-up's plan
+    batch = pa.Batch(pool, seqs, S.q.shape[1], S.tables.shape[1], part)
+    K = max(1, min(args.steps, args.e2e_steps))
+
+    def step():
+        batch.step(h_q, h_k, h_v, h_out, stream=stream)
+        batch.rollback()
+
+    for _ in range(3):
+        step()
+    batch.sync()
+    torch.cuda.synchronize()
+    dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    a.record(stream)
+    for _ in range(K):
+        step()
+    host_ms = (time.perf_counter() - t0) * 1e3 / K        # queueing the steps
+    batch.sync()
+    b.record(stream)
+    torch.cuda.synchronize()
+    wall_ms = (time.perf_counter() - t0) * 1e3 / K
+    ms = dist.max(max(a.elapsed_time(b) / K, wall_ms), device)
+    batch.close()
+    pool.plan_append(seqs, [1] * n)                       # back to the state the step assumes
+    v = dist.world * decode_bytes(w, S.lens_h, S.q8) / (ms * 1e-3) / 1e9
+    bi = (h_q.numel() * h_q.element_size() + 2 * h_k.numel() * h_k.element_size()
+          + n * (8 + 4))                                  # + the plan: slots and lengths
+    return {"value": round(v, 2), "unit": "GB/s", "h2d_bytes_per_step": int(bi),
+            "d2h_bytes_per_step": int(h_out.numel() * 4), "ms_per_step": round(ms, 5),
+            "steps": K, "host_plan_in_step": True, "api": "pa_batch_step + pa_batch_rollback",
+            "host_ms_per_step": round(host_ms, 5)}
+
+
+def run_e2e_steps(args, S, dist, device, is_prefill, part, win, sinks):
+    """Same metric through the separate calls with host buffers.  Every step
     plans its appends on the host manager (pa_plan_append), copies its inputs
     (queries, new K/V, slot mapping, copy-on-write pairs, kv_lens) from pinned
     host memory, runs the step's kernels and reads the output back; then the

@@ -423,6 +423,62 @@ pa_status pa_prefill_chunk(pa_pool* pool, const void* q, int32_t B,
                            const int32_t* d_kv_lens, float scale,
                            int32_t max_kv_splits, float* out, void* stream);
 
+/* ---- prepared decode batch --------------------------------------------- */
+
+/* A serving decode loop in one call per step.  The pages' path for one step
+ * is: plan each sequence's next token ([P1] append, [P2] preflight), copy a
+ * shared partial tail ([P1] copy-on-write), write the new token's K/V and
+ * attend over the cache ([P3] with q_tokens = 1).  A batch fixes the
+ * sequences of such a loop once, keeps their block tables, lengths and
+ * scratch on the device, and runs the whole step from host buffers.
+ *
+ * pa_batch_create: seqs (host, n distinct live sequences) of `pool`, queries
+ * with H heads, tables up to max_blocks wide (a sequence may grow to
+ * max_blocks * block_size tokens), partition_tokens as pa_decode.  Uploads
+ * the current tables and allocates the batch's device buffers (two sets of
+ * q, new K/V, output and staging), pinned staging and two copy streams.
+ * Errors: NO_DEVICE, UNKNOWN_SEQ, INVALID_ARG (n <= 0, a sequence twice, a
+ * table wider than max_blocks, H not a multiple of num_kv_heads), CUDA. */
+typedef struct pa_batch pa_batch; /* opaque */
+pa_status pa_batch_create(pa_pool* pool, const int32_t* seqs, int32_t n,
+                          int32_t H, int32_t max_blocks,
+                          int32_t partition_tokens, pa_batch** out);
+
+/* One decode step: appends one token to every sequence of the batch (the
+ * plan runs on the host manager, all-or-nothing as pa_plan_append) and
+ * decodes it.
+ *   h_q: host [n, H, head_dim], h_key / h_value: host [n, Hkv, head_dim], all
+ *   in the pool dtype (bf16 on an int8 or FP8 pool); h_out: host [n, H,
+ *   head_dim] float32.  Use pinned host memory for asynchronous copies.
+ * The plan, the table entries that changed since the previous step and the
+ * inputs are uploaded on the batch's upload stream; the table patches,
+ * copy-on-write copies and the fused append + decode (pa_decode_append) run
+ * on `stream`; the output is downloaded on the batch's download stream.
+ * Successive steps alternate two buffer sets, so a step's transfers overlap
+ * its neighbours' kernels.  The call returns once the work is queued: h_out
+ * holds the result after pa_batch_sync, and the input buffers must not change
+ * before then.  The batch's sequences change only through the batch between
+ * steps, or through pa_seq_truncate (any other change is picked up by
+ * comparing whole tables).
+ * Errors: those of pa_plan_append (nothing changes), UNKNOWN_SEQ (a sequence
+ * was released), INVALID_ARG (a null pointer, a sequence at max_blocks *
+ * block_size tokens), CUDA (the plan has been applied: treat the pool as
+ * lost), and those of pa_decode_append. */
+pa_status pa_batch_step(pa_batch* batch, const void* h_q, const void* h_key,
+                        const void* h_value, float scale, float* h_out,
+                        void* stream);
+
+/* Undo the last step's token of every sequence of the batch (drafted tokens
+ * that were not accepted): pa_seq_truncate to one token less, host-only.  A
+ * copy-on-write the step made stays. */
+pa_status pa_batch_rollback(pa_batch* batch);
+
+/* Wait until every step's output has reached its host buffer. */
+pa_status pa_batch_sync(pa_batch* batch);
+
+/* Synchronise the device and release the batch (never the pool). */
+pa_status pa_batch_free(pa_batch* batch);
+
 /* Bytes of the fixed device scratch array used by pa_decode_static_scratch. */
 #define PA_STATIC_SCRATCH_BYTES (16u << 20)
 

@@ -35,7 +35,9 @@ EXPORTS = ["pa_pool_create", "pa_free", "pa_seq_create", "pa_seq_fork", "pa_seq_
            "pa_decode_static_scratch", "pa_decode_append", "pa_seq_create_cached",
            "pa_prefix_publish", "pa_prefix_clear", "pa_prefix_entries", "pa_pool_create_int8",
            "pa_decode_window", "pa_decode_window_workspace_bytes", "pa_pool_create_layers",
-           "pa_pool_layer", "pa_decode_window_append", "pa_pool_create_fp8", "pa_seq_truncate"]
+           "pa_pool_layer", "pa_decode_window_append", "pa_pool_create_fp8", "pa_seq_truncate",
+           "pa_batch_create", "pa_batch_step", "pa_batch_rollback", "pa_batch_sync",
+           "pa_batch_free"]
 
 
 class PAError(RuntimeError):
@@ -105,6 +107,11 @@ def lib():
         "pa_decode_static_scratch": ([_P, _P, _I32, _I32, _P, _I32, _P, _F, _I32, _P, _P], C.c_int),
         "pa_decode_append": ([_P, _P, _P, _P, _P, _I32, _I32, _P, _I32, _P, _F, _I32, _P, _SZ, _P,
                               _P], C.c_int),
+        "pa_batch_create": ([_P, _PI32, _I32, _I32, _I32, _I32, C.POINTER(_P)], C.c_int),
+        "pa_batch_step": ([_P, _P, _P, _P, _F, _P, _P], C.c_int),
+        "pa_batch_rollback": ([_P], C.c_int),
+        "pa_batch_sync": ([_P], C.c_int),
+        "pa_batch_free": ([_P], C.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -558,3 +565,61 @@ class Pool:
 
     def prefill_path(self, num_heads):
         return int(lib().pa_prefill_path(self._h, num_heads))
+
+
+def _host_ptr(t, dtype, shape, name):
+    """Address of a contiguous CPU tensor of the given dtype and shape."""
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous() or t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+    return C.c_void_p(t.data_ptr())
+
+
+class Batch:
+    """A prepared decode batch (pa_batch_*): fixed sequences of ``pool``
+    whose every step appends one token and decodes, from host buffers, in one
+    C call.  ``step`` queues the work; ``sync`` waits for the outputs."""
+
+    def __init__(self, pool, seqs, num_heads, max_blocks, partition_tokens=0):
+        self.pool = pool
+        self.seqs = [int(s) for s in seqs]
+        self.num_heads, self.max_blocks = int(num_heads), int(max_blocks)
+        seqs_a, sp = _i32(self.seqs)
+        h = C.c_void_p()
+        _check(lib().pa_batch_create(pool.handle, sp, len(seqs_a), self.num_heads,
+                                     self.max_blocks, int(partition_tokens), C.byref(h)),
+               "pa_batch_create")
+        self._h = h
+
+    def step(self, q, key, value, out, scale=None, stream=None):
+        """q [n, H, d], key / value [n, Hkv, d] (pool dtype; bf16 for int8 /
+        fp8 pools) and out [n, H, d] float32: pinned CPU tensors."""
+        import torch
+        p = self.pool
+        n, d = len(self.seqs), p.head_dim
+        dt = p._torch_dtype()
+        scale = 1.0 / math.sqrt(d) if scale is None else scale
+        _check(lib().pa_batch_step(
+            self._h, _host_ptr(q, dt, (n, self.num_heads, d), "q"),
+            _host_ptr(key, dt, (n, p.num_kv_heads, d), "key"),
+            _host_ptr(value, dt, (n, p.num_kv_heads, d), "value"), float(scale),
+            _host_ptr(out, torch.float32, (n, self.num_heads, d), "out"), _stream(stream)),
+            "pa_batch_step")
+
+    def rollback(self):
+        _check(lib().pa_batch_rollback(self._h), "pa_batch_rollback")
+
+    def sync(self):
+        _check(lib().pa_batch_sync(self._h), "pa_batch_sync")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().pa_batch_free(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -8,6 +8,8 @@
 // ("abhik.ai examples/pagedattention.py", KVPool.append: keys[physical,
 // offset] = key).  K2 copies a whole block, every slot and head, of both
 // caches ("abhik.ai examples/pagedattention.py", KVPool._private_tail).
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.hpp"
 
@@ -155,6 +157,25 @@ cudaError_t launch_reshape_and_cache_q8(const void* key, const void* value, void
   kern<<<grid, 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value),
       static_cast<uint8_t*>(records), slots, T, Hkv, num_slots, err);
+  return cudaGetLastError();
+}
+
+// Block-table patches of a prepared decode batch: entry (row, index) of the
+// device tables [rows, width] takes value, for each (row, index, value) triple
+// the host found changed since the previous step.
+__global__ void __launch_bounds__(256) table_patch_kernel(int32_t* __restrict__ tables,
+                                                          int32_t width,
+                                                          const int32_t* __restrict__ patches,
+                                                          int32_t n) {
+  for (int32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    tables[int64_t(patches[3 * i]) * width + patches[3 * i + 1]] = patches[3 * i + 2];
+}
+
+cudaError_t launch_table_patch(int32_t* tables, int32_t width, const int32_t* patches,
+                               int32_t n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int grid = int(std::min<int64_t>((int64_t(n) + 255) / 256, 1024));
+  table_patch_kernel<<<grid, 256, 0, stream>>>(tables, width, patches, n);
   return cudaGetLastError();
 }
 

@@ -43,6 +43,10 @@ cudaError_t launch_cow_copy(void* k_cache, void* v_cache, const int32_t* src,
                             int32_t num_blocks, int32_t* err, int sms,
                             cudaStream_t stream);
 
+// Table patches (row, index, value) x n applied to device tables [rows, width].
+cudaError_t launch_table_patch(int32_t* tables, int32_t width, const int32_t* patches,
+                               int32_t n, cudaStream_t stream);
+
 // Generic CUDA-core paged attention: any dtype, head_dim <= 512, any block
 // size and group size, q_tokens >= 1 (causal offset rule).
 struct GenericArgs {

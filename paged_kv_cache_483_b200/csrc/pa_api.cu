@@ -868,6 +868,301 @@ pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,
   return cuda_status(pa::launch_attention_generic(g, s));
 }
 
+}  // extern "C"
+
+// ---- prepared decode batch ---------------------------------------------------
+//
+// One serving decode step per call.  The batch keeps, on the device, the
+// block tables and scratch of a fixed list of sequences, and a host mirror of
+// the tables; each step plans one new token per sequence on the host manager,
+// finds the table entries that changed (the copied tail and a new block, at
+// the end of each row), stages plan and patches in one pinned buffer, and
+// queues: the uploads (plan, patches, q, new K/V) on an upload stream, the
+// patch kernel, copy-on-write copies and the fused append + decode on the
+// caller's stream, and the download of the output on a download stream.  Two
+// sets of device buffers alternate between steps, so one step's transfers
+// overlap the neighbouring steps' kernels.
+
+namespace {
+
+constexpr int kBatchSets = 2;
+
+struct BatchSet {
+  void* d_q = nullptr;       // [n, H, d] pool dtype (bf16 on int8 / FP8 pools)
+  void* d_k = nullptr;       // [n, Hkv, d]
+  void* d_v = nullptr;
+  float* d_out = nullptr;    // [n, H, d]
+  char* d_stage = nullptr;   // slots int64 [n] | lens [n] | cow src [n] | dst [n] | patches
+  char* h_stage = nullptr;   // pinned mirror of d_stage
+  cudaEvent_t up = nullptr, done = nullptr, down = nullptr;
+  bool used = false;
+};
+
+}  // namespace
+
+struct pa_batch {
+  pa_pool* pool = nullptr;
+  std::vector<int32_t> seqs, ones;
+  int32_t n = 0, H = 0, MB = 0, part = 0;
+  size_t q_bytes = 0, kv_bytes = 0, out_bytes = 0, stage_bytes = 0;
+  int32_t patch_cap = 0;                 // (row, index, value) triples per step
+  int32_t* d_tables = nullptr;           // [n, MB]
+  void* d_ws = nullptr;
+  size_t ws_bytes = 0;
+  cudaStream_t up = nullptr, down = nullptr;
+  std::vector<int32_t> mirror;           // host copy of d_tables
+  std::vector<int32_t> mirror_blocks;    // entries of each row the device holds
+  std::vector<int64_t> mirror_len;       // sequence length the mirror reflects
+  std::vector<int64_t> slots_tmp;
+  std::vector<pa::CowPair> cow_tmp;
+  std::vector<int32_t> patches;
+  BatchSet set[kBatchSets];
+  int64_t steps = 0;
+};
+
+namespace {
+
+void free_batch(pa_batch* b) {
+  for (auto& s : b->set) {
+    cudaFree(s.d_q);
+    cudaFree(s.d_k);
+    cudaFree(s.d_v);
+    cudaFree(s.d_out);
+    cudaFree(s.d_stage);
+    if (s.h_stage) cudaFreeHost(s.h_stage);
+    if (s.up) cudaEventDestroy(s.up);
+    if (s.done) cudaEventDestroy(s.done);
+    if (s.down) cudaEventDestroy(s.down);
+  }
+  cudaFree(b->d_tables);
+  cudaFree(b->d_ws);
+  if (b->up) cudaStreamDestroy(b->up);
+  if (b->down) cudaStreamDestroy(b->down);
+  delete b;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_batch_create(pa_pool* p, const int32_t* seqs, int32_t n, int32_t H,
+                          int32_t max_blocks, int32_t partition_tokens, pa_batch** out) {
+  if (!out) return PA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!p) return PA_ERR_INVALID_ARG;
+  if (!p->device) return PA_ERR_NO_DEVICE;
+  if (n <= 0 || !seqs || H <= 0 || H % p->num_kv_heads || max_blocks <= 0 ||
+      partition_tokens < 0 || int64_t(max_blocks) * p->block_size > INT32_MAX)
+    return PA_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n; ++i) {
+    const std::vector<int32_t>* t = p->mgr->table(seqs[i]);
+    if (!t) return PA_ERR_UNKNOWN_SEQ;
+    if (int32_t(t->size()) > max_blocks) return PA_ERR_INVALID_ARG;
+    for (int32_t k = 0; k < i; ++k)
+      if (seqs[k] == seqs[i]) return PA_ERR_INVALID_ARG;   // a sequence once
+  }
+  pa::DeviceScope on_pool_device(p->dev_id);
+  pa_batch* b = new (std::nothrow) pa_batch();
+  if (!b) return PA_ERR_INVALID_ARG;
+  b->pool = p;
+  b->seqs.assign(seqs, seqs + n);
+  b->ones.assign(size_t(n), 1);
+  b->n = n;
+  b->H = H;
+  b->MB = max_blocks;
+  b->part = partition_tokens;
+  const size_t eq = p->dtype == PA_F32 ? 4 : 2;   // queries and new rows: pool dtype, bf16 for codes
+  b->q_bytes = size_t(n) * H * p->head_dim * eq;
+  b->kv_bytes = size_t(n) * p->num_kv_heads * p->head_dim * eq;
+  b->out_bytes = size_t(n) * H * p->head_dim * sizeof(float);
+  b->patch_cap = 4 * n;
+  b->stage_bytes = size_t(n) * (8 + 4 + 8) + size_t(b->patch_cap) * 12;
+  b->ws_bytes = pa_decode_workspace_bytes(p, n, H, max_blocks, partition_tokens);
+  bool ok = cudaStreamCreateWithFlags(&b->up, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&b->down, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaMalloc(&b->d_tables, size_t(n) * max_blocks * sizeof(int32_t)) == cudaSuccess &&
+            (b->ws_bytes == 0 || cudaMalloc(&b->d_ws, b->ws_bytes) == cudaSuccess);
+  for (auto& s : b->set) {
+    ok = ok && cudaMalloc(&s.d_q, b->q_bytes) == cudaSuccess &&
+         cudaMalloc(&s.d_k, b->kv_bytes) == cudaSuccess &&
+         cudaMalloc(&s.d_v, b->kv_bytes) == cudaSuccess &&
+         cudaMalloc(reinterpret_cast<void**>(&s.d_out), b->out_bytes) == cudaSuccess &&
+         cudaMalloc(reinterpret_cast<void**>(&s.d_stage), b->stage_bytes) == cudaSuccess &&
+         cudaMallocHost(reinterpret_cast<void**>(&s.h_stage), b->stage_bytes) == cudaSuccess &&
+         cudaEventCreateWithFlags(&s.up, cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&s.down, cudaEventDisableTiming) == cudaSuccess;
+  }
+  if (!ok) {
+    free_batch(b);
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  // the tables as they stand, uploaded once
+  b->mirror.assign(size_t(n) * max_blocks, 0);
+  b->mirror_blocks.assign(size_t(n), 0);
+  b->mirror_len.assign(size_t(n), 0);
+  for (int32_t i = 0; i < n; ++i) {
+    const std::vector<int32_t>* t = p->mgr->table(seqs[i]);
+    std::copy(t->begin(), t->end(), b->mirror.begin() + int64_t(i) * max_blocks);
+    b->mirror_blocks[size_t(i)] = int32_t(t->size());
+    b->mirror_len[size_t(i)] = p->mgr->length(seqs[i]);
+  }
+  if (cudaMemcpy(b->d_tables, b->mirror.data(), b->mirror.size() * sizeof(int32_t),
+                 cudaMemcpyHostToDevice) != cudaSuccess) {
+    free_batch(b);
+    return PA_ERR_CUDA;
+  }
+  *out = b;
+  return PA_OK;
+}
+
+pa_status pa_batch_step(pa_batch* b, const void* h_q, const void* h_key, const void* h_value,
+                        float scale, float* h_out, void* stream) {
+  if (!b || !h_q || !h_key || !h_value || !h_out) return PA_ERR_INVALID_ARG;
+  pa_pool* p = b->pool;
+  pa::DeviceScope on_pool_device(p->dev_id);
+  const int32_t n = b->n, MB = b->MB;
+  // every sequence must still be live and have room for one more token
+  for (int32_t i = 0; i < n; ++i) {
+    if (!p->mgr->table(b->seqs[size_t(i)])) return PA_ERR_UNKNOWN_SEQ;
+    if (p->mgr->length(b->seqs[size_t(i)]) + 1 > int64_t(MB) * p->block_size)
+      return PA_ERR_INVALID_ARG;
+  }
+  BatchSet& S = b->set[b->steps % kBatchSets];
+  // the pinned staging of this set is rewritten only after its last upload ran
+  if (S.used && cudaEventSynchronize(S.up) != cudaSuccess) return PA_ERR_CUDA;
+
+  // step a1 on the host: one token per sequence, all-or-nothing
+  b->slots_tmp.clear();
+  b->cow_tmp.clear();
+  pa_status st = from_mgr(p->mgr->append(b->seqs.data(), b->ones.data(), n, &b->slots_tmp,
+                                         &b->cow_tmp));
+  if (st != PA_OK) return st;
+
+  // table entries that differ from the device copy: the changes of an append
+  // (a copied tail, a new block) lie at the end of a row; a row whose length
+  // moved by anything but this step (a rollback) is compared whole
+  b->patches.clear();
+  bool full_upload = false;
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t seq = b->seqs[size_t(i)];
+    const std::vector<int32_t>& t = *p->mgr->table(seq);
+    const int64_t len = p->mgr->length(seq);
+    const int32_t size = int32_t(t.size());
+    int32_t from = 0;
+    if (len - 1 == b->mirror_len[size_t(i)])
+      from = std::max(0, std::min(b->mirror_blocks[size_t(i)], size) - 1);
+    int32_t* row = b->mirror.data() + int64_t(i) * MB;
+    for (int32_t j = from; j < size; ++j) {
+      if (row[j] != t[size_t(j)]) {
+        row[j] = t[size_t(j)];
+        if (int32_t(b->patches.size()) < 3 * b->patch_cap) {
+          b->patches.push_back(i);
+          b->patches.push_back(j);
+          b->patches.push_back(t[size_t(j)]);
+        } else {
+          full_upload = true;
+        }
+      }
+    }
+    b->mirror_blocks[size_t(i)] = size;
+    b->mirror_len[size_t(i)] = len;
+  }
+  const int32_t ncow = int32_t(b->cow_tmp.size());
+  const int32_t npatch = full_upload ? 0 : int32_t(b->patches.size() / 3);
+  // staging: slots | lens | cow src | cow dst | patches
+  int64_t* slots = reinterpret_cast<int64_t*>(S.h_stage);
+  int32_t* lens = reinterpret_cast<int32_t*>(slots + n);
+  int32_t* csrc = lens + n;
+  int32_t* cdst = csrc + n;
+  int32_t* pat = cdst + n;
+  std::copy(b->slots_tmp.begin(), b->slots_tmp.end(), slots);
+  for (int32_t i = 0; i < n; ++i) lens[i] = int32_t(b->mirror_len[size_t(i)]);
+  for (int32_t c = 0; c < ncow; ++c) {
+    csrc[c] = b->cow_tmp[size_t(c)].src;
+    cdst[c] = b->cow_tmp[size_t(c)].dst;
+  }
+  std::copy(b->patches.begin(), b->patches.begin() + 3 * npatch, pat);
+  const size_t staged = size_t(n) * 20 + size_t(npatch) * 12;
+  const int64_t* d_slots = reinterpret_cast<const int64_t*>(S.d_stage);
+  const int32_t* d_lens = reinterpret_cast<const int32_t*>(d_slots + n);
+  const int32_t* d_csrc = d_lens + n;
+  const int32_t* d_cdst = d_csrc + n;
+  const int32_t* d_pat = d_cdst + n;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  bool ok = true;
+  // uploads, once this set's buffers are no longer read by its last step
+  if (S.used) ok = cudaStreamWaitEvent(b->up, S.done, 0) == cudaSuccess;
+  ok = ok && cudaMemcpyAsync(S.d_stage, S.h_stage, staged, cudaMemcpyHostToDevice, b->up) ==
+                 cudaSuccess &&
+       cudaMemcpyAsync(S.d_q, h_q, b->q_bytes, cudaMemcpyHostToDevice, b->up) == cudaSuccess &&
+       cudaMemcpyAsync(S.d_k, h_key, b->kv_bytes, cudaMemcpyHostToDevice, b->up) ==
+           cudaSuccess &&
+       cudaMemcpyAsync(S.d_v, h_value, b->kv_bytes, cudaMemcpyHostToDevice, b->up) ==
+           cudaSuccess &&
+       cudaEventRecord(S.up, b->up) == cudaSuccess;
+  // kernels on the caller's stream, after the uploads and after the download
+  // of this set's previous output
+  ok = ok && cudaStreamWaitEvent(s, S.up, 0) == cudaSuccess;
+  if (S.used) ok = ok && cudaStreamWaitEvent(s, S.down, 0) == cudaSuccess;
+  if (ok && full_upload)          // many rows changed outside the batch: whole tables
+    ok = cudaMemcpyAsync(b->d_tables, b->mirror.data(), b->mirror.size() * sizeof(int32_t),
+                         cudaMemcpyHostToDevice, s) == cudaSuccess &&
+         cudaStreamSynchronize(s) == cudaSuccess;
+  if (ok) ok = pa::launch_table_patch(b->d_tables, MB, d_pat, npatch, s) == cudaSuccess;
+  if (ok) ok = cow_blocks(p, d_csrc, d_cdst, ncow, s) == cudaSuccess;
+  if (!ok) return PA_ERR_CUDA;
+  st = pa_decode_append(p, S.d_q, S.d_k, S.d_v, d_slots, n, b->H, b->d_tables, MB, d_lens,
+                        scale, b->part, b->d_ws, b->ws_bytes, S.d_out, stream);
+  if (st != PA_OK) return st;
+  // download on its own stream
+  ok = cudaEventRecord(S.done, s) == cudaSuccess &&
+       cudaStreamWaitEvent(b->down, S.done, 0) == cudaSuccess &&
+       cudaMemcpyAsync(h_out, S.d_out, b->out_bytes, cudaMemcpyDeviceToHost, b->down) ==
+           cudaSuccess &&
+       cudaEventRecord(S.down, b->down) == cudaSuccess;
+  if (!ok) return PA_ERR_CUDA;
+  S.used = true;
+  ++b->steps;
+  return PA_OK;
+}
+
+pa_status pa_batch_rollback(pa_batch* b) {
+  if (!b) return PA_ERR_INVALID_ARG;
+  pa_pool* p = b->pool;
+  std::vector<int32_t> keep(b->seqs.size());
+  for (size_t i = 0; i < b->seqs.size(); ++i) {
+    if (!p->mgr->table(b->seqs[i])) return PA_ERR_UNKNOWN_SEQ;
+    keep[i] = int32_t(std::max<int64_t>(0, p->mgr->length(b->seqs[i]) - 1));
+  }
+  pa_status st = from_mgr(p->mgr->truncate(b->seqs.data(), keep.data(), b->n));
+  if (st != PA_OK) return st;
+  // the mirror follows (entries past a row's end stay as they are, unused)
+  for (size_t i = 0; i < b->seqs.size(); ++i) {
+    b->mirror_len[i] = keep[i];
+    b->mirror_blocks[i] = int32_t(p->mgr->table(b->seqs[i])->size());
+  }
+  return PA_OK;
+}
+
+pa_status pa_batch_sync(pa_batch* b) {
+  if (!b) return PA_ERR_INVALID_ARG;
+  pa::DeviceScope on_pool_device(b->pool->dev_id);
+  for (auto& s : b->set)
+    if (s.used && cudaEventSynchronize(s.down) != cudaSuccess) return PA_ERR_CUDA;
+  return PA_OK;
+}
+
+pa_status pa_batch_free(pa_batch* b) {
+  if (!b) return PA_OK;
+  pa::DeviceScope on_pool_device(b->pool->dev_id);
+  cudaDeviceSynchronize();
+  free_batch(b);
+  return PA_OK;
+}
+
 pa_status pa_get_error(pa_pool* p, int32_t* device_code) {
   if (!p || !device_code) return PA_ERR_INVALID_ARG;
   *device_code = 0;

@@ -362,3 +362,21 @@ def test_manager_payload_takes_the_largest_fill_among_sharers():
     st = pool.stats()
     assert st["physical_payload_tokens"] == 6 and st["logical_tokens"] == 11
     assert st["internal_waste_tokens"] == 2 and st["sharing_savings_tokens"] == 5
+
+
+def test_batch_calls_on_host_pools_and_bad_arguments():
+    import ctypes as C
+    L = pa.lib()
+    p = pa.Pool(8, 4, 1, 8, "f32")
+    p.create(0)
+    seqs = np.array([0], np.int32)
+    h = C.c_void_p()
+    assert L.pa_batch_create(p.handle, seqs.ctypes.data_as(pa._PI32), 1, 1, 4, 0,
+                             C.byref(h)) == 8                       # host-only pool
+    assert h.value is None
+    assert L.pa_batch_create(p.handle, seqs.ctypes.data_as(pa._PI32), 1, 1, 4, 0, None) == 1
+    assert L.pa_batch_create(None, seqs.ctypes.data_as(pa._PI32), 1, 1, 4, 0, C.byref(h)) == 1
+    for fn in (L.pa_batch_rollback, L.pa_batch_sync):
+        assert fn(None) == 1
+    assert L.pa_batch_free(None) == 0
+    assert L.pa_batch_step(None, None, None, None, 1.0, None, None) == 1

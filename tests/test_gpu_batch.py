@@ -1,0 +1,123 @@
+"""The prepared decode batch (pa_batch_*) on a B200.
+
+A batch step is the serving decode step in one call: plan one token per
+sequence on the host manager ("abhik.ai examples/pagedattention.py", KVPool
+append and copy-on-write; "vladkulikov.com modern-llms module 9 notebook",
+the preflight), upload plan, changed table entries, queries and new K/V,
+copy shared partial tails, write and attend ("docs.rs ferrum-kv 0.4.0
+src/attention.rs", paged_attention with q_tokens = 1), download the output.
+
+Checks, over several steps with copies-on-write, block boundaries and a
+rollback: tables and lengths bit-exact against the oracle pool; outputs
+identical to the same step issued as separate calls on a second pool (same
+kernels, same partitions) and within 2e-3 of the oracle (the bf16 decode bar).
+"""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_483_b200 as pa
+import workloads
+from harness import DeviceRun, OracleRun, q64
+
+pytestmark = pytest.mark.gpu
+
+TOL_DECODE = 2e-3
+
+
+def _workload(kind):
+    # lengths that sit mid-block, one short of a boundary and on a boundary;
+    # sequence 9 shares 20 tokens of sequence 2 (a partial tail: the first
+    # step copies it)
+    lens = [1, 15, 40, 16, 47, 300, 511, 2]
+    w = workloads.custom_decode("batch", lens, 32, 8, 128, 16, "bf16", seed=71,
+                                spare_blocks=64)
+    w.setup.append(workloads.Op("share", (2, 9, 20), len(w.setup)))
+    w.decode_seqs.append(9)
+    return w
+
+
+def _step_inputs(w, step):
+    n = len(w.decode_seqs)
+    q = workloads.normal((n, w.num_heads, w.head_dim), 9000 + step)
+    k = workloads.normal((n, w.num_kv_heads, w.head_dim), 9100 + step)
+    v = workloads.normal((n, w.num_kv_heads, w.head_dim), 9200 + step)
+    return q, k, v
+
+
+@pytest.mark.parametrize("kind", ["bf16", "int8", "fp8"])
+def test_batch_steps_match_separate_calls_and_oracle(kind):
+    w = _workload(kind)
+    q8 = kind if kind != "bf16" else False
+    g = DeviceRun(w, q8=q8).apply(w.setup)           # the batch path
+    r = DeviceRun(w, q8=q8).apply(w.setup)           # the same step as separate calls
+    o = OracleRun(w, q8=q8).apply(w.setup)
+    seqs = w.decode_seqs
+    mb = 40
+    batch = pa.Batch(g.pool, seqs, w.num_heads, mb)
+    n = len(seqs)
+    h_out = torch.empty((n, w.num_heads, w.head_dim), dtype=torch.float32).pin_memory()
+    for step in range(4):
+        q, k, v = _step_inputs(w, step)
+        hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+        batch.step(hq, hk, hv, h_out)
+        batch.sync()
+        got = h_out.numpy().copy()
+        # the reference path: plan, copy-on-write, fused append + decode
+        slots, cow = r.pool.plan_append(seqs, [1] * n)
+        if cow:
+            src = torch.tensor([c[0] for c in cow], dtype=torch.int32, device="cuda")
+            dst = torch.tensor([c[1] for c in cow], dtype=torch.int32, device="cuda")
+            r.pool.cow_copy(src, dst)
+        # tables as wide as the batch's (the automatic partitions follow the width)
+        t, lens = r.pool.block_tables(seqs, mb)
+        ref = r.pool.decode_append(q.cuda(), k.cuda(), v.cuda(),
+                                   torch.tensor(slots, dtype=torch.int64, device="cuda"),
+                                   torch.from_numpy(t).cuda(),
+                                   torch.from_numpy(lens).cuda()).cpu().numpy()
+        assert np.array_equal(got, ref), step
+        # the oracle: same plan, same rows, attention over the gathered cache
+        for i, s in enumerate(seqs):
+            kk, vv = k[i:i + 1].double().numpy(), v[i:i + 1].double().numpy()
+            if q8:
+                from oracle import stored_rows, stored_rows_fp8
+                rows = stored_rows_fp8 if q8 == "fp8" else stored_rows
+                kk, vv = rows(kk)[2], rows(vv)[2]
+            o_slots, _ = o.pool.append(s, 1, kk.astype(o.pool.keys.dtype),
+                                       vv.astype(o.pool.keys.dtype))
+            assert o_slots == [slots[i]]
+        assert g.pool.refcounts() == o.pool.refs
+        for s in seqs:
+            assert g.pool.table(s) == (o.pool.tables[s], o.pool.lengths[s])
+        qd = q.to(torch.float64).numpy()
+        worst = 0.0
+        for i in range(n):
+            ref_o = o.attention(i, qd[i:i + 1])
+            for h, val in ref_o.items():
+                worst = max(worst, float(np.abs(got[i, h] - val[0]).max()))
+        assert worst <= TOL_DECODE, (step, worst)
+        if step == 1:
+            # drafted tokens rejected: every sequence gives its last token back
+            batch.rollback()
+            keep = [r.pool.table(s)[1] - 1 for s in seqs]
+            r.pool.truncate(seqs, keep)
+            for s, kl in zip(seqs, keep):
+                o.pool.truncate(s, kl)
+            assert g.pool.table(seqs[0]) == (o.pool.tables[seqs[0]], o.pool.lengths[seqs[0]])
+    assert g.pool.get_error() == 0
+    batch.close()
+
+
+def test_batch_rejects_a_full_table():
+    w = workloads.custom_decode("batchfull", [32, 5], 8, 8, 128, 16, "bf16", seed=3,
+                                spare_blocks=8)
+    g = DeviceRun(w).apply(w.setup)
+    batch = pa.Batch(g.pool, [0, 1], 8, 2)           # sequence 0 fills its 2 blocks
+    q, k, v = (workloads.normal((2, 8, 128), s) for s in (1, 2, 3))
+    out = torch.empty((2, 8, 128), dtype=torch.float32)
+    before = g.pool.table(0)
+    with pytest.raises(pa.PAError) as e:
+        batch.step(q, k[:, :8], v[:, :8], out)
+    assert e.value.code == 1
+    assert g.pool.table(0) == before                 # nothing was planned
+    batch.close()
