@@ -449,13 +449,17 @@ def run_workload(args, dist, config, kv="bf16", win=0, sinks=0, *, steps, min_ms
         metric = metric_name(w, q8, win, sinks)
         unit = "GB/s"
         achieved = kvb / (kern_ms * 1e-3) / 1e9
-        kname = (f"decode_q8_kernel<{'true' if q8 == 'fp8' else 'false'}>" if q8 else
+        # int8 / FP8 pools: the tcgen05 kernel up to 4 heads per group, the
+        # warp-level one above
+        q8tc = bool(q8) and w.num_heads // w.num_kv_heads <= 4
+        kname = (("decode_q8tc_kernel" if q8tc else "decode_q8_kernel") if q8 else
                  "decode_mma_kernel"
                  if pool.decode_path(w.num_heads) else "attention_generic_kernel")
+        kfile = ("decode_q8tc.cu" if q8tc else "decode_q8.cu") if q8 else "decode_mma.cu"
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4),
                 "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
-                "traffic": profiled_traffic("decode_q8.cu" if q8 else "decode_mma.cu",
+                "traffic": profiled_traffic(kfile,
                                             w.name + (f"_{q8}" if q8 else "")
                                             + (f"_window{win}_sinks{sinks}" if win else "")),
                 "kernel": (f"decode_order_kernel + {kname}" if order_only else
@@ -473,8 +477,9 @@ def run_workload(args, dist, config, kv="bf16", win=0, sinks=0, *, steps, min_ms
         "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": dist.world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": ("int8 KV codes (int8/fp16 MMA, fp32 softmax), bf16 Q" if q8 == "int8" else
-                  "fp8 e4m3 KV codes (fp16 MMA, fp32 softmax), bf16 Q" if q8 else "bf16"),
+        "dtype": ("int8 KV codes (int8 MMA on the codes, fp32 softmax), bf16 Q" if q8 == "int8"
+                  else "fp8 e4m3 KV codes (e4m3 MMA on the codes, fp32 softmax), bf16 Q" if q8
+                  else "bf16"),
         "data": "synthetic (seeded N(0,1), bf16-rounded)",
         "config": config_of(w, kv, win, sinks, dist),
         **extra,
