@@ -305,12 +305,15 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
     l1 += __shfl_xor_sync(0xffffffffu, l1, off);
   }
   named_bar_sync(1, 128);  // every consumer is done with the ring
-  float* so = reinterpret_cast<float*>(smem);  // [4][8][128]
-  float* sm = so + 4 * 8 * 128;                // [4][8]
+  // [4 warps][8 heads][kORow] partial O; the row pitch of 132 floats puts the
+  // four lanes c of a fragment column in four different bank octets
+  constexpr int kORow = 132;
+  float* so = reinterpret_cast<float*>(smem);
+  float* sm = so + 4 * 8 * kORow;              // [4][8]
   float* sl = sm + 32;                         // [4][8]
   {
-    float* w0 = so + (warp * 8 + 2 * c) * 128;
-    float* w1 = w0 + 128;
+    float* w0 = so + (warp * 8 + 2 * c) * kORow;
+    float* w1 = w0 + kORow;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       w0[16 * j + g] = o[j][0];
@@ -326,23 +329,34 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
     }
   }
   named_bar_sync(1, 128);
-  const int t = threadIdx.x;  // d column
+  // per (warp, head): the weight 2^(m_w - M) / sum_w l_w 2^(m_w - M) of the
+  // warp's partial O, worked out once by warp 0 (lane = warp w, head n)
   const bool zero = tail->any_bad != 0;
-  for (int n = 0; n < G; ++n) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[w * 8 + n]);
-    float num = 0.f, den = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float mw = sm[w * 8 + n];
-        const float sc = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-        num = fmaf(so[(w * 8 + n) * 128 + t], sc, num);
-        den = fmaf(sl[w * 8 + n], sc, den);
-      }
+  float* swt = sl + 32;                        // [4][8]
+  float* sM = swt + 32;                        // [8]
+  float* sden = sM + 8;                        // [8]
+  if (warp == 0) {
+    const int n = lane & 7, w = lane >> 3;
+    const float mw = sm[w * 8 + n];
+    float M = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, 8));
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 16));
+    const float sc = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+    float den = sl[w * 8 + n] * sc;
+    den += __shfl_xor_sync(0xffffffffu, den, 8);
+    den += __shfl_xor_sync(0xffffffffu, den, 16);
+    swt[w * 8 + n] = den > 0.f ? sc / den : 0.f;
+    if (w == 0) {
+      sM[n] = M;
+      sden[n] = den;
     }
-    const float val = (den > 0.f && !zero) ? num / den : 0.f;
+  }
+  named_bar_sync(1, 128);
+  const int t = threadIdx.x;  // d column
+  for (int n = 0; n < G; ++n) {
+    float val = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) val = fmaf(so[(w * 8 + n) * kORow + t], swt[w * 8 + n], val);
+    if (zero || !(sden[n] > 0.f)) val = 0.f;
     const int64_t bh = int64_t(b) * p.H + kvh * G + n;
     if (p.NP == 1) {
       p.out[bh * 128 + t] = val;
@@ -353,8 +367,8 @@ __global__ void __launch_bounds__(kDecThreads, kDecStages <= 8 ? 3 : 2) decode_m
       float* ws_o = ws_l + int64_t(p.B) * p.H * p.NP;
       ws_o[slot * 128 + t] = val;
       if (t == 0) {
-        ws_m[slot] = M;
-        ws_l[slot] = zero ? -1.f : den;  // -1 poisons the whole row
+        ws_m[slot] = sM[n];
+        ws_l[slot] = zero ? -1.f : sden[n];  // -1 poisons the whole row
       }
     }
   }
