@@ -242,24 +242,33 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t qa = smem_u32(smem + kOffQ);
+      // Descriptors of Q_A, Q_B and of each K and V stage: their high words
+      // are constants and their low words differ by fixed offsets, so each
+      // MMA needs one add.  This thread shares its issue slots with two
+      // softmax warps, and every instruction here delays the next MMA.
+      static_assert(kKStages == 2 && kVStages == 2, "two K and two V stages");
+      const uint64_t dq0 = desc_kmajor_sw128(smem_u32(smem + kOffQ));
+      const uint64_t dv0 = desc_mnmajor_sw128(smem_u32(smem + kOffV), kHalf, 1024);
+      const uint32_t hk = uint32_t(dq0 >> 32), hv = uint32_t(dv0 >> 32);
+      const uint32_t lq = uint32_t(dq0), lv = uint32_t(dv0);
+      const uint32_t lk = lq + ((kOffK - kOffQ) >> 4);
+      auto mk = [](uint32_t lo, uint32_t hi) { return (uint64_t(hi) << 32) | lo; };
       auto qk = [&](int x, int j) {                    // S_x = Q_x K(j)^T
-        const uint32_t kb = smem_u32(smem + kOffK + (j % kKStages) * kTile);
-        const uint32_t q = qa + x * kTile;
+        const uint32_t kl = lk + (j & 1) * (kTile >> 4), ql = lq + x * (kTile >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          umma_bf16(tbase + kColS + x * 128, desc_kmajor_sw128(q + off),
-                    desc_kmajor_sw128(kb + off), kIdescQK, kk > 0);
+          const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          umma_bf16(tbase + kColS + x * 128, mk(ql + off, hk), mk(kl + off, hk), kIdescQK,
+                    kk > 0);
         }
         umma_commit(&bars->s_full[x]);
       };
       auto pv = [&](int x, int j) {                    // O_x += P_x V(j)
-        const uint32_t vb = smem_u32(smem + kOffV + (j % kVStages) * kTile);
+        const uint32_t vl = lv + (j & 1) * (kTile >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_bf16_tmem_a(tbase + kColO + x * 128, tbase + kColS + x * 128 + kk * 8,
-                           desc_mnmajor_sw128(vb + kk * 2048, kHalf, 1024), kIdescPV,
+                           mk(vl + kk * (2048 >> 4), hv), kIdescPV,
                            (j > 0 || kk > 0) ? 1u : 0u);
       };
       bool ok = n_tiles > 0 && wait_or_abort(&bars->q_full, 0, bars, p.err) &&
