@@ -543,39 +543,59 @@ def run_workload(args, dist, config, kv="bf16", win=0, sinks=0, *, steps, min_ms
     return res
 
 
-def time_append(S, stream, cuda_index, n_app=300):
-    """reshape_and_cache of the step's rows at their planned slots, one launch
-    at a time with L2 flushed (a 256 MiB read) between launches."""
+def time_append(S, stream, cuda_index, n_app=300, rounds=10):
+    """reshape_and_cache of the step's rows at their planned slots with L2
+    flushed (a 256 MiB read) before every launch.  Two CUDA graphs, the flush
+    alone and the flush followed by the append, are replayed back to back in
+    alternating rounds; the append's time is the difference of their means (no
+    event between the flush and the append: an event record between two
+    launches adds microseconds, as much as this kernel takes)."""
     import torch
     pool = S.pool
+    dev = S.device
     # the flush reads a buffer larger than L2, leaving it full of clean lines
     # (a write flush would leave dirty lines for the timed kernel to evict)
-    flush = torch.ones(64 << 20, dtype=torch.float32, device=S.device)
-    sink = torch.empty(1, dtype=torch.float32, device=S.device)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    sink = torch.empty(1, dtype=torch.float32, device=dev)
     for _ in range(3):
+        torch.sum(flush, dim=0, keepdim=True, out=sink)
         pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(n_app)]
     torch.cuda.synchronize()
+    g_f, g_fa = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_f):
+        torch.sum(flush, dim=0, keepdim=True, out=sink)
+    with torch.cuda.graph(g_fa):
+        torch.sum(flush, dim=0, keepdim=True, out=sink)
+        pool.reshape_and_cache(S.step_k, S.step_v, S.slots, torch.cuda.current_stream(dev))
+    torch.cuda.synchronize()
+    per = max(1, n_app // rounds)
+    t_f, t_fa = [], []
     with SAMPLER.window() as clk:
-        for a, b in evs:
-            torch.sum(flush, dim=0, keepdim=True, out=sink)
-            a.record(stream)
-            pool.reshape_and_cache(S.step_k, S.step_v, S.slots, stream)
-            b.record(stream)
-        torch.cuda.synchronize()
+        for _ in range(rounds):
+            for g, acc in ((g_f, t_f), (g_fa, t_fa)):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(per):
+                    g.replay()
+                b.record(stream)
+                torch.cuda.synchronize()
+                acc.append(a.elapsed_time(b) / per)
     assert pool.get_error() == 0
-    app_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    del g_f, g_fa
+    app_ms = statistics.mean(t_fa) - statistics.mean(t_f)
     moved = 2 * 2 * S.step_k.numel() * S.step_k.element_size()   # K and V, read + write
     hbm, _, _, peak_kind = peaks()
     gbs = moved / (app_ms * 1e-3) / 1e9
-    return {"kernel": "reshape_and_cache_kernel<uint4>", "launches": n_app,
+    return {"kernel": "reshape_and_cache_kernel<uint4>", "launches": per * rounds,
             "kernel_ms": round(app_ms, 5), "bytes_per_launch": moved,
+            "kernel_timing": ("mean of (flush + append) graph replays minus mean of flush-alone "
+                              f"replays, {rounds} alternating rounds of {per}"),
+            "flush_ms": round(statistics.mean(t_f), 5),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4),
                          "traffic": profiled_traffic("kv_write.cu", "prefill_append"),
                          "peak_source": f"{peak_kind} hbm_gbs"},
-            "l2": "flushed between launches (a 256 MiB read, untimed)",
+            "l2": "flushed before every launch (a 256 MiB read)",
             "clocks": clk.summary()}
 
 
@@ -643,13 +663,13 @@ def run_e2e(args, S, dist, device, is_prefill, part, win, sinks):
     through the prepared batch, the rest through the separate calls."""
     w = S.w
     one_token = (not is_prefill) and bool(w.step) and all(op.args[1] == 1 for op in w.step) \
-        and not win and [op.args[0] for op in w.step] == list(w.decode_seqs)
+        and [op.args[0] for op in w.step] == list(w.decode_seqs)
     if one_token:
-        return run_e2e_batch(args, S, dist, device, part)
+        return run_e2e_batch(args, S, dist, device, part, win, sinks)
     return run_e2e_steps(args, S, dist, device, is_prefill, part, win, sinks)
 
 
-def run_e2e_batch(args, S, dist, device, part):
+def run_e2e_batch(args, S, dist, device, part, win=0, sinks=0):
     """The serving decode loop through pa_batch_step: each step is one C call
     that plans the step's appends on the host manager (step a1), uploads the
     plan, the changed table entries, the queries and the new K/V from pinned
@@ -672,7 +692,9 @@ def run_e2e_batch(args, S, dist, device, part):
     lens_now = [pool.table(s)[1] for s in seqs]
     pool.truncate(seqs, [L - 1 for L in lens_now])        # undo the set-up's plan
     batch = pa.Batch(pool, seqs, S.q.shape[1], S.tables.shape[1], part)
-    K = max(1, min(args.steps, args.e2e_steps))
+    if win:
+        batch.set_window(win, sinks)
+    K = max(1, args.e2e_steps)   # its own count: a serving loop's steady state, not the timed K
 
     def step():
         batch.step(h_q, h_k, h_v, h_out, stream=stream)
@@ -696,12 +718,14 @@ def run_e2e_batch(args, S, dist, device, part):
     ms = dist.max(max(a.elapsed_time(b) / K, wall_ms), device)
     batch.close()
     pool.plan_append(seqs, [1] * n)                       # back to the state the step assumes
-    v = dist.world * decode_bytes(w, S.lens_h, S.q8) / (ms * 1e-3) / 1e9
+    v = dist.world * decode_bytes(w, S.lens_h, S.q8, win, sinks) / (ms * 1e-3) / 1e9
     bi = (h_q.numel() * h_q.element_size() + 2 * h_k.numel() * h_k.element_size()
           + n * (8 + 4))                                  # + the plan: slots and lengths
     return {"value": round(v, 2), "unit": "GB/s", "h2d_bytes_per_step": int(bi),
             "d2h_bytes_per_step": int(h_out.numel() * 4), "ms_per_step": round(ms, 5),
-            "steps": K, "host_plan_in_step": True, "api": "pa_batch_step + pa_batch_rollback",
+            "steps": K, "host_plan_in_step": True,
+            "api": "pa_batch_step + pa_batch_rollback"
+                   + (" (after pa_batch_set_window)" if win else ""),
             "host_ms_per_step": round(host_ms, 5)}
 
 
@@ -739,7 +763,7 @@ def run_e2e_steps(args, S, dist, device, is_prefill, part, win, sinks):
         start = [L - k for L, k in zip(lens_now, n_new)]
         pool.truncate(seqs, start)                       # undo the set-up's plan
     bo = h_out.numel() * 4
-    K = max(1, min(args.steps, args.e2e_steps))
+    K = max(1, args.e2e_steps)   # its own count: a serving loop's steady state, not the timed K
     fused = (not is_prefill) and plan and not S.q8
     cow_bytes = [0]
 
@@ -974,7 +998,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=["tiny", "decode32", "ragged256", "splitk128k", "prefill"],
                     default="decode32")
-    ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--e2e-steps", type=int, default=200,
+                    help="steps of each end-to-end measurement (independent of --steps)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kv", choices=["bf16", "int8", "fp8"], default="bf16",

@@ -452,8 +452,8 @@ pa_status pa_batch_create(pa_pool* pool, const int32_t* seqs, int32_t n,
  *   head_dim] float32.  Use pinned host memory for asynchronous copies.
  * The plan, the table entries that changed since the previous step and the
  * inputs are uploaded on the batch's upload stream; the table patches,
- * copy-on-write copies and the fused append + decode (pa_decode_append) run
- * on `stream`; the output is downloaded on the batch's download stream.
+ * copy-on-write copies and the fused append + decode (pa_decode_append, or
+ * pa_decode_window_append after pa_batch_set_window) run on `stream`; the output is downloaded on the batch's download stream.
  * Successive steps alternate two buffer sets, so a step's transfers overlap
  * its neighbours' kernels.  The call returns once the work is queued: h_out
  * holds the result after pa_batch_sync, and the input buffers must not change
@@ -472,6 +472,15 @@ pa_status pa_batch_step(pa_batch* batch, const void* h_q, const void* h_key,
  * that were not accepted): pa_seq_truncate to one token less, host-only.  A
  * copy-on-write the step made stays. */
 pa_status pa_batch_rollback(pa_batch* batch);
+
+/* Decode the batch's later steps over a sink + recent window: key j is
+ * visible iff j < sinks or j >= kv_len - window ([P2] streaming_keep_indices
+ * with budget = sinks + window, as pa_decode_window_append); window = 0
+ * returns to full attention.  Waits for the device (the batch's partition
+ * scratch may be resized), so it belongs between phases of a loop, not in
+ * every step.  Errors: INVALID_ARG (window < 0, sinks < 0, sinks without a
+ * window), UNSUPPORTED (a pool without the tensor-core decode), CUDA. */
+pa_status pa_batch_set_window(pa_batch* batch, int32_t window, int32_t sinks);
 
 /* Wait until every step's output has reached its host buffer. */
 pa_status pa_batch_sync(pa_batch* batch);

@@ -36,7 +36,8 @@ EXPORTS = ["pa_pool_create", "pa_free", "pa_seq_create", "pa_seq_fork", "pa_seq_
            "pa_prefix_publish", "pa_prefix_clear", "pa_prefix_entries", "pa_pool_create_int8",
            "pa_decode_window", "pa_decode_window_workspace_bytes", "pa_pool_create_layers",
            "pa_pool_layer", "pa_decode_window_append", "pa_pool_create_fp8", "pa_seq_truncate",
-           "pa_batch_create", "pa_batch_step", "pa_batch_rollback", "pa_batch_sync",
+           "pa_batch_create", "pa_batch_step", "pa_batch_rollback", "pa_batch_set_window",
+           "pa_batch_sync",
            "pa_batch_free"]
 
 
@@ -111,6 +112,7 @@ def lib():
         "pa_batch_step": ([_P, _P, _P, _P, _F, _P, _P], C.c_int),
         "pa_batch_rollback": ([_P], C.c_int),
         "pa_batch_sync": ([_P], C.c_int),
+        "pa_batch_set_window": ([_P, _I32, _I32], C.c_int),
         "pa_batch_free": ([_P], C.c_int),
     }
     for name, (args, res) in sig.items():
@@ -609,6 +611,11 @@ class Batch:
 
     def rollback(self):
         _check(lib().pa_batch_rollback(self._h), "pa_batch_rollback")
+
+    def set_window(self, window, sinks=0):
+        """Later steps decode over a sink + recent window (window 0: full)."""
+        _check(lib().pa_batch_set_window(self._h, int(window), int(sinks)),
+               "pa_batch_set_window")
 
     def sync(self):
         _check(lib().pa_batch_sync(self._h), "pa_batch_sync")

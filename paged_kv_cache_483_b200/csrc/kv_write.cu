@@ -15,26 +15,46 @@
 
 namespace pa {
 
+// One warp per token row: the slot is read once and the lanes copy the row's
+// K and V vectors (no index division; up to four vectors of each in flight
+// per lane).
 template <typename V>
 __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const V* __restrict__ key, const V* __restrict__ value,
     V* __restrict__ k_cache, V* __restrict__ v_cache,
     const int64_t* __restrict__ slot_mapping, int32_t T, int64_t row_vecs,
     int64_t num_slots, int32_t* err) {
-  const int64_t total = int64_t(T) * row_vecs;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
-       i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t t = i / row_vecs, c = i - t * row_vecs;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
     const int64_t slot = __ldg(slot_mapping + t);
     if (slot < 0) continue;                    // padding token
     if (slot >= num_slots) {
-      if (c == 0) raise_err(err, PA_DEVERR_SLOT);
+      if (lane == 0) raise_err(err, PA_DEVERR_SLOT);
       continue;
     }
-    const V kv = key[i];
-    const V vv = value[i];
-    k_cache[slot * row_vecs + c] = kv;
-    v_cache[slot * row_vecs + c] = vv;
+    const V* ks = key + t * row_vecs;
+    const V* vs = value + t * row_vecs;
+    V* kd = k_cache + slot * row_vecs;
+    V* vd = v_cache + slot * row_vecs;
+    int64_t c = lane;
+    for (; c + 96 < row_vecs; c += 128) {
+      V k4[4], v4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        k4[u] = ks[c + 32 * u];
+        v4[u] = vs[c + 32 * u];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        kd[c + 32 * u] = k4[u];
+        vd[c + 32 * u] = v4[u];
+      }
+    }
+    for (; c < row_vecs; c += 32) {
+      kd[c] = ks[c];
+      vd[c] = vs[c];
+    }
   }
 }
 
@@ -199,17 +219,17 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value,
   if (row_bytes % 16 == 0 && aligned(key, 16) && aligned(value, 16) &&
       aligned(k_cache, 16) && aligned(v_cache, 16)) {
     int64_t rv = row_bytes / 16;
-    reshape_and_cache_kernel<uint4><<<grid_for(T * rv, sms), 256, 0, stream>>>(
+    reshape_and_cache_kernel<uint4><<<grid_for(int64_t(T) * 32, sms), 256, 0, stream>>>(
         (const uint4*)key, (const uint4*)value, (uint4*)k_cache,
         (uint4*)v_cache, slots, T, rv, num_slots, err);
   } else if (row_bytes % 4 == 0) {
     int64_t rv = row_bytes / 4;
-    reshape_and_cache_kernel<uint32_t><<<grid_for(T * rv, sms), 256, 0, stream>>>(
+    reshape_and_cache_kernel<uint32_t><<<grid_for(int64_t(T) * 32, sms), 256, 0, stream>>>(
         (const uint32_t*)key, (const uint32_t*)value, (uint32_t*)k_cache,
         (uint32_t*)v_cache, slots, T, rv, num_slots, err);
   } else {
     int64_t rv = row_bytes / 2;
-    reshape_and_cache_kernel<uint16_t><<<grid_for(T * rv, sms), 256, 0, stream>>>(
+    reshape_and_cache_kernel<uint16_t><<<grid_for(int64_t(T) * 32, sms), 256, 0, stream>>>(
         (const uint16_t*)key, (const uint16_t*)value, (uint16_t*)k_cache,
         (uint16_t*)v_cache, slots, T, rv, num_slots, err);
   }

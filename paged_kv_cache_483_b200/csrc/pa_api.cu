@@ -904,6 +904,7 @@ struct pa_batch {
   pa_pool* pool = nullptr;
   std::vector<int32_t> seqs, ones;
   int32_t n = 0, H = 0, MB = 0, part = 0;
+  int32_t window = 0, sinks = 0;         // sink + recent window (0: full attention)
   size_t q_bytes = 0, kv_bytes = 0, out_bytes = 0, stage_bytes = 0;
   int32_t patch_cap = 0;                 // (row, index, value) triples per step
   int32_t* d_tables = nullptr;           // [n, MB]
@@ -1114,8 +1115,12 @@ pa_status pa_batch_step(pa_batch* b, const void* h_q, const void* h_key, const v
   if (ok) ok = pa::launch_table_patch(b->d_tables, MB, d_pat, npatch, s) == cudaSuccess;
   if (ok) ok = cow_blocks(p, d_csrc, d_cdst, ncow, s) == cudaSuccess;
   if (!ok) return PA_ERR_CUDA;
-  st = pa_decode_append(p, S.d_q, S.d_k, S.d_v, d_slots, n, b->H, b->d_tables, MB, d_lens,
-                        scale, b->part, b->d_ws, b->ws_bytes, S.d_out, stream);
+  st = b->window > 0
+           ? pa_decode_window_append(p, S.d_q, S.d_k, S.d_v, d_slots, n, b->H, b->d_tables,
+                                     MB, d_lens, scale, b->window, b->sinks, b->part, b->d_ws,
+                                     b->ws_bytes, S.d_out, stream)
+           : pa_decode_append(p, S.d_q, S.d_k, S.d_v, d_slots, n, b->H, b->d_tables, MB,
+                              d_lens, scale, b->part, b->d_ws, b->ws_bytes, S.d_out, stream);
   if (st != PA_OK) return st;
   // download on its own stream
   ok = cudaEventRecord(S.done, s) == cudaSuccess &&
@@ -1144,6 +1149,31 @@ pa_status pa_batch_rollback(pa_batch* b) {
     b->mirror_len[i] = keep[i];
     b->mirror_blocks[i] = int32_t(p->mgr->table(b->seqs[i])->size());
   }
+  return PA_OK;
+}
+
+pa_status pa_batch_set_window(pa_batch* b, int32_t window, int32_t sinks) {
+  if (!b || window < 0 || sinks < 0 || (window == 0 && sinks > 0)) return PA_ERR_INVALID_ARG;
+  pa_pool* p = b->pool;
+  if (window > 0 && !use_fast_decode(p, b->H)) return PA_ERR_UNSUPPORTED;
+  pa::DeviceScope on_pool_device(p->dev_id);
+  const size_t need = window > 0 ? pa_decode_window_workspace_bytes(p, b->n, b->H, b->MB,
+                                                                    window, sinks, b->part)
+                                 : pa_decode_workspace_bytes(p, b->n, b->H, b->MB, b->part);
+  if (need > b->ws_bytes) {
+    // the scratch may still be read by queued steps
+    if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
+    void* ws = nullptr;
+    if (cudaMalloc(&ws, need) != cudaSuccess) {
+      cudaGetLastError();
+      return PA_ERR_CUDA;
+    }
+    cudaFree(b->d_ws);
+    b->d_ws = ws;
+    b->ws_bytes = need;
+  }
+  b->window = window;
+  b->sinks = sinks;
   return PA_OK;
 }
 

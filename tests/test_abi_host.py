@@ -380,3 +380,4 @@ def test_batch_calls_on_host_pools_and_bad_arguments():
         assert fn(None) == 1
     assert L.pa_batch_free(None) == 0
     assert L.pa_batch_step(None, None, None, None, 1.0, None, None) == 1
+    assert L.pa_batch_set_window(None, 16, 0) == 1

@@ -121,3 +121,61 @@ def test_batch_rejects_a_full_table():
     assert e.value.code == 1
     assert g.pool.table(0) == before                 # nothing was planned
     batch.close()
+
+
+@pytest.mark.parametrize("kind", ["bf16", "int8"])
+def test_batch_window_steps_match_separate_calls_and_oracle(kind):
+    """pa_batch_set_window: later steps decode over 5 sink tokens and the last
+    40 ("vladkulikov.com modern-llms module 9 notebook", streaming_keep_indices
+    with budget = sinks + window); then full attention again."""
+    from oracle import attention_window
+    w = _workload(kind)
+    q8 = kind if kind != "bf16" else False
+    g = DeviceRun(w, q8=q8).apply(w.setup)
+    r = DeviceRun(w, q8=q8).apply(w.setup)
+    o = OracleRun(w, q8=q8).apply(w.setup)
+    seqs = w.decode_seqs
+    mb, window, sinks = 40, 40, 5
+    batch = pa.Batch(g.pool, seqs, w.num_heads, mb)
+    batch.set_window(window, sinks)
+    n = len(seqs)
+    G = w.num_heads // w.num_kv_heads
+    h_out = torch.empty((n, w.num_heads, w.head_dim), dtype=torch.float32).pin_memory()
+    for step in range(3):
+        if step == 2:
+            batch.set_window(0)                      # back to full attention
+        q, k, v = _step_inputs(w, step)
+        batch.step(q.pin_memory(), k.pin_memory(), v.pin_memory(), h_out)
+        batch.sync()
+        got = h_out.numpy().copy()
+        slots, cow = r.pool.plan_append(seqs, [1] * n)
+        if cow:
+            src = torch.tensor([c[0] for c in cow], dtype=torch.int32, device="cuda")
+            dst = torch.tensor([c[1] for c in cow], dtype=torch.int32, device="cuda")
+            r.pool.cow_copy(src, dst)
+        t, lens = r.pool.block_tables(seqs, mb)
+        args = (q.cuda(), k.cuda(), v.cuda(), torch.tensor(slots, dtype=torch.int64, device="cuda"),
+                torch.from_numpy(t).cuda(), torch.from_numpy(lens).cuda())
+        ref = (r.pool.decode_window_append(*args, window, sinks) if step < 2
+               else r.pool.decode_append(*args)).cpu().numpy()
+        assert np.array_equal(got, ref), step
+        for i, s in enumerate(seqs):
+            kk, vv = k[i:i + 1].double().numpy(), v[i:i + 1].double().numpy()
+            if q8:
+                from oracle import stored_rows
+                kk, vv = stored_rows(kk)[2], stored_rows(vv)[2]
+            o.pool.append(s, 1, kk.astype(o.pool.keys.dtype), vv.astype(o.pool.keys.dtype))
+        qd = q.to(torch.float64).numpy()
+        worst = 0.0
+        for i, s in enumerate(seqs):
+            kc, vc = o.pool.gather(s)
+            for j, kvh in enumerate(o.heads):
+                hs = list(range(kvh * G, (kvh + 1) * G))
+                win = window if step < 2 else 10 ** 9
+                ref_o = attention_window(qd[i:i + 1][:, hs], kc[:, j:j + 1].astype(np.float64),
+                                         vc[:, j:j + 1].astype(np.float64), win,
+                                         sinks if step < 2 else 0)
+                worst = max(worst, float(np.abs(got[i, hs] - ref_o[0]).max()))
+        assert worst <= TOL_DECODE, (step, worst)
+    assert g.pool.get_error() == 0
+    batch.close()
