@@ -159,9 +159,10 @@ pa_status pa_pool_layer(pa_pool* pool, int32_t layer, pa_pool** layer_pool);
  * On such a pool pa_append_kv / pa_reshape_and_cache take bf16 key/value
  * [T, Hkv, 128] and quantise them into their slots; pa_cow_copy copies whole
  * records; pa_decode and pa_decode_window (and pa_decode_append /
- * pa_decode_window_append, as two launches) dequantise in the kernel for
- * H / Hkv <= 8.  pa_prefill_chunk and groups above 8 return
- * PA_ERR_UNSUPPORTED.
+ * pa_decode_window_append, as two launches) dequantise in the tensor-core
+ * kernels for H / Hkv <= 8.  pa_prefill_chunk, and pa_decode for larger
+ * groups, take the CUDA-core path, which dequantises every element it reads
+ * (correct, not fast); windows there return PA_ERR_UNSUPPORTED.
  * Errors: PA_ERR_UNSUPPORTED (block_size != 16 or head_dim != 128),
  * PA_ERR_INVALID_ARG (NULL or misaligned kv_records, bad size or order),
  * PA_ERR_CUDA. */
@@ -407,8 +408,10 @@ pa_status pa_decode_window_append(pa_pool* pool, const void* q, const void* key,
  * the chunk's q_tokens queries are its last q_tokens positions; query qt
  * sees cached positions j <= kv_lens[b] - q_tokens + qt.  The chunk's own
  * K/V must already be in the pool (pa_append_kv).
- *   q: device [B, q_tokens, H, head_dim], pool dtype.  out: device
- *   [B, q_tokens, H, head_dim] float32.  Tables/kv_lens as pa_decode.
+ *   q: device [B, q_tokens, H, head_dim], pool dtype (bf16 on an int8 or FP8
+ *   pool, whose records the CUDA-core path dequantises element by element).
+ *   out: device [B, q_tokens, H, head_dim] float32.  Tables/kv_lens as
+ *   pa_decode.
  *   max_kv_splits: on the tensor-core path, the query tiles of the last,
  *   partial wave of CTAs may be split over their keys (at most this many
  *   parts; 0 = automatic, up to 4; 1 = never) and merged with the [P4]

@@ -5,7 +5,9 @@
 // (tiled_attention).  The scores follow "docs.rs ferrum-kv 0.4.0
 // src/attention.rs" (paged_attention): kv_h = h / (H / Hkv), query qt sees
 // positions j <= kv_len - q_tokens + qt.  This is the path for fp32 pools and
-// for shapes the tensor-core kernels do not take; it is correct, not fast.
+// for shapes the tensor-core kernels do not take (also chunked prefill and
+// large groups over int8 / FP8 pools, whose elements it dequantises one by
+// one); it is correct, not fast.
 #include <math.h>
 
 #include "common.cuh"
@@ -17,6 +19,57 @@ __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) {
   return __bfloat162float(x);
 }
+
+// Value of an E4M3 code (OCP 8-bit floating point: sign, 4 exponent bits of
+// bias 7, 3 mantissa bits; exponent field 0 holds the subnormals m * 2^-9;
+// 0x7F / 0xFF are NaN).
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  float v;
+  if (e == 0u)
+    v = float(m) * 0.001953125f;                       // 2^-9
+  else if (e == 15u && m == 7u)
+    v = __int_as_float(0x7FC00000);
+  else
+    v = ldexpf(float(8u + m), int(e) - 10);            // (1 + m/8) 2^(e-7)
+  return (c & 0x80u) ? -v : v;
+}
+
+// Element (token slot off of physical block pb, KV head kvh, dimension i) of
+// a pool's K and V.
+template <typename T>
+struct PlainKV {                       // [num_blocks, bs, Hkv, d] K and V arrays
+  const T* kc;
+  const T* vc;
+  int Hkv, d, bs;
+  __device__ float k(int pb, int off, int kvh, int i) const {
+    return to_f(kc[((int64_t(pb) * bs + off) * Hkv + kvh) * d + i]);
+  }
+  __device__ float v(int pb, int off, int kvh, int i) const {
+    return to_f(vc[((int64_t(pb) * bs + off) * Hkv + kvh) * d + i]);
+  }
+};
+
+template <bool kFp8>
+struct Q8KV {                          // packed (block, head) records, bs 16, d 128
+  const uint8_t* rec;
+  int Hkv;
+  __device__ const uint8_t* at(int pb, int kvh) const {
+    return rec + (int64_t(pb) * Hkv + kvh) * kQ8RecordBytes;
+  }
+  __device__ float code(uint32_t c) const {
+    return kFp8 ? e4m3_value(c) : float(int(int8_t(uint8_t(c))));
+  }
+  __device__ float k(int pb, int off, int kvh, int i) const {
+    const uint8_t* r = at(pb, kvh);
+    const uint32_t c = r[off * 128 + ((((i >> 4) ^ (off & 7)) << 4) | (i & 15))];
+    return code(c) * reinterpret_cast<const float*>(r + 4096)[off];
+  }
+  __device__ float v(int pb, int off, int kvh, int i) const {
+    const uint8_t* r = at(pb, kvh);
+    return code(r[2048 + i * 16 + off]) * reinterpret_cast<const float*>(r + 4160)[off];
+  }
+};
 
 constexpr int kGenThreads = 128;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -41,9 +94,9 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return r;
 }
 
-template <typename T>
+template <typename T, typename KV>
 __global__ void __launch_bounds__(kGenThreads) attention_generic_kernel(
-    const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
+    const T* __restrict__ q, const KV kv,
     const int32_t* __restrict__ tables, int MB, const int32_t* __restrict__ kv_lens,
     int q_tokens, int H, int Hkv, int d, int bs, int NB, float scale_log2,
     float* __restrict__ out, int32_t* err) {
@@ -76,7 +129,6 @@ __global__ void __launch_bounds__(kGenThreads) attention_generic_kernel(
 
   float acc[4] = {0.f, 0.f, 0.f, 0.f};  // d <= 512 = 4 x 128
   float m = -INFINITY, l = 0.f;
-  const int64_t tok_stride = int64_t(Hkv) * d;
   for (int c0 = 0; c0 < visible; c0 += kGenThreads) {
     const int j = c0 + tid;
     float s = -INFINITY;
@@ -87,9 +139,9 @@ __global__ void __launch_bounds__(kGenThreads) attention_generic_kernel(
         bad = 1;
         pb = -1;
       } else {
-        const T* krow = kc + (int64_t(pb) * bs + j % bs) * tok_stride + int64_t(kvh) * d;
+        const int off = j % bs;
         float dot = 0.f;
-        for (int i = 0; i < d; ++i) dot = fmaf(qf[i], to_f(krow[i]), dot);
+        for (int i = 0; i < d; ++i) dot = fmaf(qf[i], kv.k(pb, off, kvh, i), dot);
         s = dot;
       }
     }
@@ -111,9 +163,7 @@ __global__ void __launch_bounds__(kGenThreads) attention_generic_kernel(
         const int pbj = blk[jj];
         if (pbj < 0) continue;
         const int jt = c0 + jj;
-        a = fmaf(pr[jj], to_f(vc[(int64_t(pbj) * bs + jt % bs) * tok_stride +
-                                 int64_t(kvh) * d + i]),
-                 a);
+        a = fmaf(pr[jj], kv.v(pbj, jt % bs, kvh, i), a);
       }
       acc[r] = a;
     }
@@ -131,16 +181,31 @@ cudaError_t launch_attention_generic(const GenericArgs& a, cudaStream_t s) {
   dim3 grid(a.q_tokens, a.H, a.B);
   size_t smem = sizeof(float) * (a.d + kGenThreads + 32) + sizeof(int) * kGenThreads;
   const float sl2 = a.scale * kLog2e;
-  if (a.bf16) {
-    attention_generic_kernel<__nv_bfloat16><<<grid, kGenThreads, smem, s>>>(
-        (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k_cache,
-        (const __nv_bfloat16*)a.v_cache, a.tables, a.MB, a.kv_lens, a.q_tokens,
-        a.H, a.Hkv, a.d, a.bs, a.NB, sl2, a.out, a.err);
+  const int32_t* t = a.tables;
+  if (a.q8) {                          // bf16 queries over packed int8 / FP8 records
+    const auto* q = static_cast<const __nv_bfloat16*>(a.q);
+    const auto* rec = static_cast<const uint8_t*>(a.k_cache);
+    if (a.q8 == 2)
+      attention_generic_kernel<<<grid, kGenThreads, smem, s>>>(
+          q, Q8KV<true>{rec, a.Hkv}, t, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs,
+          a.NB, sl2, a.out, a.err);
+    else
+      attention_generic_kernel<<<grid, kGenThreads, smem, s>>>(
+          q, Q8KV<false>{rec, a.Hkv}, t, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs,
+          a.NB, sl2, a.out, a.err);
+  } else if (a.bf16) {
+    using B = __nv_bfloat16;
+    attention_generic_kernel<<<grid, kGenThreads, smem, s>>>(
+        static_cast<const B*>(a.q),
+        PlainKV<B>{static_cast<const B*>(a.k_cache), static_cast<const B*>(a.v_cache), a.Hkv,
+                   a.d, a.bs},
+        t, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs, a.NB, sl2, a.out, a.err);
   } else {
-    attention_generic_kernel<float><<<grid, kGenThreads, smem, s>>>(
-        (const float*)a.q, (const float*)a.k_cache, (const float*)a.v_cache,
-        a.tables, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs, a.NB, sl2,
-        a.out, a.err);
+    attention_generic_kernel<<<grid, kGenThreads, smem, s>>>(
+        static_cast<const float*>(a.q),
+        PlainKV<float>{static_cast<const float*>(a.k_cache),
+                       static_cast<const float*>(a.v_cache), a.Hkv, a.d, a.bs},
+        t, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs, a.NB, sl2, a.out, a.err);
   }
   return cudaGetLastError();
 }

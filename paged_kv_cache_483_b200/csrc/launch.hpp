@@ -61,6 +61,7 @@ struct GenericArgs {
   float* out;  // [B, q_tokens, H, d]
   int32_t* err;
   bool bf16;
+  int32_t q8;     // 0: K/V arrays of the pool dtype; 1 / 2: int8 / FP8 records, bf16 q
 };
 cudaError_t launch_attention_generic(const GenericArgs& a, cudaStream_t s);
 

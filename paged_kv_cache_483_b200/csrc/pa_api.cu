@@ -674,6 +674,20 @@ int32_t pa_prefill_path(const pa_pool* p, int32_t H) {
   return (p && use_fast_prefill(p, H)) ? 1 : 0;
 }
 
+// The CUDA-core path: any pool dtype (int8 / FP8 records dequantised element
+// by element, bf16 queries), any head_dim <= 512, block or group size.
+static pa::GenericArgs generic_args(const pa_pool* p, const void* q, int32_t B,
+                                    int32_t q_tokens, int32_t H, const int32_t* tables,
+                                    int32_t max_blocks, const int32_t* kv_lens, float scale,
+                                    float* out) {
+  pa::GenericArgs g{q, p->k_cache, p->v_cache, tables, max_blocks,
+                    kv_lens, B, q_tokens, H, p->num_kv_heads, p->head_dim,
+                    p->block_size, p->num_blocks, scale, out, p->d_err,
+                    p->dtype == PA_BF16, 0};
+  if (is_q8(p->dtype)) g.q8 = p->dtype == PA_FP8 ? 2 : 1;
+  return g;
+}
+
 static pa_status decode_fast(pa_pool* p, const void* q, int32_t B, int32_t H,
                              const int32_t* d_block_tables, int32_t max_blocks,
                              const int32_t* d_kv_lens, float scale, int32_t partition_tokens,
@@ -755,13 +769,9 @@ pa_status pa_decode(pa_pool* p, const void* q, int32_t B, int32_t H,
     return decode_fast(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale,
                        partition_tokens, workspace, workspace_bytes, out, stream, nullptr,
                        nullptr, nullptr);
-  if (is_q8(p->dtype)) return PA_ERR_UNSUPPORTED;   // G > 8 on an int8 / FP8 pool
   if (partition_tokens % p->block_size) return PA_ERR_INVALID_ARG;
-  pa::GenericArgs g{q, p->k_cache, p->v_cache, d_block_tables, max_blocks,
-                    d_kv_lens, B, 1, H, p->num_kv_heads, p->head_dim,
-                    p->block_size, p->num_blocks, scale, out, p->d_err,
-                    p->dtype == PA_BF16};
-  return cuda_status(pa::launch_attention_generic(g, s));
+  return cuda_status(pa::launch_attention_generic(
+      generic_args(p, q, B, 1, H, d_block_tables, max_blocks, d_kv_lens, scale, out), s));
 }
 
 size_t pa_decode_window_workspace_bytes(const pa_pool* p, int32_t B, int32_t H,
@@ -850,10 +860,9 @@ pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,
   if (st != PA_OK) return st;
   pa::DeviceScope on_pool_device(p->dev_id);
   if (q_tokens <= 0 || q_tokens > 65535 || max_kv_splits < 0) return PA_ERR_INVALID_ARG;
-  if (is_q8(p->dtype)) return PA_ERR_UNSUPPORTED;
   if (B == 0) return PA_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (use_fast_prefill(p, H)) {
+  if (!is_q8(p->dtype) && use_fast_prefill(p, H)) {
     if (!aligned16(q)) return PA_ERR_INVALID_ARG;
     pa::PrefillArgs a{q, d_block_tables, max_blocks, d_kv_lens, B, q_tokens, H,
                       p->num_kv_heads, p->num_blocks, scale, out, p->d_err,
@@ -861,11 +870,9 @@ pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,
                       p->split_o ? p->sms : 0};
     return cuda_status(pa::launch_prefill_fast(&p->tmK, &p->tmV, a, p->sms, s));
   }
-  pa::GenericArgs g{q, p->k_cache, p->v_cache, d_block_tables, max_blocks,
-                    d_kv_lens, B, q_tokens, H, p->num_kv_heads, p->head_dim,
-                    p->block_size, p->num_blocks, scale, out, p->d_err,
-                    p->dtype == PA_BF16};
-  return cuda_status(pa::launch_attention_generic(g, s));
+  return cuda_status(pa::launch_attention_generic(
+      generic_args(p, q, B, q_tokens, H, d_block_tables, max_blocks, d_kv_lens, scale, out),
+      s));
 }
 
 }  // extern "C"
