@@ -162,7 +162,7 @@ pa_status pa_pool_layer(pa_pool* pool, int32_t layer, pa_pool** layer_pool);
  * pa_decode_window_append, as two launches) dequantise in the tensor-core
  * kernels for H / Hkv <= 8.  pa_prefill_chunk, and pa_decode for larger
  * groups, take the CUDA-core path, which dequantises every element it reads
- * (correct, not fast); windows there return PA_ERR_UNSUPPORTED.
+ * (correct, not fast), windows included.
  * Errors: PA_ERR_UNSUPPORTED (block_size != 16 or head_dim != 128),
  * PA_ERR_INVALID_ARG (NULL or misaligned kv_records, bad size or order),
  * PA_ERR_CUDA. */
@@ -355,10 +355,12 @@ pa_status pa_decode(pa_pool* pool, const void* q, int32_t B, int32_t H,
  * j >= kv_lens[b] - window); with kv_lens[b] <= sinks + window every key is.
  * The kernels walk only the blocks that hold a visible key, so a long
  * sequence costs about sinks + window tokens.  Arguments, layouts and errors
- * as pa_decode, plus window >= 1 and sinks >= 0 (else INVALID_ARG); the
- * tensor-core paths only (bf16, int8 or FP8 pool, block 16, head_dim 128,
- * H / Hkv <= 8), else PA_ERR_UNSUPPORTED.  partition_tokens splits the walked
- * blocks; workspace: pa_decode_window_workspace_bytes bytes. */
+ * as pa_decode, plus window >= 1 and sinks >= 0 (else INVALID_ARG).  Shapes
+ * outside the tensor-core kernels (fp32 pools, other head_dim or block sizes,
+ * groups above 8) take the CUDA-core kernel, which walks the visible keys
+ * only.  partition_tokens splits the walked blocks (tensor-core paths);
+ * workspace: pa_decode_window_workspace_bytes bytes (0 on the CUDA-core
+ * path). */
 size_t pa_decode_window_workspace_bytes(const pa_pool* pool, int32_t B, int32_t H,
                                         int32_t max_blocks, int32_t window,
                                         int32_t sinks, int32_t partition_tokens);
@@ -482,7 +484,7 @@ pa_status pa_batch_rollback(pa_batch* batch);
  * returns to full attention.  Waits for the device (the batch's partition
  * scratch may be resized), so it belongs between phases of a loop, not in
  * every step.  Errors: INVALID_ARG (window < 0, sinks < 0, sinks without a
- * window), UNSUPPORTED (a pool without the tensor-core decode), CUDA. */
+ * window), CUDA. */
 pa_status pa_batch_set_window(pa_batch* batch, int32_t window, int32_t sinks);
 
 /* Wait until every step's output has reached its host buffer. */

@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kGenThreads) attention_generic_kernel(
     const T* __restrict__ q, const KV kv,
     const int32_t* __restrict__ tables, int MB, const int32_t* __restrict__ kv_lens,
     int q_tokens, int H, int Hkv, int d, int bs, int NB, float scale_log2,
-    float* __restrict__ out, int32_t* err) {
+    float* __restrict__ out, int32_t* err, int window, int sinks) {
   extern __shared__ float gen_smem[];
   float* qf = gen_smem;              // [d]
   float* pr = qf + d;                // [128] scores, then weights
@@ -122,7 +122,17 @@ __global__ void __launch_bounds__(kGenThreads) attention_generic_kernel(
     for (int i = tid; i < d; i += kGenThreads) orow[i] = 0.f;
     return;
   }
-  const int visible = kv_len - q_tokens + qt + 1;  // keys 0 .. visible-1
+  int visible = kv_len - q_tokens + qt + 1;  // keys 0 .. visible-1
+  // Sink + recent window (decode, window > 0): the keys walked are the first
+  // `sinks` and the last `window` ("vladkulikov.com modern-llms module 9
+  // notebook", streaming_keep_indices); walk index v maps to key key_at(v).
+  int lo = 0, ns = visible;
+  if (window > 0 && visible > sinks + window) {
+    ns = sinks;
+    lo = visible - window;
+    visible = sinks + window;
+  }
+  auto key_at = [&](int v) { return v < ns ? v : lo + (v - ns); };
   const T* qrow = q + ((int64_t(b) * q_tokens + qt) * H + h) * d;
   for (int i = tid; i < d; i += kGenThreads) qf[i] = to_f(qrow[i]) * scale_log2;
   __syncthreads();
@@ -130,10 +140,10 @@ __global__ void __launch_bounds__(kGenThreads) attention_generic_kernel(
   float acc[4] = {0.f, 0.f, 0.f, 0.f};  // d <= 512 = 4 x 128
   float m = -INFINITY, l = 0.f;
   for (int c0 = 0; c0 < visible; c0 += kGenThreads) {
-    const int j = c0 + tid;
+    const int j = c0 + tid < visible ? key_at(c0 + tid) : 0;
     float s = -INFINITY;
     int pb = -1;
-    if (j < visible) {
+    if (c0 + tid < visible) {
       pb = tables[int64_t(b) * MB + j / bs];
       if (pb < 0 || pb >= NB) {
         bad = 1;
@@ -162,7 +172,7 @@ __global__ void __launch_bounds__(kGenThreads) attention_generic_kernel(
       for (int jj = 0; jj < n; ++jj) {
         const int pbj = blk[jj];
         if (pbj < 0) continue;
-        const int jt = c0 + jj;
+        const int jt = key_at(c0 + jj);
         a = fmaf(pr[jj], kv.v(pbj, jt % bs, kvh, i), a);
       }
       acc[r] = a;
@@ -188,24 +198,26 @@ cudaError_t launch_attention_generic(const GenericArgs& a, cudaStream_t s) {
     if (a.q8 == 2)
       attention_generic_kernel<<<grid, kGenThreads, smem, s>>>(
           q, Q8KV<true>{rec, a.Hkv}, t, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs,
-          a.NB, sl2, a.out, a.err);
+          a.NB, sl2, a.out, a.err, a.window, a.sinks);
     else
       attention_generic_kernel<<<grid, kGenThreads, smem, s>>>(
           q, Q8KV<false>{rec, a.Hkv}, t, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs,
-          a.NB, sl2, a.out, a.err);
+          a.NB, sl2, a.out, a.err, a.window, a.sinks);
   } else if (a.bf16) {
     using B = __nv_bfloat16;
     attention_generic_kernel<<<grid, kGenThreads, smem, s>>>(
         static_cast<const B*>(a.q),
         PlainKV<B>{static_cast<const B*>(a.k_cache), static_cast<const B*>(a.v_cache), a.Hkv,
                    a.d, a.bs},
-        t, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs, a.NB, sl2, a.out, a.err);
+        t, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs, a.NB, sl2, a.out, a.err,
+        a.window, a.sinks);
   } else {
     attention_generic_kernel<<<grid, kGenThreads, smem, s>>>(
         static_cast<const float*>(a.q),
         PlainKV<float>{static_cast<const float*>(a.k_cache),
                        static_cast<const float*>(a.v_cache), a.Hkv, a.d, a.bs},
-        t, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs, a.NB, sl2, a.out, a.err);
+        t, a.MB, a.kv_lens, a.q_tokens, a.H, a.Hkv, a.d, a.bs, a.NB, sl2, a.out, a.err,
+        a.window, a.sinks);
   }
   return cudaGetLastError();
 }

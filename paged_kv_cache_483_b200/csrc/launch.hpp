@@ -62,6 +62,7 @@ struct GenericArgs {
   int32_t* err;
   bool bf16;
   int32_t q8;     // 0: K/V arrays of the pool dtype; 1 / 2: int8 / FP8 records, bf16 q
+  int32_t window = 0, sinks = 0;   // decode only: keys j < sinks or j >= kv_len - window
 };
 cudaError_t launch_attention_generic(const GenericArgs& a, cudaStream_t s);
 

@@ -791,8 +791,15 @@ pa_status pa_decode_window(pa_pool* p, const void* q, int32_t B, int32_t H,
   if (st != PA_OK) return st;
   pa::DeviceScope on_pool_device(p->dev_id);
   if (partition_tokens < 0 || window < 1 || sinks < 0) return PA_ERR_INVALID_ARG;
-  if (!use_fast_decode(p, H)) return PA_ERR_UNSUPPORTED;
   if (B == 0) return PA_OK;
+  if (!use_fast_decode(p, H)) {
+    if (partition_tokens % p->block_size) return PA_ERR_INVALID_ARG;
+    pa::GenericArgs g =
+        generic_args(p, q, B, 1, H, d_block_tables, max_blocks, d_kv_lens, scale, out);
+    g.window = window;
+    g.sinks = sinks;
+    return cuda_status(pa::launch_attention_generic(g, static_cast<cudaStream_t>(stream)));
+  }
   return decode_fast(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale, partition_tokens,
                      workspace, workspace_bytes, out, stream, nullptr, nullptr, nullptr, window,
                      sinks);
@@ -833,10 +840,10 @@ pa_status pa_decode_window_append(pa_pool* p, const void* q, const void* key,
   pa::DeviceScope on_pool_device(p->dev_id);
   if (B > 0 && (!key || !value || !d_slot_mapping)) return PA_ERR_INVALID_ARG;
   if (partition_tokens < 0 || window < 1 || sinks < 0) return PA_ERR_INVALID_ARG;
-  if (!use_fast_decode(p, H)) return PA_ERR_UNSUPPORTED;
   if (B == 0) return PA_OK;
-  if (is_q8(p->dtype)) {
-    // the quantising append is its own launch on an int8 / FP8 pool
+  if (is_q8(p->dtype) || !use_fast_decode(p, H)) {
+    // the quantising append is its own launch on an int8 / FP8 pool, and the
+    // CUDA-core path decodes after a separate append
     st = pa_reshape_and_cache(p, key, value, d_slot_mapping, B, stream);
     if (st != PA_OK) return st;
     return pa_decode_window(p, q, B, H, d_block_tables, max_blocks, d_kv_lens, scale, window,
@@ -1162,7 +1169,6 @@ pa_status pa_batch_rollback(pa_batch* b) {
 pa_status pa_batch_set_window(pa_batch* b, int32_t window, int32_t sinks) {
   if (!b || window < 0 || sinks < 0 || (window == 0 && sinks > 0)) return PA_ERR_INVALID_ARG;
   pa_pool* p = b->pool;
-  if (window > 0 && !use_fast_decode(p, b->H)) return PA_ERR_UNSUPPORTED;
   pa::DeviceScope on_pool_device(p->dev_id);
   const size_t need = window > 0 ? pa_decode_window_workspace_bytes(p, b->n, b->H, b->MB,
                                                                     window, sinks, b->part)

@@ -92,14 +92,54 @@ def test_window_stale_slots_and_errors():
     assert g.pool.get_error() == 0
 
 
-def test_window_unsupported_on_generic_path():
-    w = workloads.custom_decode("win4", [9, 40], 8, 2, 32, 8, "f32", seed=4, spare_blocks=4)
-    g = DeviceRun(w).apply(w.setup)
+@pytest.mark.parametrize("shape", [
+    ("f32", 8, 2, 32, 8, False),      # fp32 pool, head_dim 32, block 8
+    ("f32", 6, 3, 80, 4, False),      # head_dim 80, block 4
+    ("bf16", 128, 8, 128, 16, True),  # int8 pool, group 16
+    ("bf16", 128, 8, 128, 16, "fp8"), # FP8 pool, group 16
+])
+def test_window_on_generic_path(shape):
+    # shapes outside the tensor-core kernels: the CUDA-core kernel walks the
+    # visible keys only, fp32 arithmetic, every row at 1e-4
+    dtype, H, Hkv, d, bs, q8 = shape
+    w = workloads.custom_decode("win4", LENS, H, Hkv, d, bs, dtype, seed=4 + H + d,
+                                spare_blocks=4)
+    g = DeviceRun(w, q8=q8).apply(w.setup)
+    assert g.pool.decode_path(H) == 0
+    o = OracleRun(w, q8=q8).apply(w.setup)
     tables, lens, _, _ = g.tables()
-    q = torch.zeros(2, 8, 32, dtype=torch.float32, device="cuda")
-    with pytest.raises(pa.PAError) as e:
-        g.pool.decode_window(q, tables, lens, 4, 0)
-    assert e.value.code == 7
+    qd = w.queries()[:, 0].contiguous().cuda()
+    q = q64(w)
+    for window, sinks in WINDOWS:
+        out = g.pool.decode_window(qd, tables, lens, window, sinks).cpu().numpy()
+        ref = _oracle_window(o, w, q, window, sinks)
+        worst = max(float(np.abs(out[i, h] - r).max()) for i, rows in enumerate(ref)
+                    for h, r in rows.items())
+        assert worst <= 1e-4, (window, sinks, worst)
+        assert np.all(out[LENS.index(0)] == 0)
+    assert g.pool.get_error() == 0
+
+
+def test_window_append_on_generic_path_equals_two_calls():
+    # the new token's append, then the windowed decode (group 16, int8 pool)
+    w = workloads.custom_decode("win5", [5, 40, 300], 128, 8, 128, 16, "bf16", seed=5,
+                                spare_blocks=4, split_last=1)
+    a = DeviceRun(w, q8=True).apply(w.setup)
+    b = DeviceRun(w, q8=True).apply(w.setup)
+    seqs = [op.args[0] for op in w.step]
+    slots, _ = a.pool.plan_append(seqs, [1] * len(seqs))
+    slots_b, _ = b.pool.plan_append(seqs, [1] * len(seqs))
+    assert slots == slots_b
+    ks, vs = zip(*[w.kv_for(op) for op in w.step])
+    key, val = torch.cat(ks).cuda(), torch.cat(vs).cuda()
+    d_slots = torch.tensor(slots, dtype=torch.int64, device="cuda")
+    tables, lens, _, _ = a.tables()
+    q = w.queries()[:, 0].contiguous().cuda()
+    fused = a.pool.decode_window_append(q, key, val, d_slots, tables, lens, 17, 4)
+    b.pool.reshape_and_cache(key, val, d_slots)
+    two = b.pool.decode_window(q, tables, lens, 17, 4)
+    assert torch.equal(fused, two)
+    assert a.pool.get_error() == 0 and b.pool.get_error() == 0
 
 
 @pytest.mark.parametrize("q8", [False, True, "fp8"])
