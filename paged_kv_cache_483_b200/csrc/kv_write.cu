@@ -17,7 +17,8 @@ namespace pa {
 
 // One warp per token row: the slot is read once and the lanes copy the row's
 // K and V vectors (no index division; up to four vectors of each in flight
-// per lane).
+// per lane).  The row's first vectors are loaded before the slot is known, so
+// the slot's round trip overlaps the row's.
 template <typename V>
 __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const V* __restrict__ key, const V* __restrict__ value,
@@ -28,18 +29,32 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
   const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
   for (int64_t t = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
     const int64_t slot = __ldg(slot_mapping + t);
+    const V* ks = key + t * row_vecs;
+    const V* vs = value + t * row_vecs;
+    V k4[4], v4[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (lane + 32 * u < row_vecs) {
+        k4[u] = ks[lane + 32 * u];
+        v4[u] = vs[lane + 32 * u];
+      }
+    }
     if (slot < 0) continue;                    // padding token
     if (slot >= num_slots) {
       if (lane == 0) raise_err(err, PA_DEVERR_SLOT);
       continue;
     }
-    const V* ks = key + t * row_vecs;
-    const V* vs = value + t * row_vecs;
     V* kd = k_cache + slot * row_vecs;
     V* vd = v_cache + slot * row_vecs;
-    int64_t c = lane;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (lane + 32 * u < row_vecs) {
+        kd[lane + 32 * u] = k4[u];
+        vd[lane + 32 * u] = v4[u];
+      }
+    }
+    int64_t c = lane + 128;
     for (; c + 96 < row_vecs; c += 128) {
-      V k4[4], v4[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         k4[u] = ks[c + 32 * u];
