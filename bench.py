@@ -676,10 +676,12 @@ def run_e2e_batch(args, S, dist, device, part, win=0, sinks=0):
     host memory, runs copy-on-write copies and the fused append + decode, and
     downloads the output; pa_batch_rollback then gives every sequence's token
     back (host-only) so that every step is the same step.  The timed region
-    holds K steps and the final wait for the last output.  Copies of
-    consecutive steps overlap their neighbours' kernels (two buffer sets, two
-    copy streams).  A copy-on-write of a shared partial tail happens in the
-    first step only (the tail is private afterwards), as in serving."""
+    holds K steps and the final wait for the last output.  The transfers of
+    consecutive steps overlap their neighbours' kernels (two buffer sets; the
+    uploads are one kernel that reads the pinned inputs in place, copies on
+    quantised pools; each download is queued behind the next step's
+    uploads).  A copy-on-write of a shared partial tail happens in the first
+    step only (the tail is private afterwards), as in serving."""
     import torch
     import paged_kv_cache_483_b200 as pa
     pool, w = S.pool, S.w

@@ -441,7 +441,8 @@ pa_status pa_prefill_chunk(pa_pool* pool, const void* q, int32_t B,
  * with H heads, tables up to max_blocks wide (a sequence may grow to
  * max_blocks * block_size tokens), partition_tokens as pa_decode.  Uploads
  * the current tables and allocates the batch's device buffers (two sets of
- * q, new K/V, output and staging), pinned staging and two copy streams.
+ * q, new K/V, output and staging), pinned staging mapped into the device's
+ * address space, an upload stream and a download stream.
  * Errors: NO_DEVICE, UNKNOWN_SEQ, INVALID_ARG (n <= 0, a sequence twice, a
  * table wider than max_blocks, H not a multiple of num_kv_heads), CUDA. */
 typedef struct pa_batch pa_batch; /* opaque */
@@ -456,13 +457,21 @@ pa_status pa_batch_create(pa_pool* pool, const int32_t* seqs, int32_t n,
  *   in the pool dtype (bf16 on an int8 or FP8 pool); h_out: host [n, H,
  *   head_dim] float32.  Use pinned host memory for asynchronous copies.
  * The plan, the table entries that changed since the previous step and the
- * inputs are uploaded on the batch's upload stream; the table patches,
+ * inputs are uploaded on the batch's upload stream (highest priority): by one
+ * kernel that reads the host buffers in place when all are pinned, mapped into
+ * the device's address space and 16-byte aligned and the pool is bf16 or
+ * float32, else by one copy per buffer (pageable memory works, synchronously
+ * slower); the table patches,
  * copy-on-write copies and the fused append + decode (pa_decode_append, or
- * pa_decode_window_append after pa_batch_set_window) run on `stream`; the output is downloaded on the batch's download stream.
- * Successive steps alternate two buffer sets, so a step's transfers overlap
- * its neighbours' kernels.  The call returns once the work is queued: h_out
- * holds the result after pa_batch_sync, and the input buffers must not change
- * before then.  The batch's sequences change only through the batch between
+ * pa_decode_window_append after pa_batch_set_window) run on `stream`; the
+ * output is downloaded on the batch's download stream.  That download is
+ * queued by the next pa_batch_step call, after the next step's uploads, or by
+ * pa_batch_sync: queued ahead of the next uploads, a copy that waits for this
+ * step's kernels would hold them up whenever the two copy streams share a
+ * hardware queue.  Successive steps alternate two buffer sets, so a step's
+ * transfers overlap its neighbours' kernels.  The call returns once the work
+ * is queued: h_out holds the result after pa_batch_sync (pa_batch_free also
+ * completes it), and the input buffers must not change before then.  The batch's sequences change only through the batch between
  * steps, or through pa_seq_truncate (any other change is picked up by
  * comparing whole tables).
  * Errors: those of pa_plan_append (nothing changes), UNKNOWN_SEQ (a sequence

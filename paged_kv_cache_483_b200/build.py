@@ -11,7 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpagedattn.so")
 SOURCES = ["block_manager.cpp", "pa_api.cu", "kv_write.cu", "attention_generic.cu",
            "decode_mma.cu", "decode_q8.cu", "decode_q8tc.cu", "prefill_tc.cu",
-           "decode_static.cu"]
+           "decode_static.cu", "batch_upload.cu"]
 HEADERS = ["block_manager.hpp", "common.cuh", "device_once.hpp", "launch.hpp", "tcgen05.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -43,6 +43,20 @@ cudaError_t launch_cow_copy(void* k_cache, void* v_cache, const int32_t* src,
                             int32_t num_blocks, int32_t* err, int sms,
                             cudaStream_t stream);
 
+// Up to four host -> device copies in one kernel launch: src is the mapped
+// device address of pinned host memory, both ends 16-byte aligned, n16 the
+// length in 16-byte units (0: unused).
+constexpr int kUploadSegs = 4;
+struct UploadSeg {
+  const uint4* src = nullptr;
+  uint4* dst = nullptr;
+  int64_t n16 = 0;
+};
+struct UploadArgs {
+  UploadSeg seg[kUploadSegs];
+};
+cudaError_t launch_upload(const UploadArgs& a, int sms, cudaStream_t stream);
+
 // Table patches (row, index, value) x n applied to device tables [rows, width].
 cudaError_t launch_table_patch(int32_t* tables, int32_t width, const int32_t* patches,
                                int32_t n, cudaStream_t stream);

@@ -908,6 +908,7 @@ struct BatchSet {
   float* d_out = nullptr;    // [n, H, d]
   char* d_stage = nullptr;   // slots int64 [n] | lens [n] | cow src [n] | dst [n] | patches
   char* h_stage = nullptr;   // pinned mirror of d_stage
+  const char* h_stage_dev = nullptr;   // its mapped device address (null: not mapped)
   cudaEvent_t up = nullptr, done = nullptr, down = nullptr;
   bool used = false;
 };
@@ -933,9 +934,43 @@ struct pa_batch {
   std::vector<int32_t> patches;
   BatchSet set[kBatchSets];
   int64_t steps = 0;
+  // The last step's output is downloaded by the next step call, after that
+  // step's uploads, or by pa_batch_sync: the download waits for the step's
+  // kernels, and when the two copy streams share one hardware queue a copy
+  // queued ahead of the next uploads holds them up until those kernels end.
+  int32_t pending = -1;                  // set of the step whose output is not queued yet
+  float* pending_out = nullptr;
 };
 
 namespace {
+
+// The device address of pinned host memory mapped into the current device's
+// address space, or null (pageable memory, or not visible to this device).
+const void* mapped_host(const void* h) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, h) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
+// Queue the download of the output of set k's last step into h_out, after
+// that step's kernels.
+bool queue_download(pa_batch* b, int32_t k, float* h_out) {
+  BatchSet& S = b->set[k];
+  return cudaStreamWaitEvent(b->down, S.done, 0) == cudaSuccess &&
+         cudaMemcpyAsync(h_out, S.d_out, b->out_bytes, cudaMemcpyDeviceToHost, b->down) ==
+             cudaSuccess &&
+         cudaEventRecord(S.down, b->down) == cudaSuccess;
+}
+
+bool flush_download(pa_batch* b) {
+  if (b->pending < 0) return true;
+  const bool ok = queue_download(b, b->pending, b->pending_out);
+  b->pending = -1;
+  return ok;
+}
 
 void free_batch(pa_batch* b) {
   for (auto& s : b->set) {
@@ -991,9 +1026,14 @@ pa_status pa_batch_create(pa_pool* p, const int32_t* seqs, int32_t n, int32_t H,
   b->kv_bytes = size_t(n) * p->num_kv_heads * p->head_dim * eq;
   b->out_bytes = size_t(n) * H * p->head_dim * sizeof(float);
   b->patch_cap = 4 * n;
-  b->stage_bytes = size_t(n) * (8 + 4 + 8) + size_t(b->patch_cap) * 12;
+  b->stage_bytes = (size_t(n) * (8 + 4 + 8) + size_t(b->patch_cap) * 12 + 15) & ~size_t(15);
   b->ws_bytes = pa_decode_workspace_bytes(p, n, H, max_blocks, partition_tokens);
-  bool ok = cudaStreamCreateWithFlags(&b->up, cudaStreamNonBlocking) == cudaSuccess &&
+  // the upload stream at the greatest priority: its kernel takes the first SM
+  // slot that frees up, ahead of the rest of a decode grid
+  int least_prio = 0, greatest_prio = 0;
+  cudaDeviceGetStreamPriorityRange(&least_prio, &greatest_prio);
+  bool ok = cudaStreamCreateWithPriority(&b->up, cudaStreamNonBlocking, greatest_prio) ==
+                cudaSuccess &&
             cudaStreamCreateWithFlags(&b->down, cudaStreamNonBlocking) == cudaSuccess &&
             cudaMalloc(&b->d_tables, size_t(n) * max_blocks * sizeof(int32_t)) == cudaSuccess &&
             (b->ws_bytes == 0 || cudaMalloc(&b->d_ws, b->ws_bytes) == cudaSuccess);
@@ -1012,6 +1052,13 @@ pa_status pa_batch_create(pa_pool* p, const int32_t* seqs, int32_t n, int32_t H,
     free_batch(b);
     cudaGetLastError();
     return PA_ERR_CUDA;
+  }
+  for (auto& s : b->set) {
+    void* dev = nullptr;
+    if (cudaHostGetDevicePointer(&dev, s.h_stage, 0) == cudaSuccess)
+      s.h_stage_dev = static_cast<const char*>(dev);
+    else
+      cudaGetLastError();                // not mapped: the step copies it
   }
   // the tables as they stand, uploaded once
   b->mirror.assign(size_t(n) * max_blocks, 0);
@@ -1108,16 +1155,42 @@ pa_status pa_batch_step(pa_batch* b, const void* h_q, const void* h_key, const v
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   bool ok = true;
-  // uploads, once this set's buffers are no longer read by its last step
+  // uploads, once this set's buffers are no longer read by its last step:
+  // one kernel that reads the four host buffers where all are pinned and
+  // mapped, 16-byte aligned and whole 16-byte units long; else four copies.
+  // Quantised pools keep the copies: their decode fills the SMs' shared
+  // memory, and an upload CTA beside it displaces one of its CTAs.
   if (S.used) ok = cudaStreamWaitEvent(b->up, S.done, 0) == cudaSuccess;
-  ok = ok && cudaMemcpyAsync(S.d_stage, S.h_stage, staged, cudaMemcpyHostToDevice, b->up) ==
-                 cudaSuccess &&
-       cudaMemcpyAsync(S.d_q, h_q, b->q_bytes, cudaMemcpyHostToDevice, b->up) == cudaSuccess &&
-       cudaMemcpyAsync(S.d_k, h_key, b->kv_bytes, cudaMemcpyHostToDevice, b->up) ==
-           cudaSuccess &&
-       cudaMemcpyAsync(S.d_v, h_value, b->kv_bytes, cudaMemcpyHostToDevice, b->up) ==
-           cudaSuccess &&
-       cudaEventRecord(S.up, b->up) == cudaSuccess;
+  const size_t staged16 = (staged + 15) & ~size_t(15);
+  const bool try_launch = !is_q8(p->dtype);
+  const void* src[4] = {S.h_stage_dev, try_launch ? mapped_host(h_q) : nullptr,
+                        try_launch ? mapped_host(h_key) : nullptr,
+                        try_launch ? mapped_host(h_value) : nullptr};
+  void* dst[4] = {S.d_stage, S.d_q, S.d_k, S.d_v};
+  const size_t len[4] = {staged16, b->q_bytes, b->kv_bytes, b->kv_bytes};
+  bool one_launch = try_launch;
+  for (int i = 0; i < 4; ++i)
+    one_launch = one_launch && src[i] && reinterpret_cast<uintptr_t>(src[i]) % 16 == 0 &&
+                 reinterpret_cast<uintptr_t>(dst[i]) % 16 == 0 && len[i] % 16 == 0;
+  if (ok && one_launch) {
+    pa::UploadArgs ua;
+    for (int i = 0; i < 4; ++i)
+      ua.seg[i] = {static_cast<const uint4*>(src[i]), static_cast<uint4*>(dst[i]),
+                   int64_t(len[i] / 16)};
+    ok = pa::launch_upload(ua, p->sms, b->up) == cudaSuccess;
+  } else if (ok) {
+    ok = cudaMemcpyAsync(S.d_stage, S.h_stage, staged, cudaMemcpyHostToDevice, b->up) ==
+             cudaSuccess &&
+         cudaMemcpyAsync(S.d_q, h_q, b->q_bytes, cudaMemcpyHostToDevice, b->up) ==
+             cudaSuccess &&
+         cudaMemcpyAsync(S.d_k, h_key, b->kv_bytes, cudaMemcpyHostToDevice, b->up) ==
+             cudaSuccess &&
+         cudaMemcpyAsync(S.d_v, h_value, b->kv_bytes, cudaMemcpyHostToDevice, b->up) ==
+             cudaSuccess;
+  }
+  ok = ok && cudaEventRecord(S.up, b->up) == cudaSuccess;
+  // the previous step's download, now that this step's uploads are ahead of it
+  ok = ok && flush_download(b);
   // kernels on the caller's stream, after the uploads and after the download
   // of this set's previous output
   ok = ok && cudaStreamWaitEvent(s, S.up, 0) == cudaSuccess;
@@ -1136,13 +1209,10 @@ pa_status pa_batch_step(pa_batch* b, const void* h_q, const void* h_key, const v
            : pa_decode_append(p, S.d_q, S.d_k, S.d_v, d_slots, n, b->H, b->d_tables, MB,
                               d_lens, scale, b->part, b->d_ws, b->ws_bytes, S.d_out, stream);
   if (st != PA_OK) return st;
-  // download on its own stream
-  ok = cudaEventRecord(S.done, s) == cudaSuccess &&
-       cudaStreamWaitEvent(b->down, S.done, 0) == cudaSuccess &&
-       cudaMemcpyAsync(h_out, S.d_out, b->out_bytes, cudaMemcpyDeviceToHost, b->down) ==
-           cudaSuccess &&
-       cudaEventRecord(S.down, b->down) == cudaSuccess;
-  if (!ok) return PA_ERR_CUDA;
+  // the download goes on the download stream with the next call (or sync)
+  if (cudaEventRecord(S.done, s) != cudaSuccess) return PA_ERR_CUDA;
+  b->pending = int32_t(b->steps % kBatchSets);
+  b->pending_out = h_out;
   S.used = true;
   ++b->steps;
   return PA_OK;
@@ -1193,6 +1263,7 @@ pa_status pa_batch_set_window(pa_batch* b, int32_t window, int32_t sinks) {
 pa_status pa_batch_sync(pa_batch* b) {
   if (!b) return PA_ERR_INVALID_ARG;
   pa::DeviceScope on_pool_device(b->pool->dev_id);
+  if (!flush_download(b)) return PA_ERR_CUDA;
   for (auto& s : b->set)
     if (s.used && cudaEventSynchronize(s.down) != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
@@ -1201,6 +1272,7 @@ pa_status pa_batch_sync(pa_batch* b) {
 pa_status pa_batch_free(pa_batch* b) {
   if (!b) return PA_OK;
   pa::DeviceScope on_pool_device(b->pool->dev_id);
+  flush_download(b);
   cudaDeviceSynchronize();
   free_batch(b);
   return PA_OK;

@@ -179,3 +179,37 @@ def test_batch_window_steps_match_separate_calls_and_oracle(kind):
         assert worst <= TOL_DECODE, (step, worst)
     assert g.pool.get_error() == 0
     batch.close()
+
+
+def test_batch_upload_paths_agree():
+    """The step's uploads take one kernel that reads pinned, mapped host
+    buffers, or one copy per buffer for pageable or unaligned ones: both give
+    the same tables and bit-identical outputs."""
+    w = _workload("bf16")
+    runs = [DeviceRun(w).apply(w.setup) for _ in range(2)]
+    seqs = w.decode_seqs
+    n, mb = len(seqs), 40
+    batches = [pa.Batch(r.pool, seqs, w.num_heads, mb) for r in runs]
+    outs = [torch.empty((n, w.num_heads, w.head_dim), dtype=torch.float32).pin_memory(),
+            torch.empty((n, w.num_heads, w.head_dim), dtype=torch.float32)]
+    for step in range(3):
+        q, k, v = _step_inputs(w, step)
+        # the host buffers stay referenced until the steps are synchronised
+        pinned = (q.pin_memory(), k.pin_memory(), v.pin_memory())
+        # pageable K/V and a pinned query 8 bytes off a 16-byte boundary
+        buf = torch.empty(q.numel() + 4, dtype=q.dtype).pin_memory()
+        q_off = buf[4:4 + q.numel()].view(q.shape)
+        q_off.copy_(q)
+        assert q_off.data_ptr() % 16 == 8
+        other = (q_off, k.clone(), v.clone())
+        batches[0].step(*pinned, outs[0])
+        batches[1].step(*other, outs[1])
+        for b in batches:
+            b.sync()
+        assert np.array_equal(outs[0].numpy(), outs[1].numpy()), step
+        for s in seqs:
+            assert runs[0].pool.table(s) == runs[1].pool.table(s)
+    for r in runs:
+        assert r.pool.get_error() == 0
+    for b in batches:
+        b.close()
