@@ -213,3 +213,33 @@ def test_batch_upload_paths_agree():
         assert r.pool.get_error() == 0
     for b in batches:
         b.close()
+
+
+def test_batch_pipelined_steps_deliver_every_output():
+    """Steps queued back to back with one sync at the end (each download is
+    queued by the next step call or by the sync), and a last step completed
+    by closing the batch: every output equals the same step run with a sync
+    after each call."""
+    w = _workload("bf16")
+    runs = [DeviceRun(w).apply(w.setup) for _ in range(2)]
+    seqs = w.decode_seqs
+    n, mb, steps = len(seqs), 40, 5
+    shape = (n, w.num_heads, w.head_dim)
+    inputs = [tuple(t.pin_memory() for t in _step_inputs(w, s)) for s in range(steps)]
+    piped = [torch.full(shape, float("nan")).pin_memory() for _ in range(steps)]
+    ref = [torch.empty(shape, dtype=torch.float32).pin_memory() for _ in range(steps)]
+    a = pa.Batch(runs[0].pool, seqs, w.num_heads, mb)
+    for s in range(steps - 1):
+        a.step(*inputs[s], piped[s])
+    a.sync()
+    a.step(*inputs[steps - 1], piped[steps - 1])
+    a.close()                                        # completes the last download
+    b = pa.Batch(runs[1].pool, seqs, w.num_heads, mb)
+    for s in range(steps):
+        b.step(*inputs[s], ref[s])
+        b.sync()
+    b.close()
+    for s in range(steps):
+        assert np.array_equal(piped[s].numpy(), ref[s].numpy()), s
+    for r in runs:
+        assert r.pool.get_error() == 0
