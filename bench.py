@@ -677,10 +677,10 @@ def run_e2e_batch(args, S, dist, device, part, win=0, sinks=0):
     downloads the output; pa_batch_rollback then gives every sequence's token
     back (host-only) so that every step is the same step.  The timed region
     holds K steps and the final wait for the last output.  The transfers of
-    consecutive steps overlap their neighbours' kernels (two buffer sets; the
-    uploads are one kernel that reads the pinned inputs in place, copies on
-    quantised pools; each download is queued behind the next step's
-    uploads).  A copy-on-write of a shared partial tail happens in the first
+    consecutive steps overlap their neighbours' kernels (two buffer sets; an
+    upload of up to 1 MiB is one kernel that reads the pinned inputs in place,
+    larger ones and those of quantised pools are copies; each download is
+    queued behind the next step's uploads).  A copy-on-write of a shared partial tail happens in the first
     step only (the tail is private afterwards), as in serving."""
     import torch
     import paged_kv_cache_483_b200 as pa

@@ -459,9 +459,9 @@ pa_status pa_batch_create(pa_pool* pool, const int32_t* seqs, int32_t n,
  * The plan, the table entries that changed since the previous step and the
  * inputs are uploaded on the batch's upload stream (highest priority): by one
  * kernel that reads the host buffers in place when all are pinned, mapped into
- * the device's address space and 16-byte aligned and the pool is bf16 or
- * float32, else by one copy per buffer (pageable memory works, synchronously
- * slower); the table patches,
+ * the device's address space and 16-byte aligned, the pool is bf16 or float32
+ * and the step's upload is at most 1 MiB; else by one copy per buffer
+ * (pageable memory works, synchronously slower); the table patches,
  * copy-on-write copies and the fused append + decode (pa_decode_append, or
  * pa_decode_window_append after pa_batch_set_window) run on `stream`; the
  * output is downloaded on the batch's download stream.  That download is

@@ -900,6 +900,8 @@ pa_status pa_prefill_chunk(pa_pool* p, const void* q, int32_t B,
 namespace {
 
 constexpr int kBatchSets = 2;
+// Largest step upload that one kernel reads from host memory (above it, copies).
+constexpr size_t kUploadKernelMaxBytes = size_t(1) << 20;
 
 struct BatchSet {
   void* d_q = nullptr;       // [n, H, d] pool dtype (bf16 on int8 / FP8 pools)
@@ -1158,11 +1160,14 @@ pa_status pa_batch_step(pa_batch* b, const void* h_q, const void* h_key, const v
   // uploads, once this set's buffers are no longer read by its last step:
   // one kernel that reads the four host buffers where all are pinned and
   // mapped, 16-byte aligned and whole 16-byte units long; else four copies.
-  // Quantised pools keep the copies: their decode fills the SMs' shared
-  // memory, and an upload CTA beside it displaces one of its CTAs.
+  // The kernel saves the copies' fixed costs, which dominate small uploads;
+  // its CTAs hold SM slots for as long as the PCIe reads take, so large
+  // uploads (and every upload on quantised pools, whose decode fills the SMs'
+  // shared memory) go to the copy engines, which leave the decode alone.
   if (S.used) ok = cudaStreamWaitEvent(b->up, S.done, 0) == cudaSuccess;
   const size_t staged16 = (staged + 15) & ~size_t(15);
-  const bool try_launch = !is_q8(p->dtype);
+  const bool try_launch = !is_q8(p->dtype) &&
+                          staged16 + b->q_bytes + 2 * b->kv_bytes <= kUploadKernelMaxBytes;
   const void* src[4] = {S.h_stage_dev, try_launch ? mapped_host(h_q) : nullptr,
                         try_launch ? mapped_host(h_key) : nullptr,
                         try_launch ? mapped_host(h_value) : nullptr};
