@@ -14,16 +14,16 @@
 // tile fetched into shared memory.  Keys are visited in tiles of 128 (eight
 // paged blocks, each fetched by TMA as two 64-column boxes with the 128-byte
 // swizzle, landing in the UMMA K-major layout).
-//   warp 0      TMA producer: Q_A, Q_B once; K and V tiles into 2-stage rings
-//               (K(j+1) is issued before V(j): a K stage frees after its two
-//               QK^T, well before the V stage of the same tile).
+//   warp 0      TMA producer of Q_A, Q_B (once) and of the K ring (2 stages);
+//   warp 2      TMA producer of the V ring (2 stages).  In each ring, lanes
+//               0-7 issue the two boxes of one block each.
 //   warp 1      one thread issues tcgen05.mma in the order
 //                 ... PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1) ...
 //               S_X = Q_X K^T lands in TMEM; O_X += P_X V reads P_X from TMEM
 //               (the softmax writes it over S_X) and V from shared memory.
-//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B; one thread per
-//               row = TMEM lane.  While one tile's softmax runs on the CUDA
-//               cores the tensor core works on the other tile.
+//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B; one thread
+//               per row = TMEM lane.  While one tile's softmax runs on the
+//               CUDA cores the tensor core works on the other tile.
 // TMEM (512 columns): S_A/P_A [0,128), S_B/P_B [128,256), O_A, O_B.
 // The tensor core executes one CTA's MMAs in issue order, so when QK_X(j) has
 // completed, PV_X(j-1) has too: the softmax may then rescale O_X in TMEM.  O
