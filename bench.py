@@ -738,25 +738,24 @@ def run_e2e_steps(args, S, dist, device, is_prefill, part, win, sinks):
     host memory, runs the step's kernels and reads the output back; then the
     step's tokens are rolled back (pa_seq_truncate) so that every step is the
     same step.  Plans, copies and the rollback are inside the timed region.
-    A copy-on-write of a shared partial tail happens in the first planned
-    step only (the tail is private afterwards), as in serving."""
+    Two buffer sets and two copy streams let a step's uploads and the previous
+    step's download run while the kernels of their neighbours do.  A
+    copy-on-write of a shared partial tail happens in the first planned step
+    only (the tail is private afterwards), as in serving."""
     import torch
     pool = S.pool
     stream = torch.cuda.current_stream(device)
+    up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
     w = S.w
     h_q = S.q.cpu().pin_memory()
-    h_out = torch.empty(S.out.shape, dtype=torch.float32).pin_memory()
     h_lens = S.lens.cpu().pin_memory()
-    d_q, d_lens = torch.empty_like(S.q), torch.empty_like(S.lens)
     bi = h_q.numel() * h_q.element_size() + h_lens.numel() * 4
     seqs = [op.args[0] for op in w.step]
     n_new = [op.args[1] for op in w.step]
     plan = bool(w.step)
     if plan:
         h_k, h_v = S.step_k.cpu().pin_memory(), S.step_v.cpu().pin_memory()
-        d_k, d_v = torch.empty_like(S.step_k), torch.empty_like(S.step_v)
         T = int(S.slots.numel())
-        d_slots = torch.empty_like(S.slots)
         d_cow = torch.empty(2 * len(seqs), dtype=torch.int32, device=device)
         ring = _PinnedRing(lambda: (torch.empty(T, dtype=torch.int64).pin_memory(),
                                     torch.empty(2 * len(seqs), dtype=torch.int32).pin_memory()))
@@ -764,21 +763,44 @@ def run_e2e_steps(args, S, dist, device, is_prefill, part, win, sinks):
         lens_now = [pool.table(s)[1] for s in seqs]
         start = [L - k for L, k in zip(lens_now, n_new)]
         pool.truncate(seqs, start)                       # undo the set-up's plan
-    bo = h_out.numel() * 4
+    sets = []
+    for i in range(2):
+        b = {"q": torch.empty_like(S.q), "lens": torch.empty_like(S.lens),
+             "out": S.out if i == 0 else torch.empty_like(S.out),
+             "h_out": torch.empty(S.out.shape, dtype=torch.float32).pin_memory(),
+             "up": torch.cuda.Event(), "done": torch.cuda.Event(), "down": torch.cuda.Event(),
+             "used": False}
+        if plan:
+            b.update(k=torch.empty_like(S.step_k), v=torch.empty_like(S.step_v),
+                     slots=torch.empty_like(S.slots))
+        sets.append(b)
+    bo = S.out.numel() * 4
     K = max(1, args.e2e_steps)   # its own count: a serving loop's steady state, not the timed K
     fused = (not is_prefill) and plan and not S.q8
     cow_bytes = [0]
+    count = [0]
 
     def step():
-        d_q.copy_(h_q, non_blocking=True)
-        d_lens.copy_(h_lens, non_blocking=True)
+        b = sets[count[0] % 2]
+        count[0] += 1
         if plan:
             slots, cow = pool.plan_append(seqs, n_new)            # step a1, on the host
             (hs, hc), ev = ring.take()
             hs.numpy()[:] = slots
-            d_slots.copy_(hs, non_blocking=True)
-            d_k.copy_(h_k, non_blocking=True)
-            d_v.copy_(h_v, non_blocking=True)
+        with torch.cuda.stream(up):
+            if b["used"]:
+                up.wait_event(b["done"])          # this set's last kernels have read it
+            b["q"].copy_(h_q, non_blocking=True)
+            b["lens"].copy_(h_lens, non_blocking=True)
+            if plan:
+                b["slots"].copy_(hs, non_blocking=True)
+                b["k"].copy_(h_k, non_blocking=True)
+                b["v"].copy_(h_v, non_blocking=True)
+            b["up"].record(up)
+        stream.wait_event(b["up"])
+        if b["used"]:
+            stream.wait_event(b["down"])          # and its last output has been read back
+        if plan:
             if cow:
                 n = len(cow)
                 hc.numpy()[:n] = [c[0] for c in cow]
@@ -786,23 +808,30 @@ def run_e2e_steps(args, S, dist, device, is_prefill, part, win, sinks):
                 d_cow[:2 * n].copy_(hc[:2 * n], non_blocking=True)
                 pool.cow_copy(d_cow[:n], d_cow[n:2 * n], stream)
                 cow_bytes[0] += 8 * n
-            ev.record(stream)
+            ev.record(stream)                     # after both copies of the pinned plan
             if not fused:
-                pool.reshape_and_cache(d_k, d_v, d_slots, stream)
+                pool.reshape_and_cache(b["k"], b["v"], b["slots"], stream)
         if is_prefill:
-            pool.prefill_chunk(d_q, S.tables, d_lens, out=S.out, stream=stream)
+            pool.prefill_chunk(b["q"], S.tables, b["lens"], out=b["out"], stream=stream)
         elif fused and win:
-            pool.decode_window_append(d_q, d_k, d_v, d_slots, S.tables, d_lens, win, sinks,
-                                      out=S.out, partition_tokens=part, stream=stream)
+            pool.decode_window_append(b["q"], b["k"], b["v"], b["slots"], S.tables, b["lens"],
+                                      win, sinks, out=b["out"], partition_tokens=part,
+                                      stream=stream)
         elif fused:
-            pool.decode_append(d_q, d_k, d_v, d_slots, S.tables, d_lens, out=S.out,
-                               partition_tokens=part, stream=stream)
+            pool.decode_append(b["q"], b["k"], b["v"], b["slots"], S.tables, b["lens"],
+                               out=b["out"], partition_tokens=part, stream=stream)
         elif win:
-            pool.decode_window(d_q, S.tables, d_lens, win, sinks, out=S.out,
+            pool.decode_window(b["q"], S.tables, b["lens"], win, sinks, out=b["out"],
                                partition_tokens=part, stream=stream)
         else:
-            pool.decode(d_q, S.tables, d_lens, out=S.out, partition_tokens=part, stream=stream)
-        h_out.copy_(S.out, non_blocking=True)
+            pool.decode(b["q"], S.tables, b["lens"], out=b["out"], partition_tokens=part,
+                        stream=stream)
+        b["done"].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(b["done"])
+            b["h_out"].copy_(b["out"], non_blocking=True)
+            b["down"].record(down)
+        b["used"] = True
         if plan:
             pool.truncate(seqs, start)                            # roll the step back
 
@@ -813,8 +842,10 @@ def run_e2e_steps(args, S, dist, device, is_prefill, part, win, sinks):
     cow_bytes[0] = 0
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    up.wait_stream(stream)                        # the first uploads start after a
     for _ in range(K):
         step()
+    stream.wait_stream(down)                      # b after the last download
     b.record(stream)
     torch.cuda.synchronize()
     ms = dist.max(a.elapsed_time(b) / K, device)
